@@ -1,0 +1,203 @@
+"""Plain CPU oracle for blockwise codebook quantization.
+
+TEST INFRASTRUCTURE ONLY: the tests, ``__graft_entry__.smoke()`` and the
+``cpu_baseline`` / ``--impl reference`` legs of ``bench.py`` may import this
+package. The library (``blockwise_bit_codebook_b200``) never imports it, and
+it never imports the library. Each function cites the passage it follows:
+
+* k-bit codec: bitsandbytes k-bit patch series, tests/test_kbit_quantization.py
+  (quantize_kbit_ref, dequantize_kbit_ref, pack_kbit_ref, unpack_kbit_ref) and
+  csrc/ops.cu (kQuantizeBlockwise_kbit, kDequantizeBlockwise_kbit).
+* nested 4-bit dequant: "Fuse nested 4-bit scale reconstruction on SM103",
+  Summary and Implementation.
+
+Arrays: fp32 as ``np.float32``; fp16 and bfloat16 as their raw 16-bit patterns
+in ``np.uint16`` (numpy has no bfloat16). dtype names are "f16", "bf16", "f32".
+
+Parity status of each function (see the pins in tests/test_oracle_*.py):
+every function here is pinned; none is "parity unpinned".
+"""
+import ctypes as ct
+import os
+
+import numpy as np
+
+from . import build as _build
+from .codebook import normal_float_codebook, unnormalized_quantiles  # noqa: F401
+
+_DT = {"f16": 0, "bf16": 1, "f32": 2}
+KBIT_BLOCKSIZE = 32
+
+_lib = None
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        path = _build.build()
+        L = ct.CDLL(path)
+        P = ct.c_void_p
+        I64 = ct.c_int64
+        L.orc_kbit_quantize.argtypes = [P, ct.c_int, I64, ct.c_int, P, P, P, P]
+        L.orc_kbit_quantize.restype = ct.c_int
+        L.orc_kbit_dequantize.argtypes = [P, P, P, ct.c_int, I64, ct.c_int, P]
+        L.orc_kbit_dequantize.restype = ct.c_int
+        L.orc_nested_dequantize.argtypes = [P, P, P, P, ct.c_float, P, I64, I64, I64, ct.c_int, P]
+        L.orc_nested_dequantize.restype = ct.c_int
+        L.orc_kbit_pack.argtypes = [P, I64, ct.c_int, P]
+        L.orc_kbit_unpack.argtypes = [P, I64, ct.c_int, P]
+        L.orc_nearest_entry.argtypes = [ct.c_float, P, ct.c_int]
+        L.orc_nearest_entry.restype = ct.c_int
+        L.orc_nested_scale.argtypes = [ct.c_float, ct.c_float, ct.c_float]
+        L.orc_nested_scale.restype = ct.c_float
+        for f in ("orc_f32_to_f16_array", "orc_f32_to_bf16_array"):
+            getattr(L, f).argtypes = [P, I64, P]
+        L.orc_f16_to_f32_array.argtypes = [P, I64, P]
+        _lib = L
+    return _lib
+
+
+def _p(a: np.ndarray):
+    return a.ctypes.data_as(ct.c_void_p)
+
+
+def _c(a, dtype):
+    return np.ascontiguousarray(a, dtype=dtype)
+
+
+def num_blocks(n: int, bs: int = KBIT_BLOCKSIZE) -> int:
+    return (n + bs - 1) // bs
+
+
+def f32_to_f16_bits(x) -> np.ndarray:
+    x = _c(x, np.float32).reshape(-1)
+    out = np.empty(x.size, np.uint16)
+    lib().orc_f32_to_f16_array(_p(x), x.size, _p(out))
+    return out
+
+
+def f32_to_bf16_bits(x) -> np.ndarray:
+    x = _c(x, np.float32).reshape(-1)
+    out = np.empty(x.size, np.uint16)
+    lib().orc_f32_to_bf16_array(_p(x), x.size, _p(out))
+    return out
+
+
+def f16_bits_to_f32(h) -> np.ndarray:
+    h = _c(h, np.uint16).reshape(-1)
+    out = np.empty(h.size, np.float32)
+    lib().orc_f16_to_f32_array(_p(h), h.size, _p(out))
+    return out
+
+
+def bf16_bits_to_f32(h) -> np.ndarray:
+    h = _c(h, np.uint16).reshape(-1)
+    return (h.astype(np.uint32) << 16).view(np.float32)
+
+
+def nearest_entry(xn: float, codebook) -> int:
+    cb = _c(codebook, np.float32)
+    return lib().orc_nearest_entry(ct.c_float(xn), _p(cb), cb.size)
+
+
+def kbit_pack(idx, K: int) -> np.ndarray:
+    idx = _c(idx, np.uint8).reshape(-1)
+    n = idx.size
+    out = np.empty(num_blocks(n) * K, np.uint32)
+    lib().orc_kbit_pack(_p(idx), n, K, _p(out))
+    return out
+
+
+def kbit_unpack(packed, K: int, n: int) -> np.ndarray:
+    packed = _c(packed, np.uint32).reshape(-1)
+    assert packed.size >= num_blocks(n) * K
+    out = np.empty(n, np.uint8)
+    lib().orc_kbit_unpack(_p(packed), n, K, _p(out))
+    return out
+
+
+def kbit_quantize(A, dtype: str, K: int, codebook, return_indices: bool = False):
+    """Quantize; returns (packed uint32[nb*K], absmax f32[nb]) (+ per-lane indices u8[nb*32]).
+
+    A holds fp32 values for dtype "f32", raw 16-bit patterns for "f16"/"bf16".
+    """
+    A = _c(A, np.float32 if dtype == "f32" else np.uint16).reshape(-1)
+    cb = _c(codebook, np.float32)
+    assert cb.size == (1 << K)
+    n = A.size
+    nb = num_blocks(n)
+    absmax = np.empty(nb, np.float32)
+    packed = np.empty(nb * K, np.uint32)
+    idx = np.empty(nb * KBIT_BLOCKSIZE, np.uint8) if return_indices else None
+    rc = lib().orc_kbit_quantize(_p(A), _DT[dtype], n, K, _p(cb), _p(absmax), _p(packed),
+                                 _p(idx) if idx is not None else None)
+    assert rc == 0
+    return (packed, absmax, idx) if return_indices else (packed, absmax)
+
+
+def kbit_dequantize(packed, absmax, codebook, K: int, n: int, dtype: str) -> np.ndarray:
+    """Returns fp32 values ("f32") or raw 16-bit patterns ("f16"/"bf16")."""
+    packed = _c(packed, np.uint32).reshape(-1)
+    absmax = _c(absmax, np.float32).reshape(-1)
+    cb = _c(codebook, np.float32)
+    nb = num_blocks(n)
+    assert packed.size >= nb * K and absmax.size >= nb and cb.size == (1 << K)
+    out = np.empty(n, np.float32 if dtype == "f32" else np.uint16)
+    rc = lib().orc_kbit_dequantize(_p(packed), _p(absmax), _p(cb), K, n, _DT[dtype], _p(out))
+    assert rc == 0
+    return out
+
+
+def nested_scale(code2_val: float, absmax2_val: float, offset: float) -> float:
+    """fl(fl(code2 * absmax2) + offset) in fp32, returned as a Python float."""
+    return float(np.float32(lib().orc_nested_scale(code2_val, absmax2_val, offset)))
+
+
+def nested_dequantize(codes, absmax_q, code2, absmax2, offset: float, code4,
+                      n: int, blocksize: int, blocksize2: int, dtype: str) -> np.ndarray:
+    codes = _c(codes, np.uint8).reshape(-1)
+    absmax_q = _c(absmax_q, np.uint8).reshape(-1)
+    code2 = _c(code2, np.float32)
+    absmax2 = _c(absmax2, np.float32).reshape(-1)
+    code4 = _c(code4, np.float32)
+    nbo = num_blocks(n, blocksize)
+    assert codes.size >= (n + 1) // 2 and absmax_q.size >= nbo
+    assert absmax2.size >= num_blocks(nbo, blocksize2) and code2.size == 256 and code4.size == 16
+    out = np.empty(n, np.float32 if dtype == "f32" else np.uint16)
+    rc = lib().orc_nested_dequantize(_p(codes), _p(absmax_q), _p(code2), _p(absmax2),
+                                     ct.c_float(offset), _p(code4), n, blocksize, blocksize2,
+                                     _DT[dtype], _p(out))
+    assert rc == 0
+    return out
+
+
+def kbit_quantize_threads(A, dtype: str, K: int, codebook, threads: int):
+    """The same quantize, run over contiguous block ranges on `threads` host threads.
+
+    ctypes releases the GIL during the C call, so Python threads run the C loop in
+    parallel; each range is a whole number of 32-element blocks, so the result is
+    identical to the single-threaded call.
+    """
+    import threading
+
+    A = _c(A, np.float32 if dtype == "f32" else np.uint16).reshape(-1)
+    cb = _c(codebook, np.float32)
+    n = A.size
+    nb = num_blocks(n)
+    absmax = np.empty(nb, np.float32)
+    packed = np.empty(nb * K, np.uint32)
+    per = (nb + threads - 1) // threads
+    jobs = []
+    for t in range(threads):
+        b0, b1 = t * per, min(nb, (t + 1) * per)
+        if b0 >= b1:
+            break
+        e0, e1 = b0 * KBIT_BLOCKSIZE, min(n, b1 * KBIT_BLOCKSIZE)
+        sub = A[e0:e1]
+        jobs.append(threading.Thread(target=lambda s=sub, b0=b0, b1=b1: lib().orc_kbit_quantize(
+            _p(s), _DT[dtype], s.size, K, _p(cb), _p(absmax[b0:b1]), _p(packed[b0 * K:b1 * K]), None)))
+    for j in jobs:
+        j.start()
+    for j in jobs:
+        j.join()
+    return packed, absmax
