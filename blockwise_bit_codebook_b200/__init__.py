@@ -1,0 +1,29 @@
+"""Blockwise bit-codebook quantization on NVIDIA B200 (sm_100a).
+
+Thin Python binding of the C ABI in include/bbc.h (libbbc.so, built in-tree by
+``python -m blockwise_bit_codebook_b200.build``). The functions carry the C
+names and only marshal arguments: every step of every operation runs in the
+library's CUDA kernels. torch is used for device memory and streams only.
+
+    kbit_quantize(A, K, codebook)                       -> (packed, absmax)
+    kbit_dequantize(packed, absmax, codebook, K, n, dtype) -> out
+    dequantize_4bit_nested(codes, absmax_q, code2, absmax2, offset, code4,
+                           n, blocksize, dtype)         -> out
+    bbc_nf_codebook(K)                                  -> np.float32[2^K] (host)
+
+There is no CPU fallback: if libbbc.so is missing or a call fails, an
+exception is raised.
+"""
+from ._native import (  # noqa: F401
+    BBC_BF16,
+    BBC_F16,
+    BBC_F32,
+    BBCError,
+    bbc_last_error,
+    bbc_nf_codebook,
+    dequantize_4bit_nested,
+    kbit_dequantize,
+    kbit_quantize,
+    library_path,
+    load_library,
+)

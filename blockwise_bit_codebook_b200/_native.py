@@ -1,0 +1,134 @@
+"""ctypes binding of libbbc.so (argument marshalling only)."""
+import ctypes as ct
+import os
+
+import numpy as np
+
+BBC_F16, BBC_BF16, BBC_F32 = 0, 1, 2
+_STATUS = {0: "BBC_OK", 1: "BBC_ERR_INVALID", 2: "BBC_ERR_UNSUPPORTED", 3: "BBC_ERR_CUDA"}
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_LIB_PATH = os.path.join(_HERE, "libbbc.so")
+_lib = None
+
+
+class BBCError(RuntimeError):
+    def __init__(self, fn: str, status: int, msg: str):
+        super().__init__(f"{fn} failed with {_STATUS.get(status, status)}: {msg}")
+        self.status = status
+
+
+def library_path() -> str:
+    return _LIB_PATH
+
+
+def load_library():
+    """Load libbbc.so; raises if it has not been built (there is no fallback)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(_LIB_PATH):
+        raise ImportError(f"{_LIB_PATH} is missing: build it with "
+                          "`python -m blockwise_bit_codebook_b200.build`")
+    L = ct.CDLL(_LIB_PATH)
+    P, I64, I = ct.c_void_p, ct.c_int64, ct.c_int
+    L.kbit_quantize.argtypes = [P, I, I64, I, I, P, P, P, P]
+    L.kbit_quantize.restype = I
+    L.kbit_dequantize.argtypes = [P, P, P, I, I, I64, I, P, P]
+    L.kbit_dequantize.restype = I
+    L.dequantize_4bit_nested.argtypes = [P, P, P, P, ct.c_float, P, I64, I, I, I, P, P]
+    L.dequantize_4bit_nested.restype = I
+    L.bbc_nf_codebook.argtypes = [I, P]
+    L.bbc_nf_codebook.restype = I
+    L.bbc_last_error.argtypes = []
+    L.bbc_last_error.restype = ct.c_char_p
+    _lib = L
+    return L
+
+
+def bbc_last_error() -> str:
+    return load_library().bbc_last_error().decode()
+
+
+def _check(fn: str, status: int):
+    if status != 0:
+        raise BBCError(fn, status, bbc_last_error())
+
+
+def _dt(dtype) -> int:
+    import torch
+    if isinstance(dtype, int):
+        return dtype
+    m = {torch.float16: BBC_F16, torch.bfloat16: BBC_BF16, torch.float32: BBC_F32}
+    if dtype not in m:
+        raise ValueError(f"unsupported dtype {dtype}")
+    return m[dtype]
+
+
+def _torch_dtype(dt: int):
+    import torch
+    return {BBC_F16: torch.float16, BBC_BF16: torch.bfloat16, BBC_F32: torch.float32}[dt]
+
+
+def _ptr(t):
+    return ct.c_void_p(t.data_ptr()) if t is not None else None
+
+
+def _stream(stream, device):
+    import torch
+    if stream is None:
+        stream = torch.cuda.current_stream(device)
+    return ct.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+def kbit_quantize(A, K: int, codebook, absmax=None, packed=None, blocksize: int = 32, stream=None):
+    """k-bit quantize a CUDA tensor (any shape, contiguous). Returns (packed, absmax)."""
+    import torch
+    L = load_library()
+    n = A.numel()
+    nb = (n + blocksize - 1) // blocksize if blocksize > 0 else 0
+    if absmax is None:
+        absmax = torch.empty(max(nb, 1), dtype=torch.float32, device=A.device)
+    if packed is None:
+        packed = torch.empty(max(nb * K, 1), dtype=torch.int32, device=A.device)
+    st = L.kbit_quantize(_ptr(A), _dt(A.dtype), n, K, blocksize, _ptr(codebook), _ptr(absmax),
+                         _ptr(packed), _stream(stream, A.device))
+    _check("kbit_quantize", st)
+    return packed, absmax
+
+
+def kbit_dequantize(packed, absmax, codebook, K: int, n: int, dtype, out=None, blocksize: int = 32,
+                    stream=None):
+    """Inverse of kbit_quantize; returns a 1-D CUDA tensor of n elements of `dtype`."""
+    import torch
+    L = load_library()
+    dt = _dt(dtype)
+    if out is None:
+        out = torch.empty(max(n, 1), dtype=_torch_dtype(dt), device=packed.device)
+    st = L.kbit_dequantize(_ptr(packed), _ptr(absmax), _ptr(codebook), K, blocksize, n, dt, _ptr(out),
+                           _stream(stream, packed.device))
+    _check("kbit_dequantize", st)
+    return out
+
+
+def dequantize_4bit_nested(codes, absmax_q, code2, absmax2, offset: float, code4, n: int,
+                           blocksize: int, dtype, out=None, blocksize2: int = 256, stream=None):
+    """Nested NF4/FP4 dequant; returns a 1-D CUDA tensor of n elements of `dtype`."""
+    import torch
+    L = load_library()
+    dt = _dt(dtype)
+    if out is None:
+        out = torch.empty(max(n, 1), dtype=_torch_dtype(dt), device=codes.device)
+    st = L.dequantize_4bit_nested(_ptr(codes), _ptr(absmax_q), _ptr(code2), _ptr(absmax2),
+                                  ct.c_float(offset), _ptr(code4), n, blocksize, blocksize2, dt,
+                                  _ptr(out), _stream(stream, codes.device))
+    _check("dequantize_4bit_nested", st)
+    return out
+
+
+def bbc_nf_codebook(K: int) -> np.ndarray:
+    """Host-side normal-float codebook (2^K fp32 values, ascending, max |c| = 1)."""
+    L = load_library()
+    out = np.empty(1 << K, np.float32)
+    _check("bbc_nf_codebook", L.bbc_nf_codebook(K, out.ctypes.data_as(ct.c_void_p)))
+    return out

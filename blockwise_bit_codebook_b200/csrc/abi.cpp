@@ -1,0 +1,111 @@
+// extern "C" entry points declared in include/bbc.h: host-side validation, then one launch.
+#include "bbc.h"
+
+#include <cuda_runtime.h>
+
+#include <cstdarg>
+#include <cstdio>
+#include <string>
+
+#include "launch.h"
+
+namespace {
+
+thread_local std::string g_last_error;
+
+int fail(int status, const char* fmt, ...) {
+    char buf[512];
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(buf, sizeof buf, fmt, ap);
+    va_end(ap);
+    g_last_error = buf;
+    return status;
+}
+
+int ok() {
+    g_last_error.clear();
+    return BBC_OK;
+}
+
+int cuda_status(cudaError_t e, const char* what) {
+    if (e == cudaSuccess) return ok();
+    return fail(BBC_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+bool valid_dtype(int dt) { return dt == BBC_F16 || dt == BBC_BF16 || dt == BBC_F32; }
+
+int elem_size(int dt) { return dt == BBC_F32 ? 4 : 2; }
+
+}  // namespace
+
+extern "C" {
+
+int kbit_quantize(const void* A, int dtype, int64_t n, int K, int blocksize,
+                  const float* codebook, float* absmax, uint32_t* packed, void* stream) {
+    if (!A || !codebook || !absmax || !packed)
+        return fail(BBC_ERR_INVALID, "kbit_quantize: null pointer argument");
+    if (n <= 0) return fail(BBC_ERR_INVALID, "kbit_quantize: n must be >= 1 (got %lld)", (long long)n);
+    if (K < 2 || K > 5) return fail(BBC_ERR_INVALID, "kbit_quantize: K must be 2..5 (got %d)", K);
+    if (!valid_dtype(dtype)) return fail(BBC_ERR_INVALID, "kbit_quantize: bad dtype %d", dtype);
+    if (blocksize != 32)
+        return fail(BBC_ERR_UNSUPPORTED, "kbit_quantize: blocksize must be 32 (got %d)", blocksize);
+    if (!aligned(A, elem_size(dtype)) || !aligned(codebook, 4) || !aligned(absmax, 4) || !aligned(packed, 4))
+        return fail(BBC_ERR_INVALID, "kbit_quantize: pointer not aligned to its element size");
+    const bool vec = aligned(A, 16);
+    return cuda_status(bbc::launch_kbit_quantize(A, dtype, n, K, codebook, absmax, packed, vec,
+                                                 static_cast<cudaStream_t>(stream)),
+                       "kbit_quantize launch");
+}
+
+int kbit_dequantize(const uint32_t* packed, const float* absmax, const float* codebook,
+                    int K, int blocksize, int64_t n, int out_dtype, void* out, void* stream) {
+    if (!packed || !absmax || !codebook || !out)
+        return fail(BBC_ERR_INVALID, "kbit_dequantize: null pointer argument");
+    if (n <= 0) return fail(BBC_ERR_INVALID, "kbit_dequantize: n must be >= 1 (got %lld)", (long long)n);
+    if (K < 2 || K > 5) return fail(BBC_ERR_INVALID, "kbit_dequantize: K must be 2..5 (got %d)", K);
+    if (!valid_dtype(out_dtype)) return fail(BBC_ERR_INVALID, "kbit_dequantize: bad dtype %d", out_dtype);
+    if (blocksize != 32)
+        return fail(BBC_ERR_UNSUPPORTED, "kbit_dequantize: blocksize must be 32 (got %d)", blocksize);
+    if (!aligned(out, elem_size(out_dtype)) || !aligned(codebook, 4) || !aligned(absmax, 4) || !aligned(packed, 4))
+        return fail(BBC_ERR_INVALID, "kbit_dequantize: pointer not aligned to its element size");
+    const bool vec = aligned(out, 16);
+    return cuda_status(bbc::launch_kbit_dequantize(packed, absmax, codebook, K, n, out_dtype, out, vec,
+                                                   static_cast<cudaStream_t>(stream)),
+                       "kbit_dequantize launch");
+}
+
+int dequantize_4bit_nested(const uint8_t* codes, const uint8_t* absmax_q, const float* code2,
+                           const float* absmax2, float offset, const float* code4,
+                           int64_t n, int blocksize, int blocksize2, int out_dtype, void* out,
+                           void* stream) {
+    if (!codes || !absmax_q || !code2 || !absmax2 || !code4 || !out)
+        return fail(BBC_ERR_INVALID, "dequantize_4bit_nested: null pointer argument");
+    if (n <= 0)
+        return fail(BBC_ERR_INVALID, "dequantize_4bit_nested: n must be >= 1 (got %lld)", (long long)n);
+    if (!valid_dtype(out_dtype))
+        return fail(BBC_ERR_INVALID, "dequantize_4bit_nested: bad dtype %d", out_dtype);
+    int log2_bs = -1;
+    for (int l = 5; l <= 12; l++)
+        if (blocksize == (1 << l)) log2_bs = l;
+    if (log2_bs < 0)
+        return fail(BBC_ERR_INVALID,
+                    "dequantize_4bit_nested: blocksize must be a power of two in [32, 4096] (got %d)",
+                    blocksize);
+    if (blocksize2 != 256)
+        return fail(BBC_ERR_UNSUPPORTED, "dequantize_4bit_nested: blocksize2 must be 256 (got %d)",
+                    blocksize2);
+    if (!aligned(out, elem_size(out_dtype)) || !aligned(code2, 4) || !aligned(absmax2, 4) || !aligned(code4, 4))
+        return fail(BBC_ERR_INVALID, "dequantize_4bit_nested: pointer not aligned to its element size");
+    const bool vec = aligned(out, 16) && aligned(codes, 8);
+    return cuda_status(bbc::launch_nested_dequantize(codes, absmax_q, code2, absmax2, offset, code4, n,
+                                                     log2_bs, out_dtype, out, vec,
+                                                     static_cast<cudaStream_t>(stream)),
+                       "dequantize_4bit_nested launch");
+}
+
+const char* bbc_last_error(void) { return g_last_error.c_str(); }
+
+}  // extern "C"

@@ -1,0 +1,151 @@
+// Device helpers shared by the library's kernels (sm_100a only).
+#pragma once
+#include <cstdint>
+#include <cuda_runtime.h>
+
+namespace bbc {
+
+enum DType : int { F16 = 0, BF16 = 1, F32 = 2 };
+
+__host__ __device__ constexpr int dtype_size(int dt) { return dt == F32 ? 4 : 2; }
+
+// ---- 128/256-bit streaming global accesses -------------------------------
+
+// Read-only, not kept in L1: every input byte is used exactly once.
+__device__ __forceinline__ uint4 ldg_stream_v4(const void* p) {
+    uint4 v;
+    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "l"(p));
+    return v;
+}
+
+struct u32x8 { uint32_t v[8]; };
+
+__device__ __forceinline__ u32x8 ldg_stream_v8(const void* p) {
+    u32x8 r;
+    asm volatile("ld.global.nc.L1::no_allocate.v8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+                 : "=r"(r.v[0]), "=r"(r.v[1]), "=r"(r.v[2]), "=r"(r.v[3]),
+                   "=r"(r.v[4]), "=r"(r.v[5]), "=r"(r.v[6]), "=r"(r.v[7])
+                 : "l"(p));
+    return r;
+}
+
+__device__ __forceinline__ uint2 ldg_stream_v2(const void* p) {
+    uint2 v;
+    asm volatile("ld.global.nc.L1::no_allocate.v2.u32 {%0,%1}, [%2];"
+                 : "=r"(v.x), "=r"(v.y) : "l"(p));
+    return v;
+}
+
+__device__ __forceinline__ uint32_t ldg_u32(const void* p) {
+    uint32_t v;
+    asm volatile("ld.global.nc.u32 %0, [%1];" : "=r"(v) : "l"(p));
+    return v;
+}
+
+__device__ __forceinline__ void stg_v4(void* p, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+    asm volatile("st.global.v4.u32 [%0], {%1,%2,%3,%4};" :: "l"(p), "r"(a), "r"(b), "r"(c), "r"(d)
+                 : "memory");
+}
+
+__device__ __forceinline__ void stg_v8(void* p, const uint32_t* v) {
+    asm volatile("st.global.v8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};"
+                 :: "l"(p), "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]),
+                    "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]) : "memory");
+}
+
+// ---- conversions ----------------------------------------------------------
+
+// Two fp32 -> packed pair, round to nearest even; `lo` lands at the lower address.
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+    uint32_t r;
+    asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+__device__ __forceinline__ uint32_t pack_f16x2(float lo, float hi) {
+    uint32_t r;
+    asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+    return r;
+}
+__device__ __forceinline__ uint16_t f32_to_bf16_bits(float x) {
+    uint16_t r;
+    asm("cvt.rn.bf16.f32 %0, %1;" : "=h"(r) : "f"(x));
+    return r;
+}
+__device__ __forceinline__ uint16_t f32_to_f16_bits(float x) {
+    uint16_t r;
+    asm("cvt.rn.f16.f32 %0, %1;" : "=h"(r) : "f"(x));
+    return r;
+}
+__device__ __forceinline__ float bf16_bits_to_f32(uint32_t h16) { return __uint_as_float(h16 << 16); }
+__device__ __forceinline__ float f16_bits_to_f32(uint32_t h16) {
+    float f;
+    asm("{ .reg .f16 h; mov.b16 h, %1; cvt.f32.f16 %0, h; }" : "=f"(f) : "h"((uint16_t)h16));
+    return f;
+}
+
+// Load element m of a typed array as fp32 (exact widening).
+template <int DT>
+__device__ __forceinline__ float load_as_f32(const void* A, int64_t m) {
+    if constexpr (DT == F32) return reinterpret_cast<const float*>(A)[m];
+    else {
+        uint32_t h = reinterpret_cast<const uint16_t*>(A)[m];
+        return DT == BF16 ? bf16_bits_to_f32(h) : f16_bits_to_f32(h);
+    }
+}
+
+// Store an fp32 value as element m of a typed array (one rounding to the type).
+template <int DT>
+__device__ __forceinline__ void store_from_f32(void* out, int64_t m, float v) {
+    if constexpr (DT == F32) reinterpret_cast<float*>(out)[m] = v;
+    else if constexpr (DT == BF16) reinterpret_cast<uint16_t*>(out)[m] = f32_to_bf16_bits(v);
+    else reinterpret_cast<uint16_t*>(out)[m] = f32_to_f16_bits(v);
+}
+
+// Pack 8 fp32 values (memory order) of type DT into out_words (4 words for 16-bit, 8 for fp32).
+template <int DT>
+__device__ __forceinline__ void pack8(const float* y, uint32_t* w) {
+    if constexpr (DT == F32) {
+#pragma unroll
+        for (int i = 0; i < 8; i++) w[i] = __float_as_uint(y[i]);
+    } else {
+#pragma unroll
+        for (int i = 0; i < 4; i++)
+            w[i] = DT == BF16 ? pack_bf16x2(y[2 * i], y[2 * i + 1]) : pack_f16x2(y[2 * i], y[2 * i + 1]);
+    }
+}
+
+// Store 8 packed elements of type DT (16 B for 16-bit types, 32 B for fp32), 16-byte aligned.
+template <int DT>
+__device__ __forceinline__ void store8_vec(void* p, const uint32_t* w) {
+    if constexpr (DT == F32) stg_v8(p, w);
+    else stg_v4(p, w[0], w[1], w[2], w[3]);
+}
+
+// Three-input NaN-propagating max of absolute values (sm_100 three-input form).
+__device__ __forceinline__ float max3_abs_nan(float a, float b, float c) {
+    float r;
+    asm("max.NaN.abs.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+    return r;
+}
+__device__ __forceinline__ float max_nan(float a, float b) {
+    float r;
+    asm("max.NaN.f32 %0, %1, %2;" : "=f"(r) : "f"(a), "f"(b));
+    return r;
+}
+
+// Byte permute.
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+    uint32_t r;
+    asm("prmt.b32 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(sel));
+    return r;
+}
+
+// 0xFFFFFFFF if a >= b else 0 (false for NaN).
+__device__ __forceinline__ uint32_t set_ge(float a, float b) {
+    uint32_t r;
+    asm("set.ge.u32.f32 %0, %1, %2;" : "=r"(r) : "f"(a), "f"(b));
+    return r;
+}
+
+}  // namespace bbc

@@ -1,0 +1,34 @@
+// Host-side launchers of the library's kernels (called by abi.cpp after validation).
+#pragma once
+#include <cstdint>
+#include <cuda_runtime.h>
+
+namespace bbc {
+
+// Persistent grid: enough CTAs to fill every SM at the kernel's occupancy, never more than
+// the work needs. The occupancy query runs once per (kernel, device, block, smem) and is
+// cached (grid.cpp).
+int resident_ctas(const void* kernel, int block, size_t dyn_smem);
+
+template <typename Kernel>
+inline int persistent_grid(Kernel kernel, int block, size_t dyn_smem, int64_t work_items,
+                           int items_per_cta) {
+    const int64_t cap = resident_ctas(reinterpret_cast<const void*>(kernel), block, dyn_smem);
+    int64_t need = (work_items + items_per_cta - 1) / items_per_cta;
+    if (need < 1) need = 1;
+    return (int)(need < cap ? need : cap);
+}
+
+cudaError_t launch_kbit_quantize(const void* A, int dtype, int64_t n, int K, const float* codebook,
+                                 float* absmax, uint32_t* packed, bool vec, cudaStream_t s);
+
+cudaError_t launch_kbit_dequantize(const uint32_t* packed, const float* absmax,
+                                   const float* codebook, int K, int64_t n, int out_dtype,
+                                   void* out, bool vec, cudaStream_t s);
+
+cudaError_t launch_nested_dequantize(const uint8_t* codes, const uint8_t* absmax_q,
+                                     const float* code2, const float* absmax2, float offset,
+                                     const float* code4, int64_t n, int log2_bs, int out_dtype,
+                                     void* out, bool vec, cudaStream_t s);
+
+}  // namespace bbc

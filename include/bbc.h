@@ -1,0 +1,150 @@
+/*
+ * bbc.h - C ABI of the blockwise bit-codebook library (NVIDIA B200, sm_100a).
+ *
+ * Two operations on weight tensors, both defined by the pages this library
+ * follows (cited per entry point below):
+ *   1. k-bit blockwise codebook quantization (K = 2..5, blocksize 32) and its
+ *      inverse, with bit-plane packing of the codes;
+ *   2. nested NF4/FP4 dequantization, where each outer block's fp32 scale is
+ *      rebuilt from a General8-coded absmax inside the value-decode kernel.
+ *
+ * Conventions for every entry point:
+ *   - Buffer pointers are DEVICE pointers (memory of the current CUDA device)
+ *     unless a comment says host. The caller allocates and owns every buffer;
+ *     the library never allocates, frees or keeps a pointer after returning.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = the legacy default
+ *     stream). Calls are asynchronous on that stream and never synchronize.
+ *   - Inputs are read-only. Outputs must not overlap any input.
+ *   - Arguments are validated on the host before any launch; on failure the
+ *     call returns a non-zero bbc_status, launches nothing and writes nothing.
+ *     bbc_last_error() then returns a message (per calling thread).
+ *   - A launch failure returns BBC_ERR_CUDA (message from cudaGetErrorString).
+ *   - dtype values: BBC_F16 (IEEE binary16), BBC_BF16 (bfloat16), BBC_F32.
+ *   - Conversions to fp16/bf16 round to nearest, ties to even; subnormals are
+ *     kept (no flush to zero) in every step.
+ *   - Device pointers need only the natural alignment of their element type;
+ *     16-byte-aligned buffers take the vectorised path, others a scalar path
+ *     with identical results.
+ */
+#ifndef BBC_H
+#define BBC_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum bbc_dtype { BBC_F16 = 0, BBC_BF16 = 1, BBC_F32 = 2 } bbc_dtype;
+
+typedef enum bbc_status {
+    BBC_OK = 0,
+    BBC_ERR_INVALID = 1,      /* bad argument: null pointer, n <= 0, K out of range, bad dtype */
+    BBC_ERR_UNSUPPORTED = 2,  /* valid in principle but not built: blocksize != 32, bs2 != 256 */
+    BBC_ERR_CUDA = 3          /* a CUDA runtime call or launch failed */
+} bbc_status;
+
+/*
+ * kbit_quantize - k-bit blockwise codebook quantization.
+ *
+ * Defined by: bitsandbytes k-bit patch series, PATCH 001 "Add k-bit
+ * quantization kernels (K=2-5, blocksize=32)": quantize_kbit_ref in
+ * tests/test_kbit_quantization.py and kQuantizeBlockwise_kbit in csrc/ops.cu.
+ *
+ * For each block b of 32 consecutive elements of A (the last block padded
+ * with 0.0):
+ *   absmax[b] = max_i |x_i|                       (raw, unclamped)
+ *   d         = max(absmax[b], 1e-8f)
+ *   xn_i      = x_i / d                           (IEEE fp32 division)
+ *   idx_i     = first i minimising fabsf(xn_i - codebook[i])
+ *   packed[b*K + j] bit i = bit j of idx_i        (bit-plane layout)
+ * Padding lanes of the last block are quantized like 0.0 and their bits are
+ * stored.
+ *
+ *   A          [n] elements of `dtype` (fp16, bf16 or fp32).
+ *   n          element count, >= 1.
+ *   K          bits per code, 2..5.
+ *   blocksize  must be 32 (BBC_ERR_UNSUPPORTED otherwise).
+ *   codebook   [2^K] fp32 device values. Any values give the exact result;
+ *              finite, strictly ascending entries spaced at least
+ *              2^-19 * (1 + max|c|) apart take the fast threshold search,
+ *              others a brute-force search.
+ *   absmax     [ceil(n/32)] fp32 output.
+ *   packed     [ceil(n/32) * K] uint32 output.
+ * NaN or infinite inputs give the same result as the rule above (a NaN is
+ * ignored by the max unless the whole block is NaN; NaN distances never win).
+ */
+int kbit_quantize(const void* A, int dtype, int64_t n, int K, int blocksize,
+                  const float* codebook, float* absmax, uint32_t* packed, void* stream);
+
+/*
+ * kbit_dequantize - inverse of kbit_quantize.
+ *
+ * Defined by: the same patch series, dequantize_kbit_ref and
+ * kDequantizeBlockwise_kbit: out[m] = T(codebook[idx_m] * absmax[m / 32]),
+ * one fp32 multiply then one rounding to the output type, for m < n only.
+ *
+ *   packed     [ceil(n/32) * K] uint32, layout as written by kbit_quantize.
+ *   absmax     [ceil(n/32)] fp32.
+ *   codebook   [2^K] fp32.
+ *   K          2..5.   blocksize must be 32.
+ *   n          element count, >= 1.
+ *   out_dtype  BBC_F16, BBC_BF16 or BBC_F32.
+ *   out        [n] elements of out_dtype (nothing beyond n is written).
+ */
+int kbit_dequantize(const uint32_t* packed, const float* absmax, const float* codebook,
+                    int K, int blocksize, int64_t n, int out_dtype, void* out, void* stream);
+
+/*
+ * dequantize_4bit_nested - NF4/FP4 dequantization with the nested
+ * ("compressed statistics") scale rebuilt inside the decode.
+ *
+ * Defined by: pull request "Fuse nested 4-bit scale reconstruction on SM103",
+ * Summary and Implementation: the outer-block fp32 scale is the General8 code
+ * of the quantized absmax times the inner absmax, then plus the offset, as a
+ * separately rounded fp32 multiply and add (no fused multiply-add), applied
+ * while the 4-bit values are decoded, with no intermediate scale tensor:
+ *   b        = m / blocksize
+ *   scale_b  = fl(fl(code2[absmax_q[b]] * absmax2[b / blocksize2]) + offset)
+ *   out[m]   = T(fl(code4[nibble_m] * scale_b))
+ * Nibble order (a reading; the page does not print it): element 2j is the
+ * high nibble (bits 7..4) of codes[j], element 2j+1 the low nibble.
+ *
+ *   codes       [ceil(n/2)] uint8, two 4-bit codes per byte.
+ *   absmax_q    [ceil(n/blocksize)] uint8 General8 codes of the outer absmax.
+ *   code2       [256] fp32 General8 code table.
+ *   absmax2     [ceil(ceil(n/blocksize)/blocksize2)] fp32 inner absmax.
+ *   offset      fp32 scalar added to every outer scale.
+ *   code4       [16] fp32 value table (NF4 or FP4).
+ *   n           element count, >= 1.
+ *   blocksize   outer block size: a power of two in [32, 4096].
+ *   blocksize2  inner block size: must be 256 (BBC_ERR_UNSUPPORTED otherwise).
+ *   out_dtype   BBC_F16, BBC_BF16 or BBC_F32;   out [n] elements.
+ */
+int dequantize_4bit_nested(const uint8_t* codes, const uint8_t* absmax_q, const float* code2,
+                           const float* absmax2, float offset, const float* code4,
+                           int64_t n, int blocksize, int blocksize2, int out_dtype, void* out,
+                           void* stream);
+
+/*
+ * bbc_nf_codebook - the 2^K-entry normal-float codebook, on the HOST.
+ *
+ * Defined by: the k-bit patch series, create_normal_float_codebook: standard
+ * normal quantiles at the bin midpoints (2i+1)/(2^(K+1)), computed in double,
+ * rounded to fp32, then divided (in fp32) by the largest magnitude. Sorted
+ * ascending, largest magnitude exactly 1.
+ *
+ *   K            1..8.
+ *   codebook_out HOST buffer of 2^K floats, written by the call.
+ * Host-only: no CUDA call is made.
+ */
+int bbc_nf_codebook(int K, float* codebook_out);
+
+/* Message for the last non-OK status returned on the calling thread ("" if none). */
+const char* bbc_last_error(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* BBC_H */

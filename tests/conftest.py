@@ -18,3 +18,13 @@ def orc():
     import oracle
     oracle.lib()
     return oracle
+
+
+def pytest_collection_modifyitems(config, items):
+    """`slow` tests run only when selected explicitly with -m slow."""
+    if "slow" in (config.getoption("-m") or ""):
+        return
+    skip = pytest.mark.skip(reason="slow: run with -m slow")
+    for item in items:
+        if "slow" in item.keywords:
+            item.add_marker(skip)

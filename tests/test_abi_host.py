@@ -1,0 +1,133 @@
+"""Host-only checks of the C ABI (no GPU needed, no kernel launched).
+
+* libbbc.so loads and exports every function declared in include/bbc.h;
+* argument validation happens on the host before any CUDA call, so invalid
+  calls return their status here without a device;
+* bbc_nf_codebook (host code) equals the oracle's normal-float codebook.
+"""
+import ctypes as ct
+import os
+import re
+
+import numpy as np
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "bbc.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from blockwise_bit_codebook_b200 import build, load_library
+    build.build()
+    return load_library()
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return re.findall(r"^\s*(?:const\s+)?\w+\s*\*?\s*(\w+)\s*\(", text, flags=re.M)
+
+
+def test_header_declares_the_boundary():
+    names = set(declared_functions())
+    assert {"kbit_quantize", "kbit_dequantize", "dequantize_4bit_nested",
+            "bbc_nf_codebook", "bbc_last_error"} <= names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+
+
+def test_exported_symbols_via_nm(lib):
+    import subprocess
+    from blockwise_bit_codebook_b200 import library_path
+    out = subprocess.run(["nm", "-D", "--defined-only", library_path()], capture_output=True,
+                         text=True).stdout
+    syms = {line.split()[-1] for line in out.splitlines() if line.strip()}
+    for name in declared_functions():
+        assert name in syms, name
+
+
+P = ct.c_void_p
+FAKE = P(0x1000)        # never dereferenced: every call below fails validation first
+
+
+def _q(lib, A=FAKE, dtype=2, n=64, K=4, bs=32, cb=FAKE, am=FAKE, pk=FAKE):
+    return lib.kbit_quantize(A, dtype, n, K, bs, cb, am, pk, None)
+
+
+def _dq(lib, pk=FAKE, am=FAKE, cb=FAKE, K=4, bs=32, n=64, dt=2, out=FAKE):
+    return lib.kbit_dequantize(pk, am, cb, K, bs, n, dt, out, None)
+
+
+def _nd(lib, n=64, bs=64, bs2=256, dt=1, codes=FAKE, out=FAKE):
+    return lib.dequantize_4bit_nested(codes, FAKE, FAKE, FAKE, ct.c_float(0.0), FAKE, n, bs, bs2, dt,
+                                      out, None)
+
+
+def test_quantize_validation(lib):
+    assert _q(lib, A=None) == 1
+    assert _q(lib, cb=None) == 1 and _q(lib, am=None) == 1 and _q(lib, pk=None) == 1
+    assert _q(lib, n=0) == 1 and _q(lib, n=-5) == 1
+    for K in (0, 1, 6, 8):
+        assert _q(lib, K=K) == 1
+    assert "K must be 2..5" in lib.bbc_last_error().decode()
+    assert _q(lib, dtype=3) == 1 and _q(lib, dtype=-1) == 1
+    assert _q(lib, bs=64) == 2 and _q(lib, bs=16) == 2
+    assert _q(lib, A=P(0x1001), dtype=0) == 1          # fp16 at an odd address
+    assert _q(lib, am=P(0x1002)) == 1
+
+
+def test_dequantize_validation(lib):
+    assert _dq(lib, pk=None) == 1 and _dq(lib, out=None) == 1
+    assert _dq(lib, n=0) == 1
+    assert _dq(lib, K=6) == 1 and _dq(lib, K=1) == 1
+    assert _dq(lib, dt=7) == 1
+    assert _dq(lib, bs=128) == 2
+    assert _dq(lib, out=P(0x1002), dt=2) == 1           # fp32 output at a 2-byte address
+    assert _dq(lib, pk=P(0x1001)) == 1
+
+
+def test_nested_validation(lib):
+    assert _nd(lib, codes=None) == 1 and _nd(lib, out=None) == 1
+    assert _nd(lib, n=0) == 1
+    for bs in (0, 16, 48, 100, 8192):
+        assert _nd(lib, bs=bs) == 1
+    assert _nd(lib, bs2=128) == 2
+    assert _nd(lib, dt=5) == 1
+    assert "blocksize2 must be 256" in (lib.bbc_last_error().decode() if _nd(lib, bs2=512) else "")
+
+
+def test_last_error_is_per_thread(lib):
+    import threading
+    _q(lib, K=9)
+    seen = {}
+
+    def other():
+        seen["msg"] = lib.bbc_last_error().decode()
+    t = threading.Thread(target=other)
+    t.start()
+    t.join()
+    assert seen["msg"] == "" and "K must be" in lib.bbc_last_error().decode()
+
+
+@pytest.mark.parametrize("K", [1, 2, 3, 4, 5, 6, 7, 8])
+def test_nf_codebook_matches_oracle(lib, orc, K):
+    from blockwise_bit_codebook_b200 import bbc_nf_codebook
+    ours = bbc_nf_codebook(K)
+    if K <= 5:
+        ref = orc.normal_float_codebook(K)
+    else:   # same construction through the oracle module's quantile routine
+        from oracle.codebook import unnormalized_quantiles
+        q = unnormalized_quantiles(K)
+        ref = q / np.abs(q).max()
+    assert np.array_equal(ours.view(np.uint32), ref.view(np.uint32))
+
+
+def test_nf_codebook_rejects_bad_k(lib):
+    out = np.empty(512, np.float32)
+    assert lib.bbc_nf_codebook(0, out.ctypes.data_as(P)) == 1
+    assert lib.bbc_nf_codebook(9, out.ctypes.data_as(P)) == 1
+    assert lib.bbc_nf_codebook(4, None) == 1
