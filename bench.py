@@ -1,0 +1,446 @@
+#!/usr/bin/env python
+"""Benchmark of the blockwise bit-codebook hot path on B200.
+
+One step = one pass of every operation of the path over one batch of resident
+synthetic input (default workload "c5", the large streaming case):
+    16384 x 16384 bf16 weight ~ N(0, 0.02), seed 7
+      kbit_quantize   K=3 -> kbit_dequantize K=3 (bf16 out)
+      kbit_quantize   K=5 -> kbit_dequantize K=5 (bf16 out)
+      dequantize_4bit_nested NF4 (16-entry normal-float table), outer blocksize 64,
+      inner blocksize 256, bf16 out, same element count.
+Every input is larger than the 126 MB L2, so no flush is needed between steps.
+
+Metric: achieved HBM GB/s (algorithmic bytes / time) for the whole step, plus
+per kernel GB/s, Gelem/s and the fraction of the measured HBM copy bandwidth.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl {bbc,reference}]
+
+N > 1 runs under torchrun, one rank per GPU, each rank on its own full copy of
+the workload (weak scaling; the path needs no collective). The reference arm
+(--impl reference) times the CPU oracle on a bounded sample of the workload.
+"""
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "achieved HBM GB/s and Gelem/s per kernel; fraction of B200 HBM roofline"
+FALLBACK_HBM_GBS = 6650.0
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["bbc", "reference"], default="bbc")
+    ap.add_argument("--workload", choices=["c5"], default="c5")
+    ap.add_argument("--n", type=int, default=None,
+                    help="override the element count (profiling of a smaller case)")
+    ap.add_argument("--ops", default=None,
+                    help="comma-separated subset of quantize_k3,dequantize_k3,quantize_k5,"
+                         "dequantize_k5,nested_nf4_bs64 (profiling)")
+    ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0,
+                    help="target CPU time of the oracle baseline sample")
+    return ap.parse_args()
+
+
+# ----------------------------------------------------------------------------- workload
+
+N_C5 = 16384 * 16384
+NESTED_BS = 64
+
+
+def op_bytes(kind, n, K=None, out_size=2, bs=NESTED_BS):
+    """Algorithmic bytes of one launch (the minimum the operation must move)."""
+    nb = (n + 31) // 32
+    if kind == "quantize":
+        return n * 2 + nb * K * 4 + nb * 4
+    if kind == "dequantize":
+        return nb * K * 4 + nb * 4 + n * out_size
+    nbo = (n + bs - 1) // bs
+    nbi = (nbo + 255) // 256
+    return (n + 1) // 2 + nbo + nbi * 4 + n * out_size
+
+
+ALL_OPS = [("quantize_k3", "quantize", 3), ("dequantize_k3", "dequantize", 3),
+           ("quantize_k5", "quantize", 5), ("dequantize_k5", "dequantize", 5),
+           ("nested_nf4_bs64", "nested", None)]
+
+
+def workload_ops(only=None):
+    if not only:
+        return list(ALL_OPS)
+    names = only.split(",")
+    ops = [o for o in ALL_OPS if o[0] in names]
+    assert len(ops) == len(names), f"unknown op in {only}"
+    return ops
+
+
+def workload_desc(n, ops):
+    full = n == N_C5 and len(ops) == len(ALL_OPS)
+    return {
+        "workload": ("c5: 16384x16384 bf16 weight ~ N(0,0.02) seed 7; k-bit quantize+dequantize at "
+                     "K=3 and K=5 (blocksize 32, normal-float codebooks) and nested NF4 dequant "
+                     "(outer blocksize 64, inner 256) of the same size, bf16 outputs")
+        if full else f"c5-distributed subset: n={n}, ops={[o[0] for o in ops]} (profiling case)",
+        "n": n, "io_dtype": "bf16", "blocksize": 32, "nested_blocksize": NESTED_BS,
+        "l2": "no flush: every kernel streams >= 600 MB, above the 126 MB L2",
+    }
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return float(d["hbm_gbs"]), "measured"
+    return FALLBACK_HBM_GBS, "fallback"
+
+
+def kernel_source_hash(kind):
+    files = {"quantize": ["kbit_quant.cu"], "dequantize": ["kbit_dequant.cu"],
+             "nested": ["nested_dequant.cu"]}[kind] + ["common.cuh"]
+    h = hashlib.sha256()
+    for f in files:
+        h.update(open(os.path.join(ROOT, "blockwise_bit_codebook_b200", "csrc", f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(name, kind):
+    """DRAM bytes per launch from the committed ncu summary, if the kernel source is unchanged."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    d = json.load(open(p)).get(name)
+    if not d or d.get("source_hash") != kernel_source_hash(kind):
+        return None
+    return d.get("dram_bytes_per_launch")
+
+
+# ----------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.samples = []
+        self.proc = None
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(gpu_index), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.samples.append((time.time(), [s.strip() for s in line.split(",")]))
+
+    def stop(self):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self, t0, t1):
+        rows = [r for t, r in self.samples if t0 <= t <= t1 and len(r) >= 9]
+        if not rows:
+            rows = [r for t, r in self.samples if len(r) >= 9][-3:]
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": float(rows[0][2]) if rows[0][2].replace(".", "").isdigit() else None,
+                "reasons": reasons, "samples": len(rows),
+                "power_w_max": max([float(r[3]) for r in rows if r[3].replace(".", "").isdigit()],
+                                   default=None)}
+
+
+# ----------------------------------------------------------------------------- oracle legs
+
+def oracle_sample_bytes_and_time(x_host_bits, cbs, nested, S):
+    """Run the oracle over the first S elements of each input; returns (algorithmic bytes, seconds)."""
+    import oracle
+    codes, q, a2, off, code2, code4 = nested
+    tot_bytes, t0 = 0, time.perf_counter()
+    xs = x_host_bits[:S]
+    for K in (3, 5):
+        p, a = oracle.kbit_quantize(xs, "bf16", K, cbs[K])
+        oracle.kbit_dequantize(p, a, cbs[K], K, S, "bf16")
+        tot_bytes += op_bytes("quantize", S, K) + op_bytes("dequantize", S, K)
+    nbo = (S + NESTED_BS - 1) // NESTED_BS
+    oracle.nested_dequantize(codes[: (S + 1) // 2], q[:nbo], code2, a2[: (nbo + 255) // 256], off, code4,
+                             S, NESTED_BS, 256, "bf16")
+    tot_bytes += op_bytes("nested", S)
+    return tot_bytes, time.perf_counter() - t0
+
+
+def host_inputs_for_oracle(x_dev_bf16, nested_dev, code2, code4, S):
+    import numpy as np
+    import torch
+    xb = x_dev_bf16[:S].contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
+    codes, q, a2, off = nested_dev
+    nbo = (S + NESTED_BS - 1) // NESTED_BS
+    return xb, (codes[: (S + 1) // 2].cpu().numpy(), q[:nbo].cpu().numpy(),
+                a2[: (nbo + 255) // 256].cpu().numpy(), float(off), code2, code4)
+
+
+def cpu_baseline(x_dev, nested_dev, code2, code4, cbs, seconds, n):
+    # calibrate on 2^20 elements, then size the sample for about `seconds` of CPU work
+    S0 = 1 << 20
+    xb, ns = host_inputs_for_oracle(x_dev, nested_dev, code2, code4, S0)
+    _, t = oracle_sample_bytes_and_time(xb, cbs, ns, S0)
+    S = int(min(n, max(S0, S0 * seconds / max(t, 1e-3)))) // 4096 * 4096
+    xb, ns = host_inputs_for_oracle(x_dev, nested_dev, code2, code4, S)
+    b, t = oracle_sample_bytes_and_time(xb, cbs, ns, S)
+    return {"value": b / t / 1e9, "unit": "GB/s", "cores": 1, "kind": "oracle",
+            "seconds": round(t, 2),
+            "sample": f"first {S} of the {n} elements of every input (all five operations), "
+                      "single-threaded C oracle"}
+
+
+# ----------------------------------------------------------------------------- main arm
+
+def run_bbc(args):
+    import numpy as np
+    import torch
+
+    import blockwise_bit_codebook_b200 as bbc
+    from blockwise_bit_codebook_b200 import synthetic
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    dist = None
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    bbc.load_library()
+
+    ops = workload_ops(args.ops)
+    n = args.n or N_C5
+    nb = (n + 31) // 32
+    x = synthetic.weights(n, std=0.02, seed=7, dtype=torch.bfloat16, device=dev)
+    cbs = {K: bbc.bbc_nf_codebook(K) for K in (3, 4, 5)}
+    cb_dev = {K: torch.from_numpy(cbs[K]).to(dev) for K in cbs}
+    packed = {K: torch.empty(nb * K, dtype=torch.int32, device=dev) for K in (3, 5)}
+    absmax = {K: torch.empty(nb, dtype=torch.float32, device=dev) for K in (3, 5)}
+    outs = {K: torch.empty(n, dtype=torch.bfloat16, device=dev) for K in (3, 5)}
+    nested = synthetic.nested_state(n, NESTED_BS, seed=3, device=dev)
+    codes, q, a2, off = nested
+    code2 = synthetic.general8_table()
+    code4 = cbs[4]
+    code2_dev, code4_dev = torch.from_numpy(code2).to(dev), cb_dev[4]
+    nout = torch.empty(n, dtype=torch.bfloat16, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def launch(kind, K, xin=x, cin=codes, qin=q, a2in=a2, pk=packed, am=absmax, ou=outs, no=nout):
+        if kind == "quantize":
+            bbc.kbit_quantize(xin, K, cb_dev[K], absmax=am[K], packed=pk[K], stream=stream)
+        elif kind == "dequantize":
+            bbc.kbit_dequantize(pk[K], am[K], cb_dev[K], K, n, torch.bfloat16, out=ou[K], stream=stream)
+        else:
+            bbc.dequantize_4bit_nested(cin, qin, code2_dev, a2in, float(off), code4_dev, n, NESTED_BS,
+                                       torch.bfloat16, out=no, stream=stream)
+
+    for _ in range(args.warmup):
+        for _, kind, K in ops:
+            launch(kind, K)
+    torch.cuda.synchronize()
+
+    evs = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in ops]
+           for _ in range(args.steps)]
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(local) if rank == 0 else None
+    time.sleep(0.3)
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize()
+    w0 = time.time()
+    t_start.record(stream)
+    for s in range(args.steps):
+        for i, (_, kind, K) in enumerate(ops):
+            evs[s][i][0].record(stream)
+            launch(kind, K)
+            evs[s][i][1].record(stream)
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    w1 = time.time()
+    if dist:
+        dist.barrier()
+    total_ms = t_start.elapsed_time(t_end)
+    per_op_ms = [statistics.mean(evs[s][i][0].elapsed_time(evs[s][i][1]) for s in range(args.steps))
+                 for i in range(len(ops))]
+    if dist:
+        t = torch.tensor([total_ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t.item())
+    if sampler:
+        time.sleep(0.25)
+        sampler.stop()
+    clocks = sampler.summary(w0, w1) if sampler else None
+
+    ms_per_step = total_ms / args.steps
+    bytes_step = sum(op_bytes(kind, n, K) for _, kind, K in ops)
+    value = world * bytes_step / (ms_per_step * 1e-3) / 1e9
+    peak, peak_kind = load_peaks()
+    per_kernel = {}
+    for (name, kind, K), ms in zip(ops, per_op_ms):
+        b = op_bytes(kind, n, K)
+        gbs = b / (ms * 1e-3) / 1e9
+        per_kernel[name] = {"ms": round(ms, 5), "GB/s": round(gbs, 1),
+                            "Gelem/s": round(n / (ms * 1e-3) / 1e9, 2),
+                            "frac_of_measured_hbm": round(gbs / peak, 4),
+                            "frac_of_8TBs_nominal": round(gbs / 8000.0, 4),
+                            "bytes_per_launch": b,
+                            "share_of_step": round(ms / sum(per_op_ms), 4)}
+    dom = max(range(len(ops)), key=lambda i: per_op_ms[i])
+    dname, dkind, dK = ops[dom]
+    dbytes = op_bytes(dkind, n, dK)
+    achieved = dbytes / (per_op_ms[dom] * 1e-3) / 1e9
+    roofline = {"bound": "hbm", "kernel": dname, "achieved": round(achieved, 1), "peak": peak,
+                "peak_source": f"{peak_kind} (MEASURED_PEAKS.json hbm_gbs)" if peak_kind == "measured"
+                else "fallback 6.65 TB/s", "unit": "GB/s", "frac": round(achieved / peak, 4),
+                "traffic": ncu_traffic(dname, dkind), "algorithmic_bytes_per_launch": dbytes}
+
+    result = {"metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world,
+              "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5),
+              "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
+              "data": "synthetic", "config": {**workload_desc(n, ops),
+                                              "parallelism": f"replicas{world}" if world > 1 else "single"},
+              "per_kernel": per_kernel, "roofline": roofline,
+              "gpu_launches": len(ops) * args.steps, "clocks": clocks}
+
+    # ---- end to end through the public API with host buffers
+    if not args.no_e2e:
+        pin = lambda t: t.cpu().pin_memory()  # noqa: E731
+        hx, hcodes, hq, ha2 = pin(x), pin(codes), pin(q), pin(a2)
+        hcb = {K: torch.from_numpy(cbs[K]).pin_memory() for K in (3, 4, 5)}
+        h_out = {"packed": {K: torch.empty_like(packed[K], device="cpu").pin_memory() for K in (3, 5)},
+                 "absmax": {K: torch.empty_like(absmax[K], device="cpu").pin_memory() for K in (3, 5)},
+                 "out": {K: torch.empty_like(outs[K], device="cpu").pin_memory() for K in (3, 5)},
+                 "nested": torch.empty_like(nout, device="cpu").pin_memory()}
+        dx, dcodes, dq, da2 = torch.empty_like(x), torch.empty_like(codes), torch.empty_like(q), torch.empty_like(a2)
+        h2d = sum(t.numel() * t.element_size() for t in (hx, hcodes, hq, ha2)) + \
+            sum(t.numel() * 4 for t in hcb.values())
+        d2h = sum(t.numel() * t.element_size() for K in (3, 5)
+                  for t in (packed[K], absmax[K], outs[K])) + nout.numel() * 2
+
+        def e2e_step():
+            dx.copy_(hx, non_blocking=True)
+            dcodes.copy_(hcodes, non_blocking=True)
+            dq.copy_(hq, non_blocking=True)
+            da2.copy_(ha2, non_blocking=True)
+            for K in (3, 4, 5):
+                cb_dev[K].copy_(hcb[K], non_blocking=True)
+            for _, kind, K in ops:
+                launch(kind, K, xin=dx, cin=dcodes, qin=dq, a2in=da2)
+            for K in (3, 5):
+                h_out["packed"][K].copy_(packed[K], non_blocking=True)
+                h_out["absmax"][K].copy_(absmax[K], non_blocking=True)
+                h_out["out"][K].copy_(outs[K], non_blocking=True)
+            h_out["nested"].copy_(nout, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize()
+        if dist:
+            dist.barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.e2e_steps):
+            e2e_step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        e_ms = e0.elapsed_time(e1) / args.e2e_steps
+        if dist:
+            t = torch.tensor([e_ms], device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e_ms = float(t.item())
+        result["e2e"] = {"value": round(world * bytes_step / (e_ms * 1e-3) / 1e9, 2), "unit": "GB/s",
+                         "ms_per_step": round(e_ms, 3), "h2d_bytes_per_step": h2d,
+                         "d2h_bytes_per_step": d2h, "steps": args.e2e_steps,
+                         "api": "blockwise_bit_codebook_b200 (C ABI via ctypes), pinned host buffers"}
+
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        result["cpu_baseline"] = cpu_baseline(x, nested, code2, code4, cbs, args.cpu_seconds, n)
+    elif rank == 0:
+        result["cpu_baseline"] = None
+
+    if dist:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(result), flush=True)
+
+
+# ----------------------------------------------------------------------------- reference arm
+
+def run_reference(args):
+    """The CPU oracle as the reference arm: rank 0 only, bounded samples of the c5 workload."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import numpy as np
+    import torch
+
+    import oracle
+    from blockwise_bit_codebook_b200 import synthetic
+
+    n = N_C5
+    cbs = {K: oracle.normal_float_codebook(K) for K in (3, 4, 5)}
+    code2 = synthetic.general8_table()
+    # per-step sample sized so the whole run takes about two minutes of CPU
+    budget = 120.0 / max(1, args.steps + args.warmup)
+    S = max(4096, min(n, int(budget / 170e-9)) // 4096 * 4096)
+    x = synthetic.weights(S, std=0.02, seed=7, dtype=torch.bfloat16)
+    xb = x.view(torch.int16).numpy().view(np.uint16)
+    codes, q, a2, off = synthetic.nested_state(S, NESTED_BS, seed=3)
+    ns = (codes.numpy(), q.numpy(), a2.numpy(), float(off), code2, cbs[4])
+    for _ in range(args.warmup):
+        oracle_sample_bytes_and_time(xb, cbs, ns, S)
+    tot_b, tot_t = 0, 0.0
+    for _ in range(args.steps):
+        b, t = oracle_sample_bytes_and_time(xb, cbs, ns, S)
+        tot_b += b
+        tot_t += t
+    value = tot_b / tot_t / 1e9
+    sample = f"{S} elements per step (first elements of a c5-distributed input), all five operations"
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(tot_t / args.steps * 1e3, 3), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f32", "data": "synthetic", "config": workload_desc(N_C5, ALL_OPS),
+        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }), flush=True)
+
+
+if __name__ == "__main__":
+    a = parse_args()
+    run_reference(a) if a.impl == "reference" else run_bbc(a)
