@@ -54,7 +54,7 @@ int kbit_quantize(const void* A, int dtype, int64_t n, int K, int blocksize,
         return fail(BBC_ERR_UNSUPPORTED, "kbit_quantize: blocksize must be 32 (got %d)", blocksize);
     if (!aligned(A, elem_size(dtype)) || !aligned(codebook, 4) || !aligned(absmax, 4) || !aligned(packed, 4))
         return fail(BBC_ERR_INVALID, "kbit_quantize: pointer not aligned to its element size");
-    const bool vec = aligned(A, 16);
+    const bool vec = aligned(A, 32);     // 256-bit loads of 16-element groups
     return cuda_status(bbc::launch_kbit_quantize(A, dtype, n, K, codebook, absmax, packed, vec,
                                                  static_cast<cudaStream_t>(stream)),
                        "kbit_quantize launch");

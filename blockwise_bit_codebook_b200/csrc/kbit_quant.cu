@@ -10,37 +10,38 @@
 //
 // 1. Exact decision thresholds. For a codebook that is finite, strictly
 //    ascending and spaced at least 2^-19 * (1 + max|c|) apart, a fp32 distance
-//    fl(xn - c_i) can never tie with a farther entry on the same side, so the
-//    index is a non-decreasing step function of xn:
-//        idx(xn) = #{ j >= 1 : xn >= T_j },
-//    where T_j is the smallest fp32 value at which entry j beats entry j-1
-//    under the exact rule fl(c_j - v) < fl(v - c_{j-1}). Each CTA finds the
-//    T_j by bisection over the ordered fp32 bit patterns (<= 32 steps), using
-//    the same IEEE subtractions as the rule itself. Any other codebook takes
-//    the brute-force search, which is the rule verbatim.
+//    fl(xn - c_i) never ties with a farther entry on the same side, so the index
+//    is a non-decreasing step function of xn:  idx(xn) = #{ j >= 1 : xn >= T_j },
+//    where T_j is the smallest fp32 value at which entry j beats entry j-1 under
+//    the exact rule fl(c_j - v) < fl(v - c_{j-1}). Each CTA finds the T_j by
+//    bisection over the ordered fp32 bit patterns, using the same IEEE
+//    subtractions as the rule. Any other codebook takes the brute-force search,
+//    which is the rule verbatim.
 //
-// 2. One table lookup per element instead of 2^K distance tests. The quotient
-//    is estimated as q = x * RN(1/d) (one multiply; |q - RN(x/d)| < 1.5*2^-23 |x/d|).
-//    A 256-cell table indexed by round(8192*q)/128 (cells 1/64 wide, found
-//    with one fused multiply-add and a mask) holds, per cell, the only
-//    threshold that can matter there, widened to a guard band
-//    [T - g, T + g), g = 2^-19 |T| + 2^-100, and the byte-spread bit patterns
-//    of the two possible indices. Outside the band the estimate decides
-//    exactly; inside it (about 2^-16 of elements for the normal-float
-//    codebooks) the thread redoes its 8 elements with IEEE division and the
-//    brute-force rule. Cells with two candidate thresholds are all-guard.
-//    The table is replicated 8 times so the 8 lanes of each quarter-warp
-//    phase of a 128-bit shared load always hit distinct banks.
+// 2. An exact test against one threshold without dividing. With h_T half the
+//    gap from T down to the next fp32 value, RN(x/d) >= T  <=>  x/d > T - h_T
+//    (x/d is never exactly an fp32 midpoint: its numerator would need more
+//    than 24 significant bits), i.e. x - T*d + h_T*d > 0, and the sign of that
+//    sum is computed exactly by v = fma(h_T, d, fma(-T, d, x)): when |x - T*d|
+//    is below ulp(T)*d the inner fma is exact, otherwise its rounding cannot
+//    change the sign of the sum. Two paired f32x2 FMAs per element pair.
 //
-// 3. Bit-plane packing without ballots. A thread owns 8 consecutive elements
-//    (one quarter of a block); adding spread(idx_e) << e, where spread puts
-//    bit k of idx at bit 8k, builds byte k = bits of plane k for its 8
-//    elements in one register. A 4x4 byte transpose across the block's four
-//    lanes (two xor-shuffles, two byte permutes) leaves word j in lane j.
-//    K = 5 keeps plane 4 in a second register (bit 4 of idx is xn >= T_16).
+// 3. One table lookup finds the threshold. A 256-cell table indexed by
+//    round(8192 * x/d) / 128 (cells 1/64 wide; one paired fma and a mask) holds,
+//    per cell, the only threshold that can matter there (-T, h_T) and the
+//    byte-spread bit patterns of the two possible indices. A codebook whose
+//    thresholds are closer than a cell takes the brute-force search. The table
+//    is replicated 8 times so the 8 lanes of each 128-bit shared-load phase
+//    always hit distinct banks.
 //
-// Blocks whose NaN-propagating absmax is NaN, infinite or above 2^125 (where
-// 1/d would be subnormal) take the exact path for all their elements.
+// 4. Bit-plane packing without ballots. A thread owns 16 consecutive elements
+//    (half a block); adding spread(idx) << e (bit k of idx at bit 8k) builds, per
+//    8 elements, one register whose byte k holds plane k. One xor-shuffle and
+//    four byte permutes between the two lanes of a block leave words 2h, 2h+1 in
+//    lane h. K = 5 accumulates 4 elements per register with plane 4 in bits 4..7.
+//
+// Blocks whose NaN-propagating absmax is NaN, infinite or above 2^125 take the
+// brute-force path (IEEE division and the rule verbatim) for all their elements.
 #include <cfloat>
 
 #include "common.cuh"
@@ -64,7 +65,7 @@ __device__ __forceinline__ float key_f32(int64_t k) {
 }
 
 // Smallest fp32 v in [lo, hi] where entry `hi` beats entry `lo` under the exact
-// rule; the predicate is false at lo and true at hi and monotone in v.
+// rule; the predicate is false at lo, true at hi and monotone in between.
 __device__ float bisect_threshold(float lo_c, float hi_c) {
     int64_t lo = f32_key(lo_c), hi = f32_key(hi_c);
     for (int it = 0; it < 40 && hi - lo > 1; it++) {
@@ -76,8 +77,13 @@ __device__ float bisect_threshold(float lo_c, float hi_c) {
     return key_f32(hi);
 }
 
-// Bits 0..3 of v moved to bits 0, 8, 16, 24.
-__device__ __forceinline__ uint32_t spread4(uint32_t v) { return ((v & 15u) * 0x00204081u) & 0x01010101u; }
+// Bits 0..3 of v at bits 0, 8, 16, 24; for K = 5 also bit 4 of v at bit 4.
+template <int K>
+__device__ __forceinline__ uint32_t spread(uint32_t v) {
+    uint32_t s = ((v & 15u) * 0x00204081u) & 0x01010101u;
+    if constexpr (K == 5) s |= (v & 16u);
+    return s;
+}
 
 // Brute-force nearest entry: first index with the smallest fp32 distance.
 template <int NE>
@@ -92,36 +98,73 @@ __device__ __forceinline__ uint32_t nearest_entry(float xn, const float* cb) {
     return idx;
 }
 
+// Raw input words of one half block (16 elements): 8 words for 16-bit types, 16 for fp32.
+template <int DT>
+struct Raw { uint32_t w[DT == F32 ? 16 : 8]; };
+
 template <int DT, bool VEC>
-__device__ __forceinline__ void load8(const void* A, int64_t n, int64_t Q, bool active, float* x) {
-    const int64_t m0 = Q * 8;
-    if (VEC && active && m0 + 8 <= n) {
-        if constexpr (DT == F32) {
-            const char* p = reinterpret_cast<const char*>(A) + m0 * 4;
-            const uint4 a = ldg_stream_v4(p), b = ldg_stream_v4(p + 16);
-            x[0] = __uint_as_float(a.x); x[1] = __uint_as_float(a.y);
-            x[2] = __uint_as_float(a.z); x[3] = __uint_as_float(a.w);
-            x[4] = __uint_as_float(b.x); x[5] = __uint_as_float(b.y);
-            x[6] = __uint_as_float(b.z); x[7] = __uint_as_float(b.w);
-        } else {
-            const uint4 v = ldg_stream_v4(reinterpret_cast<const char*>(A) + m0 * 2);
-            const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+__device__ __forceinline__ Raw<DT> load_raw(const void* A, int64_t n, int64_t H, bool active) {
+    Raw<DT> r;
+    const int64_t m0 = H * 16;
+    if (VEC && active && m0 + 16 <= n) {
+        const char* p = reinterpret_cast<const char*>(A) + m0 * dtype_size(DT);
+        const u32x8 a = ldg_stream_v8(p);
 #pragma unroll
-            for (int i = 0; i < 4; i++) {
-                if constexpr (DT == BF16) {
-                    x[2 * i] = __uint_as_float(w[i] << 16);
-                    x[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
-                } else {
-                    x[2 * i] = f16_bits_to_f32(w[i] & 0xffffu);
-                    x[2 * i + 1] = f16_bits_to_f32(w[i] >> 16);
-                }
+        for (int i = 0; i < 8; i++) r.w[i] = a.v[i];
+        if constexpr (DT == F32) {
+            const u32x8 b = ldg_stream_v8(p + 32);
+#pragma unroll
+            for (int i = 0; i < 8; i++) r.w[8 + i] = b.v[i];
+        }
+    } else {
+        // ragged tail or unaligned input: element-wise raw loads, zeros beyond n
+        if constexpr (DT == F32) {
+            const float* a = reinterpret_cast<const float*>(A);
+#pragma unroll
+            for (int e = 0; e < 16; e++) r.w[e] = (active && m0 + e < n) ? __float_as_uint(a[m0 + e]) : 0u;
+        } else {
+            const uint16_t* a = reinterpret_cast<const uint16_t*>(A);
+#pragma unroll
+            for (int i = 0; i < 8; i++) {
+                const uint32_t lo = (active && m0 + 2 * i < n) ? (uint32_t)a[m0 + 2 * i] : 0u;
+                const uint32_t hi = (active && m0 + 2 * i + 1 < n) ? (uint32_t)a[m0 + 2 * i + 1] : 0u;
+                r.w[i] = lo | (hi << 16);
             }
+        }
+    }
+    return r;
+}
+
+template <int DT>
+__device__ __forceinline__ void widen(const Raw<DT>& r, float* x) {
+    if constexpr (DT == F32) {
+#pragma unroll
+        for (int e = 0; e < 16; e++) x[e] = __uint_as_float(r.w[e]);
+    } else if constexpr (DT == BF16) {
+#pragma unroll
+        for (int i = 0; i < 8; i++) {
+            x[2 * i] = __uint_as_float(r.w[i] << 16);
+            x[2 * i + 1] = __uint_as_float(r.w[i] & 0xffff0000u);
         }
     } else {
 #pragma unroll
-        for (int e = 0; e < 8; e++)
-            x[e] = (active && m0 + e < n) ? load_as_f32<DT>(A, m0 + e) : 0.0f;
+        for (int i = 0; i < 8; i++) {
+            x[2 * i] = f16_bits_to_f32(r.w[i] & 0xffffu);
+            x[2 * i + 1] = f16_bits_to_f32(r.w[i] >> 16);
+        }
     }
+}
+
+__device__ __forceinline__ uint4 lds128(uint32_t saddr) {
+    uint4 v;
+    asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(saddr));
+    return v;
+}
+
+__device__ __forceinline__ float rcp_approx(float d) {
+    float r;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(d));
+    return r;
 }
 
 template <int K, int DT, bool VEC>
@@ -129,7 +172,9 @@ __global__ void __launch_bounds__(kThreads)
 kbit_quant_kernel(const void* __restrict__ A, int64_t n, const float* __restrict__ codebook,
                   float* __restrict__ absmax, uint32_t* __restrict__ packed) {
     constexpr int NE = 1 << K;
-    __shared__ __align__(16) float4 lut[kCells * kReplicas];    // 32 KB
+    constexpr int NACC = K == 5 ? 4 : 2;          // elements per accumulator: 4 (K=5) or 8
+    constexpr int EPA = 16 / NACC;
+    __shared__ __align__(16) uint4 lut[kCells * kReplicas];    // 32 KB
     __shared__ float cb[32];
     __shared__ float thr[33];
     __shared__ int fast_ok;
@@ -157,8 +202,8 @@ kbit_quant_kernel(const void* __restrict__ A, int64_t n, const float* __restrict
         if (fast && tid >= 1 && tid < NE) thr[tid] = bisect_threshold(prev, c);
     }
     __syncthreads();
-    const bool fast_cb = fast_ok != 0;
-    if (fast_cb) {
+    int multi = 0;
+    if (fast_ok) {
         for (int cell = tid; cell < kCells; cell += kThreads) {
             const int cs = cell < 128 ? cell : cell - 256;
             const float wlo = __fsub_rn((float)cs * 0.015625f, 0x1p-13f + 0x1p-12f);
@@ -169,119 +214,138 @@ kbit_quant_kernel(const void* __restrict__ A, int64_t n, const float* __restrict
                 if (T < wlo) below++;
                 else if (T <= whi) { rel++; relj = j; }
             }
-            float tlo = __int_as_float(0x7f800000), thi = tlo;               // +inf: never crossed
+            float negT = __int_as_float(0xff800000), half = 0.0f;     // -inf, 0: never crossed
             if (rel == 1) {
                 const float T = thr[relj];
-                const float g = __fadd_ru(__fmul_ru(fabsf(T), 0x1p-19f), 0x1p-100f);
-                tlo = __fsub_rd(T, g);
-                thi = __fadd_ru(T, g);
-            } else if (rel > 1) {
-                tlo = __int_as_float(0xff800000);                              // -inf: always guard
+                negT = -T;
+                half = __fmul_rn(__fsub_rn(T, key_f32(f32_key(T) - 1)), 0.5f);
             }
-            const float4 ent = make_float4(tlo, thi, __uint_as_float(spread4((uint32_t)below)),
-                                           __uint_as_float(spread4((uint32_t)below + 1)));
+            multi |= rel > 1;
+            const uint4 ent = make_uint4(__float_as_uint(negT), __float_as_uint(half),
+                                         spread<K>((uint32_t)below), spread<K>((uint32_t)below + 1));
 #pragma unroll
             for (int r = 0; r < kReplicas; r++) lut[cell * kReplicas + r] = ent;
         }
     }
-    __syncthreads();
+    const bool fast_cb = (fast_ok != 0) && !__syncthreads_or(multi);
 
-    const char* lutb = reinterpret_cast<const char*>(lut);
-    const uint32_t lutoff = (uint32_t)(lane & 7) << 4;
-    const uint32_t part = lane & 3;
-    const uint32_t sel_a = (part & 1) ? 0x3715u : 0x6240u;
-    const uint32_t sel_b = (part & 2) ? 0x3276u : 0x5410u;
-    const uint32_t grp_mask = 0xFu << (lane & ~3);
-    const float t16 = (K == 5 && fast_cb) ? thr[16] : 0.0f;
+    const uint32_t lut_s = (uint32_t)__cvta_generic_to_shared(lut) + ((uint32_t)(lane & 7) << 4);
+    const bool packed_v2 = (reinterpret_cast<uintptr_t>(packed) & 7u) == 0;
+    const uint32_t h = lane & 1;
+    const uint32_t sel_send = h ? 0x5140u : 0x7362u;
+    const uint32_t sel_keep = h ? 0x7362u : 0x5140u;
+    const uint32_t sel_wa = h ? 0x1054u : 0x5410u;
+    const uint32_t sel_wb = h ? 0x3276u : 0x7632u;
+    const uint32_t pair_mask = 3u << (lane & ~1);
+    const float2 magic = make_float2(12582912.0f, 12582912.0f);
 
-    const int64_t nq = ((n + 31) >> 5) * 4;                      // quarter blocks
+    const int64_t nh = ((n + 31) >> 5) * 2;                      // half blocks
     const int64_t stride = (int64_t)gridDim.x * kThreads;
-    for (int64_t wbase = (int64_t)blockIdx.x * kThreads + (tid & ~31); wbase < nq; wbase += stride) {
-        const int64_t Q = wbase + lane;
-        const bool active = Q < nq;                               // the 4 lanes of a block agree
-        float x[8];
-        load8<DT, VEC>(A, n, Q, active, x);
+    int64_t wbase = (int64_t)blockIdx.x * kThreads + (tid & ~31);
+    Raw<DT> cur = load_raw<DT, VEC>(A, n, wbase + lane, wbase + lane < nh);
+    for (; wbase < nh; wbase += stride) {
+        const int64_t H = wbase + lane;
+        const bool active = H < nh;                               // the 2 lanes of a block agree
+        const int64_t Hn = H + stride;
+        const Raw<DT> nxt = load_raw<DT, VEC>(A, n, Hn, Hn < nh);  // prefetch the next half block
+
+        float x[16];
+        widen<DT>(cur, x);
 
         // NaN-propagating block max decides between the fast and the exact path
         float m = max3_abs_nan(x[0], x[1], x[2]);
         m = max3_abs_nan(m, x[3], x[4]);
         m = max3_abs_nan(m, x[5], x[6]);
-        m = max_nan(m, fabsf(x[7]));
+        m = max3_abs_nan(m, x[7], x[8]);
+        m = max3_abs_nan(m, x[9], x[10]);
+        m = max3_abs_nan(m, x[11], x[12]);
+        m = max3_abs_nan(m, x[13], x[14]);
+        m = max_nan(m, fabsf(x[15]));
         m = max_nan(m, __shfl_xor_sync(0xffffffffu, m, 1));
-        m = max_nan(m, __shfl_xor_sync(0xffffffffu, m, 2));
         const bool special = !(m <= 0x1p125f);
         float amax = m;
         if (special) {   // the stored absmax ignores NaN unless the whole block is NaN
             float a = fabsf(x[0]);
 #pragma unroll
-            for (int e = 1; e < 8; e++) a = fmaxf(a, fabsf(x[e]));
-            a = fmaxf(a, __shfl_xor_sync(grp_mask, a, 1));
-            a = fmaxf(a, __shfl_xor_sync(grp_mask, a, 2));
-            amax = a;
+            for (int e = 1; e < 16; e++) a = fmaxf(a, fabsf(x[e]));
+            amax = fmaxf(a, __shfl_xor_sync(pair_mask, a, 1));
         }
         const float d = fmaxf(amax, 1e-8f);
 
-        uint32_t acc = 0, acc4 = 0;
-        bool exact = special || !fast_cb;
-        if (!exact) {
-            const float r = __frcp_rn(d);
-            bool guard = false;
+        uint32_t acc[NACC];
 #pragma unroll
-            for (int e = 0; e < 8; e++) {
-                const float q = __fmul_rn(x[e], r);
-                const float f = __fmaf_rn(q, 8192.0f, 12582912.0f);
-                const float4 ent = *reinterpret_cast<const float4*>(
-                    lutb + ((__float_as_uint(f) & 0x7f80u) | lutoff));
-                const bool a = q >= ent.x;
-                const bool b = q >= ent.y;
-                guard |= (a != b);
-                acc += (b ? __float_as_uint(ent.w) : __float_as_uint(ent.z)) << e;
-                if constexpr (K == 5) acc4 |= set_ge(q, t16) & (1u << e);
+        for (int g = 0; g < NACC; g++) acc[g] = 0;
+        if (!special && fast_cb) {
+            const float rs = __fmul_rn(rcp_approx(d), 8192.0f);
+            const float2 dd = make_float2(d, d);
+            const float2 rr = make_float2(rs, rs);
+#pragma unroll
+            for (int e = 0; e < 16; e += 2) {
+                const float2 xe = make_float2(x[e], x[e + 1]);
+                const float2 f = __ffma2_rn(xe, rr, magic);
+                const uint4 t0 = lds128(lut_s + (__float_as_uint(f.x) & 0x7f80u));
+                const uint4 t1 = lds128(lut_s + (__float_as_uint(f.y) & 0x7f80u));
+                const float2 u = __ffma2_rn(make_float2(__uint_as_float(t0.x), __uint_as_float(t1.x)), dd, xe);
+                const float2 v = __ffma2_rn(make_float2(__uint_as_float(t0.y), __uint_as_float(t1.y)), dd, u);
+                acc[e / EPA] += (v.x > 0.0f ? t0.w : t0.z) << (e % EPA);
+                acc[(e + 1) / EPA] += (v.y > 0.0f ? t1.w : t1.z) << ((e + 1) % EPA);
             }
-            exact = guard;
-        }
-        if (exact) {
-            acc = 0;
-            acc4 = 0;
+        } else {
 #pragma unroll
-            for (int e = 0; e < 8; e++) {
+            for (int e = 0; e < 16; e++) {
                 const uint32_t idx = nearest_entry<NE>(__fdiv_rn(x[e], d), cb);
-                acc |= spread4(idx) << e;
-                if constexpr (K == 5) acc4 |= ((idx >> 4) & 1u) << e;
+                acc[e / EPA] += spread<K>(idx) << (e % EPA);
             }
         }
 
-        // 4x4 byte transpose across the block's lanes: lane j ends with plane word j
-        acc = prmt(acc, __shfl_xor_sync(0xffffffffu, acc, 1), sel_a);
-        acc = prmt(acc, __shfl_xor_sync(0xffffffffu, acc, 2), sel_b);
+        // planes 0..3 of elements 0..7 (B0) and 8..15 (B1): byte j = plane j
+        uint32_t B0, B1, p4 = 0;
         if constexpr (K == 5) {
-            acc4 = prmt(acc4, __shfl_xor_sync(0xffffffffu, acc4, 1), sel_a);
-            acc4 = prmt(acc4, __shfl_xor_sync(0xffffffffu, acc4, 2), sel_b);
+            B0 = (acc[0] & 0x0f0f0f0fu) | ((acc[1] & 0x0f0f0f0fu) << 4);
+            B1 = (acc[2] & 0x0f0f0f0fu) | ((acc[3] & 0x0f0f0f0fu) << 4);
+            p4 = ((acc[0] >> 4) & 0xfu) | (acc[1] & 0xf0u) | (((acc[2] >> 4) & 0xfu) << 8) | ((acc[3] & 0xf0u) << 8);
+        } else {
+            B0 = acc[0];
+            B1 = acc[1];
         }
+        // lane h holds bytes 2h, 2h+1 of every word; swap halves so it ends with words 2h, 2h+1
+        const uint32_t send = prmt(B0, B1, sel_send);
+        const uint32_t keep = prmt(B0, B1, sel_keep);
+        const uint32_t recv = __shfl_xor_sync(0xffffffffu, send, 1);
+        const uint32_t wa = prmt(keep, recv, sel_wa);
+        const uint32_t wb = prmt(keep, recv, sel_wb);
+        uint32_t w4 = 0;
+        if constexpr (K == 5) w4 = p4 | (__shfl_xor_sync(0xffffffffu, p4, 1) << 16);
+
         if (active) {
-            const int64_t b = Q >> 2;
-            if (part < (uint32_t)(K < 4 ? K : 4)) packed[b * K + part] = acc;
-            if (part == 0) {
-                if constexpr (K == 5) packed[b * 5 + 4] = acc4;
-                absmax[b] = amax;
+            const int64_t b = H >> 1;
+            uint32_t* out = packed + b * K;
+            if (K == 4 && packed_v2) {
+                asm volatile("st.global.v2.u32 [%0], {%1,%2};" :: "l"(out + 2 * h), "r"(wa), "r"(wb) : "memory");
+            } else {
+                if (2 * h < K) out[2 * h] = wa;
+                if (2 * h + 1 < K) out[2 * h + 1] = wb;
+                if constexpr (K == 5) { if (h == 0) out[4] = w4; }
             }
+            if (h == 0) absmax[b] = amax;
         }
+        cur = nxt;
     }
 }
 
 template <int K, int DT>
 cudaError_t launch_t(const void* A, int64_t n, const float* codebook, float* absmax,
                      uint32_t* packed, bool vec, cudaStream_t s) {
-    const int64_t nq = ((n + 31) >> 5) * 4;
-    if (vec) {
-        auto k = kbit_quant_kernel<K, DT, true>;
-        int grid = persistent_grid(k, kThreads, 0, nq, kThreads);
-        k<<<grid, kThreads, 0, s>>>(A, n, codebook, absmax, packed);
-    } else {
-        auto k = kbit_quant_kernel<K, DT, false>;
-        int grid = persistent_grid(k, kThreads, 0, nq, kThreads);
-        k<<<grid, kThreads, 0, s>>>(A, n, codebook, absmax, packed);
+    const int64_t nh = ((n + 31) >> 5) * 2;
+    auto k = vec ? kbit_quant_kernel<K, DT, true> : kbit_quant_kernel<K, DT, false>;
+    static bool attr_set[2] = {false, false};
+    if (!attr_set[vec]) {
+        cudaFuncSetAttribute(k, cudaFuncAttributePreferredSharedMemoryCarveout,
+                             cudaSharedmemCarveoutMaxShared);
+        attr_set[vec] = true;
     }
+    const int grid = persistent_grid(k, kThreads, 0, nh, kThreads);
+    k<<<grid, kThreads, 0, s>>>(A, n, codebook, absmax, packed);
     return cudaGetLastError();
 }
 

@@ -22,9 +22,10 @@
  *   - dtype values: BBC_F16 (IEEE binary16), BBC_BF16 (bfloat16), BBC_F32.
  *   - Conversions to fp16/bf16 round to nearest, ties to even; subnormals are
  *     kept (no flush to zero) in every step.
- *   - Device pointers need only the natural alignment of their element type;
- *     16-byte-aligned buffers take the vectorised path, others a scalar path
- *     with identical results.
+ *   - Device pointers need only the natural alignment of their element type.
+ *     Well-aligned buffers take the vectorised path (32 bytes for the input of
+ *     kbit_quantize, 16 bytes for the outputs of the dequantizers, 8 bytes for
+ *     the nested codes), others a scalar path with identical results.
  */
 #ifndef BBC_H
 #define BBC_H
