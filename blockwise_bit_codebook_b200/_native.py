@@ -8,7 +8,7 @@ BBC_F16, BBC_BF16, BBC_F32 = 0, 1, 2
 _STATUS = {0: "BBC_OK", 1: "BBC_ERR_INVALID", 2: "BBC_ERR_UNSUPPORTED", 3: "BBC_ERR_CUDA"}
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-_LIB_PATH = os.path.join(_HERE, "libbbc.so")
+_LIB_PATH = os.environ.get("BBC_LIBRARY") or os.path.join(_HERE, "libbbc.so")
 _lib = None
 
 

@@ -16,7 +16,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
-LIB = os.path.join(HERE, "libbbc.so")
+LIB = os.environ.get("BBC_BUILD_OUTPUT") or os.path.join(HERE, "libbbc.so")
 
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
@@ -44,7 +44,8 @@ def build(force: bool = False, verbose: bool = False, extra=()) -> str:
     try:
         def compile_one(src):
             obj = os.path.join(tmp, os.path.basename(src) + ".o")
-            cmd = [NVCC, *ARCH, *FLAGS, *extra, "-c", src, "-o", obj]
+            cmd = [NVCC, *ARCH, *FLAGS, *os.environ.get("BBC_NVCC_EXTRA", "").split(), *extra,
+                   "-c", src, "-o", obj]
             r = subprocess.run(cmd, capture_output=True, text=True)
             if r.returncode != 0 or verbose:
                 sys.stderr.write(" ".join(cmd) + "\n" + r.stdout + r.stderr)

@@ -71,7 +71,7 @@ int kbit_dequantize(const uint32_t* packed, const float* absmax, const float* co
         return fail(BBC_ERR_UNSUPPORTED, "kbit_dequantize: blocksize must be 32 (got %d)", blocksize);
     if (!aligned(out, elem_size(out_dtype)) || !aligned(codebook, 4) || !aligned(absmax, 4) || !aligned(packed, 4))
         return fail(BBC_ERR_INVALID, "kbit_dequantize: pointer not aligned to its element size");
-    const bool vec = aligned(out, 16);
+    const bool vec = aligned(out, 32);     // 32-byte stores of 16-element groups
     return cuda_status(bbc::launch_kbit_dequantize(packed, absmax, codebook, K, n, out_dtype, out, vec,
                                                    static_cast<cudaStream_t>(stream)),
                        "kbit_dequantize launch");
@@ -99,7 +99,7 @@ int dequantize_4bit_nested(const uint8_t* codes, const uint8_t* absmax_q, const 
                     blocksize2);
     if (!aligned(out, elem_size(out_dtype)) || !aligned(code2, 4) || !aligned(absmax2, 4) || !aligned(code4, 4))
         return fail(BBC_ERR_INVALID, "dequantize_4bit_nested: pointer not aligned to its element size");
-    const bool vec = aligned(out, 16) && aligned(codes, 8);
+    const bool vec = aligned(out, 32) && aligned(codes, 16);   // 8/16-byte loads, 32-byte stores
     return cuda_status(bbc::launch_nested_dequantize(codes, absmax_q, code2, absmax2, offset, code4, n,
                                                      log2_bs, out_dtype, out, vec,
                                                      static_cast<cudaStream_t>(stream)),

@@ -4,15 +4,16 @@
 // kDequantizeBlockwise_kbit): out[m] = T(codebook[idx_m] * absmax[m / 32]),
 // where idx_m is gathered from the K bit-plane words of block m / 32.
 //
-// B200 layout: a thread owns one quarter block (8 consecutive elements), so
-// the four threads of a block sit in adjacent lanes and a warp covers 8 blocks
-// (256 elements): the output is written with one 16-byte store per thread per
-// 16-bit element type (two for fp32), fully coalesced. Each thread reads the K
-// words of its block (the 4 lanes of a block hit the same addresses), keeps
-// byte `part` of each, and decodes its 8 indices with one multiply-high bit
-// gather per element. The codebook lives in shared memory: 32 consecutive
-// floats occupy the 32 banks once, so the per-element lookup never conflicts.
-// The grid is persistent (SMs x resident CTAs) with a grid-stride loop.
+// B200 layout: a thread owns half a block (16 consecutive elements), so the two
+// threads of a block sit in adjacent lanes and a warp covers 16 blocks (512
+// elements). Each thread reads the block's absmax and K words (the two lanes
+// of a block hit the same addresses), keeps bytes 2h and 2h+1 of every word
+// (one byte permute per word pair), decodes each 4-bit index with one
+// multiply-high bit gather and writes its 16 outputs with one 32-byte store
+// (two for fp32). The loads of the next half block are issued before the
+// current one is decoded, so each thread keeps two round trips in flight. The
+// codebook lives in shared memory: 32 consecutive floats occupy the 32 banks
+// once, so the per-element lookup never conflicts. Persistent grid-stride loop.
 #include "common.cuh"
 #include "launch.h"
 
@@ -22,12 +23,10 @@ namespace {
 
 constexpr int kThreads = 256;
 
-// Byte offset (idx * 4) of element e of a quarter block from the gathered planes.
-// B holds byte `part` of plane word j in its byte j (j < 4); B3 = B << 3.
-// For e >= 3 the bits j*8+e are moved to bits 34+j of the 64-bit product
-// (multiplier sum_j 2^(34-7j-e)); every cross term lands outside bits 34..37,
-// on distinct positions, so no carry reaches the field. For e < 3 the same
-// gather runs on B3 with e+3.
+// Byte offset (idx * 4) of element e (0..7) of a plane group B (byte j = plane j for
+// elements 0..7; B3 = B << 3). For e >= 3 bits 8j+e are moved to bits 34+j of the 64-bit
+// product (multiplier sum_j 2^(34-7j-e)); every cross term lands outside bits 34..37 on
+// distinct positions, so no carry reaches the field. For e < 3 the same gather runs on B3.
 template <int E>
 __device__ __forceinline__ uint32_t plane_offset4(uint32_t B, uint32_t B3) {
     constexpr int e = E < 3 ? E + 3 : E;
@@ -35,6 +34,29 @@ __device__ __forceinline__ uint32_t plane_offset4(uint32_t B, uint32_t B3) {
     constexpr uint32_t mult = (1u << (34 - e)) | (1u << (27 - e)) | (1u << (20 - e)) | (1u << (13 - e));
     const uint32_t src = E < 3 ? B3 : B;
     return __umulhi(src & mask, mult) & 0x3Cu;
+}
+
+template <int K>
+struct BlockIn {
+    float am;
+    uint32_t w[K];
+};
+
+template <int K>
+__device__ __forceinline__ BlockIn<K> load_block(const uint32_t* packed, const float* absmax,
+                                                 int64_t b, bool active) {
+    BlockIn<K> r;
+    if (active) {
+        r.am = __ldg(absmax + b);
+        const uint32_t* wp = packed + b * K;
+#pragma unroll
+        for (int j = 0; j < K; j++) r.w[j] = ldg_u32(wp + j);
+    } else {
+        r.am = 0.0f;
+#pragma unroll
+        for (int j = 0; j < K; j++) r.w[j] = 0u;
+    }
+    return r;
 }
 
 template <int K, int DT, bool VEC>
@@ -46,75 +68,73 @@ kbit_dequant_kernel(const uint32_t* __restrict__ packed, const float* __restrict
     __syncthreads();
     const char* cbb = reinterpret_cast<const char*>(cb);
 
-    const int64_t nq = ((n + 31) >> 5) * 4;                       // quarter blocks
-    const uint32_t part = threadIdx.x & 3;
-    const uint32_t sel01 = part | ((4 + part) << 4);              // byte `part` of a, then of b
+    const int64_t nh = ((n + 31) >> 5) * 2;                       // half blocks
+    const uint32_t h = threadIdx.x & 1;
+    // bytes 2h and 2h+1 of two words a, b -> [a.2h, b.2h, a.2h+1, b.2h+1]
+    const uint32_t sel = (2 * h) | ((4 + 2 * h) << 4) | ((2 * h + 1) << 8) | ((5 + 2 * h) << 12);
     const int64_t stride = (int64_t)gridDim.x * kThreads;
 
-    for (int64_t Q = (int64_t)blockIdx.x * kThreads + threadIdx.x; Q < nq; Q += stride) {
-        const int64_t b = Q >> 2;
-        const float am = __ldg(absmax + b);
-        const uint32_t* wp = packed + b * K;
-        uint32_t w[K];
-#pragma unroll
-        for (int j = 0; j < K; j++) w[j] = ldg_u32(wp + j);
+    int64_t H = (int64_t)blockIdx.x * kThreads + threadIdx.x;
+    BlockIn<K> cur = load_block<K>(packed, absmax, H >> 1, H < nh);
+    for (; H < nh; H += stride) {
+        const int64_t Hn = H + stride;
+        const BlockIn<K> nxt = load_block<K>(packed, absmax, Hn >> 1, Hn < nh);
 
-        uint32_t B;
+        uint32_t B0, B1;
         if constexpr (K == 2) {
-            B = prmt(w[0], w[1], sel01) & 0xFFFFu;
-        } else if constexpr (K == 3) {
-            B = prmt(prmt(w[0], w[1], sel01), prmt(w[2], 0u, part | 0x4440u), 0x5410u);
+            const uint32_t t = prmt(cur.w[0], cur.w[1], sel);
+            B0 = prmt(t, 0u, 0x4410u);
+            B1 = prmt(t, 0u, 0x4432u);
         } else {
-            B = prmt(prmt(w[0], w[1], sel01), prmt(w[2], w[3], sel01), 0x5410u);
+            const uint32_t t01 = prmt(cur.w[0], cur.w[1], sel);
+            const uint32_t t23 = K == 3 ? prmt(cur.w[2], 0u, (2 * h) | (4u << 4) | ((2 * h + 1) << 8) | (4u << 12))
+                                        : prmt(cur.w[2], cur.w[K > 3 ? 3 : 2], sel);
+            B0 = prmt(t01, t23, 0x5410u);
+            B1 = prmt(t01, t23, 0x7632u);
         }
-        const uint32_t B3 = B << 3;
-        uint32_t hi4 = 0;
-        if constexpr (K == 5) hi4 = w[4] >> (8 * part);           // plane 4: bit e is element e
+        uint32_t p4 = 0;
+        if constexpr (K == 5) p4 = cur.w[4] >> (16 * h);           // plane 4: bit e is element e
+        const uint32_t B0s = B0 << 3, B1s = B1 << 3;
+        const float am = cur.am;
 
-        float y[8];
-#define BBC_DQ_ELEM(E)                                                              \
-        {                                                                           \
-            uint32_t off = plane_offset4<E>(B, B3);                                 \
-            if constexpr (K == 5)                                                   \
-                off |= (E <= 6 ? (hi4 << (6 - E)) : (hi4 >> 1)) & 0x40u;           \
-            y[E] = __fmul_rn(*reinterpret_cast<const float*>(cbb + off), am);       \
+        float y[16];
+#define BBC_DQ_ELEM(E)                                                                        \
+        {                                                                                     \
+            uint32_t off = (E) < 8 ? plane_offset4<(E) & 7>(B0, B0s) : plane_offset4<(E) & 7>(B1, B1s); \
+            if constexpr (K == 5)                                                             \
+                off |= ((E) <= 6 ? (p4 << (6 - (E))) : (p4 >> ((E) - 6))) & 0x40u;           \
+            y[E] = __fmul_rn(*reinterpret_cast<const float*>(cbb + off), am);                 \
         }
         BBC_DQ_ELEM(0) BBC_DQ_ELEM(1) BBC_DQ_ELEM(2) BBC_DQ_ELEM(3)
         BBC_DQ_ELEM(4) BBC_DQ_ELEM(5) BBC_DQ_ELEM(6) BBC_DQ_ELEM(7)
+        BBC_DQ_ELEM(8) BBC_DQ_ELEM(9) BBC_DQ_ELEM(10) BBC_DQ_ELEM(11)
+        BBC_DQ_ELEM(12) BBC_DQ_ELEM(13) BBC_DQ_ELEM(14) BBC_DQ_ELEM(15)
 #undef BBC_DQ_ELEM
 
-        const int64_t m0 = Q * 8;
-        if (VEC && m0 + 8 <= n) {
-            uint32_t wv[8];
+        const int64_t m0 = H * 16;
+        if (VEC && m0 + 16 <= n) {
+            uint32_t wv[16];
             pack8<DT>(y, wv);
+            pack8<DT>(y + 8, wv + (DT == F32 ? 8 : 4));
             char* dst = reinterpret_cast<char*>(out) + m0 * dtype_size(DT);
-            if constexpr (DT == F32) {
-                stg_v4(dst, wv[0], wv[1], wv[2], wv[3]);
-                stg_v4(dst + 16, wv[4], wv[5], wv[6], wv[7]);
-            } else {
-                stg_v4(dst, wv[0], wv[1], wv[2], wv[3]);
-            }
+            stg_v8(dst, wv);
+            if constexpr (DT == F32) stg_v8(dst + 32, wv + 8);
         } else {
 #pragma unroll
-            for (int e = 0; e < 8; e++)
+            for (int e = 0; e < 16; e++)
                 if (m0 + e < n) store_from_f32<DT>(out, m0 + e, y[e]);
         }
+        cur = nxt;
     }
 }
 
 template <int K, int DT>
 cudaError_t launch_t(const uint32_t* packed, const float* absmax, const float* codebook, int64_t n,
                      void* out, bool vec, cudaStream_t s) {
-    const int64_t nq = ((n + 31) >> 5) * 4;
-    if (vec) {
-        auto k = kbit_dequant_kernel<K, DT, true>;
-        int grid = persistent_grid(k, kThreads, 0, nq, kThreads);
-        k<<<grid, kThreads, 0, s>>>(packed, absmax, codebook, n, out);
-    } else {
-        auto k = kbit_dequant_kernel<K, DT, false>;
-        int grid = persistent_grid(k, kThreads, 0, nq, kThreads);
-        k<<<grid, kThreads, 0, s>>>(packed, absmax, codebook, n, out);
-    }
+    const int64_t nh = ((n + 31) >> 5) * 2;
+    auto k = vec ? kbit_dequant_kernel<K, DT, true> : kbit_dequant_kernel<K, DT, false>;
+    const int grid = persistent_grid(k, kThreads, 0, nh, kThreads);
+    k<<<grid, kThreads, 0, s>>>(packed, absmax, codebook, n, out);
     return cudaGetLastError();
 }
 

@@ -54,6 +54,10 @@ namespace {
 constexpr int kThreads = 256;
 constexpr int kCells = 256;
 constexpr int kReplicas = 8;
+#ifndef BBC_QUANT_MIN_CTAS
+#define BBC_QUANT_MIN_CTAS 3
+#endif
+constexpr int kMinCtas = BBC_QUANT_MIN_CTAS;   // resident CTAs per SM the register budget targets
 
 __device__ __forceinline__ int64_t f32_key(float f) {
     const int32_t b = __float_as_int(f);
@@ -135,6 +139,49 @@ __device__ __forceinline__ Raw<DT> load_raw(const void* A, int64_t n, int64_t H,
     return r;
 }
 
+// Exact fp32 values of the two 16-bit elements packed in w (element 2i in the low half).
+// Raw words of a half block that lies entirely inside the input (vector loads only).
+template <int DT>
+__device__ __forceinline__ Raw<DT> load_full(const void* A, int64_t H, bool active) {
+    Raw<DT> r;
+    if (active) {
+        const char* p = reinterpret_cast<const char*>(A) + H * 16 * dtype_size(DT);
+        const u32x8 a = ldg_stream_v8(p);
+#pragma unroll
+        for (int i = 0; i < 8; i++) r.w[i] = a.v[i];
+        if constexpr (DT == F32) {
+            const u32x8 b = ldg_stream_v8(p + 32);
+#pragma unroll
+            for (int i = 0; i < 8; i++) r.w[8 + i] = b.v[i];
+        }
+    } else {
+#pragma unroll
+        for (int i = 0; i < (DT == F32 ? 16 : 8); i++) r.w[i] = 0u;
+    }
+    return r;
+}
+
+template <int DT>
+__device__ __forceinline__ void widen_pair(uint32_t w, float& lo, float& hi) {
+    if constexpr (DT == BF16) {
+        lo = __uint_as_float(w << 16);
+        hi = __uint_as_float(w & 0xffff0000u);
+    } else {
+        lo = f16_bits_to_f32(w & 0xffffu);
+        hi = f16_bits_to_f32(w >> 16);
+    }
+}
+
+// Per-half NaN-propagating max of absolute values of two packed pairs (the sign bit of the
+// result is not meaningful; callers take the absolute value).
+template <int DT>
+__device__ __forceinline__ uint32_t pair_absmax(uint32_t a, uint32_t b) {
+    uint32_t r;
+    if constexpr (DT == BF16) asm("max.NaN.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+    else asm("max.NaN.xorsign.abs.f16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+    return r;
+}
+
 template <int DT>
 __device__ __forceinline__ void widen(const Raw<DT>& r, float* x) {
     if constexpr (DT == F32) {
@@ -155,25 +202,161 @@ __device__ __forceinline__ void widen(const Raw<DT>& r, float* x) {
     }
 }
 
-__device__ __forceinline__ uint4 lds128(uint32_t saddr) {
-    uint4 v;
-    asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(saddr));
-    return v;
-}
-
 __device__ __forceinline__ float rcp_approx(float d) {
     float r;
     asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(d));
     return r;
 }
 
+// Per-thread constants of the main loop.
+struct LoopCtx {
+    const char* lut;        // generic pointer to the shared table
+    uint32_t lut_s;         // its shared-window address
+    uint32_t lane16;        // this lane's replica offset
+    uint32_t h;             // which half of the block this lane owns
+    uint32_t sel_send, sel_keep, sel_wa, sel_wb, pair_mask;
+    bool fast_cb;
+    bool packed_v2;
+};
+
+#ifndef BBC_QUANT_LDS_ASM
+#define BBC_QUANT_LDS_ASM 1
+#endif
+// The table entry of the cell whose index sits in bits 7..14 of `fbits`.
+__device__ __forceinline__ uint4 lut_entry(const LoopCtx& c, uint32_t fbits) {
+    const uint32_t off = (fbits & 0x7f80u) | c.lane16;
+#if BBC_QUANT_LDS_ASM
+    uint4 v;
+    asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(c.lut_s + off));
+    return v;
+#else
+    return *reinterpret_cast<const uint4*>(__builtin_assume_aligned(c.lut + off, 16));
+#endif
+}
+
+// Fast path for one half block: thresholds via the table, exact two-FMA test per element.
+template <int K, int DT>
+__device__ __forceinline__ void fast_codes(const Raw<DT>& raw, float d, const LoopCtx& c, uint32_t* acc) {
+    constexpr int EPA = K == 5 ? 4 : 8;           // 4 elements per accumulator for K = 5, else 8
+    const float rs = __fmul_rn(rcp_approx(d), 8192.0f);
+#pragma unroll
+    for (int e = 0; e < 16; e += 2) {
+        float x0, x1;
+        if constexpr (DT == F32) {
+            x0 = __uint_as_float(raw.w[e]);
+            x1 = __uint_as_float(raw.w[e + 1]);
+        } else {
+            widen_pair<DT>(raw.w[e / 2], x0, x1);
+        }
+        const float2 f = __ffma2_rn(make_float2(x0, x1), make_float2(rs, rs),
+                                    make_float2(12582912.0f, 12582912.0f));
+        const uint4 t0 = lut_entry(c, __float_as_uint(f.x));
+        const uint4 t1 = lut_entry(c, __float_as_uint(f.y));
+        const float v0 = __fmaf_rn(__uint_as_float(t0.y), d, __fmaf_rn(__uint_as_float(t0.x), d, x0));
+        const float v1 = __fmaf_rn(__uint_as_float(t1.y), d, __fmaf_rn(__uint_as_float(t1.x), d, x1));
+        acc[e / EPA] += (v0 > 0.0f ? t0.w : t0.z) << (e % EPA);
+        acc[(e + 1) / EPA] += (v1 > 0.0f ? t1.w : t1.z) << ((e + 1) % EPA);
+    }
+}
+
+// Brute-force path for one half block: IEEE division and the nearest-entry rule verbatim.
+template <int K, int DT>
+__device__ __forceinline__ void exact_codes(const Raw<DT>& raw, float d, const float* cb, uint32_t* acc) {
+    constexpr int EPA = K == 5 ? 4 : 8;
+    float x[16];
+    widen<DT>(raw, x);
+#pragma unroll
+    for (int e = 0; e < 16; e++) {
+        const uint32_t idx = nearest_entry<1 << K>(__fdiv_rn(x[e], d), cb);
+        acc[e / EPA] += spread<K>(idx) << (e % EPA);
+    }
+}
+
+// Quantize the half block H held in `raw` (16 elements) and store its share of the block's
+// words. Every lane of the warp must call this together (it exchanges data with its pair
+// lane); `active` lanes store.
+template <int K, int DT>
+__device__ __forceinline__ void quantize_half(const Raw<DT>& raw, int64_t H, bool active, const LoopCtx& c,
+                                              const float* cb, float* __restrict__ absmax,
+                                              uint32_t* __restrict__ packed) {
+    constexpr int NACC = K == 5 ? 4 : 2;
+    // NaN-propagating block max decides between the fast and the exact path. For 16-bit
+    // inputs it runs on the packed pairs (exact: the max of values of the type is one of them).
+    float m;
+    if constexpr (DT == F32) {
+        const float* xf = reinterpret_cast<const float*>(raw.w);
+        m = max3_abs_nan(xf[0], xf[1], xf[2]);
+        m = max3_abs_nan(m, xf[3], xf[4]);
+        m = max3_abs_nan(m, xf[5], xf[6]);
+        m = max3_abs_nan(m, xf[7], xf[8]);
+        m = max3_abs_nan(m, xf[9], xf[10]);
+        m = max3_abs_nan(m, xf[11], xf[12]);
+        m = max3_abs_nan(m, xf[13], xf[14]);
+        m = max_nan(m, fabsf(xf[15]));
+    } else {
+        uint32_t p = pair_absmax<DT>(raw.w[0], raw.w[1]);
+#pragma unroll
+        for (int i = 2; i < 8; i++) p = pair_absmax<DT>(p, raw.w[i]);
+        float lo, hi;
+        widen_pair<DT>(p, lo, hi);
+        m = max_nan(fabsf(lo), fabsf(hi));
+    }
+    m = max_nan(m, __shfl_xor_sync(0xffffffffu, m, 1));
+    const bool special = !(m <= 0x1p125f);          // NaN, infinite or too large for 1/d
+    float amax = m;
+    if (special) {   // rare: the stored absmax ignores NaN unless the whole block is NaN
+        float x[16];
+        widen<DT>(raw, x);
+        float a = fabsf(x[0]);
+#pragma unroll
+        for (int e = 1; e < 16; e++) a = fmaxf(a, fabsf(x[e]));
+        amax = fmaxf(a, __shfl_xor_sync(c.pair_mask, a, 1));   // both lanes of the block are here
+    }
+    const float d = fmaxf(amax, 1e-8f);
+
+    uint32_t acc[NACC];
+#pragma unroll
+    for (int g = 0; g < NACC; g++) acc[g] = 0;
+    if (!special && c.fast_cb) fast_codes<K, DT>(raw, d, c, acc);
+    else exact_codes<K, DT>(raw, d, cb, acc);
+
+    // planes 0..3 of elements 0..7 (B0) and 8..15 (B1): byte j = plane j
+    uint32_t B0, B1, p4 = 0;
+    if constexpr (K == 5) {
+        B0 = (acc[0] & 0x0f0f0f0fu) | ((acc[1] & 0x0f0f0f0fu) << 4);
+        B1 = (acc[2] & 0x0f0f0f0fu) | ((acc[3] & 0x0f0f0f0fu) << 4);
+        p4 = ((acc[0] >> 4) & 0xfu) | (acc[1] & 0xf0u) | (((acc[2] >> 4) & 0xfu) << 8) | ((acc[3] & 0xf0u) << 8);
+    } else {
+        B0 = acc[0];
+        B1 = acc[1];
+    }
+    // lane h holds bytes 2h, 2h+1 of every word; swap halves so it ends with words 2h, 2h+1
+    const uint32_t send = prmt(B0, B1, c.sel_send);
+    const uint32_t keep = prmt(B0, B1, c.sel_keep);
+    const uint32_t recv = __shfl_xor_sync(0xffffffffu, send, 1);
+    const uint32_t wa = prmt(keep, recv, c.sel_wa);
+    const uint32_t wb = prmt(keep, recv, c.sel_wb);
+    uint32_t w4 = 0;
+    if constexpr (K == 5) w4 = p4 | (__shfl_xor_sync(0xffffffffu, p4, 1) << 16);
+
+    const int64_t b = H >> 1;
+    uint32_t* out = packed + b * K;
+    if (K == 4 && c.packed_v2) {
+        if (active) asm volatile("st.global.v2.u32 [%0], {%1,%2};" :: "l"(out + 2 * c.h), "r"(wa), "r"(wb) : "memory");
+    } else {
+        if (active && 2 * c.h < K) out[2 * c.h] = wa;
+        if (active && 2 * c.h + 1 < K) out[2 * c.h + 1] = wb;
+        if constexpr (K == 5) { if (active && c.h == 0) out[4] = w4; }
+    }
+    if (active && c.h == 0) absmax[b] = amax;
+}
+
 template <int K, int DT, bool VEC>
-__global__ void __launch_bounds__(kThreads)
+__global__ void __launch_bounds__(kThreads, kMinCtas)
 kbit_quant_kernel(const void* __restrict__ A, int64_t n, const float* __restrict__ codebook,
                   float* __restrict__ absmax, uint32_t* __restrict__ packed) {
     constexpr int NE = 1 << K;
-    constexpr int NACC = K == 5 ? 4 : 2;          // elements per accumulator: 4 (K=5) or 8
-    constexpr int EPA = 16 / NACC;
     __shared__ __align__(16) uint4 lut[kCells * kReplicas];    // 32 KB
     __shared__ float cb[32];
     __shared__ float thr[33];
@@ -223,113 +406,48 @@ kbit_quant_kernel(const void* __restrict__ A, int64_t n, const float* __restrict
             multi |= rel > 1;
             const uint4 ent = make_uint4(__float_as_uint(negT), __float_as_uint(half),
                                          spread<K>((uint32_t)below), spread<K>((uint32_t)below + 1));
+            // the 8 lanes of a store phase write 8 different replicas: distinct banks
 #pragma unroll
-            for (int r = 0; r < kReplicas; r++) lut[cell * kReplicas + r] = ent;
+            for (int r = 0; r < kReplicas; r++) lut[cell * kReplicas + ((r + tid) & (kReplicas - 1))] = ent;
         }
     }
-    const bool fast_cb = (fast_ok != 0) && !__syncthreads_or(multi);
+    LoopCtx c;
+    c.fast_cb = (fast_ok != 0) && !__syncthreads_or(multi);
+    c.lut = reinterpret_cast<const char*>(lut);
+    c.lut_s = (uint32_t)__cvta_generic_to_shared(lut);
+    c.lane16 = (uint32_t)(lane & 7) << 4;
+    c.packed_v2 = (reinterpret_cast<uintptr_t>(packed) & 7u) == 0;
+    c.h = lane & 1;
+    c.sel_send = c.h ? 0x5140u : 0x7362u;
+    c.sel_keep = c.h ? 0x7362u : 0x5140u;
+    c.sel_wa = c.h ? 0x1054u : 0x5410u;
+    c.sel_wb = c.h ? 0x3276u : 0x7632u;
+    c.pair_mask = 3u << (lane & ~1);
 
-    const uint32_t lut_s = (uint32_t)__cvta_generic_to_shared(lut) + ((uint32_t)(lane & 7) << 4);
-    const bool packed_v2 = (reinterpret_cast<uintptr_t>(packed) & 7u) == 0;
-    const uint32_t h = lane & 1;
-    const uint32_t sel_send = h ? 0x5140u : 0x7362u;
-    const uint32_t sel_keep = h ? 0x7362u : 0x5140u;
-    const uint32_t sel_wa = h ? 0x1054u : 0x5410u;
-    const uint32_t sel_wb = h ? 0x3276u : 0x7632u;
-    const uint32_t pair_mask = 3u << (lane & ~1);
-    const float2 magic = make_float2(12582912.0f, 12582912.0f);
-
-    const int64_t nh = ((n + 31) >> 5) * 2;                      // half blocks
+    // Persistent grid-stride loop over the half blocks of whole blocks (no bounds checks),
+    // unrolled by two with ping-pong prefetch; then the ragged last block, if any.
+    const int64_t nh_full = VEC ? (n >> 5) * 2 : 0;
+    const int64_t nh = ((n + 31) >> 5) * 2;
     const int64_t stride = (int64_t)gridDim.x * kThreads;
     int64_t wbase = (int64_t)blockIdx.x * kThreads + (tid & ~31);
-    Raw<DT> cur = load_raw<DT, VEC>(A, n, wbase + lane, wbase + lane < nh);
-    for (; wbase < nh; wbase += stride) {
-        const int64_t H = wbase + lane;
-        const bool active = H < nh;                               // the 2 lanes of a block agree
-        const int64_t Hn = H + stride;
-        const Raw<DT> nxt = load_raw<DT, VEC>(A, n, Hn, Hn < nh);  // prefetch the next half block
-
-        float x[16];
-        widen<DT>(cur, x);
-
-        // NaN-propagating block max decides between the fast and the exact path
-        float m = max3_abs_nan(x[0], x[1], x[2]);
-        m = max3_abs_nan(m, x[3], x[4]);
-        m = max3_abs_nan(m, x[5], x[6]);
-        m = max3_abs_nan(m, x[7], x[8]);
-        m = max3_abs_nan(m, x[9], x[10]);
-        m = max3_abs_nan(m, x[11], x[12]);
-        m = max3_abs_nan(m, x[13], x[14]);
-        m = max_nan(m, fabsf(x[15]));
-        m = max_nan(m, __shfl_xor_sync(0xffffffffu, m, 1));
-        const bool special = !(m <= 0x1p125f);
-        float amax = m;
-        if (special) {   // the stored absmax ignores NaN unless the whole block is NaN
-            float a = fabsf(x[0]);
-#pragma unroll
-            for (int e = 1; e < 16; e++) a = fmaxf(a, fabsf(x[e]));
-            amax = fmaxf(a, __shfl_xor_sync(pair_mask, a, 1));
+    if (wbase < nh_full) {
+        Raw<DT> ra = load_full<DT>(A, wbase + lane, wbase + lane < nh_full);
+        Raw<DT> rb;
+        while (true) {
+            rb = load_full<DT>(A, wbase + stride + lane, wbase + stride + lane < nh_full);
+            quantize_half<K, DT>(ra, wbase + lane, wbase + lane < nh_full, c, cb, absmax, packed);
+            wbase += stride;
+            if (wbase >= nh_full) break;
+            ra = load_full<DT>(A, wbase + stride + lane, wbase + stride + lane < nh_full);
+            quantize_half<K, DT>(rb, wbase + lane, wbase + lane < nh_full, c, cb, absmax, packed);
+            wbase += stride;
+            if (wbase >= nh_full) break;
         }
-        const float d = fmaxf(amax, 1e-8f);
-
-        uint32_t acc[NACC];
-#pragma unroll
-        for (int g = 0; g < NACC; g++) acc[g] = 0;
-        if (!special && fast_cb) {
-            const float rs = __fmul_rn(rcp_approx(d), 8192.0f);
-            const float2 dd = make_float2(d, d);
-            const float2 rr = make_float2(rs, rs);
-#pragma unroll
-            for (int e = 0; e < 16; e += 2) {
-                const float2 xe = make_float2(x[e], x[e + 1]);
-                const float2 f = __ffma2_rn(xe, rr, magic);
-                const uint4 t0 = lds128(lut_s + (__float_as_uint(f.x) & 0x7f80u));
-                const uint4 t1 = lds128(lut_s + (__float_as_uint(f.y) & 0x7f80u));
-                const float2 u = __ffma2_rn(make_float2(__uint_as_float(t0.x), __uint_as_float(t1.x)), dd, xe);
-                const float2 v = __ffma2_rn(make_float2(__uint_as_float(t0.y), __uint_as_float(t1.y)), dd, u);
-                acc[e / EPA] += (v.x > 0.0f ? t0.w : t0.z) << (e % EPA);
-                acc[(e + 1) / EPA] += (v.y > 0.0f ? t1.w : t1.z) << ((e + 1) % EPA);
-            }
-        } else {
-#pragma unroll
-            for (int e = 0; e < 16; e++) {
-                const uint32_t idx = nearest_entry<NE>(__fdiv_rn(x[e], d), cb);
-                acc[e / EPA] += spread<K>(idx) << (e % EPA);
-            }
-        }
-
-        // planes 0..3 of elements 0..7 (B0) and 8..15 (B1): byte j = plane j
-        uint32_t B0, B1, p4 = 0;
-        if constexpr (K == 5) {
-            B0 = (acc[0] & 0x0f0f0f0fu) | ((acc[1] & 0x0f0f0f0fu) << 4);
-            B1 = (acc[2] & 0x0f0f0f0fu) | ((acc[3] & 0x0f0f0f0fu) << 4);
-            p4 = ((acc[0] >> 4) & 0xfu) | (acc[1] & 0xf0u) | (((acc[2] >> 4) & 0xfu) << 8) | ((acc[3] & 0xf0u) << 8);
-        } else {
-            B0 = acc[0];
-            B1 = acc[1];
-        }
-        // lane h holds bytes 2h, 2h+1 of every word; swap halves so it ends with words 2h, 2h+1
-        const uint32_t send = prmt(B0, B1, sel_send);
-        const uint32_t keep = prmt(B0, B1, sel_keep);
-        const uint32_t recv = __shfl_xor_sync(0xffffffffu, send, 1);
-        const uint32_t wa = prmt(keep, recv, sel_wa);
-        const uint32_t wb = prmt(keep, recv, sel_wb);
-        uint32_t w4 = 0;
-        if constexpr (K == 5) w4 = p4 | (__shfl_xor_sync(0xffffffffu, p4, 1) << 16);
-
-        if (active) {
-            const int64_t b = H >> 1;
-            uint32_t* out = packed + b * K;
-            if (K == 4 && packed_v2) {
-                asm volatile("st.global.v2.u32 [%0], {%1,%2};" :: "l"(out + 2 * h), "r"(wa), "r"(wb) : "memory");
-            } else {
-                if (2 * h < K) out[2 * h] = wa;
-                if (2 * h + 1 < K) out[2 * h + 1] = wb;
-                if constexpr (K == 5) { if (h == 0) out[4] = w4; }
-            }
-            if (h == 0) absmax[b] = amax;
-        }
-        cur = nxt;
+    }
+    // remaining half blocks (the ragged last block, or everything when the input is unaligned)
+    for (int64_t t = nh_full + (int64_t)blockIdx.x * kThreads + (tid & ~31); t < nh; t += stride) {
+        const Raw<DT> r = load_raw<DT, false>(A, n, t + lane, t + lane < nh);
+        quantize_half<K, DT>(r, t + lane, t + lane < nh, c, cb, absmax, packed);
     }
 }
 

@@ -9,10 +9,13 @@
 // values it multiplies, in the one kernel that reads the codes.
 //
 // B200 layout: a thread owns 16 consecutive outputs (8 code bytes, one 8-byte
-// load); outer blocks are >= 32 elements, so the 16 share one scale. A warp
-// covers 512 outputs with coalesced 8-byte loads and 16-byte stores. Both code
-// tables sit in shared memory; the 16-entry value table lives in 16 distinct
-// banks, so the per-element lookup never conflicts. Persistent grid-stride loop.
+// load; 32 per thread measured slower on B200 because of the lower residency);
+// outer blocks are >= 32 elements and aligned, so the 16 share one scale. A
+// warp covers 512 outputs with coalesced loads and 32-byte stores, and the
+// codes, General8 code and inner absmax of the next group are loaded before
+// the current group is decoded. Both code tables sit in shared
+// memory; the 16-entry value table lives in 16 distinct banks, so the
+// per-element lookup never conflicts. Persistent grid-stride loop.
 #include "common.cuh"
 #include "launch.h"
 
@@ -21,7 +24,12 @@ namespace bbc {
 namespace {
 
 constexpr int kThreads = 256;
-constexpr int kPerThread = 16;
+#ifndef BBC_NESTED_PER_THREAD
+#define BBC_NESTED_PER_THREAD 16
+#endif
+constexpr int kPerThread = BBC_NESTED_PER_THREAD;     // 16 or 32 outputs per thread
+static_assert(kPerThread == 16 || kPerThread == 32, "16 or 32 outputs per thread");
+constexpr int kCodeBytes = kPerThread / 2;
 
 // Byte offset (code * 4) of element 2i (high nibble of byte i) and 2i+1 (low nibble)
 // of the little-endian word W holding bytes 4k..4k+3.
@@ -31,6 +39,46 @@ template <int I>
 __device__ __forceinline__ uint32_t lo_off(uint32_t W) {
     if constexpr (I == 0) return (W << 2) & 0x3Cu;
     else return (W >> (8 * I - 2)) & 0x3Cu;
+}
+
+struct GroupIn {
+    uint4 c;          // code bytes (8 or 16) of the group
+    uint32_t q;       // General8 code of the outer block
+    float a2;         // inner absmax
+};
+
+template <bool VEC>
+__device__ __forceinline__ GroupIn load_group(const uint8_t* codes, const uint8_t* absmax_q,
+                                              const float* absmax2, int64_t n, int64_t u,
+                                              int log2_bs, bool active) {
+    GroupIn g;
+    g.c = make_uint4(0u, 0u, 0u, 0u);
+    g.q = 0u;
+    g.a2 = 0.0f;
+    if (!active) return g;
+    const int64_t m0 = u * kPerThread;
+    if (VEC && m0 + kPerThread <= n) {
+        if constexpr (kCodeBytes == 16) {
+            g.c = ldg_stream_v4(codes + u * 16);
+        } else {
+            const uint2 v = ldg_stream_v2(codes + u * 8);
+            g.c = make_uint4(v.x, v.y, 0u, 0u);
+        }
+    } else {
+        const int64_t nbytes = (n + 1) >> 1;
+        uint32_t wb[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
+        for (int i = 0; i < kCodeBytes; i++) {
+            const int64_t bi = u * kCodeBytes + i;
+            const uint32_t byte = bi < nbytes ? (uint32_t)codes[bi] : 0u;
+            wb[i >> 2] |= byte << (8 * (i & 3));
+        }
+        g.c = make_uint4(wb[0], wb[1], wb[2], wb[3]);
+    }
+    const int64_t b = m0 >> log2_bs;
+    g.q = __ldg(absmax_q + b);
+    g.a2 = __ldg(absmax2 + (b >> 8));
+    return g;
 }
 
 template <int DT, bool VEC>
@@ -46,57 +94,45 @@ nested_dequant_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restri
     __syncthreads();
     const char* c4b = reinterpret_cast<const char*>(c4);
 
-    const int64_t nbytes = (n + 1) >> 1;
     const int64_t nu = (n + kPerThread - 1) / kPerThread;
     const int64_t stride = (int64_t)gridDim.x * kThreads;
-    for (int64_t u = (int64_t)blockIdx.x * kThreads + threadIdx.x; u < nu; u += stride) {
+    int64_t u = (int64_t)blockIdx.x * kThreads + threadIdx.x;
+    GroupIn cur = load_group<VEC>(codes, absmax_q, absmax2, n, u, log2_bs, u < nu);
+    for (; u < nu; u += stride) {
+        const int64_t un = u + stride;
+        const GroupIn nxt = load_group<VEC>(codes, absmax_q, absmax2, n, un, log2_bs, un < nu);
+
+        // outer scale: General8 code times inner absmax, then plus offset, each rounded
+        const float s = __fadd_rn(__fmul_rn(c2[cur.q], cur.a2), offset);
+        const uint32_t W[4] = {cur.c.x, cur.c.y, cur.c.z, cur.c.w};
         const int64_t m0 = u * kPerThread;
-        const bool full = m0 + kPerThread <= n;
-        uint32_t w0, w1;
-        if (VEC && full) {
-            const uint2 v = ldg_stream_v2(codes + u * 8);
-            w0 = v.x;
-            w1 = v.y;
-        } else {
-            uint32_t wb[2] = {0u, 0u};
 #pragma unroll
-            for (int i = 0; i < 8; i++) {
-                const int64_t bi = u * 8 + i;
-                const uint32_t byte = bi < nbytes ? (uint32_t)codes[bi] : 0u;
-                wb[i >> 2] |= byte << (8 * (i & 3));
-            }
-            w0 = wb[0];
-            w1 = wb[1];
-        }
-
-        const int64_t b = m0 >> log2_bs;
-        const float s = __fadd_rn(__fmul_rn(c2[__ldg(absmax_q + b)], __ldg(absmax2 + (b >> 8))), offset);
-
-        float y[16];
-#define BBC_ND_BYTE(I, W, BASE)                                                           \
-        y[BASE + 2 * (I)] = __fmul_rn(*reinterpret_cast<const float*>(c4b + hi_off<I>(W)), s); \
-        y[BASE + 2 * (I) + 1] = __fmul_rn(*reinterpret_cast<const float*>(c4b + lo_off<I>(W)), s);
-        BBC_ND_BYTE(0, w0, 0) BBC_ND_BYTE(1, w0, 0) BBC_ND_BYTE(2, w0, 0) BBC_ND_BYTE(3, w0, 0)
-        BBC_ND_BYTE(0, w1, 8) BBC_ND_BYTE(1, w1, 8) BBC_ND_BYTE(2, w1, 8) BBC_ND_BYTE(3, w1, 8)
+        for (int half = 0; half < kPerThread / 16; half++) {
+            float y[16];
+#pragma unroll
+            for (int k = 0; k < 2; k++) {
+                const uint32_t w = W[2 * half + k];
+#define BBC_ND_BYTE(I)                                                                       \
+                y[8 * k + 2 * (I)] = __fmul_rn(*reinterpret_cast<const float*>(c4b + hi_off<I>(w)), s); \
+                y[8 * k + 2 * (I) + 1] = __fmul_rn(*reinterpret_cast<const float*>(c4b + lo_off<I>(w)), s);
+                BBC_ND_BYTE(0) BBC_ND_BYTE(1) BBC_ND_BYTE(2) BBC_ND_BYTE(3)
 #undef BBC_ND_BYTE
-
-        if (VEC && full) {
-            uint32_t wv[16];
-            pack8<DT>(y, wv);
-            pack8<DT>(y + 8, wv + (DT == F32 ? 8 : 4));
-            char* dst = reinterpret_cast<char*>(out) + m0 * dtype_size(DT);
-            if constexpr (DT == F32) {
-#pragma unroll
-                for (int i = 0; i < 4; i++) stg_v4(dst + 16 * i, wv[4 * i], wv[4 * i + 1], wv[4 * i + 2], wv[4 * i + 3]);
-            } else {
-                stg_v4(dst, wv[0], wv[1], wv[2], wv[3]);
-                stg_v4(dst + 16, wv[4], wv[5], wv[6], wv[7]);
             }
-        } else {
+            const int64_t mh = m0 + 16 * half;
+            if (VEC && m0 + kPerThread <= n) {
+                uint32_t wv[16];
+                pack8<DT>(y, wv);
+                pack8<DT>(y + 8, wv + (DT == F32 ? 8 : 4));
+                char* dst = reinterpret_cast<char*>(out) + mh * dtype_size(DT);
+                stg_v8(dst, wv);
+                if constexpr (DT == F32) stg_v8(dst + 32, wv + 8);
+            } else {
 #pragma unroll
-            for (int e = 0; e < kPerThread; e++)
-                if (m0 + e < n) store_from_f32<DT>(out, m0 + e, y[e]);
+                for (int e = 0; e < 16; e++)
+                    if (mh + e < n) store_from_f32<DT>(out, mh + e, y[e]);
+            }
         }
+        cur = nxt;
     }
 }
 
