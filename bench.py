@@ -227,6 +227,7 @@ def run_bbc(args):
 
     import blockwise_bit_codebook_b200 as bbc
     from blockwise_bit_codebook_b200 import synthetic
+    from blockwise_bit_codebook_b200.dist import max_over_ranks
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -294,12 +295,13 @@ def run_bbc(args):
     if dist:
         dist.barrier()
     total_ms = t_start.elapsed_time(t_end)
-    per_op_ms = [statistics.mean(evs[s][i][0].elapsed_time(evs[s][i][1]) for s in range(args.steps))
-                 for i in range(len(ops))]
-    if dist:
-        t = torch.tensor([total_ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t.item())
+    samples = [[evs[s][i][0].elapsed_time(evs[s][i][1]) for s in range(args.steps)] for i in range(len(ops))]
+    per_op_ms = [statistics.mean(v) for v in samples]
+
+    def pct(v, q):
+        v = sorted(v)
+        return v[min(len(v) - 1, int(q * (len(v) - 1) + 0.5))]
+    total_ms = max_over_ranks(total_ms, device=dev)      # identity at N = 1
     if sampler:
         time.sleep(0.25)
         sampler.stop()
@@ -310,10 +312,11 @@ def run_bbc(args):
     value = world * bytes_step / (ms_per_step * 1e-3) / 1e9
     peak, peak_kind = load_peaks()
     per_kernel = {}
-    for (name, kind, K), ms in zip(ops, per_op_ms):
+    for (name, kind, K), ms, smp in zip(ops, per_op_ms, samples):
         b = op_bytes(kind, n, K)
         gbs = b / (ms * 1e-3) / 1e9
-        per_kernel[name] = {"ms": round(ms, 5), "GB/s": round(gbs, 1),
+        per_kernel[name] = {"ms": round(ms, 5), "ms_p10_p50_p90": [round(pct(smp, q), 5) for q in (0.1, 0.5, 0.9)],
+                            "GB/s": round(gbs, 1),
                             "Gelem/s": round(n / (ms * 1e-3) / 1e9, 2),
                             "frac_of_measured_hbm": round(gbs / peak, 4),
                             "frac_of_8TBs_nominal": round(gbs / 8000.0, 4),
@@ -376,11 +379,7 @@ def run_bbc(args):
             e2e_step()
         e1.record(stream)
         torch.cuda.synchronize()
-        e_ms = e0.elapsed_time(e1) / args.e2e_steps
-        if dist:
-            t = torch.tensor([e_ms], device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e_ms = float(t.item())
+        e_ms = max_over_ranks(e0.elapsed_time(e1) / args.e2e_steps, device=dev)
         result["e2e"] = {"value": round(world * bytes_step / (e_ms * 1e-3) / 1e9, 2), "unit": "GB/s",
                          "ms_per_step": round(e_ms, 3), "h2d_bytes_per_step": h2d,
                          "d2h_bytes_per_step": d2h, "steps": args.e2e_steps,

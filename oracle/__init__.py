@@ -169,35 +169,3 @@ def nested_dequantize(codes, absmax_q, code2, absmax2, offset: float, code4,
                                      _DT[dtype], _p(out))
     assert rc == 0
     return out
-
-
-def kbit_quantize_threads(A, dtype: str, K: int, codebook, threads: int):
-    """The same quantize, run over contiguous block ranges on `threads` host threads.
-
-    ctypes releases the GIL during the C call, so Python threads run the C loop in
-    parallel; each range is a whole number of 32-element blocks, so the result is
-    identical to the single-threaded call.
-    """
-    import threading
-
-    A = _c(A, np.float32 if dtype == "f32" else np.uint16).reshape(-1)
-    cb = _c(codebook, np.float32)
-    n = A.size
-    nb = num_blocks(n)
-    absmax = np.empty(nb, np.float32)
-    packed = np.empty(nb * K, np.uint32)
-    per = (nb + threads - 1) // threads
-    jobs = []
-    for t in range(threads):
-        b0, b1 = t * per, min(nb, (t + 1) * per)
-        if b0 >= b1:
-            break
-        e0, e1 = b0 * KBIT_BLOCKSIZE, min(n, b1 * KBIT_BLOCKSIZE)
-        sub = A[e0:e1]
-        jobs.append(threading.Thread(target=lambda s=sub, b0=b0, b1=b1: lib().orc_kbit_quantize(
-            _p(s), _DT[dtype], s.size, K, _p(cb), _p(absmax[b0:b1]), _p(packed[b0 * K:b1 * K]), None)))
-    for j in jobs:
-        j.start()
-    for j in jobs:
-        j.join()
-    return packed, absmax
