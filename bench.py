@@ -51,6 +51,8 @@ def parse_args():
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--nested-matrix", action="store_true",
+                    help="fused vs three-launch nested dequant on the pull request's 24-cell matrix")
     ap.add_argument("--cpu-seconds", type=float, default=15.0,
                     help="target CPU time of the oracle baseline sample")
     return ap.parse_args()
@@ -397,6 +399,90 @@ def run_bbc(args):
         print(json.dumps(result), flush=True)
 
 
+# ----------------------------------------------------------------------------- nested matrix
+
+def run_nested_matrix(args):
+    """Fused nested dequant vs the unfused three-launch chain on the pull request's matrix.
+
+    Shapes 4096x4096, 11008x4096, 4096x11008, 8192x8192; NF4 and FP4; fp16/bf16/fp32 outputs;
+    outer blocksize 64. Method as the pull request describes it: CUDA events, 20 alternating
+    warm-ups, 7 interleaved rounds of size-scaled repetitions (up to 100), medians; outputs are
+    checked bit-equal. Inputs are not flushed from L2 between repetitions (as there).
+    """
+    import math
+
+    import numpy as np
+    import torch
+
+    import blockwise_bit_codebook_b200 as bbc
+    from blockwise_bit_codebook_b200 import synthetic
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    bbc.load_library()
+    shapes = [(4096, 4096), (11008, 4096), (4096, 11008), (8192, 8192)]
+    tabs = {"nf4": bbc.bbc_nf_codebook(4), "fp4": synthetic.fp4_table()}
+    code2 = torch.from_numpy(synthetic.general8_table()).to(dev)
+    bs = 64
+    ratios = {}
+    for (r, c) in shapes:
+        n = r * c
+        codes, q, a2, off = synthetic.nested_state(n, bs, seed=3, device=dev)
+        ws = torch.empty((n + bs - 1) // bs, dtype=torch.float32, device=dev)
+        for fmt in ("nf4", "fp4"):
+            code4 = torch.from_numpy(tabs[fmt]).to(dev)
+            for dt in (torch.float16, torch.bfloat16, torch.float32):
+                out_f = torch.empty(n, dtype=dt, device=dev)
+                out_c = torch.empty(n, dtype=dt, device=dev)
+                fused = lambda: bbc.dequantize_4bit_nested(codes, q, code2, a2, float(off), code4, n, bs, dt,  # noqa: E731
+                                                           out=out_f)
+                chain = lambda: bbc.dequantize_4bit_nested_chain(codes, q, code2, a2, float(off), code4, n,  # noqa: E731
+                                                                 bs, dt, out=out_c, scale_workspace=ws)
+                for i in range(20):
+                    (fused if i % 2 == 0 else chain)()
+                torch.cuda.synchronize()
+                nbytes = op_bytes("nested", n, out_size=out_f.element_size())
+                reps = max(10, min(100, int(4e9 / nbytes)))
+                samples = {"fused": [], "chain": []}
+                for rnd in range(7):
+                    order = [("fused", fused), ("chain", chain)]
+                    if rnd % 2:
+                        order.reverse()
+                    for name, fn in order:
+                        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                        e0.record()
+                        for _ in range(reps):
+                            fn()
+                        e1.record()
+                        torch.cuda.synchronize()
+                        samples[name].append(e0.elapsed_time(e1) / reps * 1e3)
+                equal = bool(torch.equal(out_f.view(torch.int16 if dt != torch.float32 else torch.int32),
+                                         out_c.view(torch.int16 if dt != torch.float32 else torch.int32)))
+                med = {k: statistics.median(v) for k, v in samples.items()}
+                ratio = med["chain"] / med["fused"]
+                ratios.setdefault(f"{r}x{c}", []).append(ratio)
+                print(json.dumps({"cell": f"{r}x{c}", "format": fmt, "dtype": str(dt).split(".")[-1],
+                                  "blocksize": bs, "fused_us_median": round(med["fused"], 2),
+                                  "chain_us_median": round(med["chain"], 2),
+                                  "fused_us_p10_p90": [round(pct_of(samples["fused"], 0.1), 2),
+                                                       round(pct_of(samples["fused"], 0.9), 2)],
+                                  "chain_us_p10_p90": [round(pct_of(samples["chain"], 0.1), 2),
+                                                       round(pct_of(samples["chain"], 0.9), 2)],
+                                  "fused_GBs": round(nbytes / med["fused"] / 1e3, 1),
+                                  "chain_over_fused": round(ratio, 4), "bit_equal": equal}), flush=True)
+    geo = lambda v: math.exp(sum(math.log(x) for x in v) / len(v))  # noqa: E731
+    allr = [x for v in ratios.values() for x in v]
+    print(json.dumps({"summary": "chain/fused geomean per shape (outer blocksize 64)",
+                      "per_shape": {k: round(geo(v), 4) for k, v in ratios.items()},
+                      "all_cells": round(geo(allr), 4), "min": round(min(allr), 4),
+                      "max": round(max(allr), 4), "cells": len(allr)}), flush=True)
+
+
+def pct_of(v, q):
+    v = sorted(v)
+    return v[min(len(v) - 1, int(q * (len(v) - 1) + 0.5))]
+
+
 # ----------------------------------------------------------------------------- reference arm
 
 def run_reference(args):
@@ -442,4 +528,9 @@ def run_reference(args):
 
 if __name__ == "__main__":
     a = parse_args()
-    run_reference(a) if a.impl == "reference" else run_bbc(a)
+    if a.nested_matrix:
+        run_nested_matrix(a)
+    elif a.impl == "reference":
+        run_reference(a)
+    else:
+        run_bbc(a)

@@ -9,6 +9,8 @@ library's CUDA kernels. torch is used for device memory and streams only.
     kbit_dequantize(packed, absmax, codebook, K, n, dtype) -> out
     dequantize_4bit_nested(codes, absmax_q, code2, absmax2, offset, code4,
                            n, blocksize, dtype)         -> out
+    dequantize_4bit(codes, absmax, code4, n, blocksize, dtype)  -> out
+    dequantize_4bit_nested_chain(...)   the unfused three-launch form (same result)
     bbc_nf_codebook(K)                                  -> np.float32[2^K] (host)
 
 There is no CPU fallback: if libbbc.so is missing or a call fails, an
@@ -21,7 +23,9 @@ from ._native import (  # noqa: F401
     BBCError,
     bbc_last_error,
     bbc_nf_codebook,
+    dequantize_4bit,
     dequantize_4bit_nested,
+    dequantize_4bit_nested_chain,
     kbit_dequantize,
     kbit_quantize,
     library_path,

@@ -38,6 +38,10 @@ def load_library():
     L.kbit_dequantize.restype = I
     L.dequantize_4bit_nested.argtypes = [P, P, P, P, ct.c_float, P, I64, I, I, I, P, P]
     L.dequantize_4bit_nested.restype = I
+    L.dequantize_4bit.argtypes = [P, P, P, I64, I, I, P, P]
+    L.dequantize_4bit.restype = I
+    L.dequantize_4bit_nested_chain.argtypes = [P, P, P, P, ct.c_float, P, I64, I, I, I, P, P, P]
+    L.dequantize_4bit_nested_chain.restype = I
     L.bbc_nf_codebook.argtypes = [I, P]
     L.bbc_nf_codebook.restype = I
     L.bbc_last_error.argtypes = []
@@ -123,6 +127,38 @@ def dequantize_4bit_nested(codes, absmax_q, code2, absmax2, offset: float, code4
                                   ct.c_float(offset), _ptr(code4), n, blocksize, blocksize2, dt,
                                   _ptr(out), _stream(stream, codes.device))
     _check("dequantize_4bit_nested", st)
+    return out
+
+
+def dequantize_4bit(codes, absmax, code4, n: int, blocksize: int, dtype, out=None, stream=None):
+    """Plain NF4/FP4 decode with an fp32 absmax per block; returns n elements of `dtype`."""
+    import torch
+    L = load_library()
+    dt = _dt(dtype)
+    if out is None:
+        out = torch.empty(max(n, 1), dtype=_torch_dtype(dt), device=codes.device)
+    st = L.dequantize_4bit(_ptr(codes), _ptr(absmax), _ptr(code4), n, blocksize, dt, _ptr(out),
+                           _stream(stream, codes.device))
+    _check("dequantize_4bit", st)
+    return out
+
+
+def dequantize_4bit_nested_chain(codes, absmax_q, code2, absmax2, offset: float, code4, n: int,
+                                 blocksize: int, dtype, out=None, scale_workspace=None,
+                                 blocksize2: int = 256, stream=None):
+    """The unfused three-launch form of dequantize_4bit_nested (same result)."""
+    import torch
+    L = load_library()
+    dt = _dt(dtype)
+    if out is None:
+        out = torch.empty(max(n, 1), dtype=_torch_dtype(dt), device=codes.device)
+    if scale_workspace is None:
+        scale_workspace = torch.empty(max((n + blocksize - 1) // blocksize, 1), dtype=torch.float32,
+                                      device=codes.device)
+    st = L.dequantize_4bit_nested_chain(_ptr(codes), _ptr(absmax_q), _ptr(code2), _ptr(absmax2),
+                                        ct.c_float(offset), _ptr(code4), n, blocksize, blocksize2, dt,
+                                        _ptr(out), _ptr(scale_workspace), _stream(stream, codes.device))
+    _check("dequantize_4bit_nested_chain", st)
     return out
 
 

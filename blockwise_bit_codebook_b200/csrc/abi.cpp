@@ -39,6 +39,13 @@ bool valid_dtype(int dt) { return dt == BBC_F16 || dt == BBC_BF16 || dt == BBC_F
 
 int elem_size(int dt) { return dt == BBC_F32 ? 4 : 2; }
 
+// log2 of a 4-bit outer blocksize (a power of two in [32, 4096]), or -1.
+int log2_blocksize(int blocksize) {
+    for (int l = 5; l <= 12; l++)
+        if (blocksize == (1 << l)) return l;
+    return -1;
+}
+
 }  // namespace
 
 extern "C" {
@@ -87,9 +94,7 @@ int dequantize_4bit_nested(const uint8_t* codes, const uint8_t* absmax_q, const 
         return fail(BBC_ERR_INVALID, "dequantize_4bit_nested: n must be >= 1 (got %lld)", (long long)n);
     if (!valid_dtype(out_dtype))
         return fail(BBC_ERR_INVALID, "dequantize_4bit_nested: bad dtype %d", out_dtype);
-    int log2_bs = -1;
-    for (int l = 5; l <= 12; l++)
-        if (blocksize == (1 << l)) log2_bs = l;
+    const int log2_bs = log2_blocksize(blocksize);
     if (log2_bs < 0)
         return fail(BBC_ERR_INVALID,
                     "dequantize_4bit_nested: blocksize must be a power of two in [32, 4096] (got %d)",
@@ -104,6 +109,52 @@ int dequantize_4bit_nested(const uint8_t* codes, const uint8_t* absmax_q, const 
                                                      log2_bs, out_dtype, out, vec,
                                                      static_cast<cudaStream_t>(stream)),
                        "dequantize_4bit_nested launch");
+}
+
+int dequantize_4bit(const uint8_t* codes, const float* absmax, const float* code4, int64_t n,
+                    int blocksize, int out_dtype, void* out, void* stream) {
+    if (!codes || !absmax || !code4 || !out)
+        return fail(BBC_ERR_INVALID, "dequantize_4bit: null pointer argument");
+    if (n <= 0) return fail(BBC_ERR_INVALID, "dequantize_4bit: n must be >= 1 (got %lld)", (long long)n);
+    if (!valid_dtype(out_dtype)) return fail(BBC_ERR_INVALID, "dequantize_4bit: bad dtype %d", out_dtype);
+    const int log2_bs = log2_blocksize(blocksize);
+    if (log2_bs < 0)
+        return fail(BBC_ERR_INVALID, "dequantize_4bit: blocksize must be a power of two in [32, 4096] (got %d)",
+                    blocksize);
+    if (!aligned(out, elem_size(out_dtype)) || !aligned(absmax, 4) || !aligned(code4, 4))
+        return fail(BBC_ERR_INVALID, "dequantize_4bit: pointer not aligned to its element size");
+    const bool vec = aligned(out, 32) && aligned(codes, 16);
+    return cuda_status(bbc::launch_dequantize_4bit(codes, absmax, code4, n, log2_bs, out_dtype, out, vec,
+                                                   static_cast<cudaStream_t>(stream)),
+                       "dequantize_4bit launch");
+}
+
+int dequantize_4bit_nested_chain(const uint8_t* codes, const uint8_t* absmax_q, const float* code2,
+                                 const float* absmax2, float offset, const float* code4,
+                                 int64_t n, int blocksize, int blocksize2, int out_dtype, void* out,
+                                 float* scale_workspace, void* stream) {
+    if (!codes || !absmax_q || !code2 || !absmax2 || !code4 || !out || !scale_workspace)
+        return fail(BBC_ERR_INVALID, "dequantize_4bit_nested_chain: null pointer argument");
+    if (n <= 0)
+        return fail(BBC_ERR_INVALID, "dequantize_4bit_nested_chain: n must be >= 1 (got %lld)", (long long)n);
+    if (!valid_dtype(out_dtype))
+        return fail(BBC_ERR_INVALID, "dequantize_4bit_nested_chain: bad dtype %d", out_dtype);
+    const int log2_bs = log2_blocksize(blocksize);
+    if (log2_bs < 0)
+        return fail(BBC_ERR_INVALID,
+                    "dequantize_4bit_nested_chain: blocksize must be a power of two in [32, 4096] (got %d)",
+                    blocksize);
+    if (blocksize2 != 256)
+        return fail(BBC_ERR_UNSUPPORTED, "dequantize_4bit_nested_chain: blocksize2 must be 256 (got %d)",
+                    blocksize2);
+    if (!aligned(out, elem_size(out_dtype)) || !aligned(code2, 4) || !aligned(absmax2, 4) ||
+        !aligned(code4, 4) || !aligned(scale_workspace, 4))
+        return fail(BBC_ERR_INVALID, "dequantize_4bit_nested_chain: pointer not aligned to its element size");
+    const bool vec = aligned(out, 32) && aligned(codes, 16);
+    return cuda_status(bbc::launch_nested_dequantize_chain(codes, absmax_q, code2, absmax2, offset, code4, n,
+                                                           log2_bs, out_dtype, out, scale_workspace, vec,
+                                                           static_cast<cudaStream_t>(stream)),
+                       "dequantize_4bit_nested_chain launch");
 }
 
 const char* bbc_last_error(void) { return g_last_error.c_str(); }

@@ -31,4 +31,13 @@ cudaError_t launch_nested_dequantize(const uint8_t* codes, const uint8_t* absmax
                                      const float* code4, int64_t n, int log2_bs, int out_dtype,
                                      void* out, bool vec, cudaStream_t s);
 
+cudaError_t launch_dequantize_4bit(const uint8_t* codes, const float* absmax, const float* code4,
+                                   int64_t n, int log2_bs, int out_dtype, void* out, bool vec,
+                                   cudaStream_t s);
+
+cudaError_t launch_nested_dequantize_chain(const uint8_t* codes, const uint8_t* absmax_q,
+                                           const float* code2, const float* absmax2, float offset,
+                                           const float* code4, int64_t n, int log2_bs, int out_dtype,
+                                           void* out, float* scale, bool vec, cudaStream_t s);
+
 }  // namespace bbc

@@ -47,7 +47,10 @@ struct GroupIn {
     float a2;         // inner absmax
 };
 
-template <bool VEC>
+// NESTED: the group's scale inputs are a General8 code (absmax_q) and an inner absmax
+// (absmax2, one per 256 outer blocks). Otherwise `absmax2` is a plain fp32 absmax per outer
+// block (the last launch of the three-launch chain, or a non-nested 4-bit state).
+template <bool VEC, bool NESTED>
 __device__ __forceinline__ GroupIn load_group(const uint8_t* codes, const uint8_t* absmax_q,
                                               const float* absmax2, int64_t n, int64_t u,
                                               int log2_bs, bool active) {
@@ -76,12 +79,16 @@ __device__ __forceinline__ GroupIn load_group(const uint8_t* codes, const uint8_
         g.c = make_uint4(wb[0], wb[1], wb[2], wb[3]);
     }
     const int64_t b = m0 >> log2_bs;
-    g.q = __ldg(absmax_q + b);
-    g.a2 = __ldg(absmax2 + (b >> 8));
+    if constexpr (NESTED) {
+        g.q = __ldg(absmax_q + b);
+        g.a2 = __ldg(absmax2 + (b >> 8));
+    } else {
+        g.a2 = __ldg(absmax2 + b);
+    }
     return g;
 }
 
-template <int DT, bool VEC>
+template <int DT, bool VEC, bool NESTED>
 __global__ void __launch_bounds__(kThreads)
 nested_dequant_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restrict__ absmax_q,
                       const float* __restrict__ code2, const float* __restrict__ absmax2,
@@ -89,7 +96,7 @@ nested_dequant_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restri
                       void* __restrict__ out) {
     __shared__ float c2[256];
     __shared__ float c4[16];
-    c2[threadIdx.x] = code2[threadIdx.x];
+    if (NESTED) c2[threadIdx.x] = code2[threadIdx.x];
     if (threadIdx.x < 16) c4[threadIdx.x] = code4[threadIdx.x];
     __syncthreads();
     const char* c4b = reinterpret_cast<const char*>(c4);
@@ -97,13 +104,13 @@ nested_dequant_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restri
     const int64_t nu = (n + kPerThread - 1) / kPerThread;
     const int64_t stride = (int64_t)gridDim.x * kThreads;
     int64_t u = (int64_t)blockIdx.x * kThreads + threadIdx.x;
-    GroupIn cur = load_group<VEC>(codes, absmax_q, absmax2, n, u, log2_bs, u < nu);
+    GroupIn cur = load_group<VEC, NESTED>(codes, absmax_q, absmax2, n, u, log2_bs, u < nu);
     for (; u < nu; u += stride) {
         const int64_t un = u + stride;
-        const GroupIn nxt = load_group<VEC>(codes, absmax_q, absmax2, n, un, log2_bs, un < nu);
+        const GroupIn nxt = load_group<VEC, NESTED>(codes, absmax_q, absmax2, n, un, log2_bs, un < nu);
 
         // outer scale: General8 code times inner absmax, then plus offset, each rounded
-        const float s = __fadd_rn(__fmul_rn(c2[cur.q], cur.a2), offset);
+        const float s = NESTED ? __fadd_rn(__fmul_rn(c2[cur.q], cur.a2), offset) : cur.a2;
         const uint32_t W[4] = {cur.c.x, cur.c.y, cur.c.z, cur.c.w};
         const int64_t m0 = u * kPerThread;
 #pragma unroll
@@ -136,21 +143,46 @@ nested_dequant_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restri
     }
 }
 
-template <int DT>
+template <int DT, bool NESTED>
 cudaError_t launch_t(const uint8_t* codes, const uint8_t* absmax_q, const float* code2,
                      const float* absmax2, float offset, const float* code4, int64_t n,
                      int log2_bs, void* out, bool vec, cudaStream_t s) {
     const int64_t nu = (n + kPerThread - 1) / kPerThread;
-    if (vec) {
-        auto k = nested_dequant_kernel<DT, true>;
-        int grid = persistent_grid(k, kThreads, 0, nu, kThreads);
-        k<<<grid, kThreads, 0, s>>>(codes, absmax_q, code2, absmax2, offset, code4, n, log2_bs, out);
-    } else {
-        auto k = nested_dequant_kernel<DT, false>;
-        int grid = persistent_grid(k, kThreads, 0, nu, kThreads);
-        k<<<grid, kThreads, 0, s>>>(codes, absmax_q, code2, absmax2, offset, code4, n, log2_bs, out);
-    }
+    auto k = vec ? nested_dequant_kernel<DT, true, NESTED> : nested_dequant_kernel<DT, false, NESTED>;
+    const int grid = persistent_grid(k, kThreads, 0, nu, kThreads);
+    k<<<grid, kThreads, 0, s>>>(codes, absmax_q, code2, absmax2, offset, code4, n, log2_bs, out);
     return cudaGetLastError();
+}
+
+template <bool NESTED>
+cudaError_t launch_dt(const uint8_t* codes, const uint8_t* absmax_q, const float* code2,
+                      const float* absmax2, float offset, const float* code4, int64_t n, int log2_bs,
+                      int out_dtype, void* out, bool vec, cudaStream_t s) {
+    switch (out_dtype) {
+        case F16: return launch_t<F16, NESTED>(codes, absmax_q, code2, absmax2, offset, code4, n, log2_bs, out, vec, s);
+        case BF16: return launch_t<BF16, NESTED>(codes, absmax_q, code2, absmax2, offset, code4, n, log2_bs, out, vec, s);
+        default: return launch_t<F32, NESTED>(codes, absmax_q, code2, absmax2, offset, code4, n, log2_bs, out, vec, s);
+    }
+}
+
+// ---- the legacy three-launch chain: General8 scale, offset add, then plain 4-bit decode ----
+
+// scale[b] = fl(code2[absmax_q[b]] * absmax2[b / 256])
+__global__ void __launch_bounds__(kThreads)
+general8_scale_kernel(const uint8_t* __restrict__ absmax_q, const float* __restrict__ code2,
+                      const float* __restrict__ absmax2, int64_t nbo, float* __restrict__ scale) {
+    __shared__ float c2[256];
+    c2[threadIdx.x] = code2[threadIdx.x];
+    __syncthreads();
+    for (int64_t b = (int64_t)blockIdx.x * kThreads + threadIdx.x; b < nbo; b += (int64_t)gridDim.x * kThreads)
+        scale[b] = __fmul_rn(c2[__ldg(absmax_q + b)], __ldg(absmax2 + (b >> 8)));
+}
+
+// scale[b] = fl(scale[b] + offset)
+__global__ void __launch_bounds__(kThreads)
+add_offset_kernel(float* __restrict__ scale, int64_t nbo, float offset) {
+    for (int64_t b = (int64_t)blockIdx.x * kThreads + threadIdx.x; b < nbo; b += (int64_t)gridDim.x * kThreads)
+        scale[b] = __fadd_rn(scale[b], offset);
 }
 
 }  // namespace
@@ -159,11 +191,29 @@ cudaError_t launch_nested_dequantize(const uint8_t* codes, const uint8_t* absmax
                                      const float* code2, const float* absmax2, float offset,
                                      const float* code4, int64_t n, int log2_bs, int out_dtype,
                                      void* out, bool vec, cudaStream_t s) {
-    switch (out_dtype) {
-        case F16: return launch_t<F16>(codes, absmax_q, code2, absmax2, offset, code4, n, log2_bs, out, vec, s);
-        case BF16: return launch_t<BF16>(codes, absmax_q, code2, absmax2, offset, code4, n, log2_bs, out, vec, s);
-        default: return launch_t<F32>(codes, absmax_q, code2, absmax2, offset, code4, n, log2_bs, out, vec, s);
-    }
+    return launch_dt<true>(codes, absmax_q, code2, absmax2, offset, code4, n, log2_bs, out_dtype, out, vec, s);
+}
+
+cudaError_t launch_dequantize_4bit(const uint8_t* codes, const float* absmax, const float* code4,
+                                   int64_t n, int log2_bs, int out_dtype, void* out, bool vec,
+                                   cudaStream_t s) {
+    return launch_dt<false>(codes, nullptr, nullptr, absmax, 0.0f, code4, n, log2_bs, out_dtype, out, vec, s);
+}
+
+cudaError_t launch_nested_dequantize_chain(const uint8_t* codes, const uint8_t* absmax_q,
+                                           const float* code2, const float* absmax2, float offset,
+                                           const float* code4, int64_t n, int log2_bs, int out_dtype,
+                                           void* out, float* scale, bool vec, cudaStream_t s) {
+    const int64_t nbo = ((n - 1) >> log2_bs) + 1;
+    const int grid_s = persistent_grid(general8_scale_kernel, kThreads, 0, nbo, kThreads);
+    general8_scale_kernel<<<grid_s, kThreads, 0, s>>>(absmax_q, code2, absmax2, nbo, scale);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    const int grid_o = persistent_grid(add_offset_kernel, kThreads, 0, nbo, kThreads);
+    add_offset_kernel<<<grid_o, kThreads, 0, s>>>(scale, nbo, offset);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    return launch_dequantize_4bit(codes, scale, code4, n, log2_bs, out_dtype, out, vec, s);
 }
 
 }  // namespace bbc

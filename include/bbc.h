@@ -128,6 +128,41 @@ int dequantize_4bit_nested(const uint8_t* codes, const uint8_t* absmax_q, const 
                            void* stream);
 
 /*
+ * dequantize_4bit - plain NF4/FP4 dequantization with an fp32 absmax per block.
+ *
+ * Defined by: pull request "Fuse nested 4-bit scale reconstruction on SM103",
+ * Summary: the NF4/FP4 value dequantization that is the last of the three
+ * launches of the unfused path, out[m] = T(fl(code4[nibble_m] * absmax[m / blocksize])).
+ * Nibble order as in dequantize_4bit_nested.
+ *
+ *   codes      [ceil(n/2)] uint8.   absmax [ceil(n/blocksize)] fp32.
+ *   code4      [16] fp32.           n >= 1.   blocksize: power of two in [32, 4096].
+ *   out_dtype  BBC_F16, BBC_BF16 or BBC_F32;   out [n] elements.
+ */
+int dequantize_4bit(const uint8_t* codes, const float* absmax, const float* code4, int64_t n,
+                    int blocksize, int out_dtype, void* out, void* stream);
+
+/*
+ * dequantize_4bit_nested_chain - the unfused three-launch form of
+ * dequantize_4bit_nested, kept as an in-library comparator.
+ *
+ * Defined by: the same pull request, Summary: General8 scale dequantization
+ * (scale_b = fl(code2[absmax_q[b]] * absmax2[b / blocksize2]) into an fp32
+ * tensor), an offset add (scale_b = fl(scale_b + offset)), then NF4/FP4 value
+ * dequantization reading that tensor. Results are identical to
+ * dequantize_4bit_nested; the cost is the extra launches and the round trip
+ * of the scale tensor through memory.
+ *
+ * Arguments as dequantize_4bit_nested, plus:
+ *   scale_workspace  DEVICE buffer of ceil(n/blocksize) floats, caller-owned; it
+ *                    receives the scales and must not overlap any other argument.
+ */
+int dequantize_4bit_nested_chain(const uint8_t* codes, const uint8_t* absmax_q, const float* code2,
+                                 const float* absmax2, float offset, const float* code4,
+                                 int64_t n, int blocksize, int blocksize2, int out_dtype, void* out,
+                                 float* scale_workspace, void* stream);
+
+/*
  * bbc_nf_codebook - the 2^K-entry normal-float codebook, on the HOST.
  *
  * Defined by: the k-bit patch series, create_normal_float_codebook: standard

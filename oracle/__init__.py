@@ -8,8 +8,8 @@ it never imports the library. Each function cites the passage it follows:
 * k-bit codec: bitsandbytes k-bit patch series, tests/test_kbit_quantization.py
   (quantize_kbit_ref, dequantize_kbit_ref, pack_kbit_ref, unpack_kbit_ref) and
   csrc/ops.cu (kQuantizeBlockwise_kbit, kDequantizeBlockwise_kbit).
-* nested 4-bit dequant: "Fuse nested 4-bit scale reconstruction on SM103",
-  Summary and Implementation.
+* nested 4-bit dequant and the plain 4-bit decode of its unfused form: "Fuse
+  nested 4-bit scale reconstruction on SM103", Summary and Implementation.
 
 Arrays: fp32 as ``np.float32``; fp16 and bfloat16 as their raw 16-bit patterns
 in ``np.uint16`` (numpy has no bfloat16). dtype names are "f16", "bf16", "f32".
@@ -44,6 +44,8 @@ def lib():
         L.orc_kbit_dequantize.restype = ct.c_int
         L.orc_nested_dequantize.argtypes = [P, P, P, P, ct.c_float, P, I64, I64, I64, ct.c_int, P]
         L.orc_nested_dequantize.restype = ct.c_int
+        L.orc_dequantize_4bit.argtypes = [P, P, P, I64, I64, ct.c_int, P]
+        L.orc_dequantize_4bit.restype = ct.c_int
         L.orc_kbit_pack.argtypes = [P, I64, ct.c_int, P]
         L.orc_kbit_unpack.argtypes = [P, I64, ct.c_int, P]
         L.orc_nearest_entry.argtypes = [ct.c_float, P, ct.c_int]
@@ -167,5 +169,17 @@ def nested_dequantize(codes, absmax_q, code2, absmax2, offset: float, code4,
     rc = lib().orc_nested_dequantize(_p(codes), _p(absmax_q), _p(code2), _p(absmax2),
                                      ct.c_float(offset), _p(code4), n, blocksize, blocksize2,
                                      _DT[dtype], _p(out))
+    assert rc == 0
+    return out
+
+
+def dequantize_4bit(codes, absmax, code4, n: int, blocksize: int, dtype: str) -> np.ndarray:
+    """Plain 4-bit decode with an fp32 absmax per block (the last launch of the unfused chain)."""
+    codes = _c(codes, np.uint8).reshape(-1)
+    absmax = _c(absmax, np.float32).reshape(-1)
+    code4 = _c(code4, np.float32)
+    assert codes.size >= (n + 1) // 2 and absmax.size >= num_blocks(n, blocksize) and code4.size == 16
+    out = np.empty(n, np.float32 if dtype == "f32" else np.uint16)
+    rc = lib().orc_dequantize_4bit(_p(codes), _p(absmax), _p(code4), n, blocksize, _DT[dtype], _p(out))
     assert rc == 0
     return out

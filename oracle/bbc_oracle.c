@@ -268,3 +268,18 @@ int orc_nested_dequantize(const uint8_t* codes, const uint8_t* absmax_q, const f
     }
     return 0;
 }
+
+/* Plain 4-bit dequantization with an fp32 absmax per block [P2, the last launch of the
+ * unfused path]: out[m] = T(code4[nib_m] * absmax[m / bs]); same nibble order. */
+int orc_dequantize_4bit(const uint8_t* codes, const float* absmax, const float* code4,
+                        int64_t n, int64_t bs, int dtype, void* out)
+{
+    if (n <= 0 || bs <= 0) return 1;
+    for (int64_t m = 0; m < n; m++) {
+        uint8_t byte = codes[m / 2];
+        unsigned nib = (m % 2 == 0) ? (unsigned)(byte >> 4) : (unsigned)(byte & 0x0f);
+        float y = code4[nib] * absmax[m / bs];
+        store_elem(out, dtype, m, y);
+    }
+    return 0;
+}

@@ -31,8 +31,8 @@ def declared_functions():
 
 def test_header_declares_the_boundary():
     names = set(declared_functions())
-    assert {"kbit_quantize", "kbit_dequantize", "dequantize_4bit_nested",
-            "bbc_nf_codebook", "bbc_last_error"} <= names
+    assert {"kbit_quantize", "kbit_dequantize", "dequantize_4bit_nested", "dequantize_4bit",
+            "dequantize_4bit_nested_chain", "bbc_nf_codebook", "bbc_last_error"} <= names
 
 
 def test_library_exports_every_declared_symbol(lib):
@@ -98,6 +98,19 @@ def test_nested_validation(lib):
     assert _nd(lib, bs2=128) == 2
     assert _nd(lib, dt=5) == 1
     assert "blocksize2 must be 256" in (lib.bbc_last_error().decode() if _nd(lib, bs2=512) else "")
+
+
+def test_plain_and_chain_validation(lib):
+    assert lib.dequantize_4bit(None, FAKE, FAKE, 64, 64, 1, FAKE, None) == 1
+    assert lib.dequantize_4bit(FAKE, FAKE, FAKE, 0, 64, 1, FAKE, None) == 1
+    assert lib.dequantize_4bit(FAKE, FAKE, FAKE, 64, 48, 1, FAKE, None) == 1
+    assert lib.dequantize_4bit(FAKE, FAKE, FAKE, 64, 64, 9, FAKE, None) == 1
+    chain = lambda ws=FAKE, bs=64, bs2=256: lib.dequantize_4bit_nested_chain(  # noqa: E731
+        FAKE, FAKE, FAKE, FAKE, ct.c_float(0.0), FAKE, 64, bs, bs2, 1, FAKE, ws, None)
+    assert chain(ws=None) == 1
+    assert chain(ws=P(0x1002)) == 1
+    assert chain(bs=16) == 1
+    assert chain(bs2=128) == 2
 
 
 def test_last_error_is_per_thread(lib):

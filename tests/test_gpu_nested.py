@@ -143,3 +143,61 @@ def test_invalid_arguments_raise(bbc):
         bbc.dequantize_4bit_nested(z8, z8, f, f, 0.0, f, 64, 48, torch.float16)
     with pytest.raises(BBCError, match="blocksize2"):
         bbc.dequantize_4bit_nested(z8, z8, f, f, 0.0, f, 64, 64, torch.float16, blocksize2=128)
+
+
+@pytest.mark.parametrize("fmt", ["nf4", "fp4"])
+@pytest.mark.parametrize("dt", ["f16", "bf16", "f32"])
+def test_chain_equals_fused_and_oracle(bbc, fmt, dt):
+    """The unfused three-launch chain gives the fused kernel's bits and the oracle's."""
+    for n, bs in [(4096 * 4096, 64), (3 * 4096 * 256 + 37, 4096), (64 * 300 + 5, 32)]:
+        codes, q, a2, off = synthetic.nested_state(n, bs, seed=n % 1000 + bs, all_codes=True)
+        code2, code4 = tables(fmt)
+        args = (codes.cuda(), q.cuda(), torch.from_numpy(code2).cuda(), a2.cuda(), float(off),
+                torch.from_numpy(code4).cuda(), n, bs, DTYPES[dt])
+        ws = torch.full(((n + bs - 1) // bs,), float("nan"), dtype=torch.float32, device="cuda")
+        y_chain = bbc.dequantize_4bit_nested_chain(*args, scale_workspace=ws)
+        y_fused = bbc.dequantize_4bit_nested(*args)
+        torch.cuda.synchronize()
+        ref = oracle.nested_dequantize(to_host(codes), to_host(q), code2, to_host(a2), float(off), code4,
+                                       n, bs, 256, dt)
+        assert_bits_equal(to_host(y_chain)[:n], ref, f"chain n={n} {fmt} {dt}")
+        assert_bits_equal(to_host(y_fused)[:n], to_host(y_chain)[:n], f"fused vs chain {dt}")
+        # the workspace holds exactly the separately rounded scales
+        qn, a2n = to_host(q), to_host(a2)
+        sample = np.unique(np.r_[0, 1, (n - 1) // bs, np.random.default_rng(0).integers(0, (n - 1) // bs + 1, 64)])
+        want = np.array([oracle.nested_scale(float(code2[qn[b]]), float(a2n[b // 256]), float(off))
+                         for b in sample], np.float32)
+        assert_bits_equal(to_host(ws)[sample], want, "chain scales")
+
+
+@pytest.mark.parametrize("dt", ["f16", "bf16", "f32"])
+def test_plain_4bit_parity(bbc, dt):
+    rng = np.random.default_rng(41)
+    code4 = synthetic.fp4_table()
+    for n in [1, 3, 31, 32, 33, 1000, 65537, 4096 * 1024 + 7]:
+        for bs in (32, 64, 256, 4096):
+            nb = (n + bs - 1) // bs
+            codes = torch.from_numpy(rng.integers(0, 256, (n + 1) // 2, dtype=np.uint8))
+            am = rng.uniform(0, 2, nb).astype(np.float32)
+            am[:3] = [0.0, 1e-40, 7e4][: min(3, nb)]
+            ref = oracle.dequantize_4bit(codes.numpy(), am, code4, n, bs, dt)
+            y = bbc.dequantize_4bit(codes.cuda(), torch.from_numpy(am).cuda(),
+                                    torch.from_numpy(code4).cuda(), n, bs, DTYPES[dt])
+            torch.cuda.synchronize()
+            assert_bits_equal(to_host(y)[:n], ref, f"plain 4-bit n={n} bs={bs} {dt}")
+
+
+def test_chain_invalid_arguments(bbc):
+    from blockwise_bit_codebook_b200 import BBCError
+    z8 = torch.zeros(64, dtype=torch.uint8, device="cuda")
+    f = torch.zeros(256, device="cuda")
+    with pytest.raises(BBCError, match="null pointer"):
+        import ctypes as ct
+        L = bbc.load_library()
+        st = L.dequantize_4bit_nested_chain(ct.c_void_p(z8.data_ptr()), ct.c_void_p(z8.data_ptr()),
+                                            ct.c_void_p(f.data_ptr()), ct.c_void_p(f.data_ptr()),
+                                            ct.c_float(0.0), ct.c_void_p(f.data_ptr()), 64, 64, 256, 1,
+                                            ct.c_void_p(f.data_ptr()), None, None)
+        bbc._native._check("dequantize_4bit_nested_chain", st)
+    with pytest.raises(BBCError, match="power of two"):
+        bbc.dequantize_4bit(z8, f, f, 64, 100, torch.float16)

@@ -142,3 +142,43 @@ def test_full_code_sweep_exact(orc, dtype):
         assert np.array_equal(out, _cast(prod, dtype))
         # every 4-bit code appears
         assert set(nib.tolist()) == set(range(16))
+
+
+@pytest.mark.parametrize("dtype", ["f32", "f16", "bf16"])
+def test_plain_4bit_special_cases(orc, dtype):
+    """Plain 4-bit decode: unit absmax is a cast, powers of two scale exactly, general absmax is
+    one exact-rational product then a cast."""
+    rng = np.random.default_rng(23)
+    n, bs = 64 * 40 + 9, 64
+    nb = (n + bs - 1) // bs
+    code4 = rng.standard_normal(16).astype(np.float32)
+    codes = rng.integers(0, 256, (n + 1) // 2, dtype=np.uint8)
+    nib = np.empty(n, np.int64)
+    nib[0::2] = codes[: (n + 1) // 2] >> 4
+    nib[1::2] = codes[: n // 2] & 15
+    ones = np.ones(nb, np.float32)
+    assert np.array_equal(orc.dequantize_4bit(codes, ones, code4, n, bs, dtype), _cast(code4[nib], dtype))
+    p2 = (2.0 ** rng.integers(-10, 10, nb)).astype(np.float32)
+    assert np.array_equal(orc.dequantize_4bit(codes, p2, code4, n, bs, dtype),
+                          _cast((code4[nib] * p2[np.arange(n) // bs]).astype(np.float32), dtype))
+    am = rng.uniform(0.001, 3, nb).astype(np.float32)
+    prod = np.array([rn_mul(code4[nib[m]], am[m // bs]) for m in range(n)], np.float32)
+    assert np.array_equal(orc.dequantize_4bit(codes, am, code4, n, bs, dtype), _cast(prod, dtype))
+
+
+def test_plain_4bit_composes_with_nested_scale(orc):
+    """Feeding the pinned nested scale to the plain decode reproduces the nested dequant."""
+    rng = np.random.default_rng(29)
+    n, bs = 64 * 600 + 11, 64
+    nbo = (n + bs - 1) // bs
+    code2 = np.sort(rng.uniform(-1, 1, 256).astype(np.float32))
+    code4 = orc.normal_float_codebook(4)
+    codes = rng.integers(0, 256, (n + 1) // 2, dtype=np.uint8)
+    q = rng.integers(0, 256, nbo, dtype=np.uint8)
+    a2 = rng.uniform(0.01, 0.1, (nbo + 255) // 256).astype(np.float32)
+    off = float(np.float32(0.031))
+    scales = np.array([orc.nested_scale(float(code2[q[b]]), float(a2[b // 256]), off) for b in range(nbo)],
+                      np.float32)
+    for dt in ("f32", "bf16"):
+        assert np.array_equal(orc.dequantize_4bit(codes, scales, code4, n, bs, dt),
+                              orc.nested_dequantize(codes, q, code2, a2, off, code4, n, bs, 256, dt))
