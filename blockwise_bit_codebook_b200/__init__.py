@@ -26,6 +26,7 @@ from ._native import (  # noqa: F401
     dequantize_4bit,
     dequantize_4bit_nested,
     dequantize_4bit_nested_chain,
+    dequantize_4bit_nested_chain_noalloc,
     kbit_dequantize,
     kbit_quantize,
     library_path,

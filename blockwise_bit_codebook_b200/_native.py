@@ -42,6 +42,8 @@ def load_library():
     L.dequantize_4bit.restype = I
     L.dequantize_4bit_nested_chain.argtypes = [P, P, P, P, ct.c_float, P, I64, I, I, I, P, P, P]
     L.dequantize_4bit_nested_chain.restype = I
+    L.dequantize_4bit_nested_chain_noalloc.argtypes = [P, P, P, P, ct.c_float, P, I64, I, I, I, P, P]
+    L.dequantize_4bit_nested_chain_noalloc.restype = I
     L.bbc_nf_codebook.argtypes = [I, P]
     L.bbc_nf_codebook.restype = I
     L.bbc_last_error.argtypes = []
@@ -159,6 +161,27 @@ def dequantize_4bit_nested_chain(codes, absmax_q, code2, absmax2, offset: float,
                                         ct.c_float(offset), _ptr(code4), n, blocksize, blocksize2, dt,
                                         _ptr(out), _ptr(scale_workspace), _stream(stream, codes.device))
     _check("dequantize_4bit_nested_chain", st)
+    return out
+
+
+def dequantize_4bit_nested_chain_noalloc(codes, absmax_q, code2, absmax2, offset: float, code4, n: int,
+                                         blocksize: int, dtype, out=None, blocksize2: int = 256,
+                                         stream=None):
+    """The three-launch chain with its scale tensor in the library's fixed scratch.
+
+    For callers that cannot allocate device memory: nothing is allocated by the call (pass
+    `out` to allocate nothing here either). At most BBC_NOALLOC_SCRATCH_FLOATS outer blocks;
+    calls that can overlap on the GPU share the scratch and race.
+    """
+    import torch
+    L = load_library()
+    dt = _dt(dtype)
+    if out is None:
+        out = torch.empty(max(n, 1), dtype=_torch_dtype(dt), device=codes.device)
+    st = L.dequantize_4bit_nested_chain_noalloc(_ptr(codes), _ptr(absmax_q), _ptr(code2), _ptr(absmax2),
+                                                ct.c_float(offset), _ptr(code4), n, blocksize, blocksize2,
+                                                dt, _ptr(out), _stream(stream, codes.device))
+    _check("dequantize_4bit_nested_chain_noalloc", st)
     return out
 
 

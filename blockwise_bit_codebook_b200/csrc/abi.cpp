@@ -157,6 +157,36 @@ int dequantize_4bit_nested_chain(const uint8_t* codes, const uint8_t* absmax_q, 
                        "dequantize_4bit_nested_chain launch");
 }
 
+int dequantize_4bit_nested_chain_noalloc(const uint8_t* codes, const uint8_t* absmax_q,
+                                         const float* code2, const float* absmax2, float offset,
+                                         const float* code4, int64_t n, int blocksize, int blocksize2,
+                                         int out_dtype, void* out, void* stream) {
+    const char* fn = "dequantize_4bit_nested_chain_noalloc";
+    if (!codes || !absmax_q || !code2 || !absmax2 || !code4 || !out)
+        return fail(BBC_ERR_INVALID, "%s: null pointer argument", fn);
+    if (n <= 0) return fail(BBC_ERR_INVALID, "%s: n must be >= 1 (got %lld)", fn, (long long)n);
+    if (!valid_dtype(out_dtype)) return fail(BBC_ERR_INVALID, "%s: bad dtype %d", fn, out_dtype);
+    const int log2_bs = log2_blocksize(blocksize);
+    if (log2_bs < 0)
+        return fail(BBC_ERR_INVALID, "%s: blocksize must be a power of two in [32, 4096] (got %d)", fn,
+                    blocksize);
+    if (blocksize2 != 256)
+        return fail(BBC_ERR_UNSUPPORTED, "%s: blocksize2 must be 256 (got %d)", fn, blocksize2);
+    const int64_t nbo = (n + blocksize - 1) / blocksize;
+    if (nbo > BBC_NOALLOC_SCRATCH_FLOATS)
+        return fail(BBC_ERR_UNSUPPORTED,
+                    "%s: needs %lld scale slots (n=%lld, blocksize=%d) but the static scratch holds %d; "
+                    "use dequantize_4bit_nested_chain with a workspace or dequantize_4bit_nested",
+                    fn, (long long)nbo, (long long)n, blocksize, BBC_NOALLOC_SCRATCH_FLOATS);
+    if (!aligned(out, elem_size(out_dtype)) || !aligned(code2, 4) || !aligned(absmax2, 4) || !aligned(code4, 4))
+        return fail(BBC_ERR_INVALID, "%s: pointer not aligned to its element size", fn);
+    const bool vec = aligned(out, 32) && aligned(codes, 16);
+    return cuda_status(bbc::launch_nested_dequantize_chain_noalloc(codes, absmax_q, code2, absmax2, offset,
+                                                                   code4, n, log2_bs, out_dtype, out, vec,
+                                                                   static_cast<cudaStream_t>(stream)),
+                       fn);
+}
+
 const char* bbc_last_error(void) { return g_last_error.c_str(); }
 
 }  // extern "C"

@@ -40,4 +40,10 @@ cudaError_t launch_nested_dequantize_chain(const uint8_t* codes, const uint8_t* 
                                            const float* code4, int64_t n, int log2_bs, int out_dtype,
                                            void* out, float* scale, bool vec, cudaStream_t s);
 
+// The chain with its scale tensor in the library's static scratch (no allocation).
+cudaError_t launch_nested_dequantize_chain_noalloc(const uint8_t* codes, const uint8_t* absmax_q,
+                                                   const float* code2, const float* absmax2, float offset,
+                                                   const float* code4, int64_t n, int log2_bs,
+                                                   int out_dtype, void* out, bool vec, cudaStream_t s);
+
 }  // namespace bbc

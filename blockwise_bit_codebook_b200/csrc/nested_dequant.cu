@@ -16,6 +16,9 @@
 // the current group is decoded. Both code tables sit in shared
 // memory; the 16-entry value table lives in 16 distinct banks, so the
 // per-element lookup never conflicts. Persistent grid-stride loop.
+#include <mutex>
+
+#include "bbc.h"
 #include "common.cuh"
 #include "launch.h"
 
@@ -185,7 +188,45 @@ add_offset_kernel(float* __restrict__ scale, int64_t nbo, float offset) {
         scale[b] = __fadd_rn(scale[b], offset);
 }
 
+// Fixed scratch for the scale tensor of the allocation-free chain: one copy per device, kept
+// for the life of the process. Host code must not use this name as a device address; it
+// asks the runtime for the address on each device (scratch_address below).
+static __device__ __align__(256) float g_chain_scale_scratch[BBC_NOALLOC_SCRATCH_FLOATS];
+
 }  // namespace
+
+// Device address of this device's copy of the scratch array, looked up once per device with
+// that device current; nullptr if the lookup failed (the error is returned in *err).
+static float* scratch_address(cudaError_t* err) {
+    static std::mutex mu;
+    static float* addr[64] = {};
+    int dev = 0;
+    *err = cudaGetDevice(&dev);
+    if (*err != cudaSuccess) return nullptr;
+    if (dev < 0 || dev >= 64) {
+        *err = cudaErrorInvalidDevice;
+        return nullptr;
+    }
+    std::lock_guard<std::mutex> lock(mu);
+    if (!addr[dev]) {
+        void* p = nullptr;
+        *err = cudaGetSymbolAddress(&p, g_chain_scale_scratch);
+        if (*err != cudaSuccess) return nullptr;
+        addr[dev] = static_cast<float*>(p);
+    }
+    return addr[dev];
+}
+
+cudaError_t launch_nested_dequantize_chain_noalloc(const uint8_t* codes, const uint8_t* absmax_q,
+                                                   const float* code2, const float* absmax2, float offset,
+                                                   const float* code4, int64_t n, int log2_bs,
+                                                   int out_dtype, void* out, bool vec, cudaStream_t s) {
+    cudaError_t err = cudaSuccess;
+    float* scale = scratch_address(&err);
+    if (!scale) return err;
+    return launch_nested_dequantize_chain(codes, absmax_q, code2, absmax2, offset, code4, n, log2_bs,
+                                          out_dtype, out, scale, vec, s);
+}
 
 cudaError_t launch_nested_dequantize(const uint8_t* codes, const uint8_t* absmax_q,
                                      const float* code2, const float* absmax2, float offset,

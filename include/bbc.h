@@ -163,6 +163,43 @@ int dequantize_4bit_nested_chain(const uint8_t* codes, const uint8_t* absmax_q, 
                                  float* scale_workspace, void* stream);
 
 /*
+ * Capacity, in floats, of the library's static scale scratch used by
+ * dequantize_4bit_nested_chain_noalloc (4 MiB; every GPU that loads the
+ * library keeps it until the process exits).
+ */
+#define BBC_NOALLOC_SCRATCH_FLOATS 1048576
+
+/*
+ * dequantize_4bit_nested_chain_noalloc - dequantize_4bit_nested_chain without a
+ * caller-supplied workspace and without any allocation.
+ *
+ * The pages have no counterpart: this entry point exists for callers that
+ * cannot allocate device memory -- for example code hosted inside another
+ * framework that hands it only input and output buffers and owns every other
+ * byte of the GPU, or a latency-sensitive loop that must not call cudaMalloc
+ * once it is running, because allocation can block on the device. The
+ * intermediate scale tensor lives in one fixed array inside the library, so
+ * the call only needs its inputs and its output.
+ *
+ * Arguments, results and errors are those of dequantize_4bit_nested_chain
+ * without scale_workspace. In addition:
+ *   - ceil(n / blocksize) must not exceed BBC_NOALLOC_SCRATCH_FLOATS; larger
+ *     requests return BBC_ERR_UNSUPPORTED and launch nothing.
+ *   - The first call on each device looks up that device's copy of the array
+ *     (once, with the device current); make that first call before capturing
+ *     any stream. It allocates nothing.
+ *   - All calls share the one array per device and it keeps whatever the last
+ *     call left there. Each call writes every scale it later reads, so nothing
+ *     needs clearing, but calls whose work can overlap on the GPU (different
+ *     streams, or host threads that do not order their launches) race on it:
+ *     keep such calls on one stream or otherwise ordered.
+ */
+int dequantize_4bit_nested_chain_noalloc(const uint8_t* codes, const uint8_t* absmax_q,
+                                         const float* code2, const float* absmax2, float offset,
+                                         const float* code4, int64_t n, int blocksize, int blocksize2,
+                                         int out_dtype, void* out, void* stream);
+
+/*
  * bbc_nf_codebook - the 2^K-entry normal-float codebook, on the HOST.
  *
  * Defined by: the k-bit patch series, create_normal_float_codebook: standard
