@@ -34,11 +34,15 @@
 //    is replicated 8 times so the 8 lanes of each 128-bit shared-load phase
 //    always hit distinct banks.
 //
-// 4. Bit-plane packing without ballots. A thread owns 16 consecutive elements
-//    (half a block); adding spread(idx) << e (bit k of idx at bit 8k) builds, per
-//    8 elements, one register whose byte k holds plane k. One xor-shuffle and
-//    four byte permutes between the two lanes of a block leave words 2h, 2h+1 in
-//    lane h. K = 5 accumulates 4 elements per register with plane 4 in bits 4..7.
+// 4. Bit-plane packing without ballots. Adding spread(idx) << e (bit k of idx at
+//    bit 8k) builds, per 8 elements, one register whose byte k holds plane k
+//    (K = 5 accumulates 4 elements per register with plane 4 in bits 4..7). For
+//    32-byte-aligned 16-bit input a thread owns a whole block (two 32-byte loads,
+//    the next block prefetched into registers; two CTAs per SM leave room for
+//    that) and eight byte permutes turn its four registers into the K plane
+//    words. Otherwise (fp32, unaligned input, the ragged end) a thread owns half a
+//    block and one xor-shuffle plus four byte permutes between the two lanes of
+//    a block leave words 2h, 2h+1 in lane h.
 //
 // Blocks whose NaN-propagating absmax is NaN, infinite or above 2^125 take the
 // brute-force path (IEEE division and the rule verbatim) for all their elements.
@@ -54,10 +58,9 @@ namespace {
 constexpr int kThreads = 256;
 constexpr int kCells = 256;
 constexpr int kReplicas = 8;
-#ifndef BBC_QUANT_MIN_CTAS
-#define BBC_QUANT_MIN_CTAS 3
-#endif
-constexpr int kMinCtas = BBC_QUANT_MIN_CTAS;   // resident CTAs per SM the register budget targets
+// Resident CTAs per SM the register budget targets: the whole-block path (16-bit, aligned)
+// trades occupancy for per-thread parallelism; the half-block path keeps three.
+template <int DT, bool VEC> constexpr int kMinCtas = (VEC && DT != F32) ? 2 : 3;
 
 __device__ __forceinline__ int64_t f32_key(float f) {
     const int32_t b = __float_as_int(f);
@@ -217,6 +220,7 @@ struct LoopCtx {
     uint32_t sel_send, sel_keep, sel_wa, sel_wb, pair_mask;
     bool fast_cb;
     bool packed_v2;
+    bool packed_v4;
 };
 
 #ifndef BBC_QUANT_LDS_ASM
@@ -352,8 +356,119 @@ __device__ __forceinline__ void quantize_half(const Raw<DT>& raw, int64_t H, boo
     if (active && c.h == 0) absmax[b] = amax;
 }
 
+// ---- one whole block (32 elements of a 16-bit type) per thread ----
+
+// Raw words of one block of a 16-bit type (element 2i in the low half of word i).
+template <int DT>
+struct Raw32 { uint32_t w[16]; };
+
+template <int DT>
+__device__ __forceinline__ Raw32<DT> load_block(const void* A, int64_t b) {
+    Raw32<DT> r;
+    const char* p = reinterpret_cast<const char*>(A) + b * 64;
+    const u32x8 a = ldg_stream_v8(p);
+    const u32x8 q = ldg_stream_v8(p + 32);
+#pragma unroll
+    for (int i = 0; i < 8; i++) { r.w[i] = a.v[i]; r.w[8 + i] = q.v[i]; }
+    return r;
+}
+
+// Quantize block b held in `raw` and store its K plane words and absmax (no exchange
+// between lanes; the block lies entirely inside the input).
+template <int K, int DT>
+__device__ __forceinline__ void quantize_block(const Raw32<DT>& raw, int64_t b, const LoopCtx& c,
+                                               const float* cb, float* __restrict__ absmax,
+                                               uint32_t* __restrict__ packed) {
+    constexpr int EPA = K == 5 ? 4 : 8;
+    uint32_t p = pair_absmax<DT>(raw.w[0], raw.w[1]);
+#pragma unroll
+    for (int i = 2; i < 16; i++) p = pair_absmax<DT>(p, raw.w[i]);
+    float lo, hi;
+    widen_pair<DT>(p, lo, hi);
+    const float m = max_nan(fabsf(lo), fabsf(hi));
+    const bool special = !(m <= 0x1p125f);
+    float amax = m;
+    if (special) {
+        float a = 0.0f;
+#pragma unroll
+        for (int i = 0; i < 16; i++) {
+            float x0, x1;
+            widen_pair<DT>(raw.w[i], x0, x1);
+            a = i == 0 ? fabsf(x0) : fmaxf(a, fabsf(x0));
+            a = fmaxf(a, fabsf(x1));
+        }
+        amax = a;
+    }
+    const float d = fmaxf(amax, 1e-8f);
+    // B_q: byte j = plane j of elements 8q .. 8q+7; w4: plane 4 (K = 5)
+    uint32_t B[4], w4 = 0;
+    const float rs = __fmul_rn(rcp_approx(d), 8192.0f);
+    const bool fast = !special && c.fast_cb;
+    // K = 5 accumulates 4 elements per register: two passes of 16 keep 4 registers live
+    constexpr int NPASS = K == 5 ? 2 : 1;
+    constexpr int PE = 32 / NPASS;
+#pragma unroll
+    for (int pass = 0; pass < NPASS; pass++) {
+        uint32_t acc[4] = {0u, 0u, 0u, 0u};
+        if (fast) {
+#pragma unroll
+            for (int e = 0; e < PE; e += 2) {
+                float x0, x1;
+                widen_pair<DT>(raw.w[(pass * PE + e) / 2], x0, x1);
+                const float2 f = __ffma2_rn(make_float2(x0, x1), make_float2(rs, rs),
+                                            make_float2(12582912.0f, 12582912.0f));
+                const uint4 t0 = lut_entry(c, __float_as_uint(f.x));
+                const uint4 t1 = lut_entry(c, __float_as_uint(f.y));
+                const float v0 = __fmaf_rn(__uint_as_float(t0.y), d, __fmaf_rn(__uint_as_float(t0.x), d, x0));
+                const float v1 = __fmaf_rn(__uint_as_float(t1.y), d, __fmaf_rn(__uint_as_float(t1.x), d, x1));
+                acc[e / EPA] += (v0 > 0.0f ? t0.w : t0.z) << (e % EPA);
+                acc[(e + 1) / EPA] += (v1 > 0.0f ? t1.w : t1.z) << ((e + 1) % EPA);
+            }
+        } else {
+#pragma unroll
+            for (int e = 0; e < PE; e += 2) {
+                float x0, x1;
+                widen_pair<DT>(raw.w[(pass * PE + e) / 2], x0, x1);
+                acc[e / EPA] += spread<K>(nearest_entry<1 << K>(__fdiv_rn(x0, d), cb)) << (e % EPA);
+                acc[(e + 1) / EPA] += spread<K>(nearest_entry<1 << K>(__fdiv_rn(x1, d), cb)) << ((e + 1) % EPA);
+            }
+        }
+        if constexpr (K == 5) {
+#pragma unroll
+            for (int q = 0; q < 2; q++) {
+                B[2 * pass + q] = (acc[2 * q] & 0x0f0f0f0fu) | ((acc[2 * q + 1] & 0x0f0f0f0fu) << 4);
+                w4 |= (((acc[2 * q] >> 4) & 0xfu) | (acc[2 * q + 1] & 0xf0u)) << (8 * (2 * pass + q));
+            }
+        } else {
+#pragma unroll
+            for (int q = 0; q < 4; q++) B[q] = acc[q];
+        }
+    }
+    const uint32_t lo01 = prmt(B[0], B[1], 0x5140u), lo23 = prmt(B[2], B[3], 0x5140u);
+    const uint32_t w0 = prmt(lo01, lo23, 0x5410u), w1 = prmt(lo01, lo23, 0x7632u);
+    uint32_t* out = packed + b * K;
+    if constexpr (K == 2) {
+        if (c.packed_v2) asm volatile("st.global.v2.u32 [%0], {%1,%2};" :: "l"(out), "r"(w0), "r"(w1) : "memory");
+        else { out[0] = w0; out[1] = w1; }
+    } else {
+        const uint32_t hi01 = prmt(B[0], B[1], 0x7362u), hi23 = prmt(B[2], B[3], 0x7362u);
+        const uint32_t w2 = prmt(hi01, hi23, 0x5410u);
+        if constexpr (K == 4) {
+            const uint32_t w3 = prmt(hi01, hi23, 0x7632u);
+            if (c.packed_v4) stg_v4(out, w0, w1, w2, w3);
+            else { out[0] = w0; out[1] = w1; out[2] = w2; out[3] = w3; }
+        } else if constexpr (K == 3) {
+            out[0] = w0; out[1] = w1; out[2] = w2;
+        } else {
+            const uint32_t w3 = prmt(hi01, hi23, 0x7632u);
+            out[0] = w0; out[1] = w1; out[2] = w2; out[3] = w3; out[4] = w4;
+        }
+    }
+    absmax[b] = amax;
+}
+
 template <int K, int DT, bool VEC>
-__global__ void __launch_bounds__(kThreads, kMinCtas)
+__global__ void __launch_bounds__(kThreads, (kMinCtas<DT, VEC>))
 kbit_quant_kernel(const void* __restrict__ A, int64_t n, const float* __restrict__ codebook,
                   float* __restrict__ absmax, uint32_t* __restrict__ packed) {
     constexpr int NE = 1 << K;
@@ -417,6 +532,7 @@ kbit_quant_kernel(const void* __restrict__ A, int64_t n, const float* __restrict
     c.lut_s = (uint32_t)__cvta_generic_to_shared(lut);
     c.lane16 = (uint32_t)(lane & 7) << 4;
     c.packed_v2 = (reinterpret_cast<uintptr_t>(packed) & 7u) == 0;
+    c.packed_v4 = (reinterpret_cast<uintptr_t>(packed) & 15u) == 0;
     c.h = lane & 1;
     c.sel_send = c.h ? 0x5140u : 0x7362u;
     c.sel_keep = c.h ? 0x7362u : 0x5140u;
@@ -430,6 +546,35 @@ kbit_quant_kernel(const void* __restrict__ A, int64_t n, const float* __restrict
     const int64_t nh = ((n + 31) >> 5) * 2;
     const int64_t stride = (int64_t)gridDim.x * kThreads;
     int64_t wbase = (int64_t)blockIdx.x * kThreads + (tid & ~31);
+    if constexpr (VEC && DT != F32) {
+        // whole warp iterations of 32 blocks, one block per thread, the next one prefetched;
+        // what is left (at most the last partial iteration and a ragged block) goes by halves
+        const int64_t bend = (n >> 5) & ~(int64_t)31;
+        int64_t wb = wbase;                                 // in blocks
+        if (wb < bend) {
+            Raw32<DT> ra = load_block<DT>(A, wb + lane);
+            Raw32<DT> rb;
+            while (true) {
+                int64_t wn = wb + stride;
+                bool more = wn < bend;
+                if (more) rb = load_block<DT>(A, wn + lane);
+                quantize_block<K, DT>(ra, wb + lane, c, cb, absmax, packed);
+                wb = wn;
+                if (!more) break;
+                wn = wb + stride;
+                more = wn < bend;
+                if (more) ra = load_block<DT>(A, wn + lane);
+                quantize_block<K, DT>(rb, wb + lane, c, cb, absmax, packed);
+                wb = wn;
+                if (!more) break;
+            }
+        }
+        for (int64_t t = 2 * bend + (int64_t)blockIdx.x * kThreads + (tid & ~31); t < nh; t += stride) {
+            const Raw<DT> r = load_raw<DT, VEC>(A, n, t + lane, t + lane < nh);
+            quantize_half<K, DT>(r, t + lane, t + lane < nh, c, cb, absmax, packed);
+        }
+        return;
+    }
     if (wbase < nh_full) {
         Raw<DT> ra = load_full<DT>(A, wbase + lane, wbase + lane < nh_full);
         Raw<DT> rb;

@@ -109,6 +109,27 @@ def test_unaligned_pointers_take_scalar_path(bbc, dt):
     assert_bits_equal(to_host(y), oracle.kbit_dequantize(p, a, cb, K, n, dt), f"unaligned dequant {dt}")
 
 
+@pytest.mark.parametrize("K", [2, 3, 4, 5])
+@pytest.mark.parametrize("dt", ["f16", "bf16"])
+def test_whole_block_path_with_word_aligned_outputs(bbc, K, dt):
+    """Aligned 16-bit input (one block per thread) writing packed words and absmax that are
+    only 4-byte aligned: the vector stores must fall back, results identical."""
+    cb = oracle.normal_float_codebook(K)
+    n = 32 * 1024 * 3 + 32 * 5 + 9          # many warp iterations, a partial one, a ragged block
+    nb = (n + 31) // 32
+    x = synthetic.weights(n, std=0.02, seed=40 + K, dtype=DTYPES[dt], outlier_frac=0.001)
+    ref_p, ref_a = oracle.kbit_quantize(to_host(x), dt, K, cb)
+    pbuf = torch.zeros(nb * K + 4, dtype=torch.int32, device="cuda")
+    abuf = torch.zeros(nb + 4, dtype=torch.float32, device="cuda")
+    packed, absmax = pbuf[1:1 + nb * K], abuf[1:1 + nb]
+    assert packed.data_ptr() % 8 == 4
+    bbc.kbit_quantize(x.cuda(), K, torch.from_numpy(cb).cuda(), absmax=absmax, packed=packed)
+    torch.cuda.synchronize()
+    assert_bits_equal(to_host(absmax), ref_a, "absmax, word-aligned output")
+    assert_bits_equal(to_host(packed), ref_p, "packed, word-aligned output")
+    assert int(pbuf[0]) == 0 and int(pbuf[-3:].abs().sum()) == 0
+
+
 # ---------------------------------------------------------------- exactness corners
 
 def exact_thresholds(cb):
