@@ -8,6 +8,10 @@ it never imports the library. Each function cites the passage it follows:
 * k-bit codec: bitsandbytes k-bit patch series, tests/test_kbit_quantization.py
   (quantize_kbit_ref, dequantize_kbit_ref, pack_kbit_ref, unpack_kbit_ref) and
   csrc/ops.cu (kQuantizeBlockwise_kbit, kDequantizeBlockwise_kbit).
+* E4M4 uint8 absmax: the same series, PATCH 005 "Add vectorized dequant kernel
+  and E4M4 uint8 absmax support" (encode_absmax_e4m4, decode_absmax_e4m4 in
+  bitsandbytes/functional.py; decode_e4m4_absmax in csrc/ops.cu), and the
+  quantize_kbit / dequantize_kbit paths that use it.
 * nested 4-bit dequant and the plain 4-bit decode of its unfused form: "Fuse
   nested 4-bit scale reconstruction on SM103", Summary and Implementation.
 
@@ -55,6 +59,12 @@ def lib():
         for f in ("orc_f32_to_f16_array", "orc_f32_to_bf16_array"):
             getattr(L, f).argtypes = [P, I64, P]
         L.orc_f16_to_f32_array.argtypes = [P, I64, P]
+        L.orc_e4m4_encode.argtypes = [ct.c_float]
+        L.orc_e4m4_encode.restype = ct.c_uint8
+        L.orc_e4m4_decode.argtypes = [ct.c_uint8]
+        L.orc_e4m4_decode.restype = ct.c_float
+        L.orc_e4m4_encode_array.argtypes = [P, I64, P]
+        L.orc_e4m4_decode_array.argtypes = [P, I64, P]
         _lib = L
     return _lib
 
@@ -148,6 +158,34 @@ def kbit_dequantize(packed, absmax, codebook, K: int, n: int, dtype: str) -> np.
     rc = lib().orc_kbit_dequantize(_p(packed), _p(absmax), _p(cb), K, n, _DT[dtype], _p(out))
     assert rc == 0
     return out
+
+
+def e4m4_encode(absmax) -> np.ndarray:
+    """fp32 absmax -> uint8 E4M4 codes (bias 11), the pages' encode_absmax_e4m4 steps."""
+    a = _c(absmax, np.float32).reshape(-1)
+    out = np.empty(a.size, np.uint8)
+    lib().orc_e4m4_encode_array(_p(a), a.size, _p(out))
+    return out
+
+
+def e4m4_decode(codes) -> np.ndarray:
+    """uint8 E4M4 codes -> their exact fp32 values (decode_absmax_e4m4)."""
+    c = _c(codes, np.uint8).reshape(-1)
+    out = np.empty(c.size, np.float32)
+    lib().orc_e4m4_decode_array(_p(c), c.size, _p(out))
+    return out
+
+
+def kbit_quantize_e4m4(A, dtype: str, K: int, codebook):
+    """quantize_kbit with absmax_format "e4m4": the packed words are those of the fp32-absmax
+    quantize (the codes use the exact fp32 absmax); the stored absmax is its E4M4 encoding."""
+    packed, absmax = kbit_quantize(A, dtype, K, codebook)
+    return packed, e4m4_encode(absmax)
+
+
+def kbit_dequantize_e4m4(packed, absmax_e4m4, codebook, K: int, n: int, dtype: str) -> np.ndarray:
+    """dequantize_kbit with a uint8 E4M4 absmax: decode each block's absmax, then the fp32 path."""
+    return kbit_dequantize(packed, e4m4_decode(absmax_e4m4), codebook, K, n, dtype)
 
 
 def nested_scale(code2_val: float, absmax2_val: float, offset: float) -> float:

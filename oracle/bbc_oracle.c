@@ -28,6 +28,9 @@
  *    j and element 2j+1 in the low nibble.
  *  - NaN results of the float->half/bfloat16 conversions are returned as a
  *    quiet NaN with the input's sign; only the NaN class is meaningful.
+ *  - E4M4 encode: floor(log2 a) is the exact floor; an infinite absmax encodes
+ *    as 0xFF; at and above 32 the exponent field clamps to 15 while the
+ *    mantissa is rounded in a's own binade, as the pages' steps do.
  */
 #include <stdint.h>
 #include <string.h>
@@ -235,6 +238,70 @@ int orc_kbit_dequantize(const uint32_t* packed, const float* absmax, const float
         store_elem(out, dtype, m, y);
     }
     return 0;
+}
+
+/* ------------------------------------------------------------------ */
+/* E4M4 uint8 absmax [P1 PATCH 005 "Add vectorized dequant kernel and   */
+/* E4M4 uint8 absmax support": encode_absmax_e4m4, decode_absmax_e4m4,  */
+/* decode_e4m4_absmax]                                                  */
+/* ------------------------------------------------------------------ */
+
+#define ORC_E4M4_BIAS 11
+
+/*
+ * Decode: e = code >> 4, m = code & 15. e > 0: 2^(e - bias) * (1 + m/16);
+ * e == 0: 2^(1 - bias) * (m/16) (IEEE-style subnormals, code 0 is 0.0).
+ * Every such value is exact in binary32 (computed here as an integer times a
+ * power of two in double, then narrowed without rounding).
+ */
+float orc_e4m4_decode(uint8_t code)
+{
+    int e = code >> 4, m = code & 15;
+    if (e == 0) return (float)ldexp((double)m, 1 - ORC_E4M4_BIAS - 4);
+    return (float)ldexp((double)(16 + m), e - ORC_E4M4_BIAS - 4);
+}
+
+/*
+ * Encode, following the pages' steps in order:
+ *   values that are not > 0 encode as 0 (this covers 0, negatives and NaN);
+ *   e_unb = floor(log2(a));  e_biased = clamp(e_unb + bias, 0, 15);
+ *   if e_unb + bias <= 0 (subnormal): e_biased = 0, m = round(a / 2^(1-bias) * 16);
+ *   else m = round((a / 2^e_unb - 1) * 16) with the unclamped e_unb;
+ *   m is clamped to [0, 15]; code = e_biased << 4 | m.
+ * round() is round-half-to-even (torch.round). Readings: floor(log2 a) is the
+ * exact floor (frexp), not a rounded fp32 logarithm; an infinite absmax
+ * encodes as the largest code 0xFF. All arithmetic below is exact in double.
+ */
+uint8_t orc_e4m4_encode(float a)
+{
+    if (!(a > 0.0f)) return 0;
+    if (isinf(a)) return 0xFF;
+    int ex;
+    (void)frexp((double)a, &ex);          /* a = f * 2^ex, f in [0.5, 1) */
+    int e_unb = ex - 1;                   /* floor(log2 a) */
+    int e_biased = e_unb + ORC_E4M4_BIAS;
+    double m_real;
+    if (e_biased <= 0) {
+        e_biased = 0;
+        m_real = ldexp((double)a, -(1 - ORC_E4M4_BIAS)) * 16.0;
+    } else {
+        if (e_biased > 15) e_biased = 15;
+        m_real = (ldexp((double)a, -e_unb) - 1.0) * 16.0;
+    }
+    double m = nearbyint(m_real);         /* default rounding mode: to nearest, ties to even */
+    if (m < 0.0) m = 0.0;
+    if (m > 15.0) m = 15.0;
+    return (uint8_t)((e_biased << 4) | (int)m);
+}
+
+void orc_e4m4_encode_array(const float* a, int64_t n, uint8_t* out)
+{
+    for (int64_t i = 0; i < n; i++) out[i] = orc_e4m4_encode(a[i]);
+}
+
+void orc_e4m4_decode_array(const uint8_t* c, int64_t n, float* out)
+{
+    for (int64_t i = 0; i < n; i++) out[i] = orc_e4m4_decode(c[i]);
 }
 
 /* ------------------------------------------------------------------ */
