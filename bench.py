@@ -47,7 +47,8 @@ def parse_args():
                     help="override the element count (profiling of a smaller case)")
     ap.add_argument("--ops", default=None,
                     help="comma-separated subset of quantize_k3,dequantize_k3,quantize_k5,"
-                         "dequantize_k5,nested_nf4_bs64 (profiling)")
+                         "dequantize_k5,nested_nf4_bs64, or the E4M4-absmax ops "
+                         "{quantize,dequantize}_k{3,4,5}_e4m4 (profiling)")
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -71,6 +72,10 @@ def op_bytes(kind, n, K=None, out_size=2, bs=NESTED_BS):
         return n * 2 + nb * K * 4 + nb * 4
     if kind == "dequantize":
         return nb * K * 4 + nb * 4 + n * out_size
+    if kind == "quantize_e4m4":                   # one E4M4 byte of absmax per block
+        return n * 2 + nb * K * 4 + nb
+    if kind == "dequantize_e4m4":
+        return nb * K * 4 + nb + n * out_size
     nbo = (n + bs - 1) // bs
     nbi = (nbo + 255) // 256
     return (n + 1) // 2 + nbo + nbi * 4 + n * out_size
@@ -79,13 +84,15 @@ def op_bytes(kind, n, K=None, out_size=2, bs=NESTED_BS):
 ALL_OPS = [("quantize_k3", "quantize", 3), ("dequantize_k3", "dequantize", 3),
            ("quantize_k5", "quantize", 5), ("dequantize_k5", "dequantize", 5),
            ("nested_nf4_bs64", "nested", None)]
+# Selectable with --ops (not part of the default step): the E4M4-absmax codec.
+EXTRA_OPS = [(f"{k}_k{K}_e4m4", f"{k}_e4m4", K) for K in (3, 4, 5) for k in ("quantize", "dequantize")]
 
 
 def workload_ops(only=None):
     if not only:
         return list(ALL_OPS)
     names = only.split(",")
-    ops = [o for o in ALL_OPS if o[0] in names]
+    ops = [o for o in ALL_OPS + EXTRA_OPS if o[0] in names]
     assert len(ops) == len(names), f"unknown op in {only}"
     return ops
 
@@ -112,6 +119,7 @@ def load_peaks():
 
 def kernel_source_hash(kind):
     files = {"quantize": ["kbit_quant.cu"], "dequantize": ["kbit_dequant.cu"],
+             "quantize_e4m4": ["kbit_quant.cu"], "dequantize_e4m4": ["kbit_dequant.cu"],
              "nested": ["nested_dequant.cu"]}[kind] + ["common.cuh"]
     h = hashlib.sha256()
     for f in files:
@@ -251,9 +259,11 @@ def run_bbc(args):
     x = synthetic.weights(n, std=0.02, seed=7, dtype=torch.bfloat16, device=dev)
     cbs = {K: bbc.bbc_nf_codebook(K) for K in (3, 4, 5)}
     cb_dev = {K: torch.from_numpy(cbs[K]).to(dev) for K in cbs}
-    packed = {K: torch.empty(nb * K, dtype=torch.int32, device=dev) for K in (3, 5)}
-    absmax = {K: torch.empty(nb, dtype=torch.float32, device=dev) for K in (3, 5)}
-    outs = {K: torch.empty(n, dtype=torch.bfloat16, device=dev) for K in (3, 5)}
+    ks = sorted({K for _, _, K in ops if K})
+    packed = {K: torch.empty(nb * K, dtype=torch.int32, device=dev) for K in ks}
+    absmax = {K: torch.empty(nb, dtype=torch.float32, device=dev) for K in ks}
+    absmax8 = {K: torch.empty(nb, dtype=torch.uint8, device=dev) for K in ks}
+    outs = {K: torch.empty(n, dtype=torch.bfloat16, device=dev) for K in ks}
     nested = synthetic.nested_state(n, NESTED_BS, seed=3, device=dev)
     codes, q, a2, off = nested
     code2 = synthetic.general8_table()
@@ -267,6 +277,10 @@ def run_bbc(args):
             bbc.kbit_quantize(xin, K, cb_dev[K], absmax=am[K], packed=pk[K], stream=stream)
         elif kind == "dequantize":
             bbc.kbit_dequantize(pk[K], am[K], cb_dev[K], K, n, torch.bfloat16, out=ou[K], stream=stream)
+        elif kind == "quantize_e4m4":
+            bbc.kbit_quantize_e4m4(xin, K, cb_dev[K], absmax=absmax8[K], packed=pk[K], stream=stream)
+        elif kind == "dequantize_e4m4":
+            bbc.kbit_dequantize_e4m4(pk[K], absmax8[K], cb_dev[K], K, n, torch.bfloat16, out=ou[K], stream=stream)
         else:
             bbc.dequantize_4bit_nested(cin, qin, code2_dev, a2in, float(off), code4_dev, n, NESTED_BS,
                                        torch.bfloat16, out=no, stream=stream)
@@ -346,15 +360,18 @@ def run_bbc(args):
         pin = lambda t: t.cpu().pin_memory()  # noqa: E731
         hx, hcodes, hq, ha2 = pin(x), pin(codes), pin(q), pin(a2)
         hcb = {K: torch.from_numpy(cbs[K]).pin_memory() for K in (3, 4, 5)}
-        h_out = {"packed": {K: torch.empty_like(packed[K], device="cpu").pin_memory() for K in (3, 5)},
-                 "absmax": {K: torch.empty_like(absmax[K], device="cpu").pin_memory() for K in (3, 5)},
-                 "out": {K: torch.empty_like(outs[K], device="cpu").pin_memory() for K in (3, 5)},
+        k32 = sorted({K for _, kind, K in ops if kind in ("quantize", "dequantize")})
+        k8 = sorted({K for _, kind, K in ops if kind.endswith("_e4m4")})
+        h_out = {"packed": {K: torch.empty_like(packed[K], device="cpu").pin_memory() for K in ks},
+                 "absmax": {K: torch.empty_like(absmax[K], device="cpu").pin_memory() for K in k32},
+                 "absmax8": {K: torch.empty_like(absmax8[K], device="cpu").pin_memory() for K in k8},
+                 "out": {K: torch.empty_like(outs[K], device="cpu").pin_memory() for K in ks},
                  "nested": torch.empty_like(nout, device="cpu").pin_memory()}
         dx, dcodes, dq, da2 = torch.empty_like(x), torch.empty_like(codes), torch.empty_like(q), torch.empty_like(a2)
         h2d = sum(t.numel() * t.element_size() for t in (hx, hcodes, hq, ha2)) + \
             sum(t.numel() * 4 for t in hcb.values())
-        d2h = sum(t.numel() * t.element_size() for K in (3, 5)
-                  for t in (packed[K], absmax[K], outs[K])) + nout.numel() * 2
+        d2h = sum(t.numel() * t.element_size() for K in ks for t in (packed[K], outs[K])) + \
+            sum(absmax[K].numel() * 4 for K in k32) + sum(absmax8[K].numel() for K in k8) + nout.numel() * 2
 
         def e2e_step():
             dx.copy_(hx, non_blocking=True)
@@ -365,10 +382,13 @@ def run_bbc(args):
                 cb_dev[K].copy_(hcb[K], non_blocking=True)
             for _, kind, K in ops:
                 launch(kind, K, xin=dx, cin=dcodes, qin=dq, a2in=da2)
-            for K in (3, 5):
+            for K in ks:
                 h_out["packed"][K].copy_(packed[K], non_blocking=True)
-                h_out["absmax"][K].copy_(absmax[K], non_blocking=True)
                 h_out["out"][K].copy_(outs[K], non_blocking=True)
+            for K in k32:
+                h_out["absmax"][K].copy_(absmax[K], non_blocking=True)
+            for K in k8:
+                h_out["absmax8"][K].copy_(absmax8[K], non_blocking=True)
             h_out["nested"].copy_(nout, non_blocking=True)
 
         e2e_step()

@@ -7,6 +7,7 @@ library's CUDA kernels. torch is used for device memory and streams only.
 
     kbit_quantize(A, K, codebook)                       -> (packed, absmax)
     kbit_dequantize(packed, absmax, codebook, K, n, dtype) -> out
+    kbit_quantize_e4m4 / kbit_dequantize_e4m4   the same with a uint8 E4M4 absmax
     dequantize_4bit_nested(codes, absmax_q, code2, absmax2, offset, code4,
                            n, blocksize, dtype)         -> out
     dequantize_4bit(codes, absmax, code4, n, blocksize, dtype)  -> out
@@ -28,7 +29,9 @@ from ._native import (  # noqa: F401
     dequantize_4bit_nested_chain,
     dequantize_4bit_nested_chain_noalloc,
     kbit_dequantize,
+    kbit_dequantize_e4m4,
     kbit_quantize,
+    kbit_quantize_e4m4,
     library_path,
     load_library,
 )

@@ -36,6 +36,10 @@ def load_library():
     L.kbit_quantize.restype = I
     L.kbit_dequantize.argtypes = [P, P, P, I, I, I64, I, P, P]
     L.kbit_dequantize.restype = I
+    L.kbit_quantize_e4m4.argtypes = [P, I, I64, I, I, P, P, P, P]
+    L.kbit_quantize_e4m4.restype = I
+    L.kbit_dequantize_e4m4.argtypes = [P, P, P, I, I, I64, I, P, P]
+    L.kbit_dequantize_e4m4.restype = I
     L.dequantize_4bit_nested.argtypes = [P, P, P, P, ct.c_float, P, I64, I, I, I, P, P]
     L.dequantize_4bit_nested.restype = I
     L.dequantize_4bit.argtypes = [P, P, P, I64, I, I, P, P]
@@ -114,6 +118,36 @@ def kbit_dequantize(packed, absmax, codebook, K: int, n: int, dtype, out=None, b
     st = L.kbit_dequantize(_ptr(packed), _ptr(absmax), _ptr(codebook), K, blocksize, n, dt, _ptr(out),
                            _stream(stream, packed.device))
     _check("kbit_dequantize", st)
+    return out
+
+
+def kbit_quantize_e4m4(A, K: int, codebook, absmax=None, packed=None, blocksize: int = 32, stream=None):
+    """kbit_quantize with the per-block absmax stored as one E4M4 byte. Returns (packed, absmax_u8)."""
+    import torch
+    L = load_library()
+    n = A.numel()
+    nb = (n + blocksize - 1) // blocksize if blocksize > 0 else 0
+    if absmax is None:
+        absmax = torch.empty(max(nb, 1), dtype=torch.uint8, device=A.device)
+    if packed is None:
+        packed = torch.empty(max(nb * K, 1), dtype=torch.int32, device=A.device)
+    st = L.kbit_quantize_e4m4(_ptr(A), _dt(A.dtype), n, K, blocksize, _ptr(codebook), _ptr(absmax),
+                              _ptr(packed), _stream(stream, A.device))
+    _check("kbit_quantize_e4m4", st)
+    return packed, absmax
+
+
+def kbit_dequantize_e4m4(packed, absmax, codebook, K: int, n: int, dtype, out=None, blocksize: int = 32,
+                         stream=None):
+    """kbit_dequantize with a uint8 E4M4 absmax; returns a 1-D CUDA tensor of n elements of `dtype`."""
+    import torch
+    L = load_library()
+    dt = _dt(dtype)
+    if out is None:
+        out = torch.empty(max(n, 1), dtype=_torch_dtype(dt), device=packed.device)
+    st = L.kbit_dequantize_e4m4(_ptr(packed), _ptr(absmax), _ptr(codebook), K, blocksize, n, dt, _ptr(out),
+                                _stream(stream, packed.device))
+    _check("kbit_dequantize_e4m4", st)
     return out
 
 

@@ -50,17 +50,27 @@ int log2_blocksize(int blocksize) {
 
 extern "C" {
 
+// Shared validation of the k-bit entry points; `absmax` is fp32 or E4M4 bytes (`am_size`).
+static int check_kbit(const char* fn, const void* data, const void* absmax, size_t am_size, const float* codebook,
+               const uint32_t* packed, int64_t n, int K, int dtype, int blocksize, const void* typed,
+               int typed_dtype) {
+    if (!data || !absmax || !codebook || !packed)
+        return fail(BBC_ERR_INVALID, "%s: null pointer argument", fn);
+    if (n <= 0) return fail(BBC_ERR_INVALID, "%s: n must be >= 1 (got %lld)", fn, (long long)n);
+    if (K < 2 || K > 5) return fail(BBC_ERR_INVALID, "%s: K must be 2..5 (got %d)", fn, K);
+    if (!valid_dtype(dtype)) return fail(BBC_ERR_INVALID, "%s: bad dtype %d", fn, dtype);
+    if (blocksize != 32)
+        return fail(BBC_ERR_UNSUPPORTED, "%s: blocksize must be 32 (got %d)", fn, blocksize);
+    if (!aligned(typed, elem_size(typed_dtype)) || !aligned(codebook, 4) || !aligned(absmax, am_size) ||
+        !aligned(packed, 4))
+        return fail(BBC_ERR_INVALID, "%s: pointer not aligned to its element size", fn);
+    return BBC_OK;
+}
+
 int kbit_quantize(const void* A, int dtype, int64_t n, int K, int blocksize,
                   const float* codebook, float* absmax, uint32_t* packed, void* stream) {
-    if (!A || !codebook || !absmax || !packed)
-        return fail(BBC_ERR_INVALID, "kbit_quantize: null pointer argument");
-    if (n <= 0) return fail(BBC_ERR_INVALID, "kbit_quantize: n must be >= 1 (got %lld)", (long long)n);
-    if (K < 2 || K > 5) return fail(BBC_ERR_INVALID, "kbit_quantize: K must be 2..5 (got %d)", K);
-    if (!valid_dtype(dtype)) return fail(BBC_ERR_INVALID, "kbit_quantize: bad dtype %d", dtype);
-    if (blocksize != 32)
-        return fail(BBC_ERR_UNSUPPORTED, "kbit_quantize: blocksize must be 32 (got %d)", blocksize);
-    if (!aligned(A, elem_size(dtype)) || !aligned(codebook, 4) || !aligned(absmax, 4) || !aligned(packed, 4))
-        return fail(BBC_ERR_INVALID, "kbit_quantize: pointer not aligned to its element size");
+    const int st = check_kbit("kbit_quantize", A, absmax, 4, codebook, packed, n, K, dtype, blocksize, A, dtype);
+    if (st != BBC_OK) return st;
     const bool vec = aligned(A, 32);     // 256-bit loads of 16-element groups
     return cuda_status(bbc::launch_kbit_quantize(A, dtype, n, K, codebook, absmax, packed, vec,
                                                  static_cast<cudaStream_t>(stream)),
@@ -69,19 +79,35 @@ int kbit_quantize(const void* A, int dtype, int64_t n, int K, int blocksize,
 
 int kbit_dequantize(const uint32_t* packed, const float* absmax, const float* codebook,
                     int K, int blocksize, int64_t n, int out_dtype, void* out, void* stream) {
-    if (!packed || !absmax || !codebook || !out)
-        return fail(BBC_ERR_INVALID, "kbit_dequantize: null pointer argument");
-    if (n <= 0) return fail(BBC_ERR_INVALID, "kbit_dequantize: n must be >= 1 (got %lld)", (long long)n);
-    if (K < 2 || K > 5) return fail(BBC_ERR_INVALID, "kbit_dequantize: K must be 2..5 (got %d)", K);
-    if (!valid_dtype(out_dtype)) return fail(BBC_ERR_INVALID, "kbit_dequantize: bad dtype %d", out_dtype);
-    if (blocksize != 32)
-        return fail(BBC_ERR_UNSUPPORTED, "kbit_dequantize: blocksize must be 32 (got %d)", blocksize);
-    if (!aligned(out, elem_size(out_dtype)) || !aligned(codebook, 4) || !aligned(absmax, 4) || !aligned(packed, 4))
-        return fail(BBC_ERR_INVALID, "kbit_dequantize: pointer not aligned to its element size");
+    const int st = check_kbit("kbit_dequantize", out, absmax, 4, codebook, packed, n, K, out_dtype, blocksize,
+                              out, out_dtype);
+    if (st != BBC_OK) return st;
     const bool vec = aligned(out, 32);     // 32-byte stores of 16-element groups
     return cuda_status(bbc::launch_kbit_dequantize(packed, absmax, codebook, K, n, out_dtype, out, vec,
                                                    static_cast<cudaStream_t>(stream)),
                        "kbit_dequantize launch");
+}
+
+int kbit_quantize_e4m4(const void* A, int dtype, int64_t n, int K, int blocksize, const float* codebook,
+                       uint8_t* absmax_e4m4, uint32_t* packed, void* stream) {
+    const int st = check_kbit("kbit_quantize_e4m4", A, absmax_e4m4, 1, codebook, packed, n, K, dtype, blocksize,
+                              A, dtype);
+    if (st != BBC_OK) return st;
+    const bool vec = aligned(A, 32);
+    return cuda_status(bbc::launch_kbit_quantize_e4m4(A, dtype, n, K, codebook, absmax_e4m4, packed, vec,
+                                                      static_cast<cudaStream_t>(stream)),
+                       "kbit_quantize_e4m4 launch");
+}
+
+int kbit_dequantize_e4m4(const uint32_t* packed, const uint8_t* absmax_e4m4, const float* codebook, int K,
+                         int blocksize, int64_t n, int out_dtype, void* out, void* stream) {
+    const int st = check_kbit("kbit_dequantize_e4m4", out, absmax_e4m4, 1, codebook, packed, n, K, out_dtype,
+                              blocksize, out, out_dtype);
+    if (st != BBC_OK) return st;
+    const bool vec = aligned(out, 32);
+    return cuda_status(bbc::launch_kbit_dequantize_e4m4(packed, absmax_e4m4, codebook, K, n, out_dtype, out, vec,
+                                                        static_cast<cudaStream_t>(stream)),
+                       "kbit_dequantize_e4m4 launch");
 }
 
 int dequantize_4bit_nested(const uint8_t* codes, const uint8_t* absmax_q, const float* code2,

@@ -148,4 +148,35 @@ __device__ __forceinline__ uint32_t set_ge(float a, float b) {
     return r;
 }
 
+// ---- E4M4 uint8 absmax (4-bit exponent, bias 11, 4-bit mantissa, subnormals) ----
+
+// Exact value of a code: e > 0: 2^(e - 11) * (1 + m/16); e == 0: m * 2^-14.
+// t = bits (c + 1856) << 19 places e + 116 in the fp32 exponent and m in its top mantissa
+// bits, the value for e > 0. For e == 0 it is 2^-11 + m * 2^-15, and 2t - 2^-10 = m * 2^-14
+// (exact); that is below t exactly when t < 2^-10, i.e. for the 16 subnormal codes.
+__device__ __forceinline__ float e4m4_decode(uint32_t code) {
+    const float t = __uint_as_float((code << 19) + (1856u << 19));
+    return fminf(t, __fmaf_rn(t, 2.0f, -0x1p-10f));
+}
+
+// Code of an absmax: exponent floor(log2 a) + 11 clamped to [0, 15] (subnormal at <= 0), the
+// mantissa rounded half-to-even in a's own binade and clamped to 15; values that are not > 0
+// (zero, NaN) give 0, +infinity gives 0xFF.
+__device__ __forceinline__ uint32_t e4m4_encode(float a) {
+    const uint32_t u = __float_as_uint(a);
+    if (!(a > 0.0f)) return 0u;
+    if (u == 0x7f800000u) return 0xffu;
+    const int eb = (int)(u >> 23) - 127 + 11;        // fp32 subnormals land far below 0
+    if (eb <= 0) return (uint32_t)min(__float2int_rn(a * 16384.0f), 15);   // a * 2^14 is exact
+    const uint32_t f = u & 0x7fffffu;
+    const uint32_t m = min((f + 0x3ffffu + ((f >> 19) & 1u)) >> 19, 15u);    // RNE of f / 2^19
+    return ((uint32_t)min(eb, 15) << 4) | m;
+}
+
+// Per-block absmax in either storage format.
+__device__ __forceinline__ void store_absmax(float* p, int64_t b, float a) { p[b] = a; }
+__device__ __forceinline__ void store_absmax(uint8_t* p, int64_t b, float a) { p[b] = (uint8_t)e4m4_encode(a); }
+__device__ __forceinline__ float load_absmax(const float* p, int64_t b) { return __ldg(p + b); }
+__device__ __forceinline__ float load_absmax(const uint8_t* p, int64_t b) { return e4m4_decode(__ldg(p + b)); }
+
 }  // namespace bbc

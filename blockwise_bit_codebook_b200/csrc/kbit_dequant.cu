@@ -42,12 +42,12 @@ struct BlockIn {
     uint32_t w[K];
 };
 
-template <int K>
-__device__ __forceinline__ BlockIn<K> load_block(const uint32_t* packed, const float* absmax,
+template <int K, typename AT>
+__device__ __forceinline__ BlockIn<K> load_block(const uint32_t* packed, const AT* absmax,
                                                  int64_t b, bool active) {
     BlockIn<K> r;
     if (active) {
-        r.am = __ldg(absmax + b);
+        r.am = load_absmax(absmax, b);          // fp32 as stored, or the exact E4M4 value
         const uint32_t* wp = packed + b * K;
 #pragma unroll
         for (int j = 0; j < K; j++) r.w[j] = ldg_u32(wp + j);
@@ -59,9 +59,9 @@ __device__ __forceinline__ BlockIn<K> load_block(const uint32_t* packed, const f
     return r;
 }
 
-template <int K, int DT, bool VEC>
+template <int K, int DT, bool VEC, typename AT>
 __global__ void __launch_bounds__(kThreads)
-kbit_dequant_kernel(const uint32_t* __restrict__ packed, const float* __restrict__ absmax,
+kbit_dequant_kernel(const uint32_t* __restrict__ packed, const AT* __restrict__ absmax,
                     const float* __restrict__ codebook, int64_t n, void* __restrict__ out) {
     __shared__ float cb[32];
     if (threadIdx.x < 32) cb[threadIdx.x] = threadIdx.x < (1u << K) ? codebook[threadIdx.x] : 0.0f;
@@ -75,10 +75,10 @@ kbit_dequant_kernel(const uint32_t* __restrict__ packed, const float* __restrict
     const int64_t stride = (int64_t)gridDim.x * kThreads;
 
     int64_t H = (int64_t)blockIdx.x * kThreads + threadIdx.x;
-    BlockIn<K> cur = load_block<K>(packed, absmax, H >> 1, H < nh);
+    BlockIn<K> cur = load_block<K, AT>(packed, absmax, H >> 1, H < nh);
     for (; H < nh; H += stride) {
         const int64_t Hn = H + stride;
-        const BlockIn<K> nxt = load_block<K>(packed, absmax, Hn >> 1, Hn < nh);
+        const BlockIn<K> nxt = load_block<K, AT>(packed, absmax, Hn >> 1, Hn < nh);
 
         uint32_t B0, B1;
         if constexpr (K == 2) {
@@ -128,18 +128,18 @@ kbit_dequant_kernel(const uint32_t* __restrict__ packed, const float* __restrict
     }
 }
 
-template <int K, int DT>
-cudaError_t launch_t(const uint32_t* packed, const float* absmax, const float* codebook, int64_t n,
+template <int K, int DT, typename AT>
+cudaError_t launch_t(const uint32_t* packed, const AT* absmax, const float* codebook, int64_t n,
                      void* out, bool vec, cudaStream_t s) {
     const int64_t nh = ((n + 31) >> 5) * 2;
-    auto k = vec ? kbit_dequant_kernel<K, DT, true> : kbit_dequant_kernel<K, DT, false>;
+    auto k = vec ? kbit_dequant_kernel<K, DT, true, AT> : kbit_dequant_kernel<K, DT, false, AT>;
     const int grid = persistent_grid(k, kThreads, 0, nh, kThreads);
     k<<<grid, kThreads, 0, s>>>(packed, absmax, codebook, n, out);
     return cudaGetLastError();
 }
 
-template <int K>
-cudaError_t launch_k(const uint32_t* packed, const float* absmax, const float* codebook, int64_t n,
+template <int K, typename AT>
+cudaError_t launch_k(const uint32_t* packed, const AT* absmax, const float* codebook, int64_t n,
                      int dt, void* out, bool vec, cudaStream_t s) {
     switch (dt) {
         case F16: return launch_t<K, F16>(packed, absmax, codebook, n, out, vec, s);
@@ -148,17 +148,29 @@ cudaError_t launch_k(const uint32_t* packed, const float* absmax, const float* c
     }
 }
 
-}  // namespace
-
-cudaError_t launch_kbit_dequantize(const uint32_t* packed, const float* absmax,
-                                   const float* codebook, int K, int64_t n, int out_dtype,
-                                   void* out, bool vec, cudaStream_t s) {
+template <typename AT>
+cudaError_t launch_any(const uint32_t* packed, const AT* absmax, const float* codebook, int K, int64_t n,
+                       int out_dtype, void* out, bool vec, cudaStream_t s) {
     switch (K) {
         case 2: return launch_k<2>(packed, absmax, codebook, n, out_dtype, out, vec, s);
         case 3: return launch_k<3>(packed, absmax, codebook, n, out_dtype, out, vec, s);
         case 4: return launch_k<4>(packed, absmax, codebook, n, out_dtype, out, vec, s);
         default: return launch_k<5>(packed, absmax, codebook, n, out_dtype, out, vec, s);
     }
+}
+
+}  // namespace
+
+cudaError_t launch_kbit_dequantize(const uint32_t* packed, const float* absmax,
+                                   const float* codebook, int K, int64_t n, int out_dtype,
+                                   void* out, bool vec, cudaStream_t s) {
+    return launch_any(packed, absmax, codebook, K, n, out_dtype, out, vec, s);
+}
+
+cudaError_t launch_kbit_dequantize_e4m4(const uint32_t* packed, const uint8_t* absmax,
+                                        const float* codebook, int K, int64_t n, int out_dtype,
+                                        void* out, bool vec, cudaStream_t s) {
+    return launch_any(packed, absmax, codebook, K, n, out_dtype, out, vec, s);
 }
 
 }  // namespace bbc

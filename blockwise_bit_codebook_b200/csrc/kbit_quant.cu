@@ -280,9 +280,9 @@ __device__ __forceinline__ void exact_codes(const Raw<DT>& raw, float d, const f
 // Quantize the half block H held in `raw` (16 elements) and store its share of the block's
 // words. Every lane of the warp must call this together (it exchanges data with its pair
 // lane); `active` lanes store.
-template <int K, int DT>
+template <int K, int DT, typename AT>
 __device__ __forceinline__ void quantize_half(const Raw<DT>& raw, int64_t H, bool active, const LoopCtx& c,
-                                              const float* cb, float* __restrict__ absmax,
+                                              const float* cb, AT* __restrict__ absmax,
                                               uint32_t* __restrict__ packed) {
     constexpr int NACC = K == 5 ? 4 : 2;
     // NaN-propagating block max decides between the fast and the exact path. For 16-bit
@@ -353,7 +353,7 @@ __device__ __forceinline__ void quantize_half(const Raw<DT>& raw, int64_t H, boo
         if (active && 2 * c.h + 1 < K) out[2 * c.h + 1] = wb;
         if constexpr (K == 5) { if (active && c.h == 0) out[4] = w4; }
     }
-    if (active && c.h == 0) absmax[b] = amax;
+    if (active && c.h == 0) store_absmax(absmax, b, amax);
 }
 
 // ---- one whole block (32 elements of a 16-bit type) per thread ----
@@ -375,9 +375,9 @@ __device__ __forceinline__ Raw32<DT> load_block(const void* A, int64_t b) {
 
 // Quantize block b held in `raw` and store its K plane words and absmax (no exchange
 // between lanes; the block lies entirely inside the input).
-template <int K, int DT>
+template <int K, int DT, typename AT>
 __device__ __forceinline__ void quantize_block(const Raw32<DT>& raw, int64_t b, const LoopCtx& c,
-                                               const float* cb, float* __restrict__ absmax,
+                                               const float* cb, AT* __restrict__ absmax,
                                                uint32_t* __restrict__ packed) {
     constexpr int EPA = K == 5 ? 4 : 8;
     uint32_t p = pair_absmax<DT>(raw.w[0], raw.w[1]);
@@ -464,13 +464,13 @@ __device__ __forceinline__ void quantize_block(const Raw32<DT>& raw, int64_t b, 
             out[0] = w0; out[1] = w1; out[2] = w2; out[3] = w3; out[4] = w4;
         }
     }
-    absmax[b] = amax;
+    store_absmax(absmax, b, amax);
 }
 
-template <int K, int DT, bool VEC>
+template <int K, int DT, bool VEC, typename AT>
 __global__ void __launch_bounds__(kThreads, (kMinCtas<DT, VEC>))
 kbit_quant_kernel(const void* __restrict__ A, int64_t n, const float* __restrict__ codebook,
-                  float* __restrict__ absmax, uint32_t* __restrict__ packed) {
+                  AT* __restrict__ absmax, uint32_t* __restrict__ packed) {
     constexpr int NE = 1 << K;
     __shared__ __align__(16) uint4 lut[kCells * kReplicas];    // 32 KB
     __shared__ float cb[32];
@@ -558,20 +558,20 @@ kbit_quant_kernel(const void* __restrict__ A, int64_t n, const float* __restrict
                 int64_t wn = wb + stride;
                 bool more = wn < bend;
                 if (more) rb = load_block<DT>(A, wn + lane);
-                quantize_block<K, DT>(ra, wb + lane, c, cb, absmax, packed);
+                quantize_block<K, DT, AT>(ra, wb + lane, c, cb, absmax, packed);
                 wb = wn;
                 if (!more) break;
                 wn = wb + stride;
                 more = wn < bend;
                 if (more) ra = load_block<DT>(A, wn + lane);
-                quantize_block<K, DT>(rb, wb + lane, c, cb, absmax, packed);
+                quantize_block<K, DT, AT>(rb, wb + lane, c, cb, absmax, packed);
                 wb = wn;
                 if (!more) break;
             }
         }
         for (int64_t t = 2 * bend + (int64_t)blockIdx.x * kThreads + (tid & ~31); t < nh; t += stride) {
             const Raw<DT> r = load_raw<DT, VEC>(A, n, t + lane, t + lane < nh);
-            quantize_half<K, DT>(r, t + lane, t + lane < nh, c, cb, absmax, packed);
+            quantize_half<K, DT, AT>(r, t + lane, t + lane < nh, c, cb, absmax, packed);
         }
         return;
     }
@@ -580,11 +580,11 @@ kbit_quant_kernel(const void* __restrict__ A, int64_t n, const float* __restrict
         Raw<DT> rb;
         while (true) {
             rb = load_full<DT>(A, wbase + stride + lane, wbase + stride + lane < nh_full);
-            quantize_half<K, DT>(ra, wbase + lane, wbase + lane < nh_full, c, cb, absmax, packed);
+            quantize_half<K, DT, AT>(ra, wbase + lane, wbase + lane < nh_full, c, cb, absmax, packed);
             wbase += stride;
             if (wbase >= nh_full) break;
             ra = load_full<DT>(A, wbase + stride + lane, wbase + stride + lane < nh_full);
-            quantize_half<K, DT>(rb, wbase + lane, wbase + lane < nh_full, c, cb, absmax, packed);
+            quantize_half<K, DT, AT>(rb, wbase + lane, wbase + lane < nh_full, c, cb, absmax, packed);
             wbase += stride;
             if (wbase >= nh_full) break;
         }
@@ -592,15 +592,15 @@ kbit_quant_kernel(const void* __restrict__ A, int64_t n, const float* __restrict
     // remaining half blocks (the ragged last block, or everything when the input is unaligned)
     for (int64_t t = nh_full + (int64_t)blockIdx.x * kThreads + (tid & ~31); t < nh; t += stride) {
         const Raw<DT> r = load_raw<DT, false>(A, n, t + lane, t + lane < nh);
-        quantize_half<K, DT>(r, t + lane, t + lane < nh, c, cb, absmax, packed);
+        quantize_half<K, DT, AT>(r, t + lane, t + lane < nh, c, cb, absmax, packed);
     }
 }
 
-template <int K, int DT>
-cudaError_t launch_t(const void* A, int64_t n, const float* codebook, float* absmax,
+template <int K, int DT, typename AT>
+cudaError_t launch_t(const void* A, int64_t n, const float* codebook, AT* absmax,
                      uint32_t* packed, bool vec, cudaStream_t s) {
     const int64_t nh = ((n + 31) >> 5) * 2;
-    auto k = vec ? kbit_quant_kernel<K, DT, true> : kbit_quant_kernel<K, DT, false>;
+    auto k = vec ? kbit_quant_kernel<K, DT, true, AT> : kbit_quant_kernel<K, DT, false, AT>;
     static bool attr_set[2] = {false, false};
     if (!attr_set[vec]) {
         cudaFuncSetAttribute(k, cudaFuncAttributePreferredSharedMemoryCarveout,
@@ -612,8 +612,8 @@ cudaError_t launch_t(const void* A, int64_t n, const float* codebook, float* abs
     return cudaGetLastError();
 }
 
-template <int K>
-cudaError_t launch_k(const void* A, int dt, int64_t n, const float* codebook, float* absmax,
+template <int K, typename AT>
+cudaError_t launch_k(const void* A, int dt, int64_t n, const float* codebook, AT* absmax,
                      uint32_t* packed, bool vec, cudaStream_t s) {
     switch (dt) {
         case F16: return launch_t<K, F16>(A, n, codebook, absmax, packed, vec, s);
@@ -622,16 +622,27 @@ cudaError_t launch_k(const void* A, int dt, int64_t n, const float* codebook, fl
     }
 }
 
-}  // namespace
-
-cudaError_t launch_kbit_quantize(const void* A, int dtype, int64_t n, int K, const float* codebook,
-                                 float* absmax, uint32_t* packed, bool vec, cudaStream_t s) {
+template <typename AT>
+cudaError_t launch_any(const void* A, int dtype, int64_t n, int K, const float* codebook, AT* absmax,
+                       uint32_t* packed, bool vec, cudaStream_t s) {
     switch (K) {
         case 2: return launch_k<2>(A, dtype, n, codebook, absmax, packed, vec, s);
         case 3: return launch_k<3>(A, dtype, n, codebook, absmax, packed, vec, s);
         case 4: return launch_k<4>(A, dtype, n, codebook, absmax, packed, vec, s);
         default: return launch_k<5>(A, dtype, n, codebook, absmax, packed, vec, s);
     }
+}
+
+}  // namespace
+
+cudaError_t launch_kbit_quantize(const void* A, int dtype, int64_t n, int K, const float* codebook,
+                                 float* absmax, uint32_t* packed, bool vec, cudaStream_t s) {
+    return launch_any(A, dtype, n, K, codebook, absmax, packed, vec, s);
+}
+
+cudaError_t launch_kbit_quantize_e4m4(const void* A, int dtype, int64_t n, int K, const float* codebook,
+                                      uint8_t* absmax, uint32_t* packed, bool vec, cudaStream_t s) {
+    return launch_any(A, dtype, n, K, codebook, absmax, packed, vec, s);
 }
 
 }  // namespace bbc

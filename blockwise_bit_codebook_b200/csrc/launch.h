@@ -26,6 +26,14 @@ cudaError_t launch_kbit_dequantize(const uint32_t* packed, const float* absmax,
                                    const float* codebook, int K, int64_t n, int out_dtype,
                                    void* out, bool vec, cudaStream_t s);
 
+// The same two operations with the per-block absmax stored as one E4M4 byte.
+cudaError_t launch_kbit_quantize_e4m4(const void* A, int dtype, int64_t n, int K, const float* codebook,
+                                      uint8_t* absmax, uint32_t* packed, bool vec, cudaStream_t s);
+
+cudaError_t launch_kbit_dequantize_e4m4(const uint32_t* packed, const uint8_t* absmax,
+                                        const float* codebook, int K, int64_t n, int out_dtype,
+                                        void* out, bool vec, cudaStream_t s);
+
 cudaError_t launch_nested_dequantize(const uint8_t* codes, const uint8_t* absmax_q,
                                      const float* code2, const float* absmax2, float offset,
                                      const float* code4, int64_t n, int log2_bs, int out_dtype,

@@ -97,6 +97,34 @@ int kbit_dequantize(const uint32_t* packed, const float* absmax, const float* co
                     int K, int blocksize, int64_t n, int out_dtype, void* out, void* stream);
 
 /*
+ * kbit_quantize_e4m4 / kbit_dequantize_e4m4 - the k-bit codec with each block's
+ * absmax stored as one E4M4 byte instead of an fp32 word (K=4: 4.25 instead of
+ * 5 bits per element).
+ *
+ * Defined by: bitsandbytes k-bit patch series, PATCH 005 "Add vectorized
+ * dequant kernel and E4M4 uint8 absmax support" (encode_absmax_e4m4,
+ * decode_absmax_e4m4, decode_e4m4_absmax, quantize_kbit absmax_format "e4m4").
+ * Code c: e = c >> 4, m = c & 15; value 2^(e-11) * (1 + m/16) for e > 0 and
+ * m * 2^-14 for e == 0 (0.0 at c == 0; range 2^-14 .. 31.0).
+ * Encode of an absmax a: a not > 0 (zero, NaN) -> 0; +inf -> 0xFF (a reading);
+ * otherwise exponent field floor(log2 a) + 11 clamped to [0, 15] (subnormal
+ * when <= 0: m = round(a * 2^14)), mantissa round((a / 2^floor(log2 a) - 1) * 16)
+ * half-to-even, clamped to [0, 15]. At and above 32 the exponent field clamps
+ * while the mantissa stays that of a's own binade, as the page's steps compute.
+ *
+ * kbit_quantize_e4m4: as kbit_quantize; the packed words are identical to its
+ *   (indices use the exact fp32 absmax), absmax_e4m4 [ceil(n/32)] receives the
+ *   codes. Alignment: any uint8 pointer.
+ * kbit_dequantize_e4m4: as kbit_dequantize with each block's scale the exact
+ *   value of its code: out[m] = T(codebook[idx_m] * value(absmax_e4m4[m / 32])).
+ * Errors as kbit_quantize / kbit_dequantize.
+ */
+int kbit_quantize_e4m4(const void* A, int dtype, int64_t n, int K, int blocksize, const float* codebook,
+                       uint8_t* absmax_e4m4, uint32_t* packed, void* stream);
+int kbit_dequantize_e4m4(const uint32_t* packed, const uint8_t* absmax_e4m4, const float* codebook, int K,
+                         int blocksize, int64_t n, int out_dtype, void* out, void* stream);
+
+/*
  * dequantize_4bit_nested - NF4/FP4 dequantization with the nested
  * ("compressed statistics") scale rebuilt inside the decode.
  *

@@ -32,7 +32,8 @@ def declared_functions():
 def test_header_declares_the_boundary():
     names = set(declared_functions())
     assert {"kbit_quantize", "kbit_dequantize", "dequantize_4bit_nested", "dequantize_4bit",
-            "dequantize_4bit_nested_chain", "bbc_nf_codebook", "bbc_last_error"} <= names
+            "dequantize_4bit_nested_chain", "bbc_nf_codebook", "bbc_last_error",
+            "kbit_quantize_e4m4", "kbit_dequantize_e4m4"} <= names
 
 
 def test_library_exports_every_declared_symbol(lib):
@@ -88,6 +89,21 @@ def test_dequantize_validation(lib):
     assert _dq(lib, bs=128) == 2
     assert _dq(lib, out=P(0x1002), dt=2) == 1           # fp32 output at a 2-byte address
     assert _dq(lib, pk=P(0x1001)) == 1
+
+
+def test_e4m4_validation(lib):
+    q = lambda A=FAKE, dtype=1, n=64, K=4, bs=32, am=FAKE: lib.kbit_quantize_e4m4(  # noqa: E731
+        A, dtype, n, K, bs, FAKE, am, FAKE, None)
+    d = lambda am=FAKE, K=4, bs=32, n=64, dt=1, out=FAKE: lib.kbit_dequantize_e4m4(  # noqa: E731
+        FAKE, am, FAKE, K, bs, n, dt, out, None)
+    assert q(A=None) == 1 and q(am=None) == 1 and q(n=0) == 1 and q(K=6) == 1 and q(dtype=4) == 1
+    assert "kbit_quantize_e4m4" in lib.bbc_last_error().decode()
+    assert q(bs=64) == 2
+    assert q(A=P(0x1001)) == 1                           # bf16 input at an odd address
+    assert d(am=None) == 1 and d(out=None) == 1 and d(n=-1) == 1 and d(K=1) == 1 and d(dt=3) == 1
+    assert d(bs=16) == 2
+    assert d(out=P(0x1001), dt=0) == 1
+    assert "kbit_dequantize_e4m4" in lib.bbc_last_error().decode()
 
 
 def test_nested_validation(lib):
