@@ -4,16 +4,17 @@
 // kDequantizeBlockwise_kbit): out[m] = T(codebook[idx_m] * absmax[m / 32]),
 // where idx_m is gathered from the K bit-plane words of block m / 32.
 //
-// B200 layout: a thread owns half a block (16 consecutive elements), so the two
-// threads of a block sit in adjacent lanes and a warp covers 16 blocks (512
-// elements). Each thread reads the block's absmax and K words (the two lanes
-// of a block hit the same addresses), keeps bytes 2h and 2h+1 of every word
-// (one byte permute per word pair), decodes each 4-bit index with one
-// multiply-high bit gather and writes its 16 outputs with one 32-byte store
-// (two for fp32). The loads of the next half block are issued before the
-// current one is decoded, so each thread keeps two round trips in flight. The
-// codebook lives in shared memory: 32 consecutive floats occupy the 32 banks
-// once, so the per-element lookup never conflicts. Persistent grid-stride loop.
+// B200 layout. For 32-byte-aligned output a thread owns a whole block: it reads
+// the block's absmax and its K words once (one vector load when the packed array
+// allows), byte-transposes them with eight permutes into four plane groups (byte
+// j of group q = plane j of elements 8q..8q+7), decodes each 4-bit index with one
+// multiply-high bit gather, and writes 16 outputs per 32-byte store, so every lane
+// writes whole sectors. The next block's words are loaded before the current one
+// is decoded. The ragged last block and unaligned outputs go by half blocks (16
+// elements per thread; the two lanes of a block read the same words and keep
+// bytes 2h, 2h+1). The codebook lives in shared memory: 32 consecutive floats
+// occupy the 32 banks once, so the per-element lookup never conflicts.
+// Persistent grid-stride loops.
 #include "common.cuh"
 #include "launch.h"
 
@@ -59,6 +60,67 @@ __device__ __forceinline__ BlockIn<K> load_block(const uint32_t* packed, const A
     return r;
 }
 
+// One whole block's absmax and K words (block b lies inside the input); one vector load of the
+// words when `packed` allows it (K = 2: 8-byte, K = 4: 16-byte alignment of the array).
+template <int K, typename AT>
+__device__ __forceinline__ BlockIn<K> load_whole(const uint32_t* packed, const AT* absmax, int64_t b,
+                                                 bool vec_words) {
+    BlockIn<K> r;
+    r.am = load_absmax(absmax, b);
+    const uint32_t* wp = packed + b * K;
+    if (K == 4 && vec_words) {
+        const uint4 v = __ldg(reinterpret_cast<const uint4*>(wp));
+        r.w[0] = v.x; r.w[1] = v.y; r.w[2 % K] = v.z; r.w[3 % K] = v.w;
+    } else if (K == 2 && vec_words) {
+        const uint2 v = __ldg(reinterpret_cast<const uint2*>(wp));
+        r.w[0] = v.x; r.w[1 % K] = v.y;
+    } else {
+#pragma unroll
+        for (int j = 0; j < K; j++) r.w[j] = ldg_u32(wp + j);
+    }
+    return r;
+}
+
+// Decode a whole block (32 elements) and store it: byte-transpose the K words into four
+// plane groups (byte j of group q = plane j of elements 8q .. 8q+7), gather each index with one
+// multiply-high and write 64 bytes (128 for fp32) as whole 32-byte sectors.
+template <int K, int DT>
+__device__ __forceinline__ void decode_whole(const BlockIn<K>& in, const char* cbb, char* dst) {
+    const uint32_t w0 = in.w[0], w1 = in.w[1 % K];
+    const uint32_t w2 = K > 2 ? in.w[2 % K] : 0u, w3 = K > 3 ? in.w[3 % K] : 0u;
+    const uint32_t t0 = prmt(w0, w1, 0x5140u), t1 = prmt(w0, w1, 0x7362u);
+    const uint32_t t2 = prmt(w2, w3, 0x5140u), t3 = prmt(w2, w3, 0x7362u);
+    const uint32_t B[4] = {prmt(t0, t2, 0x5410u), prmt(t0, t2, 0x7632u), prmt(t1, t3, 0x5410u),
+                           prmt(t1, t3, 0x7632u)};
+    const uint32_t p4 = K == 5 ? in.w[4 % K] : 0u;             // plane 4: bit i is element i
+    const float am = in.am;
+    // 16 elements per 32-byte store (a whole sector per lane); fp32 needs two per 16
+#pragma unroll
+    for (int g = 0; g < 2; g++) {
+        uint32_t wv[DT == F32 ? 16 : 8];
+#pragma unroll
+        for (int qq = 0; qq < 2; qq++) {
+            const int q = 2 * g + qq;
+            const uint32_t Bq = B[q], Bqs = B[q] << 3;
+            const uint32_t p4q = p4 >> (8 * q);
+            float y[8];
+#define BBC_DQW_ELEM(E)                                                                       \
+            {                                                                                 \
+                uint32_t off = plane_offset4<(E)>(Bq, Bqs);                                  \
+                if constexpr (K == 5) off |= ((E) <= 6 ? (p4q << (6 - (E))) : (p4q >> ((E) - 6))) & 0x40u; \
+                y[E] = __fmul_rn(*reinterpret_cast<const float*>(cbb + off), am);             \
+            }
+            BBC_DQW_ELEM(0) BBC_DQW_ELEM(1) BBC_DQW_ELEM(2) BBC_DQW_ELEM(3)
+            BBC_DQW_ELEM(4) BBC_DQW_ELEM(5) BBC_DQW_ELEM(6) BBC_DQW_ELEM(7)
+#undef BBC_DQW_ELEM
+            pack8<DT>(y, wv + qq * (DT == F32 ? 8 : 4));
+        }
+        char* d = dst + g * 16 * dtype_size(DT);
+        stg_v8(d, wv);
+        if constexpr (DT == F32) stg_v8(d + 32, wv + 8);
+    }
+}
+
 template <int K, int DT, bool VEC, typename AT>
 __global__ void __launch_bounds__(kThreads)
 kbit_dequant_kernel(const uint32_t* __restrict__ packed, const AT* __restrict__ absmax,
@@ -74,7 +136,27 @@ kbit_dequant_kernel(const uint32_t* __restrict__ packed, const AT* __restrict__ 
     const uint32_t sel = (2 * h) | ((4 + 2 * h) << 4) | ((2 * h + 1) << 8) | ((5 + 2 * h) << 12);
     const int64_t stride = (int64_t)gridDim.x * kThreads;
 
-    int64_t H = (int64_t)blockIdx.x * kThreads + threadIdx.x;
+    int64_t H0 = 0;                                                // first half block left
+    if constexpr (VEC) {
+        // whole blocks, one per thread, the next one's words prefetched
+        const int64_t nbf = n >> 5;                                 // blocks entirely inside n
+        const bool vec_words = (reinterpret_cast<uintptr_t>(packed) & (K == 4 ? 15u : 7u)) == 0;
+        int64_t b = (int64_t)blockIdx.x * kThreads + threadIdx.x;
+        if (b < nbf) {
+            BlockIn<K> cb0 = load_whole<K, AT>(packed, absmax, b, vec_words);
+            while (true) {
+                const int64_t bn = b + stride;
+                BlockIn<K> cb1;
+                if (bn < nbf) cb1 = load_whole<K, AT>(packed, absmax, bn, vec_words);
+                decode_whole<K, DT>(cb0, cbb, reinterpret_cast<char*>(out) + b * 32 * dtype_size(DT));
+                b = bn;
+                if (b >= nbf) break;
+                cb0 = cb1;
+            }
+        }
+        H0 = 2 * nbf;
+    }
+    int64_t H = H0 + (int64_t)blockIdx.x * kThreads + threadIdx.x;
     BlockIn<K> cur = load_block<K, AT>(packed, absmax, H >> 1, H < nh);
     for (; H < nh; H += stride) {
         const int64_t Hn = H + stride;

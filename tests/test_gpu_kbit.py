@@ -130,6 +130,27 @@ def test_whole_block_path_with_word_aligned_outputs(bbc, K, dt):
     assert int(pbuf[0]) == 0 and int(pbuf[-3:].abs().sum()) == 0
 
 
+@pytest.mark.parametrize("K", [2, 3, 4, 5])
+@pytest.mark.parametrize("dt", ["f16", "bf16", "f32"])
+def test_dequant_whole_blocks_with_word_aligned_packed(bbc, K, dt):
+    """Aligned output (one block per thread) reading packed words that are only 4-byte
+    aligned: the vector word loads must fall back, results identical."""
+    rng = np.random.default_rng(60 + K)
+    n = 32 * 4096 + 32 * 3 + 21
+    nb = (n + 31) // 32
+    cb = oracle.normal_float_codebook(K)
+    packed = rng.integers(0, 2 ** 32, nb * K, dtype=np.uint64).astype(np.uint32)
+    absmax = rng.uniform(0, 3, nb).astype(np.float32)
+    ref = oracle.kbit_dequantize(packed, absmax, cb, K, n, dt)
+    buf = torch.zeros(nb * K + 1, dtype=torch.int32, device="cuda")
+    buf[1:] = torch.from_numpy(packed.view(np.int32)).cuda()
+    assert buf[1:].data_ptr() % 8 == 4
+    y = bbc.kbit_dequantize(buf[1:], torch.from_numpy(absmax).cuda(), torch.from_numpy(cb).cuda(), K, n,
+                            DTYPES[dt])
+    torch.cuda.synchronize()
+    assert_bits_equal(to_host(y)[:n], ref, f"dequant word-aligned packed K={K} {dt}")
+
+
 # ---------------------------------------------------------------- exactness corners
 
 def exact_thresholds(cb):
