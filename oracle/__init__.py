@@ -12,6 +12,9 @@ it never imports the library. Each function cites the passage it follows:
   and E4M4 uint8 absmax support" (encode_absmax_e4m4, decode_absmax_e4m4 in
   bitsandbytes/functional.py; decode_e4m4_absmax in csrc/ops.cu), and the
   quantize_kbit / dequantize_kbit paths that use it.
+* 4-bit quantize, the nested offset and the General8 absmax compression (the
+  inverse of the nested dequant): readings built from the k-bit rule and the
+  nested decode, since the nested-dequant page does not describe the quantize.
 * nested 4-bit dequant and the plain 4-bit decode of its unfused form: "Fuse
   nested 4-bit scale reconstruction on SM103", Summary and Implementation.
 
@@ -63,6 +66,12 @@ def lib():
         L.orc_e4m4_encode.restype = ct.c_uint8
         L.orc_e4m4_decode.argtypes = [ct.c_uint8]
         L.orc_e4m4_decode.restype = ct.c_float
+        L.orc_quantize_4bit.argtypes = [P, ct.c_int, I64, I64, P, P, P]
+        L.orc_quantize_4bit.restype = ct.c_int
+        L.orc_absmax_offset.argtypes = [P, I64]
+        L.orc_absmax_offset.restype = ct.c_float
+        L.orc_quantize_absmax_nested.argtypes = [P, I64, ct.c_float, P, I64, P, P]
+        L.orc_quantize_absmax_nested.restype = ct.c_int
         L.orc_e4m4_encode_array.argtypes = [P, I64, P]
         L.orc_e4m4_decode_array.argtypes = [P, I64, P]
         _lib = L
@@ -186,6 +195,46 @@ def kbit_quantize_e4m4(A, dtype: str, K: int, codebook):
 def kbit_dequantize_e4m4(packed, absmax_e4m4, codebook, K: int, n: int, dtype: str) -> np.ndarray:
     """dequantize_kbit with a uint8 E4M4 absmax: decode each block's absmax, then the fp32 path."""
     return kbit_dequantize(packed, e4m4_decode(absmax_e4m4), codebook, K, n, dtype)
+
+
+def quantize_4bit(A, dtype: str, blocksize: int, code4):
+    """Per outer block absmax (fp32) and nibble-packed 4-bit codes (uint8[ceil(n/2)], element 2j
+    in the high nibble). A: fp32 values or raw 16-bit patterns."""
+    A = _c(A, np.float32 if dtype == "f32" else np.uint16).reshape(-1)
+    c4 = _c(code4, np.float32)
+    assert c4.size == 16
+    n = A.size
+    absmax = np.empty((n + blocksize - 1) // blocksize, np.float32)
+    codes = np.empty((n + 1) // 2, np.uint8)
+    assert lib().orc_quantize_4bit(_p(A), _DT[dtype], n, blocksize, _p(c4), _p(absmax), _p(codes)) == 0
+    return codes, absmax
+
+
+def absmax_offset(absmax) -> np.float32:
+    """The nested offset: mean of the outer absmax in the fixed binary64 order (chunks of 2048)."""
+    a = _c(absmax, np.float32).reshape(-1)
+    return np.float32(lib().orc_absmax_offset(_p(a), a.size))
+
+
+def quantize_absmax_nested(absmax, offset: float, code2, blocksize2: int = 256):
+    """General8 codes of the centred outer absmax and the per-group inner absmax."""
+    a = _c(absmax, np.float32).reshape(-1)
+    c2 = _c(code2, np.float32)
+    assert c2.size == 256
+    nbi = (a.size + blocksize2 - 1) // blocksize2
+    q = np.empty(a.size, np.uint8)
+    a2 = np.empty(nbi, np.float32)
+    assert lib().orc_quantize_absmax_nested(_p(a), a.size, ct.c_float(offset), _p(c2), blocksize2, _p(q),
+                                            _p(a2)) == 0
+    return q, a2
+
+
+def quantize_4bit_nested(A, dtype: str, blocksize: int, code4, code2, blocksize2: int = 256):
+    """The nested 4-bit state of A: (codes, absmax_q, absmax2, offset)."""
+    codes, absmax = quantize_4bit(A, dtype, blocksize, code4)
+    off = absmax_offset(absmax)
+    q, a2 = quantize_absmax_nested(absmax, float(off), code2, blocksize2)
+    return codes, q, a2, off
 
 
 def nested_scale(code2_val: float, absmax2_val: float, offset: float) -> float:

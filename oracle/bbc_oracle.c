@@ -350,3 +350,82 @@ int orc_dequantize_4bit(const uint8_t* codes, const float* absmax, const float* 
     }
     return 0;
 }
+
+/* ------------------------------------------------------------------ */
+/* 4-bit quantize and nested absmax compression: the inverse of the     */
+/* nested dequant. [P2] describes only the decode ("does not change ... */
+/* quantization formats"); every step below is a reading, listed in     */
+/* the k-bit rule of [P1] applied per outer block, the       */
+/* offset as a mean of the outer absmax, General8 codes of the centred  */
+/* absmax per group of blocksize2 outer blocks.                         */
+/* ------------------------------------------------------------------ */
+
+/*
+ * Per outer block b of bs elements: absmax[b] = max |x| (raw, an fmaxf fold from
+ * the first element, so NaN only when every element is NaN); d = fmaxf(absmax,
+ * 1e-8f); code of element m = first i minimising fabsf(x_m / d - code4[i]) (IEEE
+ * fp32 division, as the k-bit codec). Codes are packed two per byte, element 2j
+ * in the high nibble of codes[j]; for odd n the last low nibble is 0.
+ */
+int orc_quantize_4bit(const void* A, int dtype, int64_t n, int64_t bs, const float* code4,
+                      float* absmax, uint8_t* codes)
+{
+    if (n <= 0 || bs <= 0) return 1;
+    memset(codes, 0, (size_t)((n + 1) / 2));
+    int64_t nbo = (n + bs - 1) / bs;
+    for (int64_t b = 0; b < nbo; b++) {
+        int64_t lo = b * bs, hi = lo + bs < n ? lo + bs : n;
+        float amax = fabsf(load_elem(A, dtype, lo));
+        for (int64_t m = lo + 1; m < hi; m++) amax = fmaxf(amax, fabsf(load_elem(A, dtype, m)));
+        absmax[b] = amax;
+        float d = fmaxf(amax, 1e-8f);
+        for (int64_t m = lo; m < hi; m++) {
+            unsigned idx = (unsigned)orc_nearest_entry(load_elem(A, dtype, m) / d, code4, 16);
+            codes[m / 2] |= (uint8_t)((m % 2 == 0) ? idx << 4 : idx);
+        }
+    }
+    return 0;
+}
+
+#define ORC_OFFSET_CHUNK 2048
+
+/*
+ * The nested offset: the mean of the nbo outer absmax values, in a fixed order in
+ * binary64: partial sums of consecutive chunks of 2048 values, each added in index
+ * order from 0.0, then the partial sums added in chunk order from 0.0; the total
+ * divided by nbo in binary64 and rounded once to binary32.
+ */
+float orc_absmax_offset(const float* absmax, int64_t nbo)
+{
+    double total = 0.0;
+    for (int64_t c = 0; c < nbo; c += ORC_OFFSET_CHUNK) {
+        double s = 0.0;
+        int64_t e = c + ORC_OFFSET_CHUNK < nbo ? c + ORC_OFFSET_CHUNK : nbo;
+        for (int64_t i = c; i < e; i++) s += (double)absmax[i];
+        total += s;
+    }
+    return (float)(total / (double)nbo);
+}
+
+/*
+ * General8 compression of the outer absmax, per group g of bs2 outer blocks:
+ * c_b = fl(absmax[b] - offset); absmax2[g] = max |c_b| over the group (fmaxf fold);
+ * absmax_q[b] = first i minimising fabsf(c_b / fmaxf(absmax2[g], 1e-8f) - code2[i])
+ * over the 256 entries. The nested dequant rebuilds fl(fl(code2[q] * absmax2) + offset).
+ */
+int orc_quantize_absmax_nested(const float* absmax, int64_t nbo, float offset, const float* code2,
+                               int64_t bs2, uint8_t* absmax_q, float* absmax2)
+{
+    if (nbo <= 0 || bs2 <= 0) return 1;
+    int64_t nbi = (nbo + bs2 - 1) / bs2;
+    for (int64_t g = 0; g < nbi; g++) {
+        int64_t lo = g * bs2, hi = lo + bs2 < nbo ? lo + bs2 : nbo;
+        float m = fabsf(absmax[lo] - offset);
+        for (int64_t b = lo + 1; b < hi; b++) m = fmaxf(m, fabsf(absmax[b] - offset));
+        absmax2[g] = m;
+        float d = fmaxf(m, 1e-8f);
+        for (int64_t b = lo; b < hi; b++)
+            absmax_q[b] = (uint8_t)orc_nearest_entry((absmax[b] - offset) / d, code2, 256);
+    }
+    return 0;
+}
