@@ -211,7 +211,8 @@ def quantize_4bit(A, dtype: str, blocksize: int, code4):
 
 
 def absmax_offset(absmax) -> np.float32:
-    """The nested offset: mean of the outer absmax in the fixed binary64 order (chunks of 2048)."""
+    """The nested offset: mean of the outer absmax, a pairwise binary64 sum over the values
+    zero-padded to a power of two, divided by the count, rounded once to fp32."""
     a = _c(absmax, np.float32).reshape(-1)
     return np.float32(lib().orc_absmax_offset(_p(a), a.size))
 

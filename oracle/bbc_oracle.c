@@ -387,24 +387,26 @@ int orc_quantize_4bit(const void* A, int dtype, int64_t n, int64_t bs, const flo
     return 0;
 }
 
-#define ORC_OFFSET_CHUNK 2048
+/* Pairwise binary64 sum of a[lo .. lo+len) (len a power of two), entries at or beyond n
+ * counting as 0.0: the sum of the lower half plus the sum of the upper half. */
+static double orc_tree_sum(const float* a, int64_t n, int64_t lo, int64_t len)
+{
+    if (lo >= n) return 0.0;
+    if (len == 1) return (double)a[lo];
+    int64_t h = len / 2;
+    return orc_tree_sum(a, n, lo, h) + orc_tree_sum(a, n, lo + h, h);
+}
 
 /*
- * The nested offset: the mean of the nbo outer absmax values, in a fixed order in
- * binary64: partial sums of consecutive chunks of 2048 values, each added in index
- * order from 0.0, then the partial sums added in chunk order from 0.0; the total
- * divided by nbo in binary64 and rounded once to binary32.
+ * The nested offset: the mean of the nbo outer absmax values, summed in binary64 by a
+ * fixed binary tree (the values zero-padded to the next power of two, each node the sum
+ * of its two halves), divided by nbo in binary64 and rounded once to binary32.
  */
 float orc_absmax_offset(const float* absmax, int64_t nbo)
 {
-    double total = 0.0;
-    for (int64_t c = 0; c < nbo; c += ORC_OFFSET_CHUNK) {
-        double s = 0.0;
-        int64_t e = c + ORC_OFFSET_CHUNK < nbo ? c + ORC_OFFSET_CHUNK : nbo;
-        for (int64_t i = c; i < e; i++) s += (double)absmax[i];
-        total += s;
-    }
-    return (float)(total / (double)nbo);
+    int64_t p = 1;
+    while (p < nbo) p <<= 1;
+    return (float)(orc_tree_sum(absmax, nbo, 0, p) / (double)nbo);
 }
 
 /*

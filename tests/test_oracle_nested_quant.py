@@ -3,7 +3,7 @@
 The nested-dequant page ("Fuse nested 4-bit scale reconstruction on SM103") defines only the
 decode; the quantize steps are readings: the k-bit rule of the bitsandbytes k-bit series
 (absmax, fmaxf(absmax, 1e-8f), IEEE division, first nearest entry) per outer block, the offset as
-the mean of the outer absmax (fixed binary64 order), and General8 codes of the centred absmax
+the mean of the outer absmax (pairwise binary64 sum), and General8 codes of the centred absmax
 per group of 256 outer blocks. Each pin checks against something other than the oracle's own
 code: numpy brute force on small inputs, exact rationals, the already-pinned dequant, and the
 error bounds the k-bit pages state.
@@ -110,11 +110,18 @@ def test_quantize_error_bound(bs):
 
 def test_offset_is_the_mean():
     rng = np.random.default_rng(4)
-    for nbo in (1, 7, 2048, 2049, 10000):
+    for nbo in (1, 2, 3, 7, 2048, 2049, 10000, 70001):
         a = np.abs(rng.standard_normal(nbo)).astype(np.float32) * np.float32(0.05)
         off = oracle.absmax_offset(a)
         exact = sum(Fraction(float(v)) for v in a) / nbo
         # within one ulp of the exact mean (the binary64 sums lose far less than that)
+        # and equal to a pairwise binary64 sum done here with numpy's own float64 adds
+        p = 1 << max(0, (nbo - 1).bit_length())
+        v = np.zeros(p, np.float64)
+        v[:nbo] = a
+        while v.size > 1:
+            v = v[0::2] + v[1::2]
+        assert off == np.float32(v[0] / nbo), nbo
         ulp = np.spacing(np.float32(float(exact)))
         assert abs(Fraction(float(off)) - exact) <= Fraction(float(ulp)), nbo
     assert oracle.absmax_offset(np.full(5000, 0.3, np.float32)) == np.float32(0.3)   # equal values
