@@ -48,7 +48,8 @@ def parse_args():
     ap.add_argument("--ops", default=None,
                     help="comma-separated subset of quantize_k3,dequantize_k3,quantize_k5,"
                          "dequantize_k5,nested_nf4_bs64, or the E4M4-absmax ops "
-                         "{quantize,dequantize}_k{3,4,5}_e4m4 (profiling)")
+                         "{quantize,dequantize}_k{3,4,5}_e4m4, or quantize_4bit_nf4_bs64, "
+                         "quantize_nested_nf4_bs64 (profiling)")
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -78,14 +79,23 @@ def op_bytes(kind, n, K=None, out_size=2, bs=NESTED_BS):
         return nb * K * 4 + nb + n * out_size
     nbo = (n + bs - 1) // bs
     nbi = (nbo + 255) // 256
+    if kind == "quantize_4bit":                   # bf16 in; nibble codes and fp32 absmax out
+        return n * 2 + (n + 1) // 2 + nbo * 4
+    if kind == "quantize_nested":                 # bf16 in; codes, absmax_q, absmax2, offset out
+        return n * 2 + (n + 1) // 2 + nbo + nbi * 4 + 4
+    nbo = (n + bs - 1) // bs
+    nbi = (nbo + 255) // 256
     return (n + 1) // 2 + nbo + nbi * 4 + n * out_size
 
 
 ALL_OPS = [("quantize_k3", "quantize", 3), ("dequantize_k3", "dequantize", 3),
            ("quantize_k5", "quantize", 5), ("dequantize_k5", "dequantize", 5),
            ("nested_nf4_bs64", "nested", None)]
+# Kernel launches per op (the nested quantize: 4-bit codes, two offset kernels, compression).
+LAUNCHES = {"quantize_nested": 4}
 # Selectable with --ops (not part of the default step): the E4M4-absmax codec.
-EXTRA_OPS = [(f"{k}_k{K}_e4m4", f"{k}_e4m4", K) for K in (3, 4, 5) for k in ("quantize", "dequantize")]
+EXTRA_OPS = [(f"{k}_k{K}_e4m4", f"{k}_e4m4", K) for K in (3, 4, 5) for k in ("quantize", "dequantize")] + \
+    [("quantize_4bit_nf4_bs64", "quantize_4bit", None), ("quantize_nested_nf4_bs64", "quantize_nested", None)]
 
 
 def workload_ops(only=None):
@@ -120,6 +130,7 @@ def load_peaks():
 def kernel_source_hash(kind):
     files = {"quantize": ["kbit_quant.cu"], "dequantize": ["kbit_dequant.cu"],
              "quantize_e4m4": ["kbit_quant.cu"], "dequantize_e4m4": ["kbit_dequant.cu"],
+             "quantize_4bit": ["kbit_quant.cu"], "quantize_nested": ["kbit_quant.cu", "nested_quant.cu"],
              "nested": ["nested_dequant.cu"]}[kind] + ["common.cuh"]
     h = hashlib.sha256()
     for f in files:
@@ -270,6 +281,16 @@ def run_bbc(args):
     code4 = cbs[4]
     code2_dev, code4_dev = torch.from_numpy(code2).to(dev), cb_dev[4]
     nout = torch.empty(n, dtype=torch.bfloat16, device=dev)
+    kinds = {kind for _, kind, _ in ops}
+    if kinds & {"quantize_4bit", "quantize_nested"}:
+        nbo4 = (n + NESTED_BS - 1) // NESTED_BS
+        q4_codes = torch.empty((n + 1) // 2, dtype=torch.uint8, device=dev)
+        q4_absmax = torch.empty(nbo4, dtype=torch.float32, device=dev)
+        nq_out = (torch.empty((n + 1) // 2, dtype=torch.uint8, device=dev),
+                  torch.empty(nbo4, dtype=torch.uint8, device=dev),
+                  torch.empty((nbo4 + 255) // 256, dtype=torch.float32, device=dev),
+                  torch.empty(1, dtype=torch.float32, device=dev))
+        nq_ws = torch.empty(bbc.quantize_4bit_nested_workspace_bytes(n, NESTED_BS), dtype=torch.uint8, device=dev)
     stream = torch.cuda.current_stream(dev)
 
     def launch(kind, K, xin=x, cin=codes, qin=q, a2in=a2, pk=packed, am=absmax, ou=outs, no=nout):
@@ -281,6 +302,11 @@ def run_bbc(args):
             bbc.kbit_quantize_e4m4(xin, K, cb_dev[K], absmax=absmax8[K], packed=pk[K], stream=stream)
         elif kind == "dequantize_e4m4":
             bbc.kbit_dequantize_e4m4(pk[K], absmax8[K], cb_dev[K], K, n, torch.bfloat16, out=ou[K], stream=stream)
+        elif kind == "quantize_4bit":
+            bbc.quantize_4bit(xin, NESTED_BS, code4_dev, absmax=q4_absmax, codes=q4_codes, stream=stream)
+        elif kind == "quantize_nested":
+            bbc.quantize_4bit_nested(xin, NESTED_BS, code4_dev, code2_dev, workspace=nq_ws, out=nq_out,
+                                     stream=stream)
         else:
             bbc.dequantize_4bit_nested(cin, qin, code2_dev, a2in, float(off), code4_dev, n, NESTED_BS,
                                        torch.bfloat16, out=no, stream=stream)
@@ -353,7 +379,7 @@ def run_bbc(args):
               "data": "synthetic", "config": {**workload_desc(n, ops),
                                               "parallelism": f"replicas{world}" if world > 1 else "single"},
               "per_kernel": per_kernel, "roofline": roofline,
-              "gpu_launches": len(ops) * args.steps, "clocks": clocks}
+              "gpu_launches": sum(LAUNCHES.get(kind, 1) for _, kind, _ in ops) * args.steps, "clocks": clocks}
 
     # ---- end to end through the public API with host buffers
     if not args.no_e2e:
@@ -370,8 +396,12 @@ def run_bbc(args):
         dx, dcodes, dq, da2 = torch.empty_like(x), torch.empty_like(codes), torch.empty_like(q), torch.empty_like(a2)
         h2d = sum(t.numel() * t.element_size() for t in (hx, hcodes, hq, ha2)) + \
             sum(t.numel() * 4 for t in hcb.values())
+        q4_dev = ([q4_codes, q4_absmax] if "quantize_4bit" in kinds else []) + \
+            (list(nq_out) if "quantize_nested" in kinds else [])
+        q4_host = [(t, torch.empty_like(t, device="cpu").pin_memory()) for t in q4_dev]
         d2h = sum(t.numel() * t.element_size() for K in ks for t in (packed[K], outs[K])) + \
-            sum(absmax[K].numel() * 4 for K in k32) + sum(absmax8[K].numel() for K in k8) + nout.numel() * 2
+            sum(absmax[K].numel() * 4 for K in k32) + sum(absmax8[K].numel() for K in k8) + nout.numel() * 2 + \
+            sum(t.numel() * t.element_size() for t in q4_dev)
 
         def e2e_step():
             dx.copy_(hx, non_blocking=True)
@@ -390,6 +420,8 @@ def run_bbc(args):
             for K in k8:
                 h_out["absmax8"][K].copy_(absmax8[K], non_blocking=True)
             h_out["nested"].copy_(nout, non_blocking=True)
+            for t, h in q4_host:
+                h.copy_(t, non_blocking=True)
 
         e2e_step()
         torch.cuda.synchronize()

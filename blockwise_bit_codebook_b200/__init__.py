@@ -11,6 +11,8 @@ library's CUDA kernels. torch is used for device memory and streams only.
     dequantize_4bit_nested(codes, absmax_q, code2, absmax2, offset, code4,
                            n, blocksize, dtype)         -> out
     dequantize_4bit(codes, absmax, code4, n, blocksize, dtype)  -> out
+    quantize_4bit(A, blocksize, code4)                  -> (codes, absmax)
+    quantize_4bit_nested(A, blocksize, code4, code2)    -> (codes, absmax_q, absmax2, offset)
     dequantize_4bit_nested_chain(...)   the unfused three-launch form (same result)
     bbc_nf_codebook(K)                                  -> np.float32[2^K] (host)
 
@@ -32,6 +34,9 @@ from ._native import (  # noqa: F401
     kbit_dequantize_e4m4,
     kbit_quantize,
     kbit_quantize_e4m4,
+    quantize_4bit,
+    quantize_4bit_nested,
+    quantize_4bit_nested_workspace_bytes,
     library_path,
     load_library,
 )

@@ -36,6 +36,12 @@ def load_library():
     L.kbit_quantize.restype = I
     L.kbit_dequantize.argtypes = [P, P, P, I, I, I64, I, P, P]
     L.kbit_dequantize.restype = I
+    L.quantize_4bit.argtypes = [P, I, I64, I, P, P, P, P]
+    L.quantize_4bit.restype = I
+    L.quantize_4bit_nested_workspace_bytes.argtypes = [I64, I]
+    L.quantize_4bit_nested_workspace_bytes.restype = ct.c_size_t
+    L.quantize_4bit_nested.argtypes = [P, I, I64, I, P, P, I, P, P, P, P, P, ct.c_size_t, P]
+    L.quantize_4bit_nested.restype = I
     L.kbit_quantize_e4m4.argtypes = [P, I, I64, I, I, P, P, P, P]
     L.kbit_quantize_e4m4.restype = I
     L.kbit_dequantize_e4m4.argtypes = [P, P, P, I, I, I64, I, P, P]
@@ -149,6 +155,51 @@ def kbit_dequantize_e4m4(packed, absmax, codebook, K: int, n: int, dtype, out=No
                                 _stream(stream, packed.device))
     _check("kbit_dequantize_e4m4", st)
     return out
+
+
+def quantize_4bit(A, blocksize: int, code4, absmax=None, codes=None, stream=None):
+    """4-bit codes (uint8[ceil(n/2)], element 2j high nibble) and fp32 absmax per outer block."""
+    import torch
+    L = load_library()
+    n = A.numel()
+    nbo = (n + blocksize - 1) // blocksize if blocksize > 0 else 1
+    if absmax is None:
+        absmax = torch.empty(max(nbo, 1), dtype=torch.float32, device=A.device)
+    if codes is None:
+        codes = torch.empty(max((n + 1) // 2, 1), dtype=torch.uint8, device=A.device)
+    st = L.quantize_4bit(_ptr(A), _dt(A.dtype), n, blocksize, _ptr(code4), _ptr(absmax), _ptr(codes),
+                         _stream(stream, A.device))
+    _check("quantize_4bit", st)
+    return codes, absmax
+
+
+def quantize_4bit_nested_workspace_bytes(n: int, blocksize: int) -> int:
+    return int(load_library().quantize_4bit_nested_workspace_bytes(n, blocksize))
+
+
+def quantize_4bit_nested(A, blocksize: int, code4, code2, blocksize2: int = 256, workspace=None,
+                         out=None, stream=None):
+    """The nested 4-bit state of A: (codes, absmax_q, absmax2, offset) with offset a 1-element
+    CUDA tensor. `out` may hold preallocated (codes, absmax_q, absmax2, offset)."""
+    import torch
+    L = load_library()
+    n = A.numel()
+    nbo = (n + blocksize - 1) // blocksize if blocksize > 0 else 1
+    nbi = (nbo + blocksize2 - 1) // blocksize2 if blocksize2 > 0 else 1
+    if out is None:
+        out = (torch.empty(max((n + 1) // 2, 1), dtype=torch.uint8, device=A.device),
+               torch.empty(max(nbo, 1), dtype=torch.uint8, device=A.device),
+               torch.empty(max(nbi, 1), dtype=torch.float32, device=A.device),
+               torch.empty(1, dtype=torch.float32, device=A.device))
+    codes, absmax_q, absmax2, offset = out
+    wsb = quantize_4bit_nested_workspace_bytes(n, blocksize) if n > 0 else 0
+    if workspace is None:
+        workspace = torch.empty(max(wsb, 1), dtype=torch.uint8, device=A.device)
+    st = L.quantize_4bit_nested(_ptr(A), _dt(A.dtype), n, blocksize, _ptr(code4), _ptr(code2), blocksize2,
+                                _ptr(codes), _ptr(absmax_q), _ptr(absmax2), _ptr(offset), _ptr(workspace),
+                                workspace.numel() * workspace.element_size(), _stream(stream, A.device))
+    _check("quantize_4bit_nested", st)
+    return codes, absmax_q, absmax2, offset
 
 
 def dequantize_4bit_nested(codes, absmax_q, code2, absmax2, offset: float, code4, n: int,

@@ -155,6 +155,55 @@ int dequantize_4bit(const uint8_t* codes, const float* absmax, const float* code
                        "dequantize_4bit launch");
 }
 
+int quantize_4bit(const void* A, int dtype, int64_t n, int blocksize, const float* code4, float* absmax,
+                  uint8_t* codes, void* stream) {
+    const char* fn = "quantize_4bit";
+    if (!A || !code4 || !absmax || !codes) return fail(BBC_ERR_INVALID, "%s: null pointer argument", fn);
+    if (n <= 0) return fail(BBC_ERR_INVALID, "%s: n must be >= 1 (got %lld)", fn, (long long)n);
+    if (!valid_dtype(dtype)) return fail(BBC_ERR_INVALID, "%s: bad dtype %d", fn, dtype);
+    const int log2_bs = log2_blocksize(blocksize);
+    if (log2_bs < 0)
+        return fail(BBC_ERR_INVALID, "%s: blocksize must be a power of two in [32, 4096] (got %d)", fn, blocksize);
+    if (!aligned(A, elem_size(dtype)) || !aligned(absmax, 4) || !aligned(code4, 4))
+        return fail(BBC_ERR_INVALID, "%s: pointer not aligned to its element size", fn);
+    const bool vec = aligned(A, 32) && aligned(codes, 16);     // 256-bit loads, 8/16-byte code stores
+    return cuda_status(bbc::launch_quantize_4bit(A, dtype, n, log2_bs, code4, absmax, codes, vec,
+                                                 static_cast<cudaStream_t>(stream)),
+                       "quantize_4bit launch");
+}
+
+size_t quantize_4bit_nested_workspace_bytes(int64_t n, int blocksize) {
+    const int log2_bs = log2_blocksize(blocksize);
+    if (n <= 0 || log2_bs < 0) return 0;
+    return bbc::nested_quant_workspace_bytes(n, log2_bs);
+}
+
+int quantize_4bit_nested(const void* A, int dtype, int64_t n, int blocksize, const float* code4,
+                         const float* code2, int blocksize2, uint8_t* codes, uint8_t* absmax_q, float* absmax2,
+                         float* offset, void* workspace, size_t workspace_bytes, void* stream) {
+    const char* fn = "quantize_4bit_nested";
+    if (!A || !code4 || !code2 || !codes || !absmax_q || !absmax2 || !offset || !workspace)
+        return fail(BBC_ERR_INVALID, "%s: null pointer argument", fn);
+    if (n <= 0) return fail(BBC_ERR_INVALID, "%s: n must be >= 1 (got %lld)", fn, (long long)n);
+    if (!valid_dtype(dtype)) return fail(BBC_ERR_INVALID, "%s: bad dtype %d", fn, dtype);
+    const int log2_bs = log2_blocksize(blocksize);
+    if (log2_bs < 0)
+        return fail(BBC_ERR_INVALID, "%s: blocksize must be a power of two in [32, 4096] (got %d)", fn, blocksize);
+    if (blocksize2 != 256)
+        return fail(BBC_ERR_UNSUPPORTED, "%s: blocksize2 must be 256 (got %d)", fn, blocksize2);
+    const size_t need = bbc::nested_quant_workspace_bytes(n, log2_bs);
+    if (workspace_bytes < need)
+        return fail(BBC_ERR_INVALID, "%s: workspace holds %zu bytes, %zu needed", fn, workspace_bytes, need);
+    if (!aligned(A, elem_size(dtype)) || !aligned(code4, 4) || !aligned(code2, 4) || !aligned(absmax2, 4) ||
+        !aligned(offset, 4) || !aligned(workspace, 256))
+        return fail(BBC_ERR_INVALID, "%s: pointer not aligned (elements; workspace to 256 bytes)", fn);
+    const bool vec = aligned(A, 32) && aligned(codes, 16);
+    return cuda_status(bbc::launch_quantize_4bit_nested(A, dtype, n, log2_bs, code4, code2, codes, absmax_q,
+                                                        absmax2, offset, workspace, vec,
+                                                        static_cast<cudaStream_t>(stream)),
+                       "quantize_4bit_nested launch");
+}
+
 int dequantize_4bit_nested_chain(const uint8_t* codes, const uint8_t* absmax_q, const float* code2,
                                  const float* absmax2, float offset, const float* code4,
                                  int64_t n, int blocksize, int blocksize2, int out_dtype, void* out,

@@ -105,6 +105,66 @@ __device__ __forceinline__ uint32_t nearest_entry(float xn, const float* cb) {
     return idx;
 }
 
+// Per-CTA set-up of the exact threshold method for a 2^K-entry codebook (every thread of the
+// CTA calls it; the result is CTA-uniform): loads the codebook into cb[], decides whether the
+// fast path applies (finite, strictly ascending, spaced >= 2^-19 (1 + max|c|), at most one
+// threshold per table cell), finds the thresholds by bisection and fills the 256-cell table
+// (8 replicas) whose entries are {-T, h_T, pattern(L), pattern(L + 1)}: the bit-plane spread of
+// the index for the k-bit codec, the index itself for nibble codes.
+template <int K, bool NIBBLE>
+__device__ __forceinline__ bool setup_exact_table(const float* __restrict__ codebook, float* cb, float* thr,
+                                                  int* fast_ok, uint4* lut) {
+    constexpr int NE = 1 << K;
+    const int tid = threadIdx.x;
+    if (tid < 32) {
+        const float c = tid < NE ? codebook[tid] : 0.0f;
+        cb[tid] = c;
+        float mag = tid < NE ? fabsf(c) : 0.0f;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) mag = max_nan(mag, __shfl_xor_sync(0xffffffffu, mag, o));
+        const float D = __fadd_rn(1.0f, mag);
+        const float prev = __shfl_up_sync(0xffffffffu, c, 1);
+        bool ok = true;
+        if (tid < NE) {
+            ok = fabsf(c) <= FLT_MAX;                                  // finite (false for NaN)
+            if (tid > 0) ok = ok && (__fsub_rn(c, prev) >= __fmul_rn(D, 0x1p-19f));
+        }
+        ok = ok && (D <= FLT_MAX);
+        const bool fast = __all_sync(0xffffffffu, ok);
+        if (tid == 0) *fast_ok = fast ? 1 : 0;
+        if (fast && tid >= 1 && tid < NE) thr[tid] = bisect_threshold(prev, c);
+    }
+    __syncthreads();
+    int multi = 0;
+    if (*fast_ok) {
+        for (int cell = tid; cell < kCells; cell += kThreads) {
+            const int cs = cell < 128 ? cell : cell - 256;
+            const float wlo = __fsub_rn((float)cs * 0.015625f, 0x1p-13f + 0x1p-12f);
+            const float whi = __fadd_rn((float)(cs + 1) * 0.015625f, 0x1p-13f + 0x1p-12f);
+            int below = 0, rel = 0, relj = 0;
+            for (int j = 1; j < NE; j++) {
+                const float T = thr[j];
+                if (T < wlo) below++;
+                else if (T <= whi) { rel++; relj = j; }
+            }
+            float negT = __int_as_float(0xff800000), half = 0.0f;     // -inf, 0: never crossed
+            if (rel == 1) {
+                const float T = thr[relj];
+                negT = -T;
+                half = __fmul_rn(__fsub_rn(T, key_f32(f32_key(T) - 1)), 0.5f);
+            }
+            multi |= rel > 1;
+            const uint32_t p0 = NIBBLE ? (uint32_t)below : spread<K>((uint32_t)below);
+            const uint32_t p1 = NIBBLE ? (uint32_t)below + 1 : spread<K>((uint32_t)below + 1);
+            const uint4 ent = make_uint4(__float_as_uint(negT), __float_as_uint(half), p0, p1);
+            // the 8 lanes of a store phase write 8 different replicas: distinct banks
+#pragma unroll
+            for (int r = 0; r < kReplicas; r++) lut[cell * kReplicas + ((r + tid) & (kReplicas - 1))] = ent;
+        }
+    }
+    return (*fast_ok != 0) && !__syncthreads_or(multi);
+}
+
 // Raw input words of one half block (16 elements): 8 words for 16-bit types, 16 for fp32.
 template <int DT>
 struct Raw { uint32_t w[DT == F32 ? 16 : 8]; };
@@ -481,53 +541,9 @@ kbit_quant_kernel(const void* __restrict__ A, int64_t n, const float* __restrict
     const int lane = tid & 31;
 
     // ---- per-CTA set-up: codebook check, thresholds, lookup table ----
-    if (tid < 32) {
-        const float c = tid < NE ? codebook[tid] : 0.0f;
-        cb[tid] = c;
-        float mag = tid < NE ? fabsf(c) : 0.0f;
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) mag = max_nan(mag, __shfl_xor_sync(0xffffffffu, mag, o));
-        const float D = __fadd_rn(1.0f, mag);
-        const float prev = __shfl_up_sync(0xffffffffu, c, 1);
-        bool ok = true;
-        if (tid < NE) {
-            ok = fabsf(c) <= FLT_MAX;                                  // finite (false for NaN)
-            if (tid > 0) ok = ok && (__fsub_rn(c, prev) >= __fmul_rn(D, 0x1p-19f));
-        }
-        ok = ok && (D <= FLT_MAX);
-        const bool fast = __all_sync(0xffffffffu, ok);
-        if (tid == 0) fast_ok = fast ? 1 : 0;
-        if (fast && tid >= 1 && tid < NE) thr[tid] = bisect_threshold(prev, c);
-    }
-    __syncthreads();
-    int multi = 0;
-    if (fast_ok) {
-        for (int cell = tid; cell < kCells; cell += kThreads) {
-            const int cs = cell < 128 ? cell : cell - 256;
-            const float wlo = __fsub_rn((float)cs * 0.015625f, 0x1p-13f + 0x1p-12f);
-            const float whi = __fadd_rn((float)(cs + 1) * 0.015625f, 0x1p-13f + 0x1p-12f);
-            int below = 0, rel = 0, relj = 0;
-            for (int j = 1; j < NE; j++) {
-                const float T = thr[j];
-                if (T < wlo) below++;
-                else if (T <= whi) { rel++; relj = j; }
-            }
-            float negT = __int_as_float(0xff800000), half = 0.0f;     // -inf, 0: never crossed
-            if (rel == 1) {
-                const float T = thr[relj];
-                negT = -T;
-                half = __fmul_rn(__fsub_rn(T, key_f32(f32_key(T) - 1)), 0.5f);
-            }
-            multi |= rel > 1;
-            const uint4 ent = make_uint4(__float_as_uint(negT), __float_as_uint(half),
-                                         spread<K>((uint32_t)below), spread<K>((uint32_t)below + 1));
-            // the 8 lanes of a store phase write 8 different replicas: distinct banks
-#pragma unroll
-            for (int r = 0; r < kReplicas; r++) lut[cell * kReplicas + ((r + tid) & (kReplicas - 1))] = ent;
-        }
-    }
+    const bool fast_cb = setup_exact_table<K, false>(codebook, cb, thr, &fast_ok, lut);
     LoopCtx c;
-    c.fast_cb = (fast_ok != 0) && !__syncthreads_or(multi);
+    c.fast_cb = fast_cb;
     c.lut = reinterpret_cast<const char*>(lut);
     c.lut_s = (uint32_t)__cvta_generic_to_shared(lut);
     c.lane16 = (uint32_t)(lane & 7) << 4;
@@ -596,6 +612,187 @@ kbit_quant_kernel(const void* __restrict__ A, int64_t n, const float* __restrict
     }
 }
 
+// ---- 4-bit codes with nibble packing (the inverse of the plain / nested 4-bit decode) ----
+//
+// A thread owns 64 bytes of input: 32 elements of a 16-bit type or 16 of fp32 (EPT), so an
+// outer block of bs elements spans bs / EPT threads, and a CTA iteration covers 256 * EPT
+// elements (at least one block of 4096). Per thread: two 32-byte loads (the next slice
+// prefetched into registers), the NaN-propagating and the NaN-ignoring max of |x| reduced over
+// the block's lanes (xor-shuffles, then shared memory for blocks wider than a warp), the exact
+// threshold search per element, and EPT / 2 bytes of codes stored at once.
+
+template <int DT> constexpr int kEpt = DT == F32 ? 16 : 32;    // elements per thread (64 bytes)
+
+struct Raw16w { uint32_t w[16]; };
+
+// The 64-byte slice U of A: vector loads when it lies inside the input, else element-wise
+// loads with zeros past n.
+template <int DT, bool VEC>
+__device__ __forceinline__ Raw16w load_slice(const void* A, int64_t n, int64_t U, bool active) {
+    Raw16w r;
+    constexpr int E = kEpt<DT>;
+    const int64_t m0 = U * E;
+    if (VEC && active && m0 + E <= n) {
+        const char* p = reinterpret_cast<const char*>(A) + U * 64;
+        const u32x8 a = ldg_stream_v8(p), b = ldg_stream_v8(p + 32);
+#pragma unroll
+        for (int i = 0; i < 8; i++) { r.w[i] = a.v[i]; r.w[8 + i] = b.v[i]; }
+    } else if constexpr (DT == F32) {
+        const float* a = reinterpret_cast<const float*>(A);
+#pragma unroll
+        for (int e = 0; e < 16; e++) r.w[e] = (active && m0 + e < n) ? __float_as_uint(a[m0 + e]) : 0u;
+    } else {
+        const uint16_t* a = reinterpret_cast<const uint16_t*>(A);
+#pragma unroll
+        for (int i = 0; i < 16; i++) {
+            const uint32_t lo = (active && m0 + 2 * i < n) ? (uint32_t)a[m0 + 2 * i] : 0u;
+            const uint32_t hi = (active && m0 + 2 * i + 1 < n) ? (uint32_t)a[m0 + 2 * i + 1] : 0u;
+            r.w[i] = lo | (hi << 16);
+        }
+    }
+    return r;
+}
+
+// Element e of the slice as fp32 (exact widening).
+template <int DT>
+__device__ __forceinline__ float slice_elem(const Raw16w& r, int e) {
+    if constexpr (DT == F32) return __uint_as_float(r.w[e]);
+    else {
+        float lo, hi;
+        widen_pair<DT>(r.w[e >> 1], lo, hi);
+        return (e & 1) ? hi : lo;
+    }
+}
+
+// NaN-propagating and NaN-ignoring max of |x| over the slice.
+template <int DT>
+__device__ __forceinline__ void slice_absmax2(const Raw16w& r, float& mnan, float& mnum) {
+    if constexpr (DT == F32) {
+        const float* xf = reinterpret_cast<const float*>(r.w);
+        float a = fabsf(xf[0]), b = fabsf(xf[0]);
+#pragma unroll
+        for (int e = 1; e < 16; e++) { a = max_nan(a, fabsf(xf[e])); b = fmaxf(b, fabsf(xf[e])); }
+        mnan = a; mnum = b;
+    } else {
+        uint32_t p = pair_absmax<DT>(r.w[0], r.w[1]), q;
+        // NaN-ignoring packed max (maxNum: a NaN operand yields the other one)
+        if constexpr (DT == BF16) asm("max.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(q) : "r"(r.w[0]), "r"(r.w[1]));
+        else asm("max.xorsign.abs.f16x2 %0, %1, %2;" : "=r"(q) : "r"(r.w[0]), "r"(r.w[1]));
+#pragma unroll
+        for (int i = 2; i < 16; i++) {
+            p = pair_absmax<DT>(p, r.w[i]);
+            if constexpr (DT == BF16) asm("max.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(q) : "r"(q), "r"(r.w[i]));
+            else asm("max.xorsign.abs.f16x2 %0, %1, %2;" : "=r"(q) : "r"(q), "r"(r.w[i]));
+        }
+        float lo, hi;
+        widen_pair<DT>(p, lo, hi);
+        mnan = max_nan(fabsf(lo), fabsf(hi));
+        widen_pair<DT>(q, lo, hi);
+        mnum = fmaxf(fabsf(lo), fabsf(hi));
+    }
+}
+
+// Bit position of element e's nibble within its 32-bit word of codes (little-endian bytes,
+// element 2j in the high nibble of byte j).
+__host__ __device__ constexpr int nib_shift(int e) { return 8 * ((e & 7) >> 1) + ((e & 1) ? 0 : 4); }
+
+template <int DT, bool VEC>
+__global__ void __launch_bounds__(kThreads, 2)
+quant4_kernel(const void* __restrict__ A, int64_t n, int log2_bs, const float* __restrict__ code4,
+              float* __restrict__ absmax, uint8_t* __restrict__ codes) {
+    constexpr int E = kEpt<DT>;
+    constexpr int NW = E / 8;                                   // code words per thread
+    __shared__ __align__(16) uint4 lut[kCells * kReplicas];    // 32 KB
+    __shared__ float cb[32];
+    __shared__ float thr[33];
+    __shared__ int fast_ok;
+    __shared__ float2 red[2][kThreads / 32];                    // per-warp maxima, two buffers
+
+    const int tid = threadIdx.x;
+    const int lane = tid & 31, warp = tid >> 5;
+    LoopCtx c;
+    c.fast_cb = setup_exact_table<4, true>(code4, cb, thr, &fast_ok, lut);
+    c.lut = reinterpret_cast<const char*>(lut);
+    c.lut_s = (uint32_t)__cvta_generic_to_shared(lut);
+    c.lane16 = (uint32_t)(lane & 7) << 4;
+
+    const int tpb_log2 = log2_bs - (DT == F32 ? 4 : 5);        // threads per outer block
+    const int tpb = 1 << tpb_log2;
+    const int64_t nu = (n + E - 1) / E;                         // 64-byte slices
+    const int64_t nbytes = (n + 1) >> 1;
+    const int64_t stride = (int64_t)gridDim.x * kThreads;
+    int buf = 0;
+    int64_t base = (int64_t)blockIdx.x * kThreads;
+    Raw16w cur = load_slice<DT, VEC>(A, n, base + tid, base + tid < nu);
+    for (; base < nu; base += stride) {                         // CTA-uniform
+        const int64_t U = base + tid;
+        const bool active = U < nu;
+        const int64_t m0 = U * E;
+        const int64_t Un = U + stride;
+        const Raw16w nxt = load_slice<DT, VEC>(A, n, Un, Un < nu);
+        float mnan, mnum;
+        slice_absmax2<DT>(cur, mnan, mnum);
+        for (int o = 1; o < tpb && o < 32; o <<= 1) {
+            mnan = max_nan(mnan, __shfl_xor_sync(0xffffffffu, mnan, o));
+            mnum = fmaxf(mnum, __shfl_xor_sync(0xffffffffu, mnum, o));
+        }
+        if (tpb > 32) {                                          // blocks wider than a warp
+            if (lane == 0) red[buf][warp] = make_float2(mnan, mnum);
+            __syncthreads();
+            const int w0 = warp & ~((tpb >> 5) - 1);
+            mnan = red[buf][w0].x; mnum = red[buf][w0].y;
+            for (int w = 1; w < (tpb >> 5); w++) {
+                mnan = max_nan(mnan, red[buf][w0 + w].x);
+                mnum = fmaxf(mnum, red[buf][w0 + w].y);
+            }
+            buf ^= 1;
+        }
+        const bool special = !(mnan <= 0x1p125f);
+        const float amax = mnum;
+        const float d = fmaxf(amax, 1e-8f);
+
+        uint32_t acc[NW];
+#pragma unroll
+        for (int g = 0; g < NW; g++) acc[g] = 0u;
+        if (!special && c.fast_cb) {
+            const float rs = __fmul_rn(rcp_approx(d), 8192.0f);
+#pragma unroll
+            for (int e = 0; e < E; e += 2) {
+                const float x0 = slice_elem<DT>(cur, e), x1 = slice_elem<DT>(cur, e + 1);
+                const float2 f = __ffma2_rn(make_float2(x0, x1), make_float2(rs, rs),
+                                            make_float2(12582912.0f, 12582912.0f));
+                const uint4 t0 = lut_entry(c, __float_as_uint(f.x));
+                const uint4 t1 = lut_entry(c, __float_as_uint(f.y));
+                const float v0 = __fmaf_rn(__uint_as_float(t0.y), d, __fmaf_rn(__uint_as_float(t0.x), d, x0));
+                const float v1 = __fmaf_rn(__uint_as_float(t1.y), d, __fmaf_rn(__uint_as_float(t1.x), d, x1));
+                acc[e / 8] += (v0 > 0.0f ? t0.w : t0.z) << nib_shift(e);
+                acc[(e + 1) / 8] += (v1 > 0.0f ? t1.w : t1.z) << nib_shift(e + 1);
+            }
+        } else {
+#pragma unroll
+            for (int e = 0; e < E; e++)
+                acc[e / 8] += nearest_entry<16>(__fdiv_rn(slice_elem<DT>(cur, e), d), cb) << nib_shift(e);
+        }
+        if (active) {
+            uint8_t* cp = codes + U * (E / 2);
+            if (VEC && m0 + E <= n) {
+                if constexpr (NW == 4) stg_v4(cp, acc[0], acc[1], acc[2], acc[3]);
+                else asm volatile("st.global.v2.u32 [%0], {%1,%2};" :: "l"(cp), "r"(acc[0]), "r"(acc[NW - 1]) : "memory");
+            } else {
+                // ragged end (or unaligned codes): nibbles of elements >= n are 0, bytes >= nbytes unwritten
+#pragma unroll
+                for (int e = 0; e < E; e++)
+                    if (m0 + e >= n) acc[e / 8] &= ~(15u << nib_shift(e));
+#pragma unroll
+                for (int j = 0; j < E / 2; j++)
+                    if (U * (E / 2) + j < nbytes) cp[j] = (uint8_t)(acc[j / 4] >> (8 * (j & 3)));
+            }
+            if ((tid & (tpb - 1)) == 0) absmax[U >> tpb_log2] = amax;
+        }
+        cur = nxt;
+    }
+}
+
 template <int K, int DT, typename AT>
 cudaError_t launch_t(const void* A, int64_t n, const float* codebook, AT* absmax,
                      uint32_t* packed, bool vec, cudaStream_t s) {
@@ -638,6 +835,21 @@ cudaError_t launch_any(const void* A, int dtype, int64_t n, int K, const float* 
 cudaError_t launch_kbit_quantize(const void* A, int dtype, int64_t n, int K, const float* codebook,
                                  float* absmax, uint32_t* packed, bool vec, cudaStream_t s) {
     return launch_any(A, dtype, n, K, codebook, absmax, packed, vec, s);
+}
+
+cudaError_t launch_quantize_4bit(const void* A, int dtype, int64_t n, int log2_bs, const float* code4,
+                                 float* absmax, uint8_t* codes, bool vec, cudaStream_t s) {
+    auto pick = [&](auto kv, auto kn) { return vec ? kv : kn; };
+    void (*k)(const void*, int64_t, int, const float*, float*, uint8_t*);
+    switch (dtype) {
+        case F16: k = pick(quant4_kernel<F16, true>, quant4_kernel<F16, false>); break;
+        case BF16: k = pick(quant4_kernel<BF16, true>, quant4_kernel<BF16, false>); break;
+        default: k = pick(quant4_kernel<F32, true>, quant4_kernel<F32, false>); break;
+    }
+    const int64_t nu = (n + 15) >> 4;                           // upper bound on 64-byte slices
+    const int grid = persistent_grid(k, kThreads, 0, nu, kThreads);
+    k<<<grid, kThreads, 0, s>>>(A, n, log2_bs, code4, absmax, codes);
+    return cudaGetLastError();
 }
 
 cudaError_t launch_kbit_quantize_e4m4(const void* A, int dtype, int64_t n, int K, const float* codebook,

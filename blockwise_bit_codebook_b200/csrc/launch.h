@@ -26,6 +26,19 @@ cudaError_t launch_kbit_dequantize(const uint32_t* packed, const float* absmax,
                                    const float* codebook, int K, int64_t n, int out_dtype,
                                    void* out, bool vec, cudaStream_t s);
 
+// 4-bit codes (two per byte, element 2j in the high nibble) and fp32 absmax per outer block of
+// 2^log2_bs elements (32 .. 4096).
+cudaError_t launch_quantize_4bit(const void* A, int dtype, int64_t n, int log2_bs, const float* code4,
+                                 float* absmax, uint8_t* codes, bool vec, cudaStream_t s);
+
+// The nested 4-bit state of A: codes, General8 codes of the centred outer absmax, inner absmax
+// per 256 outer blocks and the offset (device scalar). `workspace` holds
+// nested_quant_workspace_bytes(n, log2_bs) bytes (the fp32 outer absmax and binary64 partials).
+size_t nested_quant_workspace_bytes(int64_t n, int log2_bs);
+cudaError_t launch_quantize_4bit_nested(const void* A, int dtype, int64_t n, int log2_bs, const float* code4,
+                                        const float* code2, uint8_t* codes, uint8_t* absmax_q, float* absmax2,
+                                        float* offset, void* workspace, bool vec, cudaStream_t s);
+
 // The same two operations with the per-block absmax stored as one E4M4 byte.
 cudaError_t launch_kbit_quantize_e4m4(const void* A, int dtype, int64_t n, int K, const float* codebook,
                                       uint8_t* absmax, uint32_t* packed, bool vec, cudaStream_t s);

@@ -1,0 +1,162 @@
+// Nested 4-bit quantize: the inverse of the nested dequant.
+//
+// The nested-dequant pull request ("Fuse nested 4-bit scale reconstruction on SM103") defines
+// the decode: scale_b = fl(fl(code2[absmax_q[b]] * absmax2[b / 256]) + offset). Producing that
+// state takes three steps here (each a stated reading of the pages):
+//   1. 4-bit codes and the fp32 absmax of every outer block (quant4_kernel, kbit_quant.cu):
+//      the k-bit rule of the bitsandbytes k-bit series per outer block.
+//   2. offset = the mean of the outer absmax: a pairwise binary64 sum over the values
+//      zero-padded to a power of two (each tree node the sum of its two halves), divided by
+//      the block count, rounded once to fp32 (tree_sum_kernel). IEEE addition is commutative
+//      and adding +0.0 is exact, so a CTA that sums 8 leaves per thread as a tree, combines
+//      lanes by xor-shuffles and warps in shared memory computes exactly the nodes of that
+//      tree; each level of 2048 nodes is one launch.
+//   3. per group of 256 outer blocks, c_b = fl(absmax_b - offset): absmax2 = max |c_b| and
+//      absmax_q_b = the first nearest General8 entry to fl(c_b / fmaxf(absmax2, 1e-8f))
+//      (absmax_compress_kernel). For an ascending table the nearest entry is found exactly by
+//      binary search: fl(|xn - t_i|) does not increase up to the last t_i <= xn and does not
+//      decrease after it, so the minimum is at one of those two neighbours and the first index
+//      holding it is found by walking down a plateau of equal distances. Any other table takes
+//      the rule verbatim over all 256 entries.
+#include <cfloat>
+
+#include "common.cuh"
+#include "launch.h"
+
+namespace bbc {
+
+namespace {
+
+constexpr int kTree = 2048;            // tree leaves per CTA (256 threads x 8)
+constexpr int kGroup = 256;            // outer blocks per inner absmax
+
+// One level of the pairwise sum: node b = sum of in[2048 b .. 2048 b + 2048) (zeros past count)
+// as a binary tree. With a single CTA this is the root: it writes the fp32 mean instead.
+template <typename T>
+__global__ void __launch_bounds__(256)
+tree_sum_kernel(const T* __restrict__ in, int64_t count, double* __restrict__ nodes, int64_t nbo,
+                float* __restrict__ offset) {
+    __shared__ double ws[8];
+    const int64_t base = (int64_t)blockIdx.x * kTree + threadIdx.x * 8;
+    double v[8];
+#pragma unroll
+    for (int j = 0; j < 8; j++) v[j] = base + j < count ? (double)in[base + j] : 0.0;
+    double s = __dadd_rn(__dadd_rn(__dadd_rn(v[0], v[1]), __dadd_rn(v[2], v[3])),
+                         __dadd_rn(__dadd_rn(v[4], v[5]), __dadd_rn(v[6], v[7])));
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) s = __dadd_rn(s, __shfl_xor_sync(0xffffffffu, s, o));
+    if ((threadIdx.x & 31) == 0) ws[threadIdx.x >> 5] = s;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        const double r = __dadd_rn(__dadd_rn(__dadd_rn(ws[0], ws[1]), __dadd_rn(ws[2], ws[3])),
+                                   __dadd_rn(__dadd_rn(ws[4], ws[5]), __dadd_rn(ws[6], ws[7])));
+        if (gridDim.x == 1) *offset = __double2float_rn(__ddiv_rn(r, (double)nbo));
+        else nodes[blockIdx.x] = r;
+    }
+}
+
+// First index minimising fl(|xn - t_i|) over an ascending 256-entry table (see the header).
+__device__ __forceinline__ uint32_t nearest_ascending(float xn, const float* t) {
+    if (xn != xn) return 0;                                     // NaN: no distance is below +inf
+    int p = t[255] <= xn ? 255 : -1;                             // last index with t[p] <= xn
+    if (p < 0) {
+#pragma unroll
+        for (int step = 128; step >= 1; step >>= 1)              // p + step <= 254 throughout
+            if (t[p + step] <= xn) p += step;
+    }
+    if (p < 0) return 0;
+    const float dp = fabsf(__fsub_rn(xn, t[p]));
+    if (p < 255 && fabsf(__fsub_rn(xn, t[p + 1])) < dp) return (uint32_t)p + 1;
+    int i = p;
+    while (i > 0 && fabsf(__fsub_rn(xn, t[i - 1])) == dp) i--;
+    return (uint32_t)i;
+}
+
+__device__ __forceinline__ uint32_t nearest_any(float xn, const float* t) {
+    float best = __int_as_float(0x7f800000);
+    uint32_t idx = 0;
+    for (int i = 0; i < 256; i++) {
+        const float dist = fabsf(__fsub_rn(xn, t[i]));
+        if (dist < best) { best = dist; idx = (uint32_t)i; }
+    }
+    return idx;
+}
+
+// One warp per group of 256 outer blocks (8 per lane), persistent over the groups.
+__global__ void __launch_bounds__(256)
+absmax_compress_kernel(const float* __restrict__ absmax, int64_t nbo, const float* __restrict__ offset_p,
+                       const float* __restrict__ code2, uint8_t* __restrict__ absmax_q,
+                       float* __restrict__ absmax2) {
+    __shared__ float t[256];
+    t[threadIdx.x] = code2[threadIdx.x];
+    __syncthreads();
+    const bool ascending = __syncthreads_and(threadIdx.x == 255 || t[threadIdx.x] <= t[threadIdx.x + 1]);
+    const float off = *offset_p;
+    const int lane = threadIdx.x & 31;
+    const int64_t ngroups = (nbo + kGroup - 1) / kGroup;
+    const int64_t wstride = (int64_t)gridDim.x * (blockDim.x >> 5);
+    for (int64_t g = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); g < ngroups; g += wstride) {
+        float cv[8];
+        float m = __int_as_float(0x7fc00000);                   // NaN: ignored by fmaxf
+#pragma unroll
+        for (int j = 0; j < 8; j++) {
+            const int64_t b = g * kGroup + lane + 32 * j;
+            cv[j] = b < nbo ? __fsub_rn(__ldg(absmax + b), off) : __int_as_float(0x7fc00000);
+            m = fmaxf(m, fabsf(cv[j]));
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+        if (lane == 0) absmax2[g] = m;
+        const float d = fmaxf(m, 1e-8f);
+#pragma unroll
+        for (int j = 0; j < 8; j++) {
+            const int64_t b = g * kGroup + lane + 32 * j;
+            if (b < nbo) {
+                const float xn = __fdiv_rn(cv[j], d);
+                absmax_q[b] = (uint8_t)(ascending ? nearest_ascending(xn, t) : nearest_any(xn, t));
+            }
+        }
+    }
+}
+
+}  // namespace
+
+namespace {
+int64_t tree_nodes(int64_t count) { return (count + kTree - 1) / kTree; }
+int64_t absmax_bytes(int64_t nbo) { return ((nbo * 4 + 255) / 256) * 256; }
+}  // namespace
+
+size_t nested_quant_workspace_bytes(int64_t n, int log2_bs) {
+    const int64_t nbo = (n + (1ll << log2_bs) - 1) >> log2_bs;
+    const int64_t s1 = tree_nodes(nbo), s2 = tree_nodes(s1);
+    return (size_t)(absmax_bytes(nbo) + (s1 + s2) * 8);
+}
+
+cudaError_t launch_quantize_4bit_nested(const void* A, int dtype, int64_t n, int log2_bs, const float* code4,
+                                        const float* code2, uint8_t* codes, uint8_t* absmax_q, float* absmax2,
+                                        float* offset, void* workspace, bool vec, cudaStream_t s) {
+    const int64_t nbo = (n + (1ll << log2_bs) - 1) >> log2_bs;
+    float* absmax = static_cast<float*>(workspace);
+    double* buf_a = reinterpret_cast<double*>(static_cast<char*>(workspace) + absmax_bytes(nbo));
+    double* buf_b = buf_a + tree_nodes(nbo);
+    cudaError_t e = launch_quantize_4bit(A, dtype, n, log2_bs, code4, absmax, codes, vec, s);
+    if (e != cudaSuccess) return e;
+    // the pairwise sum, one level per launch; the single-CTA level writes the offset
+    int64_t count = tree_nodes(nbo);
+    tree_sum_kernel<float><<<(unsigned)count, 256, 0, s>>>(absmax, nbo, buf_a, nbo, offset);
+    const double* in = buf_a;
+    double* out = buf_b;
+    while (count > 1) {
+        const int64_t next = tree_nodes(count);
+        tree_sum_kernel<double><<<(unsigned)next, 256, 0, s>>>(in, count, out, nbo, offset);
+        in = out;
+        out = out == buf_b ? buf_a : buf_b;        // a level never outgrows the one before it
+        count = next;
+    }
+    const int64_t ngroups = (nbo + kGroup - 1) / kGroup;
+    const int grid = persistent_grid(absmax_compress_kernel, 256, 0, ngroups, 8);
+    absmax_compress_kernel<<<grid, 256, 0, s>>>(absmax, nbo, offset, code2, absmax_q, absmax2);
+    return cudaGetLastError();
+}
+
+}  // namespace bbc

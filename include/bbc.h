@@ -1,12 +1,16 @@
 /*
  * bbc.h - C ABI of the blockwise bit-codebook library (NVIDIA B200, sm_100a).
  *
- * Two operations on weight tensors, both defined by the pages this library
- * follows (cited per entry point below):
+ * Operations on weight tensors, defined by the pages this library follows
+ * (cited per entry point below):
  *   1. k-bit blockwise codebook quantization (K = 2..5, blocksize 32) and its
- *      inverse, with bit-plane packing of the codes;
+ *      inverse, with bit-plane packing of the codes, with an fp32 or an E4M4
+ *      byte absmax per block;
  *   2. nested NF4/FP4 dequantization, where each outer block's fp32 scale is
- *      rebuilt from a General8-coded absmax inside the value-decode kernel.
+ *      rebuilt from a General8-coded absmax inside the value-decode kernel,
+ *      its unfused three-launch form, and the plain 4-bit decode;
+ *   3. the inverse of 2: 4-bit quantization and the nested absmax state
+ *      (readings: the pages give only the decode).
  *
  * Conventions for every entry point:
  *   - Buffer pointers are DEVICE pointers (memory of the current CUDA device)
@@ -30,6 +34,7 @@
 #ifndef BBC_H
 #define BBC_H
 
+#include <stddef.h>
 #include <stdint.h>
 
 #ifdef __cplusplus
@@ -169,6 +174,58 @@ int dequantize_4bit_nested(const uint8_t* codes, const uint8_t* absmax_q, const 
  */
 int dequantize_4bit(const uint8_t* codes, const float* absmax, const float* code4, int64_t n,
                     int blocksize, int out_dtype, void* out, void* stream);
+
+/*
+ * quantize_4bit - 4-bit codes and fp32 absmax per outer block: the inverse of
+ * dequantize_4bit.
+ *
+ * Defined by: the pages give only the decode (pull request "Fuse nested 4-bit
+ * scale reconstruction on SM103"); the encode is the k-bit rule of the
+ * bitsandbytes k-bit series (PATCH 001 quantize_kbit_ref) applied per outer
+ * block of `blocksize` elements, a reading:
+ *   absmax[b] = max |x| over the block (raw; NaN only if every element is NaN)
+ *   d         = fmaxf(absmax[b], 1e-8f)
+ *   code_m    = first i minimising fabsf(fl(x_m / d) - code4[i])
+ * packed two per byte, element 2j in the high nibble of codes[j] (the unused
+ * low nibble of an odd n is 0).
+ *
+ *   A        [n] elements of dtype.   n >= 1.   blocksize: power of two in [32, 4096].
+ *   code4    [16] fp32 (NF4, FP4 or any table; ascending well-spaced tables take the
+ *            fast exact path, others the rule verbatim).
+ *   absmax   [ceil(n/blocksize)] fp32 out.   codes [ceil(n/2)] uint8 out.
+ * Fast paths need A 32-byte and codes 8-byte aligned; other alignments give the
+ * same results more slowly.
+ */
+int quantize_4bit(const void* A, int dtype, int64_t n, int blocksize, const float* code4, float* absmax,
+                  uint8_t* codes, void* stream);
+
+/*
+ * quantize_4bit_nested - the nested ("compressed statistics") 4-bit state of A,
+ * the inverse of dequantize_4bit_nested.
+ *
+ * Defined by: the same decode; the encode steps are readings (no page gives them):
+ *   1. codes and fp32 absmax per outer block as quantize_4bit;
+ *   2. offset = mean of the outer absmax, computed in binary64 in a fixed order
+ *      (partial sums of consecutive chunks of 2048 values in index order, then the
+ *      partials in chunk order; divided by the block count; rounded once to fp32);
+ *   3. per group of blocksize2 = 256 outer blocks, c_b = fl(absmax_b - offset):
+ *      absmax2[g] = max |c_b|,  absmax_q[b] = first i minimising
+ *      fabsf(fl(c_b / fmaxf(absmax2[g], 1e-8f)) - code2[i]).
+ * dequantize_4bit_nested then rebuilds each scale as fl(fl(code2[q] * absmax2) + offset).
+ *
+ *   code2      [256] fp32 General8 table.   blocksize2: must be 256.
+ *   codes      [ceil(n/2)] uint8 out.   absmax_q [ceil(n/blocksize)] uint8 out.
+ *   absmax2    [ceil(ceil(n/blocksize)/256)] fp32 out.
+ *   offset     one fp32 out, a DEVICE pointer (read it back before dequantizing).
+ *   workspace  DEVICE scratch of quantize_4bit_nested_workspace_bytes(n, blocksize)
+ *              bytes, 256-byte aligned, caller-owned, not overlapping any argument.
+ * Four launches on `stream`. Errors as quantize_4bit; a workspace that is too small
+ * is BBC_ERR_INVALID, blocksize2 != 256 BBC_ERR_UNSUPPORTED.
+ */
+size_t quantize_4bit_nested_workspace_bytes(int64_t n, int blocksize);
+int quantize_4bit_nested(const void* A, int dtype, int64_t n, int blocksize, const float* code4,
+                         const float* code2, int blocksize2, uint8_t* codes, uint8_t* absmax_q, float* absmax2,
+                         float* offset, void* workspace, size_t workspace_bytes, void* stream);
 
 /*
  * dequantize_4bit_nested_chain - the unfused three-launch form of

@@ -33,7 +33,8 @@ def test_header_declares_the_boundary():
     names = set(declared_functions())
     assert {"kbit_quantize", "kbit_dequantize", "dequantize_4bit_nested", "dequantize_4bit",
             "dequantize_4bit_nested_chain", "bbc_nf_codebook", "bbc_last_error",
-            "kbit_quantize_e4m4", "kbit_dequantize_e4m4"} <= names
+            "kbit_quantize_e4m4", "kbit_dequantize_e4m4", "quantize_4bit", "quantize_4bit_nested",
+            "quantize_4bit_nested_workspace_bytes"} <= names
 
 
 def test_library_exports_every_declared_symbol(lib):
@@ -104,6 +105,27 @@ def test_e4m4_validation(lib):
     assert d(bs=16) == 2
     assert d(out=P(0x1001), dt=0) == 1
     assert "kbit_dequantize_e4m4" in lib.bbc_last_error().decode()
+
+
+def test_quantize_4bit_validation(lib):
+    q = lambda A=FAKE, dt=1, n=64, bs=64, cb=FAKE, am=FAKE, co=FAKE: lib.quantize_4bit(  # noqa: E731
+        A, dt, n, bs, cb, am, co, None)
+    assert q(A=None) == 1 and q(co=None) == 1 and q(am=None) == 1 and q(n=0) == 1 and q(dt=3) == 1
+    for bs in (0, 16, 48, 8192):
+        assert q(bs=bs) == 1
+    assert "blocksize" in lib.bbc_last_error().decode()
+    assert q(A=P(0x1001), dt=0) == 1 and q(am=P(0x1002)) == 1
+    ws = lib.quantize_4bit_nested_workspace_bytes
+    assert ws(0, 64) == 0 and ws(100, 48) == 0
+    nbo = (10 ** 6 + 63) // 64
+    s1 = (nbo + 2047) // 2048
+    assert ws(10 ** 6, 64) == ((nbo * 4 + 255) // 256) * 256 + (s1 + (s1 + 2047) // 2048) * 8
+    nq = lambda ws_ptr=P(0x100000), wsb=1 << 20, bs2=256, n=4096, off=FAKE: lib.quantize_4bit_nested(  # noqa: E731
+        FAKE, 1, n, 64, FAKE, FAKE, bs2, FAKE, FAKE, FAKE, off, ws_ptr, wsb, None)
+    assert nq(ws_ptr=None) == 1 and nq(off=None) == 1 and nq(n=-1) == 1
+    assert nq(bs2=128) == 2
+    assert nq(wsb=10) == 1 and "workspace" in lib.bbc_last_error().decode()
+    assert nq(ws_ptr=P(0x100010)) == 1                   # workspace not 256-byte aligned
 
 
 def test_nested_validation(lib):
