@@ -15,6 +15,8 @@ it never imports the library. Each function cites the passage it follows:
 * 4-bit quantize, the nested offset and the General8 absmax compression (the
   inverse of the nested dequant): readings built from the k-bit rule and the
   nested decode, since the nested-dequant page does not describe the quantize.
+* the dequant fused into its linear consumer (the page's dequantize-plus-linear
+  public-path controls): nested_dequantize, then a float64 matmul (a library step).
 * nested 4-bit dequant and the plain 4-bit decode of its unfused form: "Fuse
   nested 4-bit scale reconstruction on SM103", Summary and Implementation.
 
@@ -236,6 +238,22 @@ def quantize_4bit_nested(A, dtype: str, blocksize: int, code4, code2, blocksize2
     off = absmax_offset(absmax)
     q, a2 = quantize_absmax_nested(absmax, float(off), code2, blocksize2)
     return codes, q, a2, off
+
+
+def linear_4bit_nested(X, x_dtype: str, N: int, K: int, state, code2, code4, blocksize: int,
+                       blocksize2: int = 256):
+    """Y = X @ W^T with W[N, K] the nested 4-bit weight dequantized to x_dtype (nested_dequantize
+    of the flattened N*K codes, rounded to the activation type as the unfused path materialises
+    it). Returns (Y64, S): the float64 product (each product of two 16-bit values is exact in
+    binary64; the binary64 sums lose at most K * 2^-53 relative) and S = |X| @ |W|^T, the scale of
+    the accumulation error bound. X: [M, K] raw 16-bit patterns of x_dtype."""
+    codes, absmax_q, absmax2, offset = state
+    Wb = nested_dequantize(codes, absmax_q, code2, absmax2, float(offset), code4, N * K, blocksize,
+                           blocksize2, x_dtype)
+    widen = f16_bits_to_f32 if x_dtype == "f16" else bf16_bits_to_f32
+    W = widen(Wb).astype(np.float64).reshape(N, K)
+    Xf = widen(_c(X, np.uint16).reshape(-1)).astype(np.float64).reshape(-1, K)
+    return Xf @ W.T, np.abs(Xf) @ np.abs(W).T
 
 
 def nested_scale(code2_val: float, absmax2_val: float, offset: float) -> float:
