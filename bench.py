@@ -53,6 +53,9 @@ def parse_args():
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--linear", action="store_true",
+                    help="fused nested 4-bit dequant + linear vs dequant then cuBLAS, on the pull "
+                         "request's public-path control shapes (one JSON line per case)")
     ap.add_argument("--nested-matrix", action="store_true",
                     help="fused vs three-launch nested dequant on the pull request's 24-cell matrix")
     ap.add_argument("--cpu-seconds", type=float, default=15.0,
@@ -453,6 +456,78 @@ def run_bbc(args):
 
 # ----------------------------------------------------------------------------- nested matrix
 
+def run_linear(args):
+    """Fused nested 4-bit dequant + linear (linear_4bit_nested) against the unfused sequence
+    (the library's fused nested dequant into a materialised weight, then torch.matmul, i.e.
+    cuBLAS) on the pull request's public-path control shapes: M = 1 and 8 (N = K = 4096) and
+    M = 32 (N = 4096 and 11008, K = 4096); bf16 activations, NF4, outer blocksize 64. CUDA events
+    around CUDA-graph replays of 200 repetitions (device time, no host launch overhead),
+    alternating order, 7 rounds, medians. Algorithmic bytes of the fused kernel: codes,
+    absmax_q, absmax2, X and Y (the weight is never written)."""
+    import torch
+
+    import blockwise_bit_codebook_b200 as bbc
+    from blockwise_bit_codebook_b200 import synthetic
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    bbc.load_library()
+    peak, peak_kind = load_peaks()
+    code4 = torch.from_numpy(bbc.bbc_nf_codebook(4)).to(dev)
+    code2 = torch.from_numpy(synthetic.general8_table()).to(dev)
+    bs = NESTED_BS
+    for (M, N, K, label) in [(1, 4096, 4096, "recurrent grad_A M=1"), (8, 4096, 4096, "recurrent grad_A M=8"),
+                             (32, 4096, 4096, "fallback forward M=32"),
+                             (32, 11008, 4096, "fallback forward M=32 N=11008")]:
+        codes, q, a2, off = synthetic.nested_state(N * K, bs, seed=3, device=dev)
+        x = synthetic.weights(M * K, std=1.0, seed=4, dtype=torch.bfloat16, device=dev).reshape(M, K)
+        w = torch.empty(N * K, dtype=torch.bfloat16, device=dev)
+        y_f = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+        y_u = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+        fused = lambda: bbc.linear_4bit_nested(x, codes, q, code2, a2, float(off), code4, N, bs, out=y_f)  # noqa: E731
+
+        def unfused():
+            bbc.dequantize_4bit_nested(codes, q, code2, a2, float(off), code4, N * K, bs, torch.bfloat16, out=w)
+            torch.matmul(x, w.view(N, K).t(), out=y_u)
+        for i in range(20):
+            (fused if i % 2 == 0 else unfused)()
+        torch.cuda.synchronize()
+        # Host-side call overhead (Python, ctypes) exceeds these kernels' device time, so each
+        # variant's repetitions are captured once in a CUDA graph and the replays are timed.
+        reps = 200
+        graphs = {}
+        for name, fn in (("fused", fused), ("unfused", unfused)):
+            gr = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(gr):
+                for _ in range(reps):
+                    fn()
+            graphs[name] = gr
+        torch.cuda.synchronize()
+        samples = {"fused": [], "unfused": []}
+        for rnd in range(7):
+            order = ["fused", "unfused"]
+            if rnd % 2:
+                order.reverse()
+            for name in order:
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                e0.record()
+                graphs[name].replay()
+                e1.record()
+                torch.cuda.synchronize()
+                samples[name].append(e0.elapsed_time(e1) / reps * 1e3)
+        del graphs
+        med = {k: statistics.median(v) for k, v in samples.items()}
+        nbo = (N * K + bs - 1) // bs
+        nbytes = N * K // 2 + nbo + ((nbo + 255) // 256) * 4 + M * K * 2 + M * N * 2
+        rel = float((y_f.float() - y_u.float()).abs().max() / y_u.float().abs().max())
+        print(json.dumps({"case": label, "M": M, "N": N, "K": K, "dtype": "bf16", "format": "nf4", "blocksize": bs,
+                          "fused_us_median": round(med["fused"], 2), "unfused_us_median": round(med["unfused"], 2),
+                          "unfused_over_fused": round(med["unfused"] / med["fused"], 3),
+                          "fused_GBs": round(nbytes / med["fused"] / 1e3, 1),
+                          "fused_frac_of_measured_hbm": round(nbytes / med["fused"] / 1e3 / peak, 4),
+                          "max_rel_diff_vs_unfused": round(rel, 6)}), flush=True)
+
+
 def run_nested_matrix(args):
     """Fused nested dequant vs the unfused three-launch chain on the pull request's matrix.
 
@@ -580,7 +655,9 @@ def run_reference(args):
 
 if __name__ == "__main__":
     a = parse_args()
-    if a.nested_matrix:
+    if a.linear:
+        run_linear(a)
+    elif a.nested_matrix:
         run_nested_matrix(a)
     elif a.impl == "reference":
         run_reference(a)

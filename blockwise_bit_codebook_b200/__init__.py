@@ -38,5 +38,6 @@ from ._native import (  # noqa: F401
     quantize_4bit_nested,
     quantize_4bit_nested_workspace_bytes,
     library_path,
+    linear_4bit_nested,
     load_library,
 )

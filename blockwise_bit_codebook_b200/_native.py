@@ -42,6 +42,8 @@ def load_library():
     L.quantize_4bit_nested_workspace_bytes.restype = ct.c_size_t
     L.quantize_4bit_nested.argtypes = [P, I, I64, I, P, P, I, P, P, P, P, P, ct.c_size_t, P]
     L.quantize_4bit_nested.restype = I
+    L.linear_4bit_nested.argtypes = [P, I, I64, I64, I64, P, P, P, P, ct.c_float, P, I, I, P, P]
+    L.linear_4bit_nested.restype = I
     L.kbit_quantize_e4m4.argtypes = [P, I, I64, I, I, P, P, P, P]
     L.kbit_quantize_e4m4.restype = I
     L.kbit_dequantize_e4m4.argtypes = [P, P, P, I, I, I64, I, P, P]
@@ -200,6 +202,22 @@ def quantize_4bit_nested(A, blocksize: int, code4, code2, blocksize2: int = 256,
                                 workspace.numel() * workspace.element_size(), _stream(stream, A.device))
     _check("quantize_4bit_nested", st)
     return codes, absmax_q, absmax2, offset
+
+
+def linear_4bit_nested(X, codes, absmax_q, code2, absmax2, offset: float, code4, N: int, blocksize: int,
+                       blocksize2: int = 256, out=None, stream=None):
+    """Y = X @ W^T for X [M, K] (fp16/bf16, M <= 32) and W [N, K] the nested 4-bit weight, decoded
+    in registers (never materialised). Returns Y [M, N] in X's dtype."""
+    import torch
+    L = load_library()
+    M, K = X.shape
+    if out is None:
+        out = torch.empty((M, N), dtype=X.dtype, device=X.device)
+    st = L.linear_4bit_nested(_ptr(X), _dt(X.dtype), M, N, K, _ptr(codes), _ptr(absmax_q), _ptr(code2),
+                              _ptr(absmax2), ct.c_float(offset), _ptr(code4), blocksize, blocksize2, _ptr(out),
+                              _stream(stream, X.device))
+    _check("linear_4bit_nested", st)
+    return out
 
 
 def dequantize_4bit_nested(codes, absmax_q, code2, absmax2, offset: float, code4, n: int,

@@ -204,6 +204,33 @@ int quantize_4bit_nested(const void* A, int dtype, int64_t n, int blocksize, con
                        "quantize_4bit_nested launch");
 }
 
+int linear_4bit_nested(const void* X, int dtype, int64_t M, int64_t N, int64_t K, const uint8_t* codes,
+                       const uint8_t* absmax_q, const float* code2, const float* absmax2, float offset,
+                       const float* code4, int blocksize, int blocksize2, void* Y, void* stream) {
+    const char* fn = "linear_4bit_nested";
+    if (!X || !codes || !absmax_q || !code2 || !absmax2 || !code4 || !Y)
+        return fail(BBC_ERR_INVALID, "%s: null pointer argument", fn);
+    if (M <= 0 || N <= 0 || K <= 0)
+        return fail(BBC_ERR_INVALID, "%s: M, N, K must be >= 1 (got %lld, %lld, %lld)", fn, (long long)M,
+                    (long long)N, (long long)K);
+    if (dtype != BBC_F16 && dtype != BBC_BF16)
+        return fail(BBC_ERR_UNSUPPORTED, "%s: activations must be fp16 or bf16 (got dtype %d)", fn, dtype);
+    if (M > 32 || N % 16 != 0 || K % 64 != 0)
+        return fail(BBC_ERR_UNSUPPORTED, "%s: needs M <= 32, N %% 16 == 0, K %% 64 == 0 (got %lld, %lld, %lld)",
+                    fn, (long long)M, (long long)N, (long long)K);
+    const int log2_bs = log2_blocksize(blocksize);
+    if (log2_bs < 0)
+        return fail(BBC_ERR_INVALID, "%s: blocksize must be a power of two in [32, 4096] (got %d)", fn, blocksize);
+    if (blocksize2 != 256)
+        return fail(BBC_ERR_UNSUPPORTED, "%s: blocksize2 must be 256 (got %d)", fn, blocksize2);
+    if (!aligned(X, 16) || !aligned(codes, 8) || !aligned(Y, 2) || !aligned(code2, 4) || !aligned(absmax2, 4) ||
+        !aligned(code4, 4))
+        return fail(BBC_ERR_INVALID, "%s: X must be 16-byte, codes 8-byte aligned (others: element size)", fn);
+    return cuda_status(bbc::launch_linear_4bit_nested(X, dtype, (int)M, N, K, codes, absmax_q, code2, absmax2,
+                                                      offset, code4, log2_bs, Y, static_cast<cudaStream_t>(stream)),
+                       "linear_4bit_nested launch");
+}
+
 int dequantize_4bit_nested_chain(const uint8_t* codes, const uint8_t* absmax_q, const float* code2,
                                  const float* absmax2, float offset, const float* code4,
                                  int64_t n, int blocksize, int blocksize2, int out_dtype, void* out,

@@ -39,6 +39,13 @@ cudaError_t launch_quantize_4bit_nested(const void* A, int dtype, int64_t n, int
                                         const float* code2, uint8_t* codes, uint8_t* absmax_q, float* absmax2,
                                         float* offset, void* workspace, bool vec, cudaStream_t s);
 
+// Y[M, N] = X[M, K] @ W^T with W the nested 4-bit weight decoded in registers (M <= 32,
+// N % 16 == 0, K % 64 == 0; X 16-byte and codes 8-byte aligned; dtype F16 or BF16).
+cudaError_t launch_linear_4bit_nested(const void* X, int dtype, int M, int64_t N, int64_t K,
+                                      const uint8_t* codes, const uint8_t* absmax_q, const float* code2,
+                                      const float* absmax2, float offset, const float* code4, int log2_bs,
+                                      void* Y, cudaStream_t s);
+
 // The same two operations with the per-block absmax stored as one E4M4 byte.
 cudaError_t launch_kbit_quantize_e4m4(const void* A, int dtype, int64_t n, int K, const float* codebook,
                                       uint8_t* absmax, uint32_t* packed, bool vec, cudaStream_t s);

@@ -1,0 +1,76 @@
+"""GPU parity of the fused nested 4-bit dequant + linear against the float64 oracle.
+
+The fused kernel accumulates in fp32 on the tensor cores, so it is not bit-exact; the tolerance
+comes from the arithmetic: every product of two 16-bit values is exact, the K additions in fp32
+lose at most 2 K 2^-24 sum|x w| (twice the RN bound, allowing for the tensor core's internal
+accumulation), and the result is rounded once to the activation type (half an ulp)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from blockwise_bit_codebook_b200 import synthetic
+from tests.gpu_util import DTYPES, to_host
+
+pytestmark = pytest.mark.gpu
+NF4 = oracle.normal_float_codebook(4)
+G8 = synthetic.general8_table()
+
+
+@pytest.fixture(scope="module")
+def bbc():
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    from blockwise_bit_codebook_b200 import build
+    build.build()
+    import blockwise_bit_codebook_b200 as m
+    m.load_library()
+    return m
+
+
+def run_case(bbc, M, N, K, bs, dt, seed=0):
+    codes, q, a2, off = synthetic.nested_state(N * K, bs, seed=seed)
+    x = synthetic.weights(M * K, std=1.0, seed=seed + 100, dtype=DTYPES[dt]).reshape(M, K)
+    Y64, S = oracle.linear_4bit_nested(to_host(x), dt, N, K, (to_host(codes), to_host(q), to_host(a2), off),
+                                       G8, NF4, bs)
+    y = bbc.linear_4bit_nested(x.cuda(), codes.cuda(), q.cuda(), torch.from_numpy(G8).cuda(), a2.cuda(),
+                               float(off), torch.from_numpy(NF4).cuda(), N, bs)
+    torch.cuda.synchronize()
+    got = y.float().cpu().numpy().astype(np.float64)
+    acc_err = 2 * K * 2.0 ** -24 * S
+    half_ulp = (2.0 ** -8 if dt == "bf16" else 2.0 ** -11) * (np.abs(Y64) + acc_err)
+    err = np.abs(got - Y64)
+    bound = acc_err + half_ulp + 1e-30
+    assert np.all(err <= bound), (M, N, K, bs, dt, float(np.max(err / bound)))
+    return float(np.max(err / bound))
+
+
+@pytest.mark.parametrize("dt", ["bf16", "f16"])
+@pytest.mark.parametrize("M,N", [(1, 4096), (8, 4096), (32, 4096), (32, 11008)])
+def test_public_path_control_shapes(bbc, M, N, dt):
+    """The page's dequantize-plus-linear controls: M = 1, 8, 32; N = 4096 / 11008; K = 4096."""
+    run_case(bbc, M, N, 4096, 64, dt, seed=M)
+
+
+@pytest.mark.parametrize("dt", ["bf16", "f16"])
+def test_ragged_m_and_blocksizes(bbc, dt):
+    # (8, 32, 8192, 64): X too large to stage in shared memory, read from global memory instead
+    for M, N, K, bs in [(3, 64, 640, 64), (9, 256, 1024, 32), (17, 128, 4096, 4096), (31, 48, 192, 128),
+                        (2, 16, 64, 32), (8, 32, 8192, 64), (16, 64, 2048, 256)]:
+        run_case(bbc, M, N, K, bs, dt, seed=M + N)
+
+
+def test_invalid_arguments(bbc):
+    from blockwise_bit_codebook_b200 import BBCError
+    x = torch.zeros(33, 64, dtype=torch.bfloat16, device="cuda")
+    z8 = torch.zeros(4096, dtype=torch.uint8, device="cuda")
+    f = torch.zeros(256, device="cuda")
+    with pytest.raises(BBCError, match="M <= 32"):
+        bbc.linear_4bit_nested(x, z8, z8, f, f, 0.0, f, 16, 64)
+    with pytest.raises(BBCError, match="N % 16"):
+        bbc.linear_4bit_nested(x[:4], z8, z8, f, f, 0.0, f, 24, 64)
+    with pytest.raises(BBCError, match="K % 64"):
+        bbc.linear_4bit_nested(x[:4, :48].contiguous(), z8, z8, f, f, 0.0, f, 16, 64)
+    with pytest.raises(BBCError, match="aligned"):
+        bbc.linear_4bit_nested(x[:4], z8[1:], z8, f, f, 0.0, f, 16, 64)
+    with pytest.raises(BBCError, match="fp16 or bf16"):
+        bbc.linear_4bit_nested(x[:4].float(), z8, z8, f, f, 0.0, f, 16, 64)
