@@ -55,20 +55,25 @@ tree_sum_kernel(const T* __restrict__ in, int64_t count, double* __restrict__ no
     }
 }
 
+// The General8 table in shared memory as 32 lane-interleaved replicas (entry i of replica r at
+// i * 32 + r): each lane reads its own replica, so the data-dependent probes of a binary search
+// never conflict. `t` below is a lane's replica base; entry i is t[i * kRep].
+constexpr int kRep = 32;
+
 // First index minimising fl(|xn - t_i|) over an ascending 256-entry table (see the header).
 __device__ __forceinline__ uint32_t nearest_ascending(float xn, const float* t) {
     if (xn != xn) return 0;                                     // NaN: no distance is below +inf
-    int p = t[255] <= xn ? 255 : -1;                             // last index with t[p] <= xn
+    int p = t[255 * kRep] <= xn ? 255 : -1;                     // last index with entry p <= xn
     if (p < 0) {
 #pragma unroll
         for (int step = 128; step >= 1; step >>= 1)              // p + step <= 254 throughout
-            if (t[p + step] <= xn) p += step;
+            if (t[(p + step) * kRep] <= xn) p += step;
     }
     if (p < 0) return 0;
-    const float dp = fabsf(__fsub_rn(xn, t[p]));
-    if (p < 255 && fabsf(__fsub_rn(xn, t[p + 1])) < dp) return (uint32_t)p + 1;
+    const float dp = fabsf(__fsub_rn(xn, t[p * kRep]));
+    if (p < 255 && fabsf(__fsub_rn(xn, t[(p + 1) * kRep])) < dp) return (uint32_t)p + 1;
     int i = p;
-    while (i > 0 && fabsf(__fsub_rn(xn, t[i - 1])) == dp) i--;
+    while (i > 0 && fabsf(__fsub_rn(xn, t[(i - 1) * kRep])) == dp) i--;
     return (uint32_t)i;
 }
 
@@ -76,7 +81,7 @@ __device__ __forceinline__ uint32_t nearest_any(float xn, const float* t) {
     float best = __int_as_float(0x7f800000);
     uint32_t idx = 0;
     for (int i = 0; i < 256; i++) {
-        const float dist = fabsf(__fsub_rn(xn, t[i]));
+        const float dist = fabsf(__fsub_rn(xn, t[i * kRep]));
         if (dist < best) { best = dist; idx = (uint32_t)i; }
     }
     return idx;
@@ -87,10 +92,14 @@ __global__ void __launch_bounds__(256)
 absmax_compress_kernel(const float* __restrict__ absmax, int64_t nbo, const float* __restrict__ offset_p,
                        const float* __restrict__ code2, uint8_t* __restrict__ absmax_q,
                        float* __restrict__ absmax2) {
-    __shared__ float t[256];
-    t[threadIdx.x] = code2[threadIdx.x];
-    __syncthreads();
-    const bool ascending = __syncthreads_and(threadIdx.x == 255 || t[threadIdx.x] <= t[threadIdx.x + 1]);
+    __shared__ float tr[256 * kRep];                            // 32 KB
+    const float v = code2[threadIdx.x];
+    const float next = threadIdx.x < 255 ? code2[threadIdx.x + 1] : v;
+#pragma unroll 8
+    for (int r = 0; r < kRep; r++) tr[threadIdx.x * kRep + ((r + threadIdx.x) & (kRep - 1))] = v;
+    // the barrier also makes the replicas visible
+    const bool ascending = __syncthreads_and(v <= next);        // false if any entry is NaN
+    const float* t = tr + (threadIdx.x & (kRep - 1));
     const float off = *offset_p;
     const int lane = threadIdx.x & 31;
     const int64_t ngroups = (nbo + kGroup - 1) / kGroup;
