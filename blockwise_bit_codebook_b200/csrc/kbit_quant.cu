@@ -34,6 +34,18 @@
 //    is replicated 8 times so the 8 lanes of each 128-bit shared-load phase
 //    always hit distinct banks.
 //
+//    Whole-block threads (32-byte-aligned 16-bit input) use an 8-byte entry instead:
+//    {-A, spread(L)} with A = prev(T) for T > 0 and A = T for T < 0, so that the
+//    decision midpoint is always A + copysign(ulp(|A|) / 2, A); that half-ulp is
+//    rebuilt from A's bits (sign and exponent, exponent minus 24: two integer
+//    operations), the test becomes v = fma(-H, d, fma(-A, d, x)) with the same
+//    exactness argument, and instead of selecting spread(L) or spread(L + 1) the
+//    sign bits of v are collected (one funnel shift per element) and added to the
+//    K plane words of the block at the end as a bit-sliced increment. Half the
+//    shared-memory bytes per element, one select fewer. The thresholds must lie at
+//    least 2^-100 from zero (they do for any codebook the fast path accepts; the set-
+//    up checks it).
+//
 // 4. Bit-plane packing without ballots. Adding spread(idx) << e (bit k of idx at
 //    bit 8k) builds, per 8 elements, one register whose byte k holds plane k
 //    (K = 5 accumulates 4 elements per register with plane 4 in bits 4..7). For
@@ -58,6 +70,7 @@ namespace {
 constexpr int kThreads = 256;
 constexpr int kCells = 256;
 constexpr int kReplicas = 8;
+constexpr int kReplicas8 = 16;           // the 8-byte table: 16 lanes per shared-load phase
 // Resident CTAs per SM the register budget targets: the whole-block path (16-bit, aligned)
 // trades occupancy for per-thread parallelism; the half-block path keeps three.
 template <int DT, bool VEC> constexpr int kMinCtas = (VEC && DT != F32) ? 2 : 3;
@@ -110,10 +123,11 @@ __device__ __forceinline__ uint32_t nearest_entry(float xn, const float* cb) {
 // fast path applies (finite, strictly ascending, spaced >= 2^-19 (1 + max|c|), at most one
 // threshold per table cell), finds the thresholds by bisection and fills the 256-cell table
 // (8 replicas) whose entries are {-T, h_T, pattern(L), pattern(L + 1)}: the bit-plane spread of
-// the index for the k-bit codec, the index itself for nibble codes.
+// the index for the k-bit codec, the index itself for nibble codes. With `lut8` it fills the
+// 8-byte table {-A, pattern(L)} (16 replicas) instead (see step 3 of the header).
 template <int K, bool NIBBLE>
 __device__ __forceinline__ bool setup_exact_table(const float* __restrict__ codebook, float* cb, float* thr,
-                                                  int* fast_ok, uint4* lut) {
+                                                  int* fast_ok, uint4* lut, uint2* lut8 = nullptr) {
     constexpr int NE = 1 << K;
     const int tid = threadIdx.x;
     if (tid < 32) {
@@ -157,9 +171,22 @@ __device__ __forceinline__ bool setup_exact_table(const float* __restrict__ code
             const uint32_t p0 = NIBBLE ? (uint32_t)below : spread<K>((uint32_t)below);
             const uint32_t p1 = NIBBLE ? (uint32_t)below + 1 : spread<K>((uint32_t)below + 1);
             const uint4 ent = make_uint4(__float_as_uint(negT), __float_as_uint(half), p0, p1);
-            // the 8 lanes of a store phase write 8 different replicas: distinct banks
+            if (!lut8) {
+                // the 8 lanes of a store phase write 8 different replicas: distinct banks
 #pragma unroll
-            for (int r = 0; r < kReplicas; r++) lut[cell * kReplicas + ((r + tid) & (kReplicas - 1))] = ent;
+                for (int r = 0; r < kReplicas; r++) lut[cell * kReplicas + ((r + tid) & (kReplicas - 1))] = ent;
+            } else {
+                float nA = __int_as_float(0xff800000);               // -inf: never crossed
+                if (rel == 1) {
+                    const float T = thr[relj];
+                    const float Av = T > 0.0f ? key_f32(f32_key(T) - 1) : T;
+                    nA = -Av;
+                    multi |= !(fabsf(Av) >= 0x1p-100f);              // keep the rebuilt half-ulp normal
+                }
+                const uint2 e8 = make_uint2(__float_as_uint(nA), p0);
+#pragma unroll
+                for (int r = 0; r < kReplicas8; r++) lut8[cell * kReplicas8 + ((r + tid) & (kReplicas8 - 1))] = e8;
+            }
         }
     }
     return (*fast_ok != 0) && !__syncthreads_or(multi);
@@ -276,6 +303,8 @@ struct LoopCtx {
     const char* lut;        // generic pointer to the shared table
     uint32_t lut_s;         // its shared-window address
     uint32_t lane16;        // this lane's replica offset
+    uint32_t lut8_s;        // shared address of the 8-byte table (whole-block path)
+    uint32_t lane8;         // this lane's replica offset in it
     uint32_t h;             // which half of the block this lane owns
     uint32_t sel_send, sel_keep, sel_wa, sel_wb, pair_mask;
     bool fast_cb;
@@ -297,6 +326,14 @@ __device__ __forceinline__ uint4 lut_entry(const LoopCtx& c, uint32_t fbits) {
 #else
     return *reinterpret_cast<const uint4*>(__builtin_assume_aligned(c.lut + off, 16));
 #endif
+}
+
+// The 8-byte table entry {-A, spread(L)} of the cell in bits 7..14 of `fbits` (128 bytes per
+// cell, as the 16-byte table: the same cell offset).
+__device__ __forceinline__ uint2 lut8_entry(const LoopCtx& c, uint32_t fbits) {
+    uint2 v;
+    asm volatile("ld.shared.v2.u32 {%0,%1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(c.lut8_s + ((fbits & 0x7f80u) | c.lane8)));
+    return v;
 }
 
 // Fast path for one half block: thresholds via the table, exact two-FMA test per element.
@@ -464,6 +501,7 @@ __device__ __forceinline__ void quantize_block(const Raw32<DT>& raw, int64_t b, 
     uint32_t B[4], w4 = 0;
     const float rs = __fmul_rn(rcp_approx(d), 8192.0f);
     const bool fast = !special && c.fast_cb;
+    uint32_t sv = 0;                     // fast path: sign of v per element, element 0 shifted in first
     // K = 5 accumulates 4 elements per register: two passes of 16 keep 4 registers live
     constexpr int NPASS = K == 5 ? 2 : 1;
     constexpr int PE = 32 / NPASS;
@@ -477,12 +515,16 @@ __device__ __forceinline__ void quantize_block(const Raw32<DT>& raw, int64_t b, 
                 widen_pair<DT>(raw.w[(pass * PE + e) / 2], x0, x1);
                 const float2 f = __ffma2_rn(make_float2(x0, x1), make_float2(rs, rs),
                                             make_float2(12582912.0f, 12582912.0f));
-                const uint4 t0 = lut_entry(c, __float_as_uint(f.x));
-                const uint4 t1 = lut_entry(c, __float_as_uint(f.y));
-                const float v0 = __fmaf_rn(__uint_as_float(t0.y), d, __fmaf_rn(__uint_as_float(t0.x), d, x0));
-                const float v1 = __fmaf_rn(__uint_as_float(t1.y), d, __fmaf_rn(__uint_as_float(t1.x), d, x1));
-                acc[e / EPA] += (v0 > 0.0f ? t0.w : t0.z) << (e % EPA);
-                acc[(e + 1) / EPA] += (v1 > 0.0f ? t1.w : t1.z) << ((e + 1) % EPA);
+                const uint2 t0 = lut8_entry(c, __float_as_uint(f.x));
+                const uint2 t1 = lut8_entry(c, __float_as_uint(f.y));
+                const float h0 = __uint_as_float((t0.x & 0xff800000u) - 0x0c000000u);   // -H
+                const float h1 = __uint_as_float((t1.x & 0xff800000u) - 0x0c000000u);
+                const float v0 = __fmaf_rn(h0, d, __fmaf_rn(__uint_as_float(t0.x), d, x0));
+                const float v1 = __fmaf_rn(h1, d, __fmaf_rn(__uint_as_float(t1.x), d, x1));
+                sv = __funnelshift_l(__float_as_uint(v0), sv, 1);                         // sign bits
+                sv = __funnelshift_l(__float_as_uint(v1), sv, 1);
+                acc[e / EPA] += t0.y << (e % EPA);
+                acc[(e + 1) / EPA] += t1.y << ((e + 1) % EPA);
             }
         } else {
 #pragma unroll
@@ -505,24 +547,30 @@ __device__ __forceinline__ void quantize_block(const Raw32<DT>& raw, int64_t b, 
         }
     }
     const uint32_t lo01 = prmt(B[0], B[1], 0x5140u), lo23 = prmt(B[2], B[3], 0x5140u);
-    const uint32_t w0 = prmt(lo01, lo23, 0x5410u), w1 = prmt(lo01, lo23, 0x7632u);
+    const uint32_t hi01 = prmt(B[0], B[1], 0x7362u), hi23 = prmt(B[2], B[3], 0x7362u);
+    uint32_t w[5] = {prmt(lo01, lo23, 0x5410u), prmt(lo01, lo23, 0x7632u), prmt(hi01, hi23, 0x5410u),
+                     prmt(hi01, hi23, 0x7632u), w4};
+    if (fast) {
+        // planes of L + 1 where v > 0: a bit-sliced increment (the bit-reversed signs put
+        // element i at bit i; L + 1 never exceeds 2^K - 1)
+        uint32_t cy = ~__brev(sv);
+#pragma unroll
+        for (int j = 0; j < K; j++) {
+            const uint32_t carry = w[j] & cy;
+            w[j] ^= cy;
+            cy = carry;
+        }
+    }
     uint32_t* out = packed + b * K;
     if constexpr (K == 2) {
-        if (c.packed_v2) asm volatile("st.global.v2.u32 [%0], {%1,%2};" :: "l"(out), "r"(w0), "r"(w1) : "memory");
-        else { out[0] = w0; out[1] = w1; }
+        if (c.packed_v2) asm volatile("st.global.v2.u32 [%0], {%1,%2};" :: "l"(out), "r"(w[0]), "r"(w[1]) : "memory");
+        else { out[0] = w[0]; out[1] = w[1]; }
+    } else if constexpr (K == 4) {
+        if (c.packed_v4) stg_v4(out, w[0], w[1], w[2], w[3]);
+        else { out[0] = w[0]; out[1] = w[1]; out[2] = w[2]; out[3] = w[3]; }
     } else {
-        const uint32_t hi01 = prmt(B[0], B[1], 0x7362u), hi23 = prmt(B[2], B[3], 0x7362u);
-        const uint32_t w2 = prmt(hi01, hi23, 0x5410u);
-        if constexpr (K == 4) {
-            const uint32_t w3 = prmt(hi01, hi23, 0x7632u);
-            if (c.packed_v4) stg_v4(out, w0, w1, w2, w3);
-            else { out[0] = w0; out[1] = w1; out[2] = w2; out[3] = w3; }
-        } else if constexpr (K == 3) {
-            out[0] = w0; out[1] = w1; out[2] = w2;
-        } else {
-            const uint32_t w3 = prmt(hi01, hi23, 0x7632u);
-            out[0] = w0; out[1] = w1; out[2] = w2; out[3] = w3; out[4] = w4;
-        }
+#pragma unroll
+        for (int j = 0; j < K; j++) out[j] = w[j];
     }
     store_absmax(absmax, b, amax);
 }
@@ -532,7 +580,9 @@ __global__ void __launch_bounds__(kThreads, (kMinCtas<DT, VEC>))
 kbit_quant_kernel(const void* __restrict__ A, int64_t n, const float* __restrict__ codebook,
                   AT* __restrict__ absmax, uint32_t* __restrict__ packed) {
     constexpr int NE = 1 << K;
-    __shared__ __align__(16) uint4 lut[kCells * kReplicas];    // 32 KB
+    constexpr bool WHOLE = VEC && DT != F32;                   // whole blocks per thread: 8-byte table
+    __shared__ __align__(16) uint4 lut[WHOLE ? 1 : kCells * kReplicas];     // 32 KB
+    __shared__ __align__(16) uint2 lut8[WHOLE ? kCells * kReplicas8 : 1];   // 32 KB
     __shared__ float cb[32];
     __shared__ float thr[33];
     __shared__ int fast_ok;
@@ -541,12 +591,14 @@ kbit_quant_kernel(const void* __restrict__ A, int64_t n, const float* __restrict
     const int lane = tid & 31;
 
     // ---- per-CTA set-up: codebook check, thresholds, lookup table ----
-    const bool fast_cb = setup_exact_table<K, false>(codebook, cb, thr, &fast_ok, lut);
+    const bool fast_cb = setup_exact_table<K, false>(codebook, cb, thr, &fast_ok, lut, WHOLE ? lut8 : nullptr);
     LoopCtx c;
     c.fast_cb = fast_cb;
     c.lut = reinterpret_cast<const char*>(lut);
     c.lut_s = (uint32_t)__cvta_generic_to_shared(lut);
     c.lane16 = (uint32_t)(lane & 7) << 4;
+    c.lut8_s = (uint32_t)__cvta_generic_to_shared(lut8);
+    c.lane8 = (uint32_t)(lane & (kReplicas8 - 1)) << 3;
     c.packed_v2 = (reinterpret_cast<uintptr_t>(packed) & 7u) == 0;
     c.packed_v4 = (reinterpret_cast<uintptr_t>(packed) & 15u) == 0;
     c.h = lane & 1;
@@ -585,6 +637,7 @@ kbit_quant_kernel(const void* __restrict__ A, int64_t n, const float* __restrict
                 if (!more) break;
             }
         }
+        c.fast_cb = false;                  // the ragged end (under one warp iteration): the rule verbatim
         for (int64_t t = 2 * bend + (int64_t)blockIdx.x * kThreads + (tid & ~31); t < nh; t += stride) {
             const Raw<DT> r = load_raw<DT, VEC>(A, n, t + lane, t + lane < nh);
             quantize_half<K, DT, AT>(r, t + lane, t + lane < nh, c, cb, absmax, packed);

@@ -203,6 +203,35 @@ def test_quotients_on_thresholds(bbc, K):
     check_quantize(bbc, torch.from_numpy(x), K, cb, what=f"thresholds K{K}")
 
 
+@pytest.mark.parametrize("K", [2, 3, 4, 5])
+@pytest.mark.parametrize("dt", ["bf16", "f16"])
+def test_every_16bit_quotient_for_several_absmax(bbc, K, dt):
+    """Every value of the 16-bit type in [-d, d] as a numerator, for several block maxima d (the
+    block's first element): all quotients these d can produce, those on and beside every
+    threshold included. The length is whole warp iterations of 32 blocks, so the aligned
+    one-block-per-thread path (8-byte table, sign-bit increment) decides all of them."""
+    cb = oracle.normal_float_codebook(K)
+    bits = np.arange(1 << 16, dtype=np.uint32).astype(np.uint16)
+    widen = oracle.bf16_bits_to_f32 if dt == "bf16" else oracle.f16_bits_to_f32
+    narrow = oracle.f32_to_bf16_bits if dt == "bf16" else oracle.f32_to_f16_bits
+    vals = widen(bits)
+    blocks = []
+    for d_req in (1.0, 0.7373, 3.25e-3, 1234.5):
+        d_bits = narrow(np.array([d_req], np.float32))[0]
+        d = widen(np.array([d_bits], np.uint16))[0]
+        xs = bits[np.isfinite(vals) & (np.abs(vals) <= d)]
+        for i in range(0, xs.size, 31):
+            blk = np.zeros(32, np.uint16)
+            blk[0] = d_bits
+            blk[1:1 + xs[i:i + 31].size] = xs[i:i + 31]
+            blocks.append(blk)
+    while len(blocks) % 32:
+        blocks.append(np.zeros(32, np.uint16))
+    x = np.concatenate(blocks)
+    xt = torch.from_numpy(x.view(np.int16)).view(DTYPES[dt])
+    check_quantize(bbc, xt, K, cb, what=f"every {dt} quotient K{K}")
+
+
 def test_quotients_on_thresholds_wide_codebook(bbc):
     """Thresholds beyond [-1, 1] and a codebook not symmetric about zero."""
     cb = np.array([-3.0, -1.7, -0.9, -0.2, 0.05, 0.4, 1.1, 2.5], np.float32)
