@@ -755,7 +755,8 @@ quant4_kernel(const void* __restrict__ A, int64_t n, int log2_bs, const float* _
               float* __restrict__ absmax, uint8_t* __restrict__ codes) {
     constexpr int E = kEpt<DT>;
     constexpr int NW = E / 8;                                   // code words per thread
-    __shared__ __align__(16) uint4 lut[kCells * kReplicas];    // 32 KB
+    __shared__ __align__(16) uint2 lut8[kCells * kReplicas8];  // 32 KB: {-A, L}
+    __shared__ uint32_t nib_spread[256];                         // bit i of a byte -> nibble i's low bit
     __shared__ float cb[32];
     __shared__ float thr[33];
     __shared__ int fast_ok;
@@ -763,11 +764,16 @@ quant4_kernel(const void* __restrict__ A, int64_t n, int log2_bs, const float* _
 
     const int tid = threadIdx.x;
     const int lane = tid & 31, warp = tid >> 5;
+    {
+        uint32_t v = 0;
+#pragma unroll
+        for (int i = 0; i < 8; i++) v |= ((uint32_t)(tid >> i) & 1u) << nib_shift(i);
+        nib_spread[tid] = v;                                     // kThreads == 256
+    }
     LoopCtx c;
-    c.fast_cb = setup_exact_table<4, true>(code4, cb, thr, &fast_ok, lut);
-    c.lut = reinterpret_cast<const char*>(lut);
-    c.lut_s = (uint32_t)__cvta_generic_to_shared(lut);
-    c.lane16 = (uint32_t)(lane & 7) << 4;
+    c.fast_cb = setup_exact_table<4, true>(code4, cb, thr, &fast_ok, nullptr, lut8);
+    c.lut8_s = (uint32_t)__cvta_generic_to_shared(lut8);
+    c.lane8 = (uint32_t)(lane & (kReplicas8 - 1)) << 3;
 
     const int tpb_log2 = log2_bs - (DT == F32 ? 4 : 5);        // threads per outer block
     const int tpb = 1 << tpb_log2;
@@ -809,18 +815,27 @@ quant4_kernel(const void* __restrict__ A, int64_t n, int log2_bs, const float* _
         for (int g = 0; g < NW; g++) acc[g] = 0u;
         if (!special && c.fast_cb) {
             const float rs = __fmul_rn(rcp_approx(d), 8192.0f);
+            uint32_t sv = 0;                                     // signs of v, element 0 shifted in first
 #pragma unroll
             for (int e = 0; e < E; e += 2) {
                 const float x0 = slice_elem<DT>(cur, e), x1 = slice_elem<DT>(cur, e + 1);
                 const float2 f = __ffma2_rn(make_float2(x0, x1), make_float2(rs, rs),
                                             make_float2(12582912.0f, 12582912.0f));
-                const uint4 t0 = lut_entry(c, __float_as_uint(f.x));
-                const uint4 t1 = lut_entry(c, __float_as_uint(f.y));
-                const float v0 = __fmaf_rn(__uint_as_float(t0.y), d, __fmaf_rn(__uint_as_float(t0.x), d, x0));
-                const float v1 = __fmaf_rn(__uint_as_float(t1.y), d, __fmaf_rn(__uint_as_float(t1.x), d, x1));
-                acc[e / 8] += (v0 > 0.0f ? t0.w : t0.z) << nib_shift(e);
-                acc[(e + 1) / 8] += (v1 > 0.0f ? t1.w : t1.z) << nib_shift(e + 1);
+                const uint2 t0 = lut8_entry(c, __float_as_uint(f.x));
+                const uint2 t1 = lut8_entry(c, __float_as_uint(f.y));
+                const float h0 = __uint_as_float((t0.x & 0xff800000u) - 0x0c000000u);   // -H
+                const float h1 = __uint_as_float((t1.x & 0xff800000u) - 0x0c000000u);
+                const float v0 = __fmaf_rn(h0, d, __fmaf_rn(__uint_as_float(t0.x), d, x0));
+                const float v1 = __fmaf_rn(h1, d, __fmaf_rn(__uint_as_float(t1.x), d, x1));
+                sv = __funnelshift_l(__float_as_uint(v0), sv, 1);
+                sv = __funnelshift_l(__float_as_uint(v1), sv, 1);
+                acc[e / 8] += t0.y << nib_shift(e);
+                acc[(e + 1) / 8] += t1.y << nib_shift(e + 1);
             }
+            // L + 1 where v > 0 (never beyond 15): element i's increment at bit i of ~brev(sv)
+            const uint32_t inc = ~__brev(sv) >> (32 - E);
+#pragma unroll
+            for (int g = 0; g < NW; g++) acc[g] += nib_spread[(inc >> (8 * g)) & 0xffu];
         } else {
 #pragma unroll
             for (int e = 0; e < E; e++)

@@ -121,3 +121,28 @@ def test_nested_state_small_and_constant(bbc):
     # every outer absmax equal: absmax2 = 0, the divisor clamps to 1e-8
     x = torch.ones(64 * 300, dtype=torch.float32) * 0.25
     check_nested(bbc, x, 64, what="constant")
+
+
+@pytest.mark.parametrize("table", ["nf4", "fp4"])
+@pytest.mark.parametrize("dt", ["bf16", "f16"])
+def test_every_16bit_quotient_4bit(bbc, table, dt):
+    """Every value of the 16-bit type in [-d, d] as a numerator for several block maxima d
+    (blocksize 32: the block's first element is d), so every quotient these d produce, on and
+    beside each threshold of the table, is decided by the kernel's exact search."""
+    code4 = NF4 if table == "nf4" else FP4
+    bits = np.arange(1 << 16, dtype=np.uint32).astype(np.uint16)
+    widen = oracle.bf16_bits_to_f32 if dt == "bf16" else oracle.f16_bits_to_f32
+    narrow = oracle.f32_to_bf16_bits if dt == "bf16" else oracle.f32_to_f16_bits
+    vals = widen(bits)
+    blocks = []
+    for d_req in (1.0, 0.7373, 3.25e-3, 1234.5):
+        d_bits = narrow(np.array([d_req], np.float32))[0]
+        d = widen(np.array([d_bits], np.uint16))[0]
+        xs = bits[np.isfinite(vals) & (np.abs(vals) <= d)]
+        for i in range(0, xs.size, 31):
+            blk = np.zeros(32, np.uint16)
+            blk[0] = d_bits
+            blk[1:1 + xs[i:i + 31].size] = xs[i:i + 31]
+            blocks.append(blk)
+    x = np.concatenate(blocks)
+    check_q4(bbc, torch.from_numpy(x.view(np.int16)).view(DTYPES[dt]), 32, code4, what=f"every {dt} quotient")
