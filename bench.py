@@ -462,7 +462,9 @@ def run_linear(args):
     cuBLAS) on the pull request's public-path control shapes: M = 1 and 8 (N = K = 4096) and
     M = 32 (N = 4096 and 11008, K = 4096); bf16 activations, NF4, outer blocksize 64. CUDA events
     around CUDA-graph replays of 200 repetitions (device time, no host launch overhead),
-    alternating order, 7 rounds, medians. Algorithmic bytes of the fused kernel: codes,
+    alternating order, 7 rounds, medians. Two regimes: the same weight every call (it stays in
+    L2, as in the page's timing loop) and "cold", where the calls cycle through copies of the
+    weight state totalling more than L2. Algorithmic bytes of the fused kernel: codes,
     absmax_q, absmax2, X and Y (the weight is never written)."""
     import torch
 
@@ -484,28 +486,35 @@ def run_linear(args):
         w = torch.empty(N * K, dtype=torch.bfloat16, device=dev)
         y_f = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
         y_u = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
-        fused = lambda: bbc.linear_4bit_nested(x, codes, q, code2, a2, float(off), code4, N, bs, out=y_f)  # noqa: E731
+        # "cold": the calls cycle through copies of the weight state that together exceed the
+        # 126 MB L2, so every call reads its weight from HBM (as successive layers of a model do)
+        ncopy = max(2, -(-160 * 2**20 // (N * K // 2)))
+        copies = [(codes.clone(), q.clone()) for _ in range(ncopy)]
 
-        def unfused():
-            bbc.dequantize_4bit_nested(codes, q, code2, a2, float(off), code4, N * K, bs, torch.bfloat16, out=w)
+        def fused_on(c, qq):
+            bbc.linear_4bit_nested(x, c, qq, code2, a2, float(off), code4, N, bs, out=y_f)
+
+        def unfused_on(c, qq):
+            bbc.dequantize_4bit_nested(c, qq, code2, a2, float(off), code4, N * K, bs, torch.bfloat16, out=w)
             torch.matmul(x, w.view(N, K).t(), out=y_u)
         for i in range(20):
-            (fused if i % 2 == 0 else unfused)()
+            (fused_on if i % 2 == 0 else unfused_on)(codes, q)
         torch.cuda.synchronize()
         # Host-side call overhead (Python, ctypes) exceeds these kernels' device time, so each
         # variant's repetitions are captured once in a CUDA graph and the replays are timed.
         reps = 200
         graphs = {}
-        for name, fn in (("fused", fused), ("unfused", unfused)):
+        for name, fn, cold in (("fused", fused_on, False), ("unfused", unfused_on, False),
+                               ("fused_cold", fused_on, True), ("unfused_cold", unfused_on, True)):
             gr = torch.cuda.CUDAGraph()
             with torch.cuda.graph(gr):
-                for _ in range(reps):
-                    fn()
+                for r in range(reps):
+                    fn(*(copies[r % ncopy] if cold else (codes, q)))
             graphs[name] = gr
         torch.cuda.synchronize()
-        samples = {"fused": [], "unfused": []}
+        samples = {k: [] for k in graphs}
         for rnd in range(7):
-            order = ["fused", "unfused"]
+            order = list(graphs)
             if rnd % 2:
                 order.reverse()
             for name in order:
@@ -525,6 +534,12 @@ def run_linear(args):
                           "unfused_over_fused": round(med["unfused"] / med["fused"], 3),
                           "fused_GBs": round(nbytes / med["fused"] / 1e3, 1),
                           "fused_frac_of_measured_hbm": round(nbytes / med["fused"] / 1e3 / peak, 4),
+                          "cold_weight_copies": ncopy,
+                          "fused_cold_us_median": round(med["fused_cold"], 2),
+                          "unfused_cold_us_median": round(med["unfused_cold"], 2),
+                          "cold_unfused_over_fused": round(med["unfused_cold"] / med["fused_cold"], 3),
+                          "fused_cold_GBs": round(nbytes / med["fused_cold"] / 1e3, 1),
+                          "fused_cold_frac_of_measured_hbm": round(nbytes / med["fused_cold"] / 1e3 / peak, 4),
                           "max_rel_diff_vs_unfused": round(rel, 6)}), flush=True)
 
 

@@ -223,9 +223,9 @@ int linear_4bit_nested(const void* X, int dtype, int64_t M, int64_t N, int64_t K
         return fail(BBC_ERR_INVALID, "%s: blocksize must be a power of two in [32, 4096] (got %d)", fn, blocksize);
     if (blocksize2 != 256)
         return fail(BBC_ERR_UNSUPPORTED, "%s: blocksize2 must be 256 (got %d)", fn, blocksize2);
-    if (!aligned(X, 16) || !aligned(codes, 8) || !aligned(Y, 2) || !aligned(code2, 4) || !aligned(absmax2, 4) ||
+    if (!aligned(X, 16) || !aligned(codes, 16) || !aligned(Y, 2) || !aligned(code2, 4) || !aligned(absmax2, 4) ||
         !aligned(code4, 4))
-        return fail(BBC_ERR_INVALID, "%s: X must be 16-byte, codes 8-byte aligned (others: element size)", fn);
+        return fail(BBC_ERR_INVALID, "%s: X and codes must be 16-byte aligned (others: element size)", fn);
     return cuda_status(bbc::launch_linear_4bit_nested(X, dtype, (int)M, N, K, codes, absmax_q, code2, absmax2,
                                                       offset, code4, log2_bs, Y, static_cast<cudaStream_t>(stream)),
                        "linear_4bit_nested launch");

@@ -579,7 +579,6 @@ template <int K, int DT, bool VEC, typename AT>
 __global__ void __launch_bounds__(kThreads, (kMinCtas<DT, VEC>))
 kbit_quant_kernel(const void* __restrict__ A, int64_t n, const float* __restrict__ codebook,
                   AT* __restrict__ absmax, uint32_t* __restrict__ packed) {
-    constexpr int NE = 1 << K;
     constexpr bool WHOLE = VEC && DT != F32;                   // whole blocks per thread: 8-byte table
     __shared__ __align__(16) uint4 lut[WHOLE ? 1 : kCells * kReplicas];     // 32 KB
     __shared__ __align__(16) uint2 lut8[WHOLE ? kCells * kReplicas8 : 1];   // 32 KB

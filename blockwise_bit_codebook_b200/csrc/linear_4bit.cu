@@ -9,15 +9,20 @@
 //
 // Layout of the work: a CTA owns a tile of 16 rows of W (16 outputs per activation row) and
 // its 8 warps split K; partial sums meet in shared memory and are added in warp order. Each
-// warp walks 64-wide windows of K with mma.sync m16n8k16 (T inputs, fp32 accumulators), one
-// n-tile per 8 activation rows (M <= 32). Both operands use the same permutation of the 16
-// k-slots of each mma step s (slot of lane-quad t -> k = 16 t + 4 s + 0..3), so a lane needs
-// 16 consecutive k of a window: 8 contiguous code bytes per W row and 32 contiguous bytes of
-// each activation row. Each code byte is decoded through a 256-entry shared table of the pair
-// (code4[hi], code4[lo]), multiplied by the block scale (paired fp32 multiply) and rounded to T.
-// The loads of the next window (code bytes, scale codes, activation fragments) are issued
-// before the current window is decoded and multiplied.
+// warp walks windows of K (a 64-wide window ends the row when 128-wide windows leave 64) with
+// mma.sync m16n8k16 (T inputs, fp32 accumulators), one n-tile per 8 activation rows (M <= 32).
+// Both operands use the same permutation of the 16 k-slots of each mma step s: the slots of
+// lane-quad t are k = (W/4) t + 4 s + 0..3 for a window of width W, so a lane needs W/4
+// consecutive k of a window: one 16-byte (8-byte) load of code bytes per W row, all inside one
+// outer block (blocksize >= 32), so one scale per row per window, and W/2 contiguous bytes of
+// each activation row. Windows are 128 wide when the activations are staged in shared memory
+// (M <= 8) and 64 wide when they are read from global memory (the quad's loads of a row then
+// stay within one 128-byte line). Each code byte is decoded through a 256-entry shared table of
+// the pair (code4[hi], code4[lo]) (one shift and one logic operation form the table address),
+// multiplied by the block scale (paired fp32 multiply) and rounded to T. The code loads of the
+// next windows are in flight while the current one is decoded and multiplied.
 #include <atomic>
+#include <type_traits>
 
 #include "common.cuh"
 #include "launch.h"
@@ -27,6 +32,7 @@ namespace bbc {
 namespace {
 
 constexpr int kLinThreads = 256;          // two CTAs per SM: one wave for N <= 4736
+constexpr int kNWarp = kLinThreads / 32;
 
 template <int DT>
 __device__ __forceinline__ void mma16816(float* c, const uint32_t* a, uint32_t b0, uint32_t b1) {
@@ -42,109 +48,166 @@ __device__ __forceinline__ void mma16816(float* c, const uint32_t* a, uint32_t b
                      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
-// The decode table: entry (byte, r) = (code4[byte >> 4], code4[byte & 15]) at index byte * 16 + r,
-// 16 interleaved replicas: the 16 lanes of an 8-byte shared-load phase read replica lane & 15,
-// so they always hit 16 different bank pairs.
+// The decode table: entry (byte, r) = (code4[byte >> 4], code4[byte & 15]) at byte offset
+// byte * 128 + r * 8, 16 interleaved replicas: the 16 lanes of an 8-byte shared-load phase read
+// replica lane & 15, so they always hit 16 different bank pairs.
 constexpr int kPairReplicas = 16;
+constexpr int kPairBytes = 256 * kPairReplicas * 8;      // 32 KB
+static_assert(kPairReplicas * 8 == 128, "one table entry spans bits 7..14 of the byte offset");
 
-// 16 weights of one W row from 8 code bytes (element 2j in the high nibble of byte j), as 8
-// packed pairs of T: word j = (w[2j], w[2j+1]) with w[2j] in the low half.
-template <int DT>
-__device__ __forceinline__ void decode16(uint2 cw, float scale, const float2* pairs_r, uint32_t* w) {
-#pragma unroll
-    for (int j = 0; j < 8; j++) {
-        const uint32_t byte = ((j < 4 ? cw.x : cw.y) >> (8 * (j & 3))) & 0xffu;
-        const float2 v = pairs_r[byte * kPairReplicas];             // (code4[hi], code4[lo])
-        const float2 p = __fmul2_rn(v, make_float2(scale, scale));
-        w[j] = DT == BF16 ? pack_bf16x2(p.x, p.y) : pack_f16x2(p.x, p.y);
-    }
+// Two weights (w[2j], w[2j+1] of this lane's run, w[2j] in the low half) from byte J of `word`:
+// the byte moved to bits 7..14 is the entry's offset, the lane's replica is or-ed in.
+template <int DT, int J>
+__device__ __forceinline__ uint32_t decode_byte(uint32_t word, uint32_t lane_off, float2 scale,
+                                                const unsigned char* table) {
+    const uint32_t sel = (J == 0 ? (word << 7) : (word >> (8 * J - 7))) & 0x7f80u;
+    const float2 v = *reinterpret_cast<const float2*>(table + (sel | lane_off));
+    const float2 p = __fmul2_rn(v, scale);
+    return DT == BF16 ? pack_bf16x2(p.x, p.y) : pack_f16x2(p.x, p.y);
 }
 
-// Code bytes and scale inputs of one window for this lane's two W rows.
-struct WinCodes {
-    uint2 ca, cb;                 // 8 code bytes of W rows g and g + 8
-    uint32_t qa, qb;              // their outer blocks' General8 codes
-    float a2a, a2b;               // and inner absmax
+// Code bytes and scale inputs of one window for this lane's two W rows (g and g + 8). Lane t of
+// a row quad takes the W/4 consecutive k from (W/4) t: one 16-byte (8-byte) code load per row,
+// all inside one outer block (blocksize >= 32 >= W/4, and the run starts at a multiple of W/4),
+// so one scale per row per window.
+template <int W>
+struct Win {
+    uint32_t ca[W / 32], cb[W / 32];      // code word c: the lane's k 8c .. 8c + 7 of the window
+    uint32_t qa, qb;                      // the General8 code of each row's outer block
+    float a2a, a2b;                       // and its inner absmax
 };
 
-__device__ __forceinline__ WinCodes load_codes(int64_t K, const uint8_t* codes, const uint8_t* absmax_q,
-                                               const float* absmax2, int log2_bs, int64_t ra, int64_t rb,
-                                               int64_t win, int t) {
-    WinCodes r;
-    const int64_t k0 = win * 64 + 16 * t;                           // this lane's 16 k
-    const int64_t ea = ra * K + k0, eb = rb * K + k0;               // flattened element indices
-    r.ca = __ldg(reinterpret_cast<const uint2*>(codes + (ea >> 1)));
-    r.cb = __ldg(reinterpret_cast<const uint2*>(codes + (eb >> 1)));
-    const int64_t ba = ea >> log2_bs, bb = eb >> log2_bs;           // outer blocks (16 k inside one)
+// ea, eb: flattened index of the window's first weight in rows g and g + 8.
+template <int W>
+__device__ __forceinline__ void load_win(Win<W>& r, const uint8_t* codes, const uint8_t* absmax_q,
+                                         const float* absmax2, int log2_bs, int64_t ea, int64_t eb, int t) {
+    const int64_t la = ea + (W / 4) * t, lb = eb + (W / 4) * t;
+    if constexpr (W == 128) {
+        const uint4 a = __ldg(reinterpret_cast<const uint4*>(codes + (la >> 1)));
+        const uint4 b = __ldg(reinterpret_cast<const uint4*>(codes + (lb >> 1)));
+        r.ca[0] = a.x; r.ca[1] = a.y; r.ca[2] = a.z; r.ca[3] = a.w;
+        r.cb[0] = b.x; r.cb[1] = b.y; r.cb[2] = b.z; r.cb[3] = b.w;
+    } else {
+        const uint2 a = __ldg(reinterpret_cast<const uint2*>(codes + (la >> 1)));
+        const uint2 b = __ldg(reinterpret_cast<const uint2*>(codes + (lb >> 1)));
+        r.ca[0] = a.x; r.ca[1] = a.y;
+        r.cb[0] = b.x; r.cb[1] = b.y;
+    }
+    const int64_t ba = la >> log2_bs, bb = lb >> log2_bs;
     r.qa = __ldg(absmax_q + ba);
     r.qb = __ldg(absmax_q + bb);
     r.a2a = __ldg(absmax2 + (ba >> 8));
     r.a2b = __ldg(absmax2 + (bb >> 8));
-    return r;
 }
 
-// 16 consecutive k of activation row m (zeros past M), from global memory or shared staging.
-template <bool SMEM>
-__device__ __forceinline__ void load_x(const uint16_t* X, const uint16_t* xs, int64_t xs_stride, int M,
-                                       int64_t K, int m, int64_t k0, uint32_t* xb) {
-    if (m < M) {
-        const uint4* xp = SMEM ? reinterpret_cast<const uint4*>(xs + (int64_t)m * xs_stride + k0)
-                               : reinterpret_cast<const uint4*>(X + (int64_t)m * K + k0);
-        const uint4 x0 = SMEM ? xp[0] : __ldg(xp), x1 = SMEM ? xp[1] : __ldg(xp + 1);
-        xb[0] = x0.x; xb[1] = x0.y; xb[2] = x0.z; xb[3] = x0.w;
-        xb[4] = x1.x; xb[5] = x1.y; xb[6] = x1.z; xb[7] = x1.w;
-    } else {
+// Code words W0 .. W1-1 of a window of width W for this lane: the activation words xw (word 4c + i:
+// the lane's k 8c + 2i, 8c + 2i + 1) and the rows' scales; decodes both rows' codes and runs their
+// mma steps (two per word).
+template <int DT, int NT, int W, int W0, int W1>
+__device__ __forceinline__ void mma_win(float (&acc)[NT][4], const Win<W>& wc, float2 sa2, float2 sb2,
+                                        const uint32_t (&xw)[NT][W / 8], const unsigned char* table,
+                                        uint32_t lane_off) {
 #pragma unroll
-        for (int j = 0; j < 8; j++) xb[j] = 0u;
+    for (int w = W0; w < W1; w++) {
+        // code word w holds the bytes of mma steps 2w and 2w + 1
+        const uint32_t wa = wc.ca[w], wb = wc.cb[w];
+        uint32_t a[2][4];
+        a[0][0] = decode_byte<DT, 0>(wa, lane_off, sa2, table);
+        a[0][1] = decode_byte<DT, 0>(wb, lane_off, sb2, table);
+        a[0][2] = decode_byte<DT, 1>(wa, lane_off, sa2, table);
+        a[0][3] = decode_byte<DT, 1>(wb, lane_off, sb2, table);
+        a[1][0] = decode_byte<DT, 2>(wa, lane_off, sa2, table);
+        a[1][1] = decode_byte<DT, 2>(wb, lane_off, sb2, table);
+        a[1][2] = decode_byte<DT, 3>(wa, lane_off, sa2, table);
+        a[1][3] = decode_byte<DT, 3>(wb, lane_off, sb2, table);
+#pragma unroll
+        for (int q = 0; q < NT; q++) {
+            mma16816<DT>(acc[q], a[0], xw[q][4 * w], xw[q][4 * w + 1]);
+            mma16816<DT>(acc[q], a[1], xw[q][4 * w + 2], xw[q][4 * w + 3]);
+        }
     }
 }
 
-// Windows whose code loads are issued together (registers allow fewer as M grows).
-template <int NT> constexpr int kBatch = NT == 1 ? 4 : 2;
+// One window: xr[q] is the lane's activation row of n-tile q (rows past M repeat row M - 1:
+// their outputs are never stored), in shared or global memory; kw is the window's first k.
+template <int DT, int NT, int W>
+__device__ __forceinline__ void run_win(float (&acc)[NT][4], const Win<W>& wc, const float* c2s, float offset,
+                                        const unsigned char* table, uint32_t lane_off,
+                                        const uint16_t* const (&xr)[NT], int64_t kw, int t) {
+    // activation words of chunks C0 .. C1-1 (chunk c: the lane's k 8c .. 8c + 7)
+    uint32_t xw[NT][W / 8];
+    auto load_x = [&](auto c0, auto c1) {
+#pragma unroll
+        for (int q = 0; q < NT; q++)
+#pragma unroll
+            for (int c = decltype(c0)::value; c < decltype(c1)::value; c++) {
+                const uint4 x = *reinterpret_cast<const uint4*>(xr[q] + kw + (W / 4) * t + 8 * c);
+                xw[q][4 * c + 0] = x.x; xw[q][4 * c + 1] = x.y; xw[q][4 * c + 2] = x.z; xw[q][4 * c + 3] = x.w;
+            }
+    };
+    // with three or four n-tiles the second half of a 128-wide window is fetched after the first
+    // half's mma steps (registers)
+    constexpr int CH = (NT >= 3 && W == 128) ? 2 : W / 32;
+    load_x(std::integral_constant<int, 0>{}, std::integral_constant<int, CH>{});
+    const float sa = __fadd_rn(__fmul_rn(c2s[wc.qa], wc.a2a), offset);
+    const float sb = __fadd_rn(__fmul_rn(c2s[wc.qb], wc.a2b), offset);
+    const float2 sa2 = make_float2(sa, sa), sb2 = make_float2(sb, sb);
+    mma_win<DT, NT, W, 0, CH>(acc, wc, sa2, sb2, xw, table, lane_off);
+    if constexpr (CH < W / 32) {
+        load_x(std::integral_constant<int, CH>{}, std::integral_constant<int, W / 32>{});
+        mma_win<DT, NT, W, CH, W / 32>(acc, wc, sa2, sb2, xw, table, lane_off);
+    }
+}
+
+// Windows whose code loads are issued together: 512, 256 or 128 k of codes in flight per lane
+// (registers allow fewer as M grows).
+template <int NT, int W> constexpr int kBatch = (NT == 1 ? 512 : NT == 2 ? 256 : 128) / W;
 constexpr size_t kMaxXs = 72 * 1024;        // largest shared staging of X (two CTAs per SM)
 
-// With XS (M <= 8 and X small enough) X is staged in shared memory (rows padded by 8 elements:
-// conflict-free fragment reads); otherwise it is read from global memory (it stays in L2).
+// With XS (M <= 8 and X small enough) X is staged in shared memory (rows padded by 8 elements);
+// otherwise it is read from global memory (it stays in L2).
 template <int DT, int NT, bool XS>
 __global__ void __launch_bounds__(kLinThreads, 2)
 linear4_nested_kernel(const uint16_t* __restrict__ X, int M, int64_t N, int64_t K,
                       const uint8_t* __restrict__ codes, const uint8_t* __restrict__ absmax_q,
                       const float* __restrict__ code2, const float* __restrict__ absmax2, float offset,
                       const float* __restrict__ code4, int log2_bs, uint16_t* __restrict__ Y) {
-    constexpr int NWARP = kLinThreads / 32;
-    constexpr int B = kBatch<NT>;
-    __shared__ float c2[256];
-    __shared__ float red[NWARP][32][4 * NT];
-    extern __shared__ __align__(16) unsigned char dsm[];       // decode table (32 KB), then X
-    float2* pairs = reinterpret_cast<float2*>(dsm);
-    uint16_t* xs = reinterpret_cast<uint16_t*>(dsm + 256 * kPairReplicas * sizeof(float2));   // [M][K + 8]
+    static_assert(kLinThreads == 256, "the table build gives one thread to each of the 256 code bytes");
+    // windows of 128 k with X in shared memory; of 64 k with X in global memory, where a lane's
+    // 32-byte run keeps the quad's activation loads of a row within one 128-byte line
+    constexpr int WM = XS ? 128 : 64;
+    constexpr int B = kBatch<NT, WM>;
+    __shared__ __align__(16) unsigned char table[kPairBytes];   // decode table; then the split-K partials
+    __shared__ float c2s[256];
+    extern __shared__ __align__(16) uint16_t xs[];              // [M][K + 8] staged X (XS only)
 
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int g = lane >> 2, t = lane & 3;
     const int64_t r0 = (int64_t)blockIdx.x * 16;
     const int64_t ra = r0 + g, rb = r0 + g + 8;
-    const int64_t nwin = K >> 6;
-    const int64_t w_lo = nwin * warp / NWARP, w_hi = nwin * (warp + 1) / NWARP;
+    const int64_t nwin = K / WM;                                 // full-width windows
+    const int64_t w_lo = nwin * warp / kNWarp, w_hi = nwin * (warp + 1) / kNWarp;
     const int64_t xs_stride = K + 8;
+    const int64_t ea0 = ra * K, eb0 = rb * K;                    // first weight of rows g, g + 8
 
     // the first batch of code loads goes out before the tables and X are staged
-    WinCodes wc[B];
+    Win<WM> wc[B];
 #pragma unroll
     for (int i = 0; i < B; i++)
-        if (w_lo + i < w_hi) wc[i] = load_codes(K, codes, absmax_q, absmax2, log2_bs, ra, rb, w_lo + i, t);
+        if (w_lo + i < w_hi)
+            load_win<WM>(wc[i], codes, absmax_q, absmax2, log2_bs, ea0 + (w_lo + i) * WM,
+                         eb0 + (w_lo + i) * WM, t);
     {
-        // code4 held once per warp (lane l: entry l & 15); table entries built by shuffles
-        const float c4 = __ldg(code4 + (lane & 15));
-        if (threadIdx.x < 256) c2[threadIdx.x] = __ldg(code2 + threadIdx.x);
-#pragma unroll 4
-        for (int i = threadIdx.x; i < 256 * kPairReplicas; i += kLinThreads) {
-            const int byte = i / kPairReplicas;
-            const float hi = __shfl_sync(0xffffffffu, c4, byte >> 4);
-            const float lo = __shfl_sync(0xffffffffu, c4, byte & 15);
-            pairs[i] = make_float2(hi, lo);
-        }
+        // thread i writes the 16 replicas of entry i as 8 rotated 16-byte stores (each store
+        // phase of 8 threads covers all 32 banks)
+        const int byte = threadIdx.x;
+        const float hi = __ldg(code4 + (byte >> 4)), lo = __ldg(code4 + (byte & 15));
+        const float4 v = make_float4(hi, lo, hi, lo);
+#pragma unroll
+        for (int r = 0; r < kPairReplicas / 2; r++)
+            *reinterpret_cast<float4*>(table + byte * 128 + ((r + byte) & 7) * 16) = v;
+        c2s[byte] = __ldg(code2 + byte);
     }
-    const float2* pairs_r = pairs + (lane & (kPairReplicas - 1));
     if (XS) {
         // asynchronous 16-byte copies (L2 -> shared), all in flight at once
         const int64_t chunks = (int64_t)M * (K / 8);               // 16-byte chunks of X
@@ -158,6 +221,13 @@ linear4_nested_kernel(const uint16_t* __restrict__ X, int M, int64_t N, int64_t 
     }
     __syncthreads();
 
+    const uint32_t lane_off = (uint32_t)(lane & (kPairReplicas - 1)) * 8u;
+    const uint16_t* xr[NT];
+#pragma unroll
+    for (int q = 0; q < NT; q++) {
+        const int m = min(q * 8 + g, M - 1);
+        xr[q] = XS ? xs + m * xs_stride : X + (int64_t)m * K;
+    }
     float acc[NT][4];
 #pragma unroll
     for (int q = 0; q < NT; q++) acc[q][0] = acc[q][1] = acc[q][2] = acc[q][3] = 0.0f;
@@ -167,28 +237,25 @@ linear4_nested_kernel(const uint16_t* __restrict__ X, int M, int64_t N, int64_t 
         for (int i = 0; i < B; i++) {
             const int64_t win = wb0 + i;
             if (win >= w_hi) break;
-            const int64_t k0 = win * 64 + 16 * t;
-            uint32_t xb[NT][8];
-#pragma unroll
-            for (int q = 0; q < NT; q++) load_x<XS>(X, xs, xs_stride, M, K, q * 8 + g, k0, xb[q]);
-            const float sa = __fadd_rn(__fmul_rn(c2[wc[i].qa], wc[i].a2a), offset);
-            const float sb = __fadd_rn(__fmul_rn(c2[wc[i].qb], wc[i].a2b), offset);
-            uint32_t wa[8], wbv[8];
-            decode16<DT>(wc[i].ca, sa, pairs_r, wa);
-            decode16<DT>(wc[i].cb, sb, pairs_r, wbv);
-            // the same slot of the next batch can be refilled as soon as this one is decoded
-            if (win + B < w_hi) wc[i] = load_codes(K, codes, absmax_q, absmax2, log2_bs, ra, rb, win + B, t);
-#pragma unroll
-            for (int q = 0; q < NT; q++)
-#pragma unroll
-                for (int s = 0; s < 4; s++) {
-                    const uint32_t a[4] = {wa[2 * s], wbv[2 * s], wa[2 * s + 1], wbv[2 * s + 1]};
-                    mma16816<DT>(acc[q], a, xb[q][2 * s], xb[q][2 * s + 1]);
-                }
+            run_win<DT, NT, WM>(acc, wc[i], c2s, offset, table, lane_off, xr, win * WM, t);
+            // the slot is refilled with the window B ahead once this one is decoded
+            if (win + B < w_hi)
+                load_win<WM>(wc[i], codes, absmax_q, absmax2, log2_bs, ea0 + (win + B) * WM,
+                             eb0 + (win + B) * WM, t);
         }
     }
+    if (WM == 128 && (K & 64) && warp == kNWarp - 1) {
+        // the last 64 k of every row
+        Win<64> tw;
+        load_win<64>(tw, codes, absmax_q, absmax2, log2_bs, ea0 + K - 64, eb0 + K - 64, t);
+        run_win<DT, NT, 64>(acc, tw, c2s, offset, table, lane_off, xr, K - 64, t);
+    }
 
-    // split-K partials: warp w's fragment in red[w], summed in warp order by warp 0
+    // split-K partials: warp w's fragment in red[w] (over the table, no longer read), summed in
+    // warp order by warp 0
+    __syncthreads();
+    float (*red)[32][4 * NT] = reinterpret_cast<float (*)[32][4 * NT]>(table);
+    static_assert(kNWarp * 32 * 4 * 4 * sizeof(float) <= kPairBytes, "partials fit over the table");
 #pragma unroll
     for (int q = 0; q < NT; q++)
 #pragma unroll
@@ -201,7 +268,7 @@ linear4_nested_kernel(const uint16_t* __restrict__ X, int M, int64_t N, int64_t 
 #pragma unroll
         for (int i = 0; i < 4; i++) {
             float s = red[0][lane][4 * q + i];
-            for (int w = 1; w < NWARP; w++) s = __fadd_rn(s, red[w][lane][4 * q + i]);
+            for (int w = 1; w < kNWarp; w++) s = __fadd_rn(s, red[w][lane][4 * q + i]);
             y[i] = s;
         }
         // c0, c1: W row g, activation rows 2t, 2t+1; c2, c3: W row g + 8
@@ -223,8 +290,7 @@ cudaError_t launch_nt(const uint16_t* X, int M, int64_t N, int64_t K, const uint
                       const uint8_t* absmax_q, const float* code2, const float* absmax2, float offset,
                       const float* code4, int log2_bs, uint16_t* Y, cudaStream_t s) {
     auto k = linear4_nested_kernel<DT, NT, XS>;
-    constexpr size_t kTable = 256 * kPairReplicas * sizeof(float2);
-    const size_t dyn = kTable + (XS ? (size_t)M * (size_t)(K + 8) * 2 : 0);
+    const size_t dyn = XS ? (size_t)M * (size_t)(K + 8) * 2 : 0;
     {
         // the dynamic shared-memory limit is set once per device (function attributes are per device)
         static std::atomic<uint64_t> attr_set{0};
@@ -233,7 +299,7 @@ cudaError_t launch_nt(const uint16_t* X, int M, int64_t N, int64_t K, const uint
         const uint64_t bit = 1ull << (dev & 63);
         if (!(attr_set.load() & bit)) {
             const cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                       (int)(kTable + (XS ? kMaxXs : 0)));
+                                                       (int)(XS ? kMaxXs : 0));
             if (e != cudaSuccess) return e;
             attr_set.fetch_or(bit);
         }

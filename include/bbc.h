@@ -10,7 +10,9 @@
  *      rebuilt from a General8-coded absmax inside the value-decode kernel,
  *      its unfused three-launch form, and the plain 4-bit decode;
  *   3. the inverse of 2: 4-bit quantization and the nested absmax state
- *      (readings: the pages give only the decode).
+ *      (readings: the pages give only the decode);
+ *   4. the nested 4-bit decode fused into its linear consumer (Y = X W^T with
+ *      the weight decoded in registers, never written to memory).
  *
  * Conventions for every entry point:
  *   - Buffer pointers are DEVICE pointers (memory of the current CUDA device)
@@ -205,9 +207,9 @@ int quantize_4bit(const void* A, int dtype, int64_t n, int blocksize, const floa
  *
  * Defined by: the same decode; the encode steps are readings (no page gives them):
  *   1. codes and fp32 absmax per outer block as quantize_4bit;
- *   2. offset = mean of the outer absmax, computed in binary64 in a fixed order
- *      (partial sums of consecutive chunks of 2048 values in index order, then the
- *      partials in chunk order; divided by the block count; rounded once to fp32);
+ *   2. offset = mean of the outer absmax, summed in binary64 by a fixed pairwise
+ *      tree (the values zero-padded to the next power of two, each node the sum of
+ *      its two halves), divided by the block count, rounded once to fp32;
  *   3. per group of blocksize2 = 256 outer blocks, c_b = fl(absmax_b - offset):
  *      absmax2[g] = max |c_b|,  absmax_q[b] = first i minimising
  *      fabsf(fl(c_b / fmaxf(absmax2[g], 1e-8f)) - code2[i]).
@@ -283,6 +285,40 @@ int dequantize_4bit_nested_chain_noalloc(const uint8_t* codes, const uint8_t* ab
                                          const float* code2, const float* absmax2, float offset,
                                          const float* code4, int64_t n, int blocksize, int blocksize2,
                                          int out_dtype, void* out, void* stream);
+
+/*
+ * linear_4bit_nested - Y = X W^T, with W the nested 4-bit weight of
+ * dequantize_4bit_nested decoded on the fly (W is never written to memory).
+ *
+ * Defined by: "Fuse nested 4-bit scale reconstruction on SM103", Summary and
+ * its timing of the public dequantize-plus-linear paths (the "recurrent grad_A"
+ * and "fallback forward" controls at M = 1, 8 and 32 activation rows). Each
+ * weight is exactly the element dequantize_4bit_nested would write in the
+ * activation type T: w[n][k] = T(fl(code4[nibble(n*K + k)] * scale_b)),
+ * scale_b = fl(fl(code2[absmax_q[b]] * absmax2[b / 256]) + offset),
+ * b = (n*K + k) / blocksize (the weight is the flattened N x K row-major tensor).
+ * The products x*w are exact in fp32 and are summed in fp32 (tensor-core
+ * accumulation, a fixed order: the same inputs give the same bits); each Y
+ * element is rounded once to T. Not bit-exact against a float64 sum: the error
+ * is at most 2*K*2^-24*sum_k |x w| plus half an ulp of T.
+ *
+ *   X        [M][K] activations, row-major, dtype BBC_F16 or BBC_BF16 (T),
+ *            16-byte aligned.
+ *   M        1..32.   N: a multiple of 16.   K: a multiple of 64.
+ *   codes    [N*K/2] uint8 (element 2j in the high nibble of byte j),
+ *            16-byte aligned.
+ *   absmax_q [ceil(N*K/blocksize)] uint8.   code2 [256] fp32.
+ *   absmax2  [ceil(ceil(N*K/blocksize)/256)] fp32.   offset: fp32 by value.
+ *   code4    [16] fp32 value table (NF4 or FP4).
+ *   blocksize  power of two in [32, 4096].   blocksize2: must be 256.
+ *   Y        [M][N] out, row-major, dtype T.
+ * One launch on `stream`. Errors: null pointers, M/N/K < 1, a bad blocksize or
+ * misaligned X/codes -> BBC_ERR_INVALID; another dtype, M > 32, N % 16 != 0,
+ * K % 64 != 0 or blocksize2 != 256 -> BBC_ERR_UNSUPPORTED.
+ */
+int linear_4bit_nested(const void* X, int dtype, int64_t M, int64_t N, int64_t K, const uint8_t* codes,
+                       const uint8_t* absmax_q, const float* code2, const float* absmax2, float offset,
+                       const float* code4, int blocksize, int blocksize2, void* Y, void* stream);
 
 /*
  * bbc_nf_codebook - the 2^K-entry normal-float codebook, on the HOST.

@@ -55,7 +55,9 @@ def test_public_path_control_shapes(bbc, M, N, dt):
 def test_ragged_m_and_blocksizes(bbc, dt):
     # (8, 32, 8192, 64): X too large to stage in shared memory, read from global memory instead
     for M, N, K, bs in [(3, 64, 640, 64), (9, 256, 1024, 32), (17, 128, 4096, 4096), (31, 48, 192, 128),
-                        (2, 16, 64, 32), (8, 32, 8192, 64), (16, 64, 2048, 256)]:
+                        (2, 16, 64, 32), (8, 32, 8192, 64), (16, 64, 2048, 256),
+                        # K % 128 == 64: a 64-wide window ends every row (staged X, X from L2)
+                        (1, 272, 4160, 64), (8, 48, 4160, 32), (24, 32, 1088, 128)]:
         run_case(bbc, M, N, K, bs, dt, seed=M + N)
 
 
@@ -72,5 +74,7 @@ def test_invalid_arguments(bbc):
         bbc.linear_4bit_nested(x[:4, :48].contiguous(), z8, z8, f, f, 0.0, f, 16, 64)
     with pytest.raises(BBCError, match="aligned"):
         bbc.linear_4bit_nested(x[:4], z8[1:], z8, f, f, 0.0, f, 16, 64)
+    with pytest.raises(BBCError, match="aligned"):
+        bbc.linear_4bit_nested(x[:4], z8[8:], z8, f, f, 0.0, f, 16, 64)
     with pytest.raises(BBCError, match="fp16 or bf16"):
         bbc.linear_4bit_nested(x[:4].float(), z8, z8, f, f, 0.0, f, 16, 64)
