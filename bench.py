@@ -58,6 +58,9 @@ def parse_args():
                          "request's public-path control shapes (one JSON line per case)")
     ap.add_argument("--nested-matrix", action="store_true",
                     help="fused vs three-launch nested dequant on the pull request's 24-cell matrix")
+    ap.add_argument("--matrix", action="store_true",
+                    help="the timed configuration cells besides c5: c1 (L2-resident), the c2 k-bit sweep "
+                         "(K=2..5 x fp16/bf16/fp32) and the c4 nested blocksize sweep")
     ap.add_argument("--cpu-seconds", type=float, default=15.0,
                     help="target CPU time of the oracle baseline sample")
     return ap.parse_args()
@@ -543,6 +546,110 @@ def run_linear(args):
                           "max_rel_diff_vs_unfused": round(rel, 6)}), flush=True)
 
 
+def _graph_time(fns, rounds=7):
+    """Median, p10 and p90 device time (us) of one call, from CUDA-graph replays of `fns` (one
+    call per element, cycling through buffer sets), 7 rounds."""
+    import torch
+    for f in fns[:4]:
+        f()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        for f in fns:
+            f()
+    torch.cuda.synchronize()
+    samples = []
+    for _ in range(rounds):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        g.replay()
+        e1.record()
+        torch.cuda.synchronize()
+        samples.append(e0.elapsed_time(e1) / len(fns) * 1e3)
+    del g
+    return statistics.median(samples), pct_of(samples, 0.1), pct_of(samples, 0.9)
+
+
+def run_matrix(args):
+    """The timed configuration cells other than the c5 step.
+
+    c1: 1,048,576 fp32 ~ N(0,1) (seed 0), K=4 quantize and dequantize to fp32: 4.9 MB, so
+        L2-resident: reported as latency, not against the HBM roofline.
+    c2: 4096x4096 ~ N(0,0.02) (seed 1) with 0.1 % outliers x20 (seed 2), K = 2..5 x fp16 / bf16 /
+        fp32, quantize then dequantize; every cell cycles through >= 4 buffer sets holding more
+        than twice the 126 MB L2, so each launch streams from HBM.
+    c4: nested dequant of 8192x8192 (every General8 code present, all 16 value codes), NF4 and
+        FP4, outer blocksizes 32 .. 4096, bf16 and fp32 outputs (>= 168 MB per launch, no reuse).
+    Each cell: CUDA-graph replays (one call per buffer set, host launch cost excluded), 7 rounds,
+    median / p10 / p90; GB/s = algorithmic bytes / median time."""
+    import torch
+
+    import blockwise_bit_codebook_b200 as bbc
+    from blockwise_bit_codebook_b200 import synthetic
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    bbc.load_library()
+    peak, _ = load_peaks()
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    sizes = {torch.float16: 2, torch.bfloat16: 2, torch.float32: 4}
+    names = {torch.float16: "fp16", torch.bfloat16: "bf16", torch.float32: "fp32"}
+
+    def emit(cfg, op, dt, K, n, nbytes, t, nsets, **extra):
+        med, p10, p90 = t
+        print(json.dumps({"config": cfg, "op": op, "dtype": names[dt], "K": K, "n": n, **extra,
+                          "us_median": round(med, 2), "us_p10_p90": [round(p10, 2), round(p90, 2)],
+                          "GB/s": round(nbytes / med / 1e3, 1), "Gelem/s": round(n / med / 1e3, 1),
+                          "frac_of_measured_hbm": round(nbytes / med / 1e3 / peak, 4),
+                          "buffer_sets": nsets}), flush=True)
+
+    def kbit_cells(cfg, n, dt, Ks, x0, l2_resident, reps_per_set):
+        s_in = sizes[dt]
+        nb = (n + 31) // 32
+        for K in Ks:
+            cb = torch.from_numpy(bbc.bbc_nf_codebook(K)).to(dev)
+            qb = n * s_in + nb * K * 4 + nb * 4
+            nsets = 1 if l2_resident else max(4, -(-2 * l2 // qb))
+            xs = [x0.clone() for _ in range(nsets)]
+            packed = [torch.empty(nb * K, dtype=torch.int32, device=dev) for _ in range(nsets)]
+            absmax = [torch.empty(nb, dtype=torch.float32, device=dev) for _ in range(nsets)]
+            outs = [torch.empty(n, dtype=dt, device=dev) for _ in range(nsets)]
+            qf = [(lambda i=i: bbc.kbit_quantize(xs[i], K, cb, absmax=absmax[i], packed=packed[i]))
+                  for i in range(nsets)] * reps_per_set
+            emit(cfg, "quantize", dt, K, n, qb, _graph_time(qf), nsets)
+            df = [(lambda i=i: bbc.kbit_dequantize(packed[i], absmax[i], cb, K, n, dt, out=outs[i]))
+                  for i in range(nsets)] * reps_per_set
+            emit(cfg, "dequantize", dt, K, n, qb, _graph_time(df), nsets)
+            del xs, packed, absmax, outs
+            torch.cuda.empty_cache()
+
+    # c1: L2-resident, one buffer set
+    n1 = 1 << 20
+    x1 = synthetic.weights(n1, std=1.0, seed=0, dtype=torch.float32, device=dev)
+    kbit_cells("c1", n1, torch.float32, [4], x1, True, 200)
+    # c2: the k-bit sweep
+    n2 = 4096 * 4096
+    for dt in (torch.float16, torch.bfloat16, torch.float32):
+        x2 = synthetic.weights(n2, std=0.02, seed=1, dtype=dt, device=dev, outlier_frac=0.001)
+        kbit_cells("c2", n2, dt, [2, 3, 4, 5], x2, False, 8)
+        del x2
+    # c4: nested dequant, blocksize sweep
+    n4 = 8192 * 8192
+    code2 = torch.from_numpy(synthetic.general8_table()).to(dev)
+    tabs = {"nf4": bbc.bbc_nf_codebook(4), "fp4": synthetic.fp4_table()}
+    for bs in (32, 64, 128, 256, 1024, 4096):
+        codes, q, a2, off = synthetic.nested_state(n4, bs, seed=3, device=dev, all_codes=True)
+        for fmt, tab in tabs.items():
+            code4 = torch.from_numpy(tab).to(dev)
+            for dt in (torch.bfloat16, torch.float32):
+                out = torch.empty(n4, dtype=dt, device=dev)
+                nbytes = op_bytes("nested", n4, out_size=sizes[dt], bs=bs)
+                fns = [lambda: bbc.dequantize_4bit_nested(codes, q, code2, a2, float(off), code4, n4, bs, dt,
+                                                          out=out)] * 20
+                emit("c4", "nested_dequant", dt, None, n4, nbytes, _graph_time(fns), 1, format=fmt, blocksize=bs)
+                del out
+
+
 def run_nested_matrix(args):
     """Fused nested dequant vs the unfused three-launch chain on the pull request's matrix.
 
@@ -672,6 +779,8 @@ if __name__ == "__main__":
     a = parse_args()
     if a.linear:
         run_linear(a)
+    elif a.matrix:
+        run_matrix(a)
     elif a.nested_matrix:
         run_nested_matrix(a)
     elif a.impl == "reference":
