@@ -460,15 +460,15 @@ def run_bbc(args):
 # ----------------------------------------------------------------------------- nested matrix
 
 def run_linear(args):
-    """Fused nested 4-bit dequant + linear (linear_4bit_nested) against the unfused sequence
-    (the library's fused nested dequant into a materialised weight, then torch.matmul, i.e.
-    cuBLAS) on the pull request's public-path control shapes: M = 1 and 8 (N = K = 4096) and
-    M = 32 (N = 4096 and 11008, K = 4096); bf16 activations, NF4, outer blocksize 64. CUDA events
-    around CUDA-graph replays of 200 repetitions (device time, no host launch overhead),
-    alternating order, 7 rounds, medians. Two regimes: the same weight every call (it stays in
-    L2, as in the page's timing loop) and "cold", where the calls cycle through copies of the
-    weight state totalling more than L2. Algorithmic bytes of the fused kernel: codes,
-    absmax_q, absmax2, X and Y (the weight is never written)."""
+    """Fused dequant + linear (linear_4bit_nested, linear_kbit) against the unfused sequence (the
+    library's dequant into a materialised weight, then torch.matmul, i.e. cuBLAS) on the pull
+    request's public-path control shapes: M = 1 and 8 (N = K = 4096) and M = 32 (N = 4096 and
+    11008, K = 4096); bf16 activations; the nested NF4 weight (outer blocksize 64) and the k-bit
+    K = 4 weight (blocksize 32). CUDA events around CUDA-graph replays of 200 repetitions (device
+    time, no host launch overhead), alternating order, 7 rounds, medians. Two regimes: the same
+    weight every call (it stays in L2, as in the page's timing loop) and "cold", where the calls
+    cycle through copies of the weight state totalling more than L2. Algorithmic bytes of a fused
+    call: the weight state, X and Y (the weight is never written)."""
     import torch
 
     import blockwise_bit_codebook_b200 as bbc
@@ -481,69 +481,86 @@ def run_linear(args):
     code4 = torch.from_numpy(bbc.bbc_nf_codebook(4)).to(dev)
     code2 = torch.from_numpy(synthetic.general8_table()).to(dev)
     bs = NESTED_BS
+    KB = 4
+    cbk = torch.from_numpy(bbc.bbc_nf_codebook(KB)).to(dev)
     for (M, N, K, label) in [(1, 4096, 4096, "recurrent grad_A M=1"), (8, 4096, 4096, "recurrent grad_A M=8"),
                              (32, 4096, 4096, "fallback forward M=32"),
                              (32, 11008, 4096, "fallback forward M=32 N=11008")]:
-        codes, q, a2, off = synthetic.nested_state(N * K, bs, seed=3, device=dev)
         x = synthetic.weights(M * K, std=1.0, seed=4, dtype=torch.bfloat16, device=dev).reshape(M, K)
         w = torch.empty(N * K, dtype=torch.bfloat16, device=dev)
         y_f = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
         y_u = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
-        # "cold": the calls cycle through copies of the weight state that together exceed the
-        # 126 MB L2, so every call reads its weight from HBM (as successive layers of a model do)
-        ncopy = max(2, -(-160 * 2**20 // (N * K // 2)))
-        copies = [(codes.clone(), q.clone()) for _ in range(ncopy)]
+        for fmt in ("nested_nf4_bs64", f"kbit{KB}"):
+            if fmt.startswith("nested"):
+                codes, q, a2, off = synthetic.nested_state(N * K, bs, seed=3, device=dev)
+                state = (codes, q)
+                nbo = (N * K + bs - 1) // bs
+                wbytes = N * K // 2 + nbo + ((nbo + 255) // 256) * 4
 
-        def fused_on(c, qq):
-            bbc.linear_4bit_nested(x, c, qq, code2, a2, float(off), code4, N, bs, out=y_f)
+                def fused_on(c, qq):
+                    bbc.linear_4bit_nested(x, c, qq, code2, a2, float(off), code4, N, bs, out=y_f)
 
-        def unfused_on(c, qq):
-            bbc.dequantize_4bit_nested(c, qq, code2, a2, float(off), code4, N * K, bs, torch.bfloat16, out=w)
-            torch.matmul(x, w.view(N, K).t(), out=y_u)
-        for i in range(20):
-            (fused_on if i % 2 == 0 else unfused_on)(codes, q)
-        torch.cuda.synchronize()
-        # Host-side call overhead (Python, ctypes) exceeds these kernels' device time, so each
-        # variant's repetitions are captured once in a CUDA graph and the replays are timed.
-        reps = 200
-        graphs = {}
-        for name, fn, cold in (("fused", fused_on, False), ("unfused", unfused_on, False),
-                               ("fused_cold", fused_on, True), ("unfused_cold", unfused_on, True)):
-            gr = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(gr):
-                for r in range(reps):
-                    fn(*(copies[r % ncopy] if cold else (codes, q)))
-            graphs[name] = gr
-        torch.cuda.synchronize()
-        samples = {k: [] for k in graphs}
-        for rnd in range(7):
-            order = list(graphs)
-            if rnd % 2:
-                order.reverse()
-            for name in order:
-                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-                e0.record()
-                graphs[name].replay()
-                e1.record()
-                torch.cuda.synchronize()
-                samples[name].append(e0.elapsed_time(e1) / reps * 1e3)
-        del graphs
-        med = {k: statistics.median(v) for k, v in samples.items()}
-        nbo = (N * K + bs - 1) // bs
-        nbytes = N * K // 2 + nbo + ((nbo + 255) // 256) * 4 + M * K * 2 + M * N * 2
-        rel = float((y_f.float() - y_u.float()).abs().max() / y_u.float().abs().max())
-        print(json.dumps({"case": label, "M": M, "N": N, "K": K, "dtype": "bf16", "format": "nf4", "blocksize": bs,
-                          "fused_us_median": round(med["fused"], 2), "unfused_us_median": round(med["unfused"], 2),
-                          "unfused_over_fused": round(med["unfused"] / med["fused"], 3),
-                          "fused_GBs": round(nbytes / med["fused"] / 1e3, 1),
-                          "fused_frac_of_measured_hbm": round(nbytes / med["fused"] / 1e3 / peak, 4),
-                          "cold_weight_copies": ncopy,
-                          "fused_cold_us_median": round(med["fused_cold"], 2),
-                          "unfused_cold_us_median": round(med["unfused_cold"], 2),
-                          "cold_unfused_over_fused": round(med["unfused_cold"] / med["fused_cold"], 3),
-                          "fused_cold_GBs": round(nbytes / med["fused_cold"] / 1e3, 1),
-                          "fused_cold_frac_of_measured_hbm": round(nbytes / med["fused_cold"] / 1e3 / peak, 4),
-                          "max_rel_diff_vs_unfused": round(rel, 6)}), flush=True)
+                def unfused_on(c, qq):
+                    bbc.dequantize_4bit_nested(c, qq, code2, a2, float(off), code4, N * K, bs, torch.bfloat16,
+                                               out=w)
+                    torch.matmul(x, w.view(N, K).t(), out=y_u)
+            else:
+                state = synthetic.kbit_state(N * K, KB, seed=3, device=dev)
+                wbytes = N * K * KB // 8 + (N * K // 32) * 4
+
+                def fused_on(pk, am):
+                    bbc.linear_kbit(x, pk, am, cbk, KB, N, out=y_f)
+
+                def unfused_on(pk, am):
+                    bbc.kbit_dequantize(pk, am, cbk, KB, N * K, torch.bfloat16, out=w)
+                    torch.matmul(x, w.view(N, K).t(), out=y_u)
+            # "cold": the calls cycle through copies of the weight state that together exceed the
+            # 126 MB L2, so every call reads its weight from HBM (as successive layers of a model do)
+            ncopy = max(2, -(-160 * 2**20 // wbytes))
+            copies = [tuple(t.clone() for t in state) for _ in range(ncopy)]
+            for i in range(20):
+                (fused_on if i % 2 == 0 else unfused_on)(*state)
+            torch.cuda.synchronize()
+            # Host-side call overhead (Python, ctypes) exceeds these kernels' device time, so each
+            # variant's repetitions are captured once in a CUDA graph and the replays are timed.
+            reps = 200
+            graphs = {}
+            for name, fn, cold in (("fused", fused_on, False), ("unfused", unfused_on, False),
+                                   ("fused_cold", fused_on, True), ("unfused_cold", unfused_on, True)):
+                gr = torch.cuda.CUDAGraph()
+                with torch.cuda.graph(gr):
+                    for r in range(reps):
+                        fn(*(copies[r % ncopy] if cold else state))
+                graphs[name] = gr
+            torch.cuda.synchronize()
+            samples = {k: [] for k in graphs}
+            for rnd in range(7):
+                order = list(graphs)
+                if rnd % 2:
+                    order.reverse()
+                for name in order:
+                    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                    e0.record()
+                    graphs[name].replay()
+                    e1.record()
+                    torch.cuda.synchronize()
+                    samples[name].append(e0.elapsed_time(e1) / reps * 1e3)
+            del graphs, copies
+            med = {k: statistics.median(v) for k, v in samples.items()}
+            nbytes = wbytes + M * K * 2 + M * N * 2
+            rel = float((y_f.float() - y_u.float()).abs().max() / y_u.float().abs().max())
+            print(json.dumps({"case": label, "format": fmt, "M": M, "N": N, "K": K, "dtype": "bf16",
+                              "fused_us_median": round(med["fused"], 2), "unfused_us_median": round(med["unfused"], 2),
+                              "unfused_over_fused": round(med["unfused"] / med["fused"], 3),
+                              "fused_GBs": round(nbytes / med["fused"] / 1e3, 1),
+                              "fused_frac_of_measured_hbm": round(nbytes / med["fused"] / 1e3 / peak, 4),
+                              "cold_weight_copies": ncopy,
+                              "fused_cold_us_median": round(med["fused_cold"], 2),
+                              "unfused_cold_us_median": round(med["unfused_cold"], 2),
+                              "cold_unfused_over_fused": round(med["unfused_cold"] / med["fused_cold"], 3),
+                              "fused_cold_GBs": round(nbytes / med["fused_cold"] / 1e3, 1),
+                              "fused_cold_frac_of_measured_hbm": round(nbytes / med["fused_cold"] / 1e3 / peak, 4),
+                              "max_rel_diff_vs_unfused": round(rel, 6)}), flush=True)
 
 
 def _graph_time(fns, rounds=7):

@@ -39,5 +39,6 @@ from ._native import (  # noqa: F401
     quantize_4bit_nested_workspace_bytes,
     library_path,
     linear_4bit_nested,
+    linear_kbit,
     load_library,
 )

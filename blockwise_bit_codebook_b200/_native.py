@@ -44,6 +44,8 @@ def load_library():
     L.quantize_4bit_nested.restype = I
     L.linear_4bit_nested.argtypes = [P, I, I64, I64, I64, P, P, P, P, ct.c_float, P, I, I, P, P]
     L.linear_4bit_nested.restype = I
+    L.linear_kbit.argtypes = [P, I, I64, I64, I64, P, P, P, I, I, P, P]
+    L.linear_kbit.restype = I
     L.kbit_quantize_e4m4.argtypes = [P, I, I64, I, I, P, P, P, P]
     L.kbit_quantize_e4m4.restype = I
     L.kbit_dequantize_e4m4.argtypes = [P, P, P, I, I, I64, I, P, P]
@@ -217,6 +219,20 @@ def linear_4bit_nested(X, codes, absmax_q, code2, absmax2, offset: float, code4,
                               _ptr(absmax2), ct.c_float(offset), _ptr(code4), blocksize, blocksize2, _ptr(out),
                               _stream(stream, X.device))
     _check("linear_4bit_nested", st)
+    return out
+
+
+def linear_kbit(X, packed, absmax, codebook, K: int, N: int, blocksize: int = 32, out=None, stream=None):
+    """Y = X @ W^T for X [M, Kin] (fp16/bf16, M <= 32) and W [N, Kin] the k-bit weight of
+    kbit_quantize (K bits, blocksize 32), decoded in registers. Returns Y [M, N] in X's dtype."""
+    import torch
+    L = load_library()
+    M, Kin = X.shape
+    if out is None:
+        out = torch.empty((M, N), dtype=X.dtype, device=X.device)
+    st = L.linear_kbit(_ptr(X), _dt(X.dtype), M, N, Kin, _ptr(packed), _ptr(absmax), _ptr(codebook), K, blocksize,
+                       _ptr(out), _stream(stream, X.device))
+    _check("linear_kbit", st)
     return out
 
 

@@ -231,6 +231,27 @@ int linear_4bit_nested(const void* X, int dtype, int64_t M, int64_t N, int64_t K
                        "linear_4bit_nested launch");
 }
 
+int linear_kbit(const void* X, int dtype, int64_t M, int64_t N, int64_t K, const uint32_t* packed,
+                const float* absmax, const float* codebook, int bits, int blocksize, void* Y, void* stream) {
+    const char* fn = "linear_kbit";
+    if (!X || !packed || !absmax || !codebook || !Y) return fail(BBC_ERR_INVALID, "%s: null pointer argument", fn);
+    if (M <= 0 || N <= 0 || K <= 0)
+        return fail(BBC_ERR_INVALID, "%s: M, N, K must be >= 1 (got %lld, %lld, %lld)", fn, (long long)M,
+                    (long long)N, (long long)K);
+    if (bits < 2 || bits > 5) return fail(BBC_ERR_INVALID, "%s: bits must be 2..5 (got %d)", fn, bits);
+    if (blocksize != 32) return fail(BBC_ERR_UNSUPPORTED, "%s: blocksize must be 32 (got %d)", fn, blocksize);
+    if (dtype != BBC_F16 && dtype != BBC_BF16)
+        return fail(BBC_ERR_UNSUPPORTED, "%s: activations must be fp16 or bf16 (got dtype %d)", fn, dtype);
+    if (M > 32 || N % 16 != 0 || K % 64 != 0)
+        return fail(BBC_ERR_UNSUPPORTED, "%s: needs M <= 32, N %% 16 == 0, K %% 64 == 0 (got %lld, %lld, %lld)",
+                    fn, (long long)M, (long long)N, (long long)K);
+    if (!aligned(X, 16) || !aligned(packed, 16) || !aligned(Y, 2) || !aligned(absmax, 4) || !aligned(codebook, 4))
+        return fail(BBC_ERR_INVALID, "%s: X and packed must be 16-byte aligned (others: element size)", fn);
+    return cuda_status(bbc::launch_linear_kbit(X, dtype, (int)M, N, K, packed, absmax, codebook, bits, Y,
+                                               static_cast<cudaStream_t>(stream)),
+                       "linear_kbit launch");
+}
+
 int dequantize_4bit_nested_chain(const uint8_t* codes, const uint8_t* absmax_q, const float* code2,
                                  const float* absmax2, float offset, const float* code4,
                                  int64_t n, int blocksize, int blocksize2, int out_dtype, void* out,

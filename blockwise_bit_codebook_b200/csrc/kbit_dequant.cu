@@ -24,19 +24,6 @@ namespace {
 
 constexpr int kThreads = 256;
 
-// Byte offset (idx * 4) of element e (0..7) of a plane group B (byte j = plane j for
-// elements 0..7; B3 = B << 3). For e >= 3 bits 8j+e are moved to bits 34+j of the 64-bit
-// product (multiplier sum_j 2^(34-7j-e)); every cross term lands outside bits 34..37 on
-// distinct positions, so no carry reaches the field. For e < 3 the same gather runs on B3.
-template <int E>
-__device__ __forceinline__ uint32_t plane_offset4(uint32_t B, uint32_t B3) {
-    constexpr int e = E < 3 ? E + 3 : E;
-    constexpr uint32_t mask = 0x01010101u << e;
-    constexpr uint32_t mult = (1u << (34 - e)) | (1u << (27 - e)) | (1u << (20 - e)) | (1u << (13 - e));
-    const uint32_t src = E < 3 ? B3 : B;
-    return __umulhi(src & mask, mult) & 0x3Cu;
-}
-
 template <int K>
 struct BlockIn {
     float am;

@@ -46,6 +46,9 @@ cudaError_t launch_linear_4bit_nested(const void* X, int dtype, int M, int64_t N
                                       const float* absmax2, float offset, const float* code4, int log2_bs,
                                       void* Y, cudaStream_t s);
 
+cudaError_t launch_linear_kbit(const void* X, int dtype, int M, int64_t N, int64_t K, const uint32_t* packed,
+                               const float* absmax, const float* codebook, int KB, void* Y, cudaStream_t s);
+
 // The same two operations with the per-block absmax stored as one E4M4 byte.
 cudaError_t launch_kbit_quantize_e4m4(const void* A, int dtype, int64_t n, int K, const float* codebook,
                                       uint8_t* absmax, uint32_t* packed, bool vec, cudaStream_t s);

@@ -164,6 +164,53 @@ __device__ __forceinline__ void run_win(float (&acc)[NT][4], const Win<W>& wc, c
 template <int NT, int W> constexpr int kBatch = (NT == 1 ? 512 : NT == 2 ? 256 : 128) / W;
 constexpr size_t kMaxXs = 72 * 1024;        // largest shared staging of X (two CTAs per SM)
 
+// X[M][K] into shared memory rows of K + 8 elements with asynchronous 16-byte copies (L2 ->
+// shared), all in flight at once; the caller's barrier publishes them.
+__device__ __forceinline__ void stage_x(const uint16_t* X, uint16_t* xs, int M, int64_t K) {
+    const int64_t chunks = (int64_t)M * (K / 8);
+    const int64_t xs_stride = K + 8;
+    const uint32_t xs_s = (uint32_t)__cvta_generic_to_shared(xs);
+    for (int64_t c = threadIdx.x; c < chunks; c += kLinThreads) {
+        const int64_t m = c / (K / 8), kk = (c % (K / 8)) * 8;
+        asm volatile("cp.async.cg.shared.global [%0], [%1], 16;"
+                     :: "r"(xs_s + (uint32_t)((m * xs_stride + kk) * 2)), "l"(X + m * K + kk) : "memory");
+    }
+    asm volatile("cp.async.commit_group;\ncp.async.wait_group 0;" ::: "memory");
+}
+
+// Split-K partials: warp w's fragment in red[w], summed in warp order by warp 0, which rounds
+// each sum once to T and stores it (c0, c1: W row g, activation rows 2t, 2t + 1; c2, c3: row
+// g + 8). Called by every thread of the CTA after the last read of whatever `red` overlays.
+template <int DT, int NT>
+__device__ __forceinline__ void reduce_store(float (*red)[32][4 * NT], const float (&acc)[NT][4], int M,
+                                             int64_t N, int64_t ra, int64_t rb, uint16_t* Y) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, t = lane & 3;
+    __syncthreads();
+#pragma unroll
+    for (int q = 0; q < NT; q++)
+#pragma unroll
+        for (int i = 0; i < 4; i++) red[warp][lane][4 * q + i] = acc[q][i];
+    __syncthreads();
+    if (warp != 0) return;
+#pragma unroll
+    for (int q = 0; q < NT; q++) {
+        float y[4];
+#pragma unroll
+        for (int i = 0; i < 4; i++) {
+            float s = red[0][lane][4 * q + i];
+            for (int w = 1; w < kNWarp; w++) s = __fadd_rn(s, red[w][lane][4 * q + i]);
+            y[i] = s;
+        }
+        const int m0 = q * 8 + 2 * t;
+#pragma unroll
+        for (int i = 0; i < 4; i++) {
+            const int m = m0 + (i & 1);
+            const int64_t nn = (i < 2) ? ra : rb;
+            if (m < M) Y[(int64_t)m * N + nn] = DT == BF16 ? f32_to_bf16_bits(y[i]) : f32_to_f16_bits(y[i]);
+        }
+    }
+}
+
 // With XS (M <= 8 and X small enough) X is staged in shared memory (rows padded by 8 elements);
 // otherwise it is read from global memory (it stays in L2).
 template <int DT, int NT, bool XS>
@@ -187,7 +234,6 @@ linear4_nested_kernel(const uint16_t* __restrict__ X, int M, int64_t N, int64_t 
     const int64_t ra = r0 + g, rb = r0 + g + 8;
     const int64_t nwin = K / WM;                                 // full-width windows
     const int64_t w_lo = nwin * warp / kNWarp, w_hi = nwin * (warp + 1) / kNWarp;
-    const int64_t xs_stride = K + 8;
     const int64_t ea0 = ra * K, eb0 = rb * K;                    // first weight of rows g, g + 8
 
     // the first batch of code loads goes out before the tables and X are staged
@@ -208,17 +254,7 @@ linear4_nested_kernel(const uint16_t* __restrict__ X, int M, int64_t N, int64_t 
             *reinterpret_cast<float4*>(table + byte * 128 + ((r + byte) & 7) * 16) = v;
         c2s[byte] = __ldg(code2 + byte);
     }
-    if (XS) {
-        // asynchronous 16-byte copies (L2 -> shared), all in flight at once
-        const int64_t chunks = (int64_t)M * (K / 8);               // 16-byte chunks of X
-        const uint32_t xs_s = (uint32_t)__cvta_generic_to_shared(xs);
-        for (int64_t c = threadIdx.x; c < chunks; c += kLinThreads) {
-            const int64_t m = c / (K / 8), kk = (c % (K / 8)) * 8;
-            asm volatile("cp.async.cg.shared.global [%0], [%1], 16;"
-                         :: "r"(xs_s + (uint32_t)((m * xs_stride + kk) * 2)), "l"(X + m * K + kk) : "memory");
-        }
-        asm volatile("cp.async.commit_group;\ncp.async.wait_group 0;" ::: "memory");
-    }
+    if (XS) stage_x(X, xs, M, K);
     __syncthreads();
 
     const uint32_t lane_off = (uint32_t)(lane & (kPairReplicas - 1)) * 8u;
@@ -226,7 +262,7 @@ linear4_nested_kernel(const uint16_t* __restrict__ X, int M, int64_t N, int64_t 
 #pragma unroll
     for (int q = 0; q < NT; q++) {
         const int m = min(q * 8 + g, M - 1);
-        xr[q] = XS ? xs + m * xs_stride : X + (int64_t)m * K;
+        xr[q] = XS ? xs + m * (K + 8) : X + (int64_t)m * K;
     }
     float acc[NT][4];
 #pragma unroll
@@ -250,60 +286,207 @@ linear4_nested_kernel(const uint16_t* __restrict__ X, int M, int64_t N, int64_t 
         load_win<64>(tw, codes, absmax_q, absmax2, log2_bs, ea0 + K - 64, eb0 + K - 64, t);
         run_win<DT, NT, 64>(acc, tw, c2s, offset, table, lane_off, xr, K - 64, t);
     }
-
-    // split-K partials: warp w's fragment in red[w] (over the table, no longer read), summed in
-    // warp order by warp 0
-    __syncthreads();
-    float (*red)[32][4 * NT] = reinterpret_cast<float (*)[32][4 * NT]>(table);
+    // the partials overlay the decode table, which no warp reads any more after the barrier
     static_assert(kNWarp * 32 * 4 * 4 * sizeof(float) <= kPairBytes, "partials fit over the table");
+    reduce_store<DT, NT>(reinterpret_cast<float (*)[32][4 * NT]>(table), acc, M, N, ra, rb, Y);
+}
+
+// ---- k-bit weights (K = 2..5, blocksize 32, bit-plane packed, fp32 absmax) ----
+//
+// The weight of the k-bit patch series' dequantize_kbit: w[n][k] = T(fl(codebook[idx] *
+// absmax[b])) for flattened element m = n*K + k in block b = m / 32, idx gathered from the K
+// plane words of block b. With K % 64 == 0 blocks never straddle rows, and the lane's run of a
+// window (32 k for 128-wide windows, 16 for 64-wide) lies in one block: one absmax and the
+// block's K words per row per window. Each element's index is gathered from the byte-transposed
+// plane groups with one multiply-high (as in the dequant kernel), looked up in a 32-float shared
+// codebook (every entry its own bank), multiplied by the absmax and rounded to T in pairs.
+
+template <int KB>
+struct KWin {
+    uint32_t wa[KB], wb[KB];              // plane words of the block holding the lane's run, rows g, g + 8
+    float ama, amb;                       // and the blocks' absmax
+};
+
+// ea, eb: flattened index of the window's first weight in rows g and g + 8. `packed` is 16-byte
+// aligned, so block b's words start on a 16-byte (K = 4) or 8-byte (K = 2) boundary.
+template <int KB, int W>
+__device__ __forceinline__ void load_kwin(KWin<KB>& r, const uint32_t* packed, const float* absmax, int64_t ea,
+                                          int64_t eb, int t) {
+    const int64_t ba = (ea + (W / 4) * t) >> 5, bb = (eb + (W / 4) * t) >> 5;
+    const uint32_t* pa = packed + ba * KB;
+    const uint32_t* pb = packed + bb * KB;
+    if constexpr (KB == 4) {
+        const uint4 a = __ldg(reinterpret_cast<const uint4*>(pa)), b = __ldg(reinterpret_cast<const uint4*>(pb));
+        r.wa[0] = a.x; r.wa[1] = a.y; r.wa[2 % KB] = a.z; r.wa[3 % KB] = a.w;
+        r.wb[0] = b.x; r.wb[1] = b.y; r.wb[2 % KB] = b.z; r.wb[3 % KB] = b.w;
+    } else if constexpr (KB == 2) {
+        const uint2 a = __ldg(reinterpret_cast<const uint2*>(pa)), b = __ldg(reinterpret_cast<const uint2*>(pb));
+        r.wa[0] = a.x; r.wa[1 % KB] = a.y;
+        r.wb[0] = b.x; r.wb[1 % KB] = b.y;
+    } else {
+#pragma unroll
+        for (int j = 0; j < KB; j++) { r.wa[j] = ldg_u32(pa + j); r.wb[j] = ldg_u32(pb + j); }
+    }
+    r.ama = __ldg(absmax + ba);
+    r.amb = __ldg(absmax + bb);
+}
+
+// Eight weights (elements 8q .. 8q+7 of a block) as four packed pairs of T, from plane group Bq
+// (byte j = plane j of those elements) and, for K = 5, p4q (bit i = plane 4 of element 8q + i).
+template <int KB, int DT, int E>
+__device__ __forceinline__ float kbit_elem(uint32_t Bq, uint32_t Bqs, uint32_t p4q, float am, const char* cbb) {
+    uint32_t off = plane_offset4<E>(Bq, Bqs);
+    if constexpr (KB == 5) off |= (E <= 6 ? (p4q << (6 - E)) : (p4q >> (E - 6))) & 0x40u;
+    return __fmul_rn(*reinterpret_cast<const float*>(cbb + off), am);
+}
+template <int KB, int DT>
+__device__ __forceinline__ void kbit_group(uint32_t Bq, uint32_t p4q, float am, const char* cbb, uint32_t (&pr)[4]) {
+    const uint32_t Bqs = Bq << 3;
+    const float y0 = kbit_elem<KB, DT, 0>(Bq, Bqs, p4q, am, cbb), y1 = kbit_elem<KB, DT, 1>(Bq, Bqs, p4q, am, cbb);
+    const float y2 = kbit_elem<KB, DT, 2>(Bq, Bqs, p4q, am, cbb), y3 = kbit_elem<KB, DT, 3>(Bq, Bqs, p4q, am, cbb);
+    const float y4 = kbit_elem<KB, DT, 4>(Bq, Bqs, p4q, am, cbb), y5 = kbit_elem<KB, DT, 5>(Bq, Bqs, p4q, am, cbb);
+    const float y6 = kbit_elem<KB, DT, 6>(Bq, Bqs, p4q, am, cbb), y7 = kbit_elem<KB, DT, 7>(Bq, Bqs, p4q, am, cbb);
+    pr[0] = DT == BF16 ? pack_bf16x2(y0, y1) : pack_f16x2(y0, y1);
+    pr[1] = DT == BF16 ? pack_bf16x2(y2, y3) : pack_f16x2(y2, y3);
+    pr[2] = DT == BF16 ? pack_bf16x2(y4, y5) : pack_f16x2(y4, y5);
+    pr[3] = DT == BF16 ? pack_bf16x2(y6, y7) : pack_f16x2(y6, y7);
+}
+
+// The plane groups of a lane's run: all four for a 32-element run; for a 16-element run, the
+// two groups of half h of the block.
+template <int KB, int R>
+__device__ __forceinline__ void kbit_groups(const uint32_t (&w)[KB], int h, uint32_t (&G)[R / 8], uint32_t& p4) {
+    const uint32_t w0 = w[0], w1 = w[1 % KB], w2 = KB > 2 ? w[2 % KB] : 0u, w3 = KB > 3 ? w[3 % KB] : 0u;
+    p4 = KB == 5 ? w[4 % KB] : 0u;
+    if constexpr (R == 32) {
+        const uint32_t t0 = prmt(w0, w1, 0x5140u), t1 = prmt(w0, w1, 0x7362u);
+        const uint32_t t2 = prmt(w2, w3, 0x5140u), t3 = prmt(w2, w3, 0x7362u);
+        G[0] = prmt(t0, t2, 0x5410u);
+        G[1] = prmt(t0, t2, 0x7632u);
+        G[2] = prmt(t1, t3, 0x5410u);
+        G[3] = prmt(t1, t3, 0x7632u);
+    } else {
+        const uint32_t sel = h ? 0x7362u : 0x5140u;            // bytes 2h, 2h + 1 of two words
+        const uint32_t tl = prmt(w0, w1, sel), th = prmt(w2, w3, sel);
+        G[0] = prmt(tl, th, 0x5410u);
+        G[1] = prmt(tl, th, 0x7632u);
+        p4 >>= 16 * h;
+    }
+}
+
+// One window of width W: the lane's run of W/4 weights in rows g and g + 8, decoded group by
+// group (8 weights = one code word's worth of mma steps) into the same fragments as the nested
+// kernel's.
+template <int DT, int NT, int KB, int W>
+__device__ __forceinline__ void run_kwin(float (&acc)[NT][4], const KWin<KB>& wc, const char* cbb,
+                                         const uint16_t* const (&xr)[NT], int64_t kw, int t) {
+    constexpr int R = W / 4;
+    uint32_t xw[NT][W / 8];
 #pragma unroll
     for (int q = 0; q < NT; q++)
 #pragma unroll
-        for (int i = 0; i < 4; i++) red[warp][lane][4 * q + i] = acc[q][i];
-    __syncthreads();
-    if (warp != 0) return;
-#pragma unroll
-    for (int q = 0; q < NT; q++) {
-        float y[4];
-#pragma unroll
-        for (int i = 0; i < 4; i++) {
-            float s = red[0][lane][4 * q + i];
-            for (int w = 1; w < kNWarp; w++) s = __fadd_rn(s, red[w][lane][4 * q + i]);
-            y[i] = s;
+        for (int c = 0; c < R / 8; c++) {
+            const uint4 x = *reinterpret_cast<const uint4*>(xr[q] + kw + R * t + 8 * c);
+            xw[q][4 * c + 0] = x.x; xw[q][4 * c + 1] = x.y; xw[q][4 * c + 2] = x.z; xw[q][4 * c + 3] = x.w;
         }
-        // c0, c1: W row g, activation rows 2t, 2t+1; c2, c3: W row g + 8
-        const int m0 = q * 8 + 2 * t;
+    uint32_t Ga[R / 8], Gb[R / 8], p4a, p4b;
+    kbit_groups<KB, R>(wc.wa, t & 1, Ga, p4a);
+    kbit_groups<KB, R>(wc.wb, t & 1, Gb, p4b);
 #pragma unroll
-        for (int i = 0; i < 4; i++) {
-            const int m = m0 + (i & 1);
-            const int64_t nn = (i < 2) ? ra : rb;
-            if (m < M) {
-                const uint16_t h = DT == BF16 ? f32_to_bf16_bits(y[i]) : f32_to_f16_bits(y[i]);
-                Y[(int64_t)m * N + nn] = h;
-            }
+    for (int w = 0; w < R / 8; w++) {
+        uint32_t pa[4], pb[4];
+        kbit_group<KB, DT>(Ga[w], p4a >> (8 * w), wc.ama, cbb, pa);
+        kbit_group<KB, DT>(Gb[w], p4b >> (8 * w), wc.amb, cbb, pb);
+        const uint32_t a0[4] = {pa[0], pb[0], pa[1], pb[1]};
+        const uint32_t a1[4] = {pa[2], pb[2], pa[3], pb[3]};
+#pragma unroll
+        for (int q = 0; q < NT; q++) {
+            mma16816<DT>(acc[q], a0, xw[q][4 * w], xw[q][4 * w + 1]);
+            mma16816<DT>(acc[q], a1, xw[q][4 * w + 2], xw[q][4 * w + 3]);
         }
     }
 }
+
+template <int DT, int NT, bool XS, int KB>
+__global__ void __launch_bounds__(kLinThreads, 2)
+linear_kbit_kernel(const uint16_t* __restrict__ X, int M, int64_t N, int64_t K,
+                   const uint32_t* __restrict__ packed, const float* __restrict__ absmax,
+                   const float* __restrict__ codebook, uint16_t* __restrict__ Y) {
+    constexpr int WM = XS ? 128 : 64;
+    constexpr int B = kBatch<NT, WM> < 4 ? kBatch<NT, WM> : 4;   // a window holds 2 (K + 1) registers
+    __shared__ float cbs[32];
+    __shared__ __align__(16) float red[kNWarp][32][4 * NT];    // the split-K partials
+    extern __shared__ __align__(16) uint16_t xs[];              // [M][K + 8] staged X (XS only)
+
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int g = lane >> 2, t = lane & 3;
+    const int64_t r0 = (int64_t)blockIdx.x * 16;
+    const int64_t ra = r0 + g, rb = r0 + g + 8;
+    const int64_t nwin = K / WM;
+    const int64_t w_lo = nwin * warp / kNWarp, w_hi = nwin * (warp + 1) / kNWarp;
+    const int64_t ea0 = ra * K, eb0 = rb * K;
+
+    KWin<KB> wc[B];
+#pragma unroll
+    for (int i = 0; i < B; i++)
+        if (w_lo + i < w_hi) load_kwin<KB, WM>(wc[i], packed, absmax, ea0 + (w_lo + i) * WM, eb0 + (w_lo + i) * WM, t);
+    if (threadIdx.x < 32) cbs[threadIdx.x] = threadIdx.x < (1 << KB) ? __ldg(codebook + threadIdx.x) : 0.0f;
+    if (XS) stage_x(X, xs, M, K);
+    __syncthreads();
+
+    const char* cbb = reinterpret_cast<const char*>(cbs);
+    const uint16_t* xr[NT];
+#pragma unroll
+    for (int q = 0; q < NT; q++) {
+        const int m = min(q * 8 + g, M - 1);
+        xr[q] = XS ? xs + m * (K + 8) : X + (int64_t)m * K;
+    }
+    float acc[NT][4];
+#pragma unroll
+    for (int q = 0; q < NT; q++) acc[q][0] = acc[q][1] = acc[q][2] = acc[q][3] = 0.0f;
+
+    for (int64_t wb0 = w_lo; wb0 < w_hi; wb0 += B) {
+#pragma unroll
+        for (int i = 0; i < B; i++) {
+            const int64_t win = wb0 + i;
+            if (win >= w_hi) break;
+            run_kwin<DT, NT, KB, WM>(acc, wc[i], cbb, xr, win * WM, t);
+            if (win + B < w_hi)
+                load_kwin<KB, WM>(wc[i], packed, absmax, ea0 + (win + B) * WM, eb0 + (win + B) * WM, t);
+        }
+    }
+    if (WM == 128 && (K & 64) && warp == kNWarp - 1) {
+        KWin<KB> tw;
+        load_kwin<KB, 64>(tw, packed, absmax, ea0 + K - 64, eb0 + K - 64, t);
+        run_kwin<DT, NT, KB, 64>(acc, tw, cbb, xr, K - 64, t);
+    }
+    reduce_store<DT, NT>(red, acc, M, N, ra, rb, Y);
+}
+
+// The dynamic shared-memory limit of kernel `k` raised to `bytes`, once per device (function
+// attributes are per device); one flag word per kernel instantiation.
+template <typename Kernel>
+cudaError_t allow_dyn_smem(Kernel k, std::atomic<uint64_t>& done, size_t bytes) {
+    int dev = 0;
+    cudaGetDevice(&dev);
+    const uint64_t bit = 1ull << (dev & 63);
+    if (done.load() & bit) return cudaSuccess;
+    const cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+    if (e == cudaSuccess) done.fetch_or(bit);
+    return e;
+}
+
+bool stage_in_smem(int M, int64_t K) { return M <= 8 && (size_t)M * (size_t)(K + 8) * 2 <= kMaxXs; }
 
 template <int DT, int NT, bool XS>
 cudaError_t launch_nt(const uint16_t* X, int M, int64_t N, int64_t K, const uint8_t* codes,
                       const uint8_t* absmax_q, const float* code2, const float* absmax2, float offset,
                       const float* code4, int log2_bs, uint16_t* Y, cudaStream_t s) {
     auto k = linear4_nested_kernel<DT, NT, XS>;
+    static std::atomic<uint64_t> attr{0};
+    const cudaError_t e = allow_dyn_smem(k, attr, XS ? kMaxXs : 0);
+    if (e != cudaSuccess) return e;
     const size_t dyn = XS ? (size_t)M * (size_t)(K + 8) * 2 : 0;
-    {
-        // the dynamic shared-memory limit is set once per device (function attributes are per device)
-        static std::atomic<uint64_t> attr_set{0};
-        int dev = 0;
-        cudaGetDevice(&dev);
-        const uint64_t bit = 1ull << (dev & 63);
-        if (!(attr_set.load() & bit)) {
-            const cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                       (int)(XS ? kMaxXs : 0));
-            if (e != cudaSuccess) return e;
-            attr_set.fetch_or(bit);
-        }
-    }
     k<<<(unsigned)(N / 16), kLinThreads, dyn, s>>>(X, M, N, K, codes, absmax_q, code2, absmax2, offset, code4,
                                                    log2_bs, Y);
     return cudaGetLastError();
@@ -315,12 +498,48 @@ cudaError_t launch_dt(const uint16_t* X, int M, int64_t N, int64_t K, const uint
                       const float* code4, int log2_bs, uint16_t* Y, cudaStream_t s) {
     switch ((M + 7) / 8) {
         case 1:
-            if ((size_t)M * (size_t)(K + 8) * 2 <= kMaxXs)
+            if (stage_in_smem(M, K))
                 return launch_nt<DT, 1, true>(X, M, N, K, codes, absmax_q, code2, absmax2, offset, code4, log2_bs, Y, s);
             return launch_nt<DT, 1, false>(X, M, N, K, codes, absmax_q, code2, absmax2, offset, code4, log2_bs, Y, s);
         case 2: return launch_nt<DT, 2, false>(X, M, N, K, codes, absmax_q, code2, absmax2, offset, code4, log2_bs, Y, s);
         case 3: return launch_nt<DT, 3, false>(X, M, N, K, codes, absmax_q, code2, absmax2, offset, code4, log2_bs, Y, s);
         default: return launch_nt<DT, 4, false>(X, M, N, K, codes, absmax_q, code2, absmax2, offset, code4, log2_bs, Y, s);
+    }
+}
+
+template <int DT, int NT, bool XS, int KB>
+cudaError_t launch_kbit_nt(const uint16_t* X, int M, int64_t N, int64_t K, const uint32_t* packed,
+                           const float* absmax, const float* codebook, uint16_t* Y, cudaStream_t s) {
+    auto k = linear_kbit_kernel<DT, NT, XS, KB>;
+    static std::atomic<uint64_t> attr{0};
+    const cudaError_t e = allow_dyn_smem(k, attr, XS ? kMaxXs : 0);
+    if (e != cudaSuccess) return e;
+    const size_t dyn = XS ? (size_t)M * (size_t)(K + 8) * 2 : 0;
+    k<<<(unsigned)(N / 16), kLinThreads, dyn, s>>>(X, M, N, K, packed, absmax, codebook, Y);
+    return cudaGetLastError();
+}
+
+template <int DT, int KB>
+cudaError_t launch_kbit_k(const uint16_t* X, int M, int64_t N, int64_t K, const uint32_t* packed,
+                          const float* absmax, const float* codebook, uint16_t* Y, cudaStream_t s) {
+    switch ((M + 7) / 8) {
+        case 1:
+            if (stage_in_smem(M, K)) return launch_kbit_nt<DT, 1, true, KB>(X, M, N, K, packed, absmax, codebook, Y, s);
+            return launch_kbit_nt<DT, 1, false, KB>(X, M, N, K, packed, absmax, codebook, Y, s);
+        case 2: return launch_kbit_nt<DT, 2, false, KB>(X, M, N, K, packed, absmax, codebook, Y, s);
+        case 3: return launch_kbit_nt<DT, 3, false, KB>(X, M, N, K, packed, absmax, codebook, Y, s);
+        default: return launch_kbit_nt<DT, 4, false, KB>(X, M, N, K, packed, absmax, codebook, Y, s);
+    }
+}
+
+template <int DT>
+cudaError_t launch_kbit_dt(const uint16_t* X, int M, int64_t N, int64_t K, const uint32_t* packed,
+                           const float* absmax, const float* codebook, int KB, uint16_t* Y, cudaStream_t s) {
+    switch (KB) {
+        case 2: return launch_kbit_k<DT, 2>(X, M, N, K, packed, absmax, codebook, Y, s);
+        case 3: return launch_kbit_k<DT, 3>(X, M, N, K, packed, absmax, codebook, Y, s);
+        case 4: return launch_kbit_k<DT, 4>(X, M, N, K, packed, absmax, codebook, Y, s);
+        default: return launch_kbit_k<DT, 5>(X, M, N, K, packed, absmax, codebook, Y, s);
     }
 }
 
@@ -334,6 +553,14 @@ cudaError_t launch_linear_4bit_nested(const void* X, int dtype, int M, int64_t N
     uint16_t* y = static_cast<uint16_t*>(Y);
     if (dtype == BF16) return launch_dt<BF16>(x, M, N, K, codes, absmax_q, code2, absmax2, offset, code4, log2_bs, y, s);
     return launch_dt<F16>(x, M, N, K, codes, absmax_q, code2, absmax2, offset, code4, log2_bs, y, s);
+}
+
+cudaError_t launch_linear_kbit(const void* X, int dtype, int M, int64_t N, int64_t K, const uint32_t* packed,
+                               const float* absmax, const float* codebook, int KB, void* Y, cudaStream_t s) {
+    const uint16_t* x = static_cast<const uint16_t*>(X);
+    uint16_t* y = static_cast<uint16_t*>(Y);
+    if (dtype == BF16) return launch_kbit_dt<BF16>(x, M, N, K, packed, absmax, codebook, KB, y, s);
+    return launch_kbit_dt<F16>(x, M, N, K, packed, absmax, codebook, KB, y, s);
 }
 
 }  // namespace bbc

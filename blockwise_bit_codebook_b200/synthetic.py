@@ -71,3 +71,13 @@ def nested_state(n: int, blocksize: int, seed: int = 3, device="cpu", all_codes:
                          dtype=torch.float32) * 0.09 + 0.01
     offset = float(torch.randn(1, generator=_gen(seed + 3, "cpu"), dtype=torch.float32)[0] * 0.005 + 0.03)
     return codes, absmax_q, absmax2, np.float32(offset)
+
+
+def kbit_state(n: int, K: int, seed: int = 5, device="cpu"):
+    """A k-bit weight state for n elements (blocksize 32): uniformly random bit-plane words, so
+    every index 0 .. 2^K - 1 occurs, and per-block absmax ~ U(0.01, 0.1)."""
+    nb = (n + 31) // 32
+    packed = torch.randint(-2 ** 31, 2 ** 31, (nb * K,), generator=_gen(seed, device), device=device,
+                           dtype=torch.int64).to(torch.int32)
+    absmax = torch.rand(nb, generator=_gen(seed + 1, device), device=device, dtype=torch.float32) * 0.09 + 0.01
+    return packed, absmax

@@ -11,8 +11,8 @@
  *      its unfused three-launch form, and the plain 4-bit decode;
  *   3. the inverse of 2: 4-bit quantization and the nested absmax state
  *      (readings: the pages give only the decode);
- *   4. the nested 4-bit decode fused into its linear consumer (Y = X W^T with
- *      the weight decoded in registers, never written to memory).
+ *   4. the nested 4-bit and the k-bit decode fused into their linear consumer
+ *      (Y = X W^T with the weight decoded in registers, never written to memory).
  *
  * Conventions for every entry point:
  *   - Buffer pointers are DEVICE pointers (memory of the current CUDA device)
@@ -319,6 +319,34 @@ int dequantize_4bit_nested_chain_noalloc(const uint8_t* codes, const uint8_t* ab
 int linear_4bit_nested(const void* X, int dtype, int64_t M, int64_t N, int64_t K, const uint8_t* codes,
                        const uint8_t* absmax_q, const float* code2, const float* absmax2, float offset,
                        const float* code4, int blocksize, int blocksize2, void* Y, void* stream);
+
+/*
+ * linear_kbit - Y = X W^T, with W the k-bit weight of kbit_quantize decoded on
+ * the fly (W is never written to memory).
+ *
+ * Defined by: the k-bit patch series, dequantize_kbit (the decode) followed by
+ * a linear layer, the consumer the nested-dequant pull request times on its
+ * public paths ("Fuse nested 4-bit scale reconstruction on SM103", Summary).
+ * Each weight is exactly the element kbit_dequantize would write in the
+ * activation type T: w[n][k] = T(fl(codebook[idx(m)] * absmax[m / 32])) for the
+ * flattened element m = n*K + k of the N x K row-major weight. Accumulation and
+ * error bound as linear_4bit_nested (fp32 tensor-core sums in a fixed order,
+ * at most 2*K*2^-24*sum_k |x w| plus half an ulp of T from the float64 result).
+ *
+ *   X        [M][K] activations, row-major, dtype BBC_F16 or BBC_BF16 (T),
+ *            16-byte aligned.
+ *   M        1..32.   N: a multiple of 16.   K: a multiple of 64.
+ *   packed   [N*K/32 * bits] uint32 bit-plane words (kbit_quantize layout),
+ *            16-byte aligned.
+ *   absmax   [N*K/32] fp32.   codebook: [2^bits] fp32.
+ *   bits     2..5 (the K of kbit_quantize).   blocksize: must be 32.
+ *   Y        [M][N] out, row-major, dtype T.
+ * One launch on `stream`. Errors: null pointers, M/N/K < 1, bits outside 2..5
+ * or misaligned X/packed -> BBC_ERR_INVALID; another dtype, M > 32,
+ * N % 16 != 0, K % 64 != 0 or blocksize != 32 -> BBC_ERR_UNSUPPORTED.
+ */
+int linear_kbit(const void* X, int dtype, int64_t M, int64_t N, int64_t K, const uint32_t* packed,
+                const float* absmax, const float* codebook, int bits, int blocksize, void* Y, void* stream);
 
 /*
  * bbc_nf_codebook - the 2^K-entry normal-float codebook, on the HOST.

@@ -256,6 +256,17 @@ def linear_4bit_nested(X, x_dtype: str, N: int, K: int, state, code2, code4, blo
     return Xf @ W.T, np.abs(Xf) @ np.abs(W).T
 
 
+def linear_kbit(X, x_dtype: str, N: int, Kin: int, packed, absmax, codebook, K: int):
+    """Y = X @ W^T with W[N, Kin] the k-bit weight dequantized to x_dtype (kbit_dequantize of the
+    flattened N*Kin codes, as the unfused dequantize-then-linear path materialises it). Returns
+    (Y64, S) as linear_4bit_nested. X: [M, Kin] raw 16-bit patterns of x_dtype."""
+    Wb = kbit_dequantize(packed, absmax, codebook, K, N * Kin, x_dtype)
+    widen = f16_bits_to_f32 if x_dtype == "f16" else bf16_bits_to_f32
+    W = widen(Wb).astype(np.float64).reshape(N, Kin)
+    Xf = widen(_c(X, np.uint16).reshape(-1)).astype(np.float64).reshape(-1, Kin)
+    return Xf @ W.T, np.abs(Xf) @ np.abs(W).T
+
+
 def nested_scale(code2_val: float, absmax2_val: float, offset: float) -> float:
     """fl(fl(code2 * absmax2) + offset) in fp32, returned as a Python float."""
     return float(np.float32(lib().orc_nested_scale(code2_val, absmax2_val, offset)))

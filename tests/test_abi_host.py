@@ -34,7 +34,7 @@ def test_header_declares_the_boundary():
     assert {"kbit_quantize", "kbit_dequantize", "dequantize_4bit_nested", "dequantize_4bit",
             "dequantize_4bit_nested_chain", "bbc_nf_codebook", "bbc_last_error",
             "kbit_quantize_e4m4", "kbit_dequantize_e4m4", "quantize_4bit", "quantize_4bit_nested",
-            "quantize_4bit_nested_workspace_bytes"} <= names
+            "quantize_4bit_nested_workspace_bytes", "linear_4bit_nested", "linear_kbit"} <= names
 
 
 def test_library_exports_every_declared_symbol(lib):
@@ -149,6 +149,26 @@ def test_plain_and_chain_validation(lib):
     assert chain(ws=P(0x1002)) == 1
     assert chain(bs=16) == 1
     assert chain(bs2=128) == 2
+
+
+def test_linear_validation(lib):
+    """Both fused linear entries reject bad arguments on the host (the pointers are never read)."""
+    lib.linear_kbit.argtypes = [ct.c_void_p, ct.c_int, ct.c_int64, ct.c_int64, ct.c_int64, ct.c_void_p,
+                                ct.c_void_p, ct.c_void_p, ct.c_int, ct.c_int, ct.c_void_p, ct.c_void_p]
+    kl = lambda X=FAKE, dt=1, M=1, N=16, K=64, pk=FAKE, am=FAKE, cb=FAKE, bits=4, bs=32, Y=FAKE: lib.linear_kbit(  # noqa: E731
+        X, dt, M, N, K, pk, am, cb, bits, bs, Y, None)
+    assert kl(X=None) == 1 and kl(pk=None) == 1 and kl(Y=None) == 1 and kl(M=0) == 1
+    assert kl(bits=1) == 1 and kl(bits=6) == 1 and "bits" in lib.bbc_last_error().decode()
+    assert kl(bs=64) == 2 and kl(dt=2) == 2 and kl(M=33) == 2 and kl(N=24) == 2 and kl(K=96) == 2
+    assert kl(pk=P(0x100008)) == 1 and kl(X=P(0x100008)) == 1
+    assert "16-byte" in lib.bbc_last_error().decode()
+    lib.linear_4bit_nested.argtypes = [ct.c_void_p, ct.c_int, ct.c_int64, ct.c_int64, ct.c_int64, ct.c_void_p,
+                                       ct.c_void_p, ct.c_void_p, ct.c_void_p, ct.c_float, ct.c_void_p, ct.c_int,
+                                       ct.c_int, ct.c_void_p, ct.c_void_p]
+    nl = lambda X=FAKE, dt=1, M=1, N=16, K=64, co=FAKE, bs=64, bs2=256: lib.linear_4bit_nested(  # noqa: E731
+        X, dt, M, N, K, co, FAKE, FAKE, FAKE, 0.0, FAKE, bs, bs2, FAKE, None)
+    assert nl(X=None) == 1 and nl(K=0) == 1 and nl(bs=48) == 1 and nl(co=P(0x100008)) == 1
+    assert nl(dt=2) == 2 and nl(M=40) == 2 and nl(K=32) == 2 and nl(bs2=128) == 2
 
 
 def test_last_error_is_per_thread(lib):

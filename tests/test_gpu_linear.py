@@ -1,4 +1,5 @@
-"""GPU parity of the fused nested 4-bit dequant + linear against the float64 oracle.
+"""GPU parity of the fused dequant + linear layers (nested 4-bit and k-bit weights) against the
+float64 oracle.
 
 The fused kernel accumulates in fp32 on the tensor cores, so it is not bit-exact; the tolerance
 comes from the arithmetic: every product of two 16-bit values is exact, the K additions in fp32
@@ -61,6 +62,36 @@ def test_ragged_m_and_blocksizes(bbc, dt):
         run_case(bbc, M, N, K, bs, dt, seed=M + N)
 
 
+def run_kbit_case(bbc, M, N, Kin, K, dt, seed=0):
+    packed, absmax = synthetic.kbit_state(N * Kin, K, seed=seed)
+    cb = oracle.normal_float_codebook(K)
+    x = synthetic.weights(M * Kin, std=1.0, seed=seed + 100, dtype=DTYPES[dt]).reshape(M, Kin)
+    Y64, S = oracle.linear_kbit(to_host(x), dt, N, Kin, to_host(packed), to_host(absmax), cb, K)
+    y = bbc.linear_kbit(x.cuda(), packed.cuda(), absmax.cuda(), torch.from_numpy(cb).cuda(), K, N)
+    torch.cuda.synchronize()
+    got = y.float().cpu().numpy().astype(np.float64)
+    acc_err = 2 * Kin * 2.0 ** -24 * S
+    half_ulp = (2.0 ** -8 if dt == "bf16" else 2.0 ** -11) * (np.abs(Y64) + acc_err)
+    bound = acc_err + half_ulp + 1e-30
+    assert np.all(np.abs(got - Y64) <= bound), (M, N, Kin, K, dt, float(np.max(np.abs(got - Y64) / bound)))
+
+
+@pytest.mark.parametrize("K", [2, 3, 4, 5])
+@pytest.mark.parametrize("M", [1, 8, 32])
+def test_kbit_control_shapes(bbc, M, K):
+    """The public-path control shapes (N = K = 4096) with a k-bit weight, every code width."""
+    run_kbit_case(bbc, M, 4096, 4096, K, "bf16", seed=M * 10 + K)
+
+
+@pytest.mark.parametrize("dt", ["bf16", "f16"])
+def test_kbit_ragged_shapes(bbc, dt):
+    # staged X with 128-wide windows, X from L2 with 64-wide windows, 64-wide row tails, n-tiles 1..4
+    cases = [(3, 64, 640), (9, 256, 1024), (17, 128, 4096), (31, 48, 192), (2, 16, 64), (8, 32, 8192),
+             (1, 272, 4160), (8, 48, 4160), (24, 32, 1088), (16, 64, 2048)]
+    for i, (M, N, Kin) in enumerate(cases):
+        run_kbit_case(bbc, M, N, Kin, 2 + i % 4, dt, seed=i)
+
+
 def test_invalid_arguments(bbc):
     from blockwise_bit_codebook_b200 import BBCError
     x = torch.zeros(33, 64, dtype=torch.bfloat16, device="cuda")
@@ -78,3 +109,18 @@ def test_invalid_arguments(bbc):
         bbc.linear_4bit_nested(x[:4], z8[8:], z8, f, f, 0.0, f, 16, 64)
     with pytest.raises(BBCError, match="fp16 or bf16"):
         bbc.linear_4bit_nested(x[:4].float(), z8, z8, f, f, 0.0, f, 16, 64)
+
+
+def test_kbit_invalid_arguments(bbc):
+    from blockwise_bit_codebook_b200 import BBCError
+    x = torch.zeros(4, 64, dtype=torch.bfloat16, device="cuda")
+    pk = torch.zeros(4096, dtype=torch.int32, device="cuda")
+    f = torch.zeros(256, device="cuda")
+    with pytest.raises(BBCError, match="bits"):
+        bbc.linear_kbit(x, pk, f, f, 6, 16)
+    with pytest.raises(BBCError, match="M <= 32"):
+        bbc.linear_kbit(torch.zeros(33, 64, dtype=torch.bfloat16, device="cuda"), pk, f, f, 4, 16)
+    with pytest.raises(BBCError, match="aligned"):
+        bbc.linear_kbit(x, pk[2:], f, f, 4, 16)
+    with pytest.raises(BBCError, match="blocksize"):
+        bbc.linear_kbit(x, pk, f, f, 4, 16, blocksize=64)
