@@ -300,7 +300,6 @@ __device__ __forceinline__ float rcp_approx(float d) {
 
 // Per-thread constants of the main loop.
 struct LoopCtx {
-    const char* lut;        // generic pointer to the shared table
     uint32_t lut_s;         // its shared-window address
     uint32_t lane16;        // this lane's replica offset
     uint32_t lut8_s;        // shared address of the 8-byte table (whole-block path)
@@ -312,20 +311,13 @@ struct LoopCtx {
     bool packed_v4;
 };
 
-#ifndef BBC_QUANT_LDS_ASM
-#define BBC_QUANT_LDS_ASM 1
-#endif
 // The table entry of the cell whose index sits in bits 7..14 of `fbits`.
 __device__ __forceinline__ uint4 lut_entry(const LoopCtx& c, uint32_t fbits) {
     const uint32_t off = (fbits & 0x7f80u) | c.lane16;
-#if BBC_QUANT_LDS_ASM
     uint4 v;
     asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];"
                  : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(c.lut_s + off));
     return v;
-#else
-    return *reinterpret_cast<const uint4*>(__builtin_assume_aligned(c.lut + off, 16));
-#endif
 }
 
 // The 8-byte table entry {-A, spread(L)} of the cell in bits 7..14 of `fbits` (128 bytes per
@@ -593,7 +585,6 @@ kbit_quant_kernel(const void* __restrict__ A, int64_t n, const float* __restrict
     const bool fast_cb = setup_exact_table<K, false>(codebook, cb, thr, &fast_ok, lut, WHOLE ? lut8 : nullptr);
     LoopCtx c;
     c.fast_cb = fast_cb;
-    c.lut = reinterpret_cast<const char*>(lut);
     c.lut_s = (uint32_t)__cvta_generic_to_shared(lut);
     c.lane16 = (uint32_t)(lane & 7) << 4;
     c.lut8_s = (uint32_t)__cvta_generic_to_shared(lut8);

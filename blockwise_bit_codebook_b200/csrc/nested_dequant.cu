@@ -27,10 +27,7 @@ namespace bbc {
 namespace {
 
 constexpr int kThreads = 256;
-#ifndef BBC_NESTED_PER_THREAD
-#define BBC_NESTED_PER_THREAD 16
-#endif
-constexpr int kPerThread = BBC_NESTED_PER_THREAD;     // 16 or 32 outputs per thread
+constexpr int kPerThread = 16;                        // outputs per thread (16 or 32 supported)
 static_assert(kPerThread == 16 || kPerThread == 32, "16 or 32 outputs per thread");
 constexpr int kCodeBytes = kPerThread / 2;
 
