@@ -309,6 +309,8 @@ struct LoopCtx {
     bool fast_cb;
     bool packed_v2;
     bool packed_v4;
+    uint32_t* stage;        // this warp's 32 * 5 words (whole-block path, K = 5)
+    int lane;
 };
 
 // The table entry of the cell whose index sits in bits 7..14 of `fbits`.
@@ -560,6 +562,18 @@ __device__ __forceinline__ void quantize_block(const Raw32<DT>& raw, int64_t b, 
     } else if constexpr (K == 4) {
         if (c.packed_v4) stg_v4(out, w[0], w[1], w[2], w[3]);
         else { out[0] = w[0]; out[1] = w[1]; out[2] = w[2]; out[3] = w[3]; }
+    } else if constexpr (K == 5) {
+        // the warp's 32 consecutive blocks are 160 contiguous words: transposed through shared
+        // memory so that each store instruction writes 128 contiguous bytes (five 4-byte stores
+        // at a 20-byte lane stride left the K = 5 kernel 2-3 points slower)
+        uint32_t* st = c.stage;
+#pragma unroll
+        for (int j = 0; j < K; j++) st[c.lane * K + j] = w[j];
+        __syncwarp();
+        uint32_t* outw = packed + (b - c.lane) * K;
+#pragma unroll
+        for (int j = 0; j < K; j++) outw[j * 32 + c.lane] = st[j * 32 + c.lane];
+        __syncwarp();
     } else {
 #pragma unroll
         for (int j = 0; j < K; j++) out[j] = w[j];
@@ -577,6 +591,7 @@ kbit_quant_kernel(const void* __restrict__ A, int64_t n, const float* __restrict
     __shared__ float cb[32];
     __shared__ float thr[33];
     __shared__ int fast_ok;
+    __shared__ uint32_t stage[WHOLE && K == 5 ? kThreads * K : 1];   // per-warp store staging
 
     const int tid = threadIdx.x;
     const int lane = tid & 31;
@@ -584,6 +599,8 @@ kbit_quant_kernel(const void* __restrict__ A, int64_t n, const float* __restrict
     // ---- per-CTA set-up: codebook check, thresholds, lookup table ----
     const bool fast_cb = setup_exact_table<K, false>(codebook, cb, thr, &fast_ok, lut, WHOLE ? lut8 : nullptr);
     LoopCtx c;
+    c.stage = stage + (WHOLE && K == 5 ? (tid & ~31) * K : 0);
+    c.lane = lane;
     c.fast_cb = fast_cb;
     c.lut_s = (uint32_t)__cvta_generic_to_shared(lut);
     c.lane16 = (uint32_t)(lane & 7) << 4;
