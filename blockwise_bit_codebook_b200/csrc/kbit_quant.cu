@@ -71,9 +71,10 @@ constexpr int kThreads = 256;
 constexpr int kCells = 256;
 constexpr int kReplicas = 8;
 constexpr int kReplicas8 = 16;           // the 8-byte table: 16 lanes per shared-load phase
-// Resident CTAs per SM the register budget targets: the whole-block path (16-bit, aligned)
-// trades occupancy for per-thread parallelism; the half-block path keeps three.
-template <int DT, bool VEC> constexpr int kMinCtas = (VEC && DT != F32) ? 2 : 3;
+// Resident CTAs per SM the register budget targets: the vector paths (the whole-block 16-bit
+// path and the fp32 half-block path) trade occupancy for per-thread parallelism (at three CTAs
+// the fp32 path spilled and ran 2-10 % slower); the unaligned path keeps three.
+template <int DT, bool VEC> constexpr int kMinCtas = VEC ? 2 : 3;
 
 __device__ __forceinline__ int64_t f32_key(float f) {
     const int32_t b = __float_as_int(f);
