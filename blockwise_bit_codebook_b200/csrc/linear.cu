@@ -352,6 +352,26 @@ __device__ __forceinline__ void kbit_group(uint32_t Bq, uint32_t p4q, float am, 
     pr[3] = DT == BF16 ? pack_bf16x2(y6, y7) : pack_f16x2(y6, y7);
 }
 
+// K <= 4: the same eight weights through a table of (codebook[a], codebook[b]) pairs. The 8 plane
+// bits of elements 2i, 2i + 1 (bits 8j + 2i + s of Bq) are gathered by one wide multiply into an
+// 8-bit index: multiplier 2^30 + 2^20 + 2^10 + 1 moves bit 8j + 2i + s to bit 24 + 2i + 2(3 - j) + s;
+// every cross term lands outside those 8 bits on a position of its own, so no carry reaches them
+// (checked over all 256 bit patterns at each i). Entry i of the table is (codebook[a], codebook[b])
+// with a = sum_j bit(i, 6 - 2j) 2^j, b = sum_j bit(i, 7 - 2j) 2^j, 16 lane-interleaved replicas.
+template <int DT>
+__device__ __forceinline__ void kbit_group_pairs(uint32_t Bq, float am, uint32_t lane_off, const unsigned char* table,
+                                                 uint32_t (&pr)[4]) {
+    const float2 sc = make_float2(am, am);
+#pragma unroll
+    for (int i = 0; i < 4; i++) {
+        const uint64_t prod = (uint64_t)(Bq & (0x03030303u << (2 * i))) * 0x40100401u;
+        const uint32_t sel = (uint32_t)(prod >> (17 + 2 * i)) & 0x7f80u;          // index * 128
+        const float2 v = *reinterpret_cast<const float2*>(table + (sel | lane_off));
+        const float2 p = __fmul2_rn(v, sc);
+        pr[i] = DT == BF16 ? pack_bf16x2(p.x, p.y) : pack_f16x2(p.x, p.y);
+    }
+}
+
 // The plane groups of a lane's run: all four for a 32-element run; for a 16-element run, the
 // two groups of half h of the block.
 template <int KB, int R>
@@ -379,6 +399,7 @@ __device__ __forceinline__ void kbit_groups(const uint32_t (&w)[KB], int h, uint
 // kernel's.
 template <int DT, int NT, int KB, int W>
 __device__ __forceinline__ void run_kwin(float (&acc)[NT][4], const KWin<KB>& wc, const char* cbb,
+                                         const unsigned char* table, uint32_t lane_off,
                                          const uint16_t* const (&xr)[NT], int64_t kw, int t) {
     constexpr int R = W / 4;
     uint32_t xw[NT][W / 8];
@@ -395,8 +416,13 @@ __device__ __forceinline__ void run_kwin(float (&acc)[NT][4], const KWin<KB>& wc
 #pragma unroll
     for (int w = 0; w < R / 8; w++) {
         uint32_t pa[4], pb[4];
-        kbit_group<KB, DT>(Ga[w], p4a >> (8 * w), wc.ama, cbb, pa);
-        kbit_group<KB, DT>(Gb[w], p4b >> (8 * w), wc.amb, cbb, pb);
+        if constexpr (KB <= 4) {
+            kbit_group_pairs<DT>(Ga[w], wc.ama, lane_off, table, pa);
+            kbit_group_pairs<DT>(Gb[w], wc.amb, lane_off, table, pb);
+        } else {
+            kbit_group<KB, DT>(Ga[w], p4a >> (8 * w), wc.ama, cbb, pa);
+            kbit_group<KB, DT>(Gb[w], p4b >> (8 * w), wc.amb, cbb, pb);
+        }
         const uint32_t a0[4] = {pa[0], pb[0], pa[1], pb[1]};
         const uint32_t a1[4] = {pa[2], pb[2], pa[3], pb[3]};
 #pragma unroll
@@ -414,8 +440,10 @@ linear_kbit_kernel(const uint16_t* __restrict__ X, int M, int64_t N, int64_t K,
                    const float* __restrict__ codebook, uint16_t* __restrict__ Y) {
     constexpr int WM = XS ? 128 : 64;
     constexpr int B = kBatch<NT, WM> < 4 ? kBatch<NT, WM> : 4;   // a window holds 2 (K + 1) registers
+    constexpr bool PAIRS = KB <= 4;                              // pair table (else per-weight codebook)
     __shared__ float cbs[32];
-    __shared__ __align__(16) float red[kNWarp][32][4 * NT];    // the split-K partials
+    __shared__ __align__(16) unsigned char table[PAIRS ? kPairBytes : 16];     // then the split-K partials
+    __shared__ __align__(16) float red5[PAIRS ? 1 : kNWarp * 32 * 4 * NT];     // split-K partials (K = 5)
     extern __shared__ __align__(16) uint16_t xs[];              // [M][K + 8] staged X (XS only)
 
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -431,10 +459,26 @@ linear_kbit_kernel(const uint16_t* __restrict__ X, int M, int64_t N, int64_t K,
     for (int i = 0; i < B; i++)
         if (w_lo + i < w_hi) load_kwin<KB, WM>(wc[i], packed, absmax, ea0 + (w_lo + i) * WM, eb0 + (w_lo + i) * WM, t);
     if (threadIdx.x < 32) cbs[threadIdx.x] = threadIdx.x < (1 << KB) ? __ldg(codebook + threadIdx.x) : 0.0f;
+    if constexpr (PAIRS) {
+        // thread i writes the 16 replicas of entry i (rotated 16-byte stores, as the nested table)
+        const int i = threadIdx.x;
+        int a = 0, b = 0;
+#pragma unroll
+        for (int j = 0; j < 4; j++) {
+            a |= ((i >> (6 - 2 * j)) & 1) << j;
+            b |= ((i >> (7 - 2 * j)) & 1) << j;
+        }
+        const float ca = __ldg(codebook + (a & ((1 << KB) - 1))), cbv = __ldg(codebook + (b & ((1 << KB) - 1)));
+        const float4 v = make_float4(ca, cbv, ca, cbv);
+#pragma unroll
+        for (int r = 0; r < kPairReplicas / 2; r++)
+            *reinterpret_cast<float4*>(table + i * 128 + ((r + i) & 7) * 16) = v;
+    }
     if (XS) stage_x(X, xs, M, K);
     __syncthreads();
 
     const char* cbb = reinterpret_cast<const char*>(cbs);
+    const uint32_t lane_off = (uint32_t)(lane & (kPairReplicas - 1)) * 8u;
     const uint16_t* xr[NT];
 #pragma unroll
     for (int q = 0; q < NT; q++) {
@@ -450,7 +494,7 @@ linear_kbit_kernel(const uint16_t* __restrict__ X, int M, int64_t N, int64_t K,
         for (int i = 0; i < B; i++) {
             const int64_t win = wb0 + i;
             if (win >= w_hi) break;
-            run_kwin<DT, NT, KB, WM>(acc, wc[i], cbb, xr, win * WM, t);
+            run_kwin<DT, NT, KB, WM>(acc, wc[i], cbb, table, lane_off, xr, win * WM, t);
             if (win + B < w_hi)
                 load_kwin<KB, WM>(wc[i], packed, absmax, ea0 + (win + B) * WM, eb0 + (win + B) * WM, t);
         }
@@ -458,9 +502,12 @@ linear_kbit_kernel(const uint16_t* __restrict__ X, int M, int64_t N, int64_t K,
     if (WM == 128 && (K & 64) && warp == kNWarp - 1) {
         KWin<KB> tw;
         load_kwin<KB, 64>(tw, packed, absmax, ea0 + K - 64, eb0 + K - 64, t);
-        run_kwin<DT, NT, KB, 64>(acc, tw, cbb, xr, K - 64, t);
+        run_kwin<DT, NT, KB, 64>(acc, tw, cbb, table, lane_off, xr, K - 64, t);
     }
-    reduce_store<DT, NT>(red, acc, M, N, ra, rb, Y);
+    // with the pair table the partials overlay it (no warp reads it after the barrier)
+    reduce_store<DT, NT>(reinterpret_cast<float (*)[32][4 * NT]>(PAIRS ? static_cast<void*>(table)
+                                                                       : static_cast<void*>(red5)),
+                         acc, M, N, ra, rb, Y);
 }
 
 // The dynamic shared-memory limit of kernel `k` raised to `bytes`, once per device (function
