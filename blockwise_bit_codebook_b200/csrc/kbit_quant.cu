@@ -627,7 +627,21 @@ kbit_quant_kernel(const void* __restrict__ A, int64_t n, const float* __restrict
         // what is left (at most the last partial iteration and a ragged block) goes by halves
         const int64_t bend = (n >> 5) & ~(int64_t)31;
         int64_t wb = wbase;                                 // in blocks
-        if (wb < bend) {
+        if (K == 5 && wb < bend) {
+            // K = 5: one copy of the block code in the loop and a register copy of the prefetched
+            // block (two unrolled copies of its larger body stalled on instruction fetch)
+            Raw32<DT> ra = load_block<DT>(A, wb + lane);
+            while (true) {
+                const int64_t wn = wb + stride;
+                const bool more = wn < bend;
+                Raw32<DT> rb;
+                if (more) rb = load_block<DT>(A, wn + lane);
+                quantize_block<K, DT, AT>(ra, wb + lane, c, cb, absmax, packed);
+                wb = wn;
+                if (!more) break;
+                ra = rb;
+            }
+        } else if (wb < bend) {
             Raw32<DT> ra = load_block<DT>(A, wb + lane);
             Raw32<DT> rb;
             while (true) {
