@@ -36,10 +36,11 @@
 //
 //    Whole-block threads (32-byte-aligned 16-bit input) use an 8-byte entry instead:
 //    {-A, spread(L)} with A = prev(T) for T > 0 and A = T for T < 0, so that the
-//    decision midpoint is always A + copysign(ulp(|A|) / 2, A); that half-ulp is
-//    rebuilt from A's bits (sign and exponent, exponent minus 24: two integer
-//    operations), the test becomes v = fma(-H, d, fma(-A, d, x)) with the same
-//    exactness argument, and instead of selecting spread(L) or spread(L + 1) the
+//    decision midpoint is always A + copysign(ulp(|A|) / 2, A); that half-ulp H is
+//    2^-24 times the sign and exponent bits of A, so -H * d is (the masked bits of
+//    -A) * (d * 2^-24), both exact (one mask per element, one multiply per block);
+//    the test becomes v = fma(-H, d, fma(-A, d, x)) with the same exactness argument,
+//    and instead of selecting spread(L) or spread(L + 1) the
 //    sign bits of v are collected (one funnel shift per element) and added to the
 //    K plane words of the block at the end as a bit-sliced increment. Half the
 //    shared-memory bytes per element, one select fewer. The thresholds must lie at
@@ -495,6 +496,7 @@ __device__ __forceinline__ void quantize_block(const Raw32<DT>& raw, int64_t b, 
     // B_q: byte j = plane j of elements 8q .. 8q+7; w4: plane 4 (K = 5)
     uint32_t B[4], w4 = 0;
     const float rs = __fmul_rn(rcp_approx(d), 8192.0f);
+    const float d24 = __fmul_rn(d, 0x1p-24f);                  // exact: d >= 1e-8 stays normal
     const bool fast = !special && c.fast_cb;
     uint32_t sv = 0;                     // fast path: sign of v per element, element 0 shifted in first
     // K = 5 accumulates 4 elements per register: two passes of 16 keep 4 registers live
@@ -512,10 +514,11 @@ __device__ __forceinline__ void quantize_block(const Raw32<DT>& raw, int64_t b, 
                                             make_float2(12582912.0f, 12582912.0f));
                 const uint2 t0 = lut8_entry(c, __float_as_uint(f.x));
                 const uint2 t1 = lut8_entry(c, __float_as_uint(f.y));
-                const float h0 = __uint_as_float((t0.x & 0xff800000u) - 0x0c000000u);   // -H
-                const float h1 = __uint_as_float((t1.x & 0xff800000u) - 0x0c000000u);
-                const float v0 = __fmaf_rn(h0, d, __fmaf_rn(__uint_as_float(t0.x), d, x0));
-                const float v1 = __fmaf_rn(h1, d, __fmaf_rn(__uint_as_float(t1.x), d, x1));
+                // -H * d = (sign and exponent bits of -A) * (d * 2^-24), both factors exact
+                const float h0 = __uint_as_float(t0.x & 0xff800000u);
+                const float h1 = __uint_as_float(t1.x & 0xff800000u);
+                const float v0 = __fmaf_rn(h0, d24, __fmaf_rn(__uint_as_float(t0.x), d, x0));
+                const float v1 = __fmaf_rn(h1, d24, __fmaf_rn(__uint_as_float(t1.x), d, x1));
                 sv = __funnelshift_l(__float_as_uint(v0), sv, 1);                         // sign bits
                 sv = __funnelshift_l(__float_as_uint(v1), sv, 1);
                 acc[e / EPA] += t0.y << (e % EPA);
@@ -837,6 +840,7 @@ quant4_kernel(const void* __restrict__ A, int64_t n, int log2_bs, const float* _
         for (int g = 0; g < NW; g++) acc[g] = 0u;
         if (!special && c.fast_cb) {
             const float rs = __fmul_rn(rcp_approx(d), 8192.0f);
+            const float d24 = __fmul_rn(d, 0x1p-24f);           // exact: d >= 1e-8 stays normal
             uint32_t sv = 0;                                     // signs of v, element 0 shifted in first
 #pragma unroll
             for (int e = 0; e < E; e += 2) {
@@ -845,10 +849,11 @@ quant4_kernel(const void* __restrict__ A, int64_t n, int log2_bs, const float* _
                                             make_float2(12582912.0f, 12582912.0f));
                 const uint2 t0 = lut8_entry(c, __float_as_uint(f.x));
                 const uint2 t1 = lut8_entry(c, __float_as_uint(f.y));
-                const float h0 = __uint_as_float((t0.x & 0xff800000u) - 0x0c000000u);   // -H
-                const float h1 = __uint_as_float((t1.x & 0xff800000u) - 0x0c000000u);
-                const float v0 = __fmaf_rn(h0, d, __fmaf_rn(__uint_as_float(t0.x), d, x0));
-                const float v1 = __fmaf_rn(h1, d, __fmaf_rn(__uint_as_float(t1.x), d, x1));
+                // -H * d = (sign and exponent bits of -A) * (d * 2^-24), both factors exact
+                const float h0 = __uint_as_float(t0.x & 0xff800000u);
+                const float h1 = __uint_as_float(t1.x & 0xff800000u);
+                const float v0 = __fmaf_rn(h0, d24, __fmaf_rn(__uint_as_float(t0.x), d, x0));
+                const float v1 = __fmaf_rn(h1, d24, __fmaf_rn(__uint_as_float(t1.x), d, x1));
                 sv = __funnelshift_l(__float_as_uint(v0), sv, 1);
                 sv = __funnelshift_l(__float_as_uint(v1), sv, 1);
                 acc[e / 8] += t0.y << nib_shift(e);
