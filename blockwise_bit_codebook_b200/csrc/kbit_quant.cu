@@ -34,7 +34,11 @@
 //    is replicated 8 times so the 8 lanes of each 128-bit shared-load phase
 //    always hit distinct banks.
 //
-//    Whole-block threads (32-byte-aligned 16-bit input) use an 8-byte entry instead:
+//    Whole-block threads (32-byte-aligned 16-bit input) use an 8-byte entry instead, with
+//    cells centred on multiples of 1/64 (cell c = round(64 x/d), one fma with the same
+//    magic constant, stored at slot c + 128) so that the entry's shared address is one
+//    multiply-add of the fma's bits (bits * 128 plus a per-lane constant) in place of a
+//    mask, an or and an add:
 //    {-A, spread(L)} with A = prev(T) for T > 0 and A = T for T < 0, so that the
 //    decision midpoint is always A + copysign(ulp(|A|) / 2, A); that half-ulp H is
 //    2^-24 times the sign and exponent bits of A, so -H * d is (the masked bits of
@@ -154,9 +158,13 @@ __device__ __forceinline__ bool setup_exact_table(const float* __restrict__ code
     int multi = 0;
     if (*fast_ok) {
         for (int cell = tid; cell < kCells; cell += kThreads) {
-            const int cs = cell < 128 ? cell : cell - 256;
-            const float wlo = __fsub_rn((float)cs * 0.015625f, 0x1p-13f + 0x1p-12f);
-            const float whi = __fadd_rn((float)(cs + 1) * 0.015625f, 0x1p-13f + 0x1p-12f);
+            // 16-byte table: cell cs = floor(64 xn) (two's complement, slots 128..255 negative);
+            // 8-byte table: cell cs = round(64 xn), slot cs + 128
+            const int cs = lut8 ? cell - 128 : (cell < 128 ? cell : cell - 256);
+            const float lo_edge = lut8 ? ((float)cs - 0.5f) * 0.015625f : (float)cs * 0.015625f;
+            const float hi_edge = lut8 ? ((float)cs + 0.5f) * 0.015625f : (float)(cs + 1) * 0.015625f;
+            const float wlo = __fsub_rn(lo_edge, 0x1p-13f + 0x1p-12f);
+            const float whi = __fadd_rn(hi_edge, 0x1p-13f + 0x1p-12f);
             int below = 0, rel = 0, relj = 0;
             for (int j = 1; j < NE; j++) {
                 const float T = thr[j];
@@ -306,6 +314,7 @@ struct LoopCtx {
     uint32_t lane16;        // this lane's replica offset
     uint32_t lut8_s;        // shared address of the 8-byte table (whole-block path)
     uint32_t lane8;         // this lane's replica offset in it
+    uint32_t lut8_c;        // address of slot 0 of this lane's replica minus the magic constant's bits * 128
     uint32_t h;             // which half of the block this lane owns
     uint32_t sel_send, sel_keep, sel_wa, sel_wb, pair_mask;
     bool fast_cb;
@@ -328,7 +337,7 @@ __device__ __forceinline__ uint4 lut_entry(const LoopCtx& c, uint32_t fbits) {
 // cell, as the 16-byte table: the same cell offset).
 __device__ __forceinline__ uint2 lut8_entry(const LoopCtx& c, uint32_t fbits) {
     uint2 v;
-    asm volatile("ld.shared.v2.u32 {%0,%1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(c.lut8_s + ((fbits & 0x7f80u) | c.lane8)));
+    asm volatile("ld.shared.v2.u32 {%0,%1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(fbits * 128u + c.lut8_c));
     return v;
 }
 
@@ -495,7 +504,7 @@ __device__ __forceinline__ void quantize_block(const Raw32<DT>& raw, int64_t b, 
     const float d = fmaxf(amax, 1e-8f);
     // B_q: byte j = plane j of elements 8q .. 8q+7; w4: plane 4 (K = 5)
     uint32_t B[4], w4 = 0;
-    const float rs = __fmul_rn(rcp_approx(d), 8192.0f);
+    const float rs = __fmul_rn(rcp_approx(d), 64.0f);
     const float d24 = __fmul_rn(d, 0x1p-24f);                  // exact: d >= 1e-8 stays normal
     const bool fast = !special && c.fast_cb;
     uint32_t sv = 0;                     // fast path: sign of v per element, element 0 shifted in first
@@ -610,6 +619,7 @@ kbit_quant_kernel(const void* __restrict__ A, int64_t n, const float* __restrict
     c.lane16 = (uint32_t)(lane & 7) << 4;
     c.lut8_s = (uint32_t)__cvta_generic_to_shared(lut8);
     c.lane8 = (uint32_t)(lane & (kReplicas8 - 1)) << 3;
+    c.lut8_c = c.lut8_s + c.lane8 + 128u * 128u - 0x4B400000u * 128u;     // mod 2^32
     c.packed_v2 = (reinterpret_cast<uintptr_t>(packed) & 7u) == 0;
     c.packed_v4 = (reinterpret_cast<uintptr_t>(packed) & 15u) == 0;
     c.h = lane & 1;
@@ -799,6 +809,7 @@ quant4_kernel(const void* __restrict__ A, int64_t n, int log2_bs, const float* _
     c.fast_cb = setup_exact_table<4, true>(code4, cb, thr, &fast_ok, nullptr, lut8);
     c.lut8_s = (uint32_t)__cvta_generic_to_shared(lut8);
     c.lane8 = (uint32_t)(lane & (kReplicas8 - 1)) << 3;
+    c.lut8_c = c.lut8_s + c.lane8 + 128u * 128u - 0x4B400000u * 128u;     // mod 2^32
 
     const int tpb_log2 = log2_bs - (DT == F32 ? 4 : 5);        // threads per outer block
     const int tpb = 1 << tpb_log2;
@@ -839,7 +850,7 @@ quant4_kernel(const void* __restrict__ A, int64_t n, int log2_bs, const float* _
 #pragma unroll
         for (int g = 0; g < NW; g++) acc[g] = 0u;
         if (!special && c.fast_cb) {
-            const float rs = __fmul_rn(rcp_approx(d), 8192.0f);
+            const float rs = __fmul_rn(rcp_approx(d), 64.0f);
             const float d24 = __fmul_rn(d, 0x1p-24f);           // exact: d >= 1e-8 stays normal
             uint32_t sv = 0;                                     // signs of v, element 0 shifted in first
 #pragma unroll
