@@ -26,30 +26,28 @@
 //    is below ulp(T)*d the inner fma is exact, otherwise its rounding cannot
 //    change the sign of the sum. Two paired f32x2 FMAs per element pair.
 //
-// 3. One table lookup finds the threshold. A 256-cell table indexed by
-//    round(8192 * x/d) / 128 (cells 1/64 wide; one paired fma and a mask) holds,
-//    per cell, the only threshold that can matter there (-T, h_T) and the
-//    byte-spread bit patterns of the two possible indices. A codebook whose
-//    thresholds are closer than a cell takes the brute-force search. The table
-//    is replicated 8 times so the 8 lanes of each 128-bit shared-load phase
-//    always hit distinct banks.
+// 3. One table lookup finds the threshold. A 256-cell table indexed by the cell
+//    c = round(64 x/d) (cells 1/64 wide, centred on multiples of 1/64; one paired fma
+//    with a magic constant, stored at slot c + 128) holds, per cell, the only threshold
+//    that can matter there and the byte-spread bit pattern of the index below it. The
+//    entry's shared address is one multiply-add of the fma's bits (bits * 128 plus a
+//    per-lane constant that absorbs the magic constant, the table base and the lane's
+//    replica). A codebook whose thresholds are closer than a cell takes the brute-force
+//    search. Half-block threads (fp32, unaligned input) read 16-byte entries (-T, h_T,
+//    spread(L), spread(L + 1)), 8 replicas so that the 8 lanes of each 128-bit
+//    shared-load phase always hit distinct banks.
 //
-//    Whole-block threads (32-byte-aligned 16-bit input) use an 8-byte entry instead, with
-//    cells centred on multiples of 1/64 (cell c = round(64 x/d), one fma with the same
-//    magic constant, stored at slot c + 128) so that the entry's shared address is one
-//    multiply-add of the fma's bits (bits * 128 plus a per-lane constant) in place of a
-//    mask, an or and an add:
-//    {-A, spread(L)} with A = prev(T) for T > 0 and A = T for T < 0, so that the
-//    decision midpoint is always A + copysign(ulp(|A|) / 2, A); that half-ulp H is
-//    2^-24 times the sign and exponent bits of A, so -H * d is (the masked bits of
-//    -A) * (d * 2^-24), both exact (one mask per element, one multiply per block);
-//    the test becomes v = fma(-H, d, fma(-A, d, x)) with the same exactness argument,
-//    and instead of selecting spread(L) or spread(L + 1) the
-//    sign bits of v are collected (one funnel shift per element) and added to the
-//    K plane words of the block at the end as a bit-sliced increment. Half the
-//    shared-memory bytes per element, one select fewer. The thresholds must lie at
-//    least 2^-100 from zero (they do for any codebook the fast path accepts; the set-
-//    up checks it).
+//    Whole-block threads (32-byte-aligned 16-bit input) use an 8-byte entry instead
+//    (16 replicas): {-A, spread(L)} with A = prev(T) for T > 0 and A = T for T < 0, so
+//    that the decision midpoint is always A + copysign(ulp(|A|) / 2, A); that half-ulp H
+//    is 2^-24 times the sign and exponent bits of A, so -H * d is (the masked bits of
+//    -A) * (d * 2^-24), both exact (one mask per element, one multiply per block); the
+//    test becomes v = fma(-H, d, fma(-A, d, x)) with the same exactness argument, and
+//    instead of selecting spread(L) or spread(L + 1) the sign bits of v are collected
+//    (one funnel shift per element) and added to the K plane words of the block at the
+//    end as a bit-sliced increment. Half the shared-memory bytes per element, one
+//    select fewer. The thresholds must lie at least 2^-100 from zero (they do for any
+//    codebook the fast path accepts; the set-up checks it).
 //
 // 4. Bit-plane packing without ballots. Adding spread(idx) << e (bit k of idx at
 //    bit 8k) builds, per 8 elements, one register whose byte k holds plane k
@@ -158,11 +156,10 @@ __device__ __forceinline__ bool setup_exact_table(const float* __restrict__ code
     int multi = 0;
     if (*fast_ok) {
         for (int cell = tid; cell < kCells; cell += kThreads) {
-            // 16-byte table: cell cs = floor(64 xn) (two's complement, slots 128..255 negative);
-            // 8-byte table: cell cs = round(64 xn), slot cs + 128
-            const int cs = lut8 ? cell - 128 : (cell < 128 ? cell : cell - 256);
-            const float lo_edge = lut8 ? ((float)cs - 0.5f) * 0.015625f : (float)cs * 0.015625f;
-            const float hi_edge = lut8 ? ((float)cs + 0.5f) * 0.015625f : (float)(cs + 1) * 0.015625f;
+            // cell cs = round(64 xn) at slot cs + 128: it holds every xn within half a cell
+            const int cs = cell - 128;
+            const float lo_edge = ((float)cs - 0.5f) * 0.015625f;
+            const float hi_edge = ((float)cs + 0.5f) * 0.015625f;
             const float wlo = __fsub_rn(lo_edge, 0x1p-13f + 0x1p-12f);
             const float whi = __fadd_rn(hi_edge, 0x1p-13f + 0x1p-12f);
             int below = 0, rel = 0, relj = 0;
@@ -310,8 +307,8 @@ __device__ __forceinline__ float rcp_approx(float d) {
 
 // Per-thread constants of the main loop.
 struct LoopCtx {
-    uint32_t lut_s;         // its shared-window address
-    uint32_t lane16;        // this lane's replica offset
+    uint32_t lut_c;         // address of slot 0 of this lane's replica (16-byte table) minus the
+                            // magic constant's bits * 128
     uint32_t lut8_s;        // shared address of the 8-byte table (whole-block path)
     uint32_t lane8;         // this lane's replica offset in it
     uint32_t lut8_c;        // address of slot 0 of this lane's replica minus the magic constant's bits * 128
@@ -326,10 +323,9 @@ struct LoopCtx {
 
 // The table entry of the cell whose index sits in bits 7..14 of `fbits`.
 __device__ __forceinline__ uint4 lut_entry(const LoopCtx& c, uint32_t fbits) {
-    const uint32_t off = (fbits & 0x7f80u) | c.lane16;
     uint4 v;
     asm volatile("ld.shared.v4.u32 {%0,%1,%2,%3}, [%4];"
-                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(c.lut_s + off));
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(fbits * 128u + c.lut_c));
     return v;
 }
 
@@ -345,7 +341,7 @@ __device__ __forceinline__ uint2 lut8_entry(const LoopCtx& c, uint32_t fbits) {
 template <int K, int DT>
 __device__ __forceinline__ void fast_codes(const Raw<DT>& raw, float d, const LoopCtx& c, uint32_t* acc) {
     constexpr int EPA = K == 5 ? 4 : 8;           // 4 elements per accumulator for K = 5, else 8
-    const float rs = __fmul_rn(rcp_approx(d), 8192.0f);
+    const float rs = __fmul_rn(rcp_approx(d), 64.0f);
 #pragma unroll
     for (int e = 0; e < 16; e += 2) {
         float x0, x1;
@@ -615,8 +611,8 @@ kbit_quant_kernel(const void* __restrict__ A, int64_t n, const float* __restrict
     c.stage = stage + (WHOLE && K == 5 ? (tid & ~31) * K : 0);
     c.lane = lane;
     c.fast_cb = fast_cb;
-    c.lut_s = (uint32_t)__cvta_generic_to_shared(lut);
-    c.lane16 = (uint32_t)(lane & 7) << 4;
+    c.lut_c = (uint32_t)__cvta_generic_to_shared(lut) + ((uint32_t)(lane & 7) << 4) + 128u * 128u -
+              0x4B400000u * 128u;                                 // mod 2^32
     c.lut8_s = (uint32_t)__cvta_generic_to_shared(lut8);
     c.lane8 = (uint32_t)(lane & (kReplicas8 - 1)) << 3;
     c.lut8_c = c.lut8_s + c.lane8 + 128u * 128u - 0x4B400000u * 128u;     // mod 2^32
