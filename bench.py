@@ -100,7 +100,15 @@ ALL_OPS = [("quantize_k3", "quantize", 3), ("dequantize_k3", "dequantize", 3),
            ("quantize_k5", "quantize", 5), ("dequantize_k5", "dequantize", 5),
            ("nested_nf4_bs64", "nested", None)]
 # Kernel launches per op (the nested quantize: 4-bit codes, two offset kernels, compression).
-LAUNCHES = {"quantize_nested": 4}
+def nested_quant_launches(n, bs=NESTED_BS):
+    """Launches of one quantize_4bit_nested call: the 4-bit codes, one per level of the offset
+    tree while more than 2048 values remain, and the compression (which forms the root)."""
+    count, levels = (n + bs - 1) // bs, 0
+    while count > 2048:
+        count = (count + 2047) // 2048
+        levels += 1
+    return 2 + levels
+
 # Selectable with --ops (not part of the default step): the E4M4-absmax codec.
 EXTRA_OPS = [(f"{k}_k{K}_e4m4", f"{k}_e4m4", K) for K in (3, 4, 5) for k in ("quantize", "dequantize")] + \
     [("quantize_4bit_nf4_bs64", "quantize_4bit", None), ("quantize_nested_nf4_bs64", "quantize_nested", None)]
@@ -418,7 +426,8 @@ def run_bbc(args):
               "data": "synthetic", "config": {**workload_desc(n, ops),
                                               "parallelism": f"replicas{world}" if world > 1 else "single"},
               "per_kernel": per_kernel, "roofline": roofline,
-              "gpu_launches": sum(LAUNCHES.get(kind, 1) for _, kind, _ in ops) * args.steps, "clocks": clocks}
+              "gpu_launches": sum(nested_quant_launches(n) if kind == "quantize_nested" else 1
+                                  for _, kind, _ in ops) * args.steps, "clocks": clocks}
 
     # ---- end to end through the public API with host buffers
     if not args.no_e2e:

@@ -19,6 +19,7 @@
 //      holding it is found by walking down a plateau of equal distances. Any other table takes
 //      the rule verbatim over all 256 entries.
 #include <cfloat>
+#include <type_traits>
 
 #include "common.cuh"
 #include "launch.h"
@@ -30,14 +31,12 @@ namespace {
 constexpr int kTree = 2048;            // tree leaves per CTA (256 threads x 8)
 constexpr int kGroup = 256;            // outer blocks per inner absmax
 
-// One level of the pairwise sum: node b = sum of in[2048 b .. 2048 b + 2048) (zeros past count)
-// as a binary tree. With a single CTA this is the root: it writes the fp32 mean instead.
+// Node `blk` of one level of the pairwise sum: in[2048 blk .. 2048 blk + 2048) (zeros past
+// count) summed as a binary tree by the whole CTA (8 leaves per thread as a tree, lanes by
+// xor-shuffles, warps in shared memory); the result is returned to every thread.
 template <typename T>
-__global__ void __launch_bounds__(256)
-tree_sum_kernel(const T* __restrict__ in, int64_t count, double* __restrict__ nodes, int64_t nbo,
-                float* __restrict__ offset) {
-    __shared__ double ws[8];
-    const int64_t base = (int64_t)blockIdx.x * kTree + threadIdx.x * 8;
+__device__ __forceinline__ double tree_node(const T* __restrict__ in, int64_t count, int64_t blk, double* ws) {
+    const int64_t base = blk * kTree + threadIdx.x * 8;
     double v[8];
 #pragma unroll
     for (int j = 0; j < 8; j++) v[j] = base + j < count ? (double)in[base + j] : 0.0;
@@ -45,14 +44,20 @@ tree_sum_kernel(const T* __restrict__ in, int64_t count, double* __restrict__ no
                          __dadd_rn(__dadd_rn(v[4], v[5]), __dadd_rn(v[6], v[7])));
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) s = __dadd_rn(s, __shfl_xor_sync(0xffffffffu, s, o));
+    __syncthreads();                                            // ws may hold a previous use
     if ((threadIdx.x & 31) == 0) ws[threadIdx.x >> 5] = s;
     __syncthreads();
-    if (threadIdx.x == 0) {
-        const double r = __dadd_rn(__dadd_rn(__dadd_rn(ws[0], ws[1]), __dadd_rn(ws[2], ws[3])),
-                                   __dadd_rn(__dadd_rn(ws[4], ws[5]), __dadd_rn(ws[6], ws[7])));
-        if (gridDim.x == 1) *offset = __double2float_rn(__ddiv_rn(r, (double)nbo));
-        else nodes[blockIdx.x] = r;
-    }
+    return __dadd_rn(__dadd_rn(__dadd_rn(ws[0], ws[1]), __dadd_rn(ws[2], ws[3])),
+                     __dadd_rn(__dadd_rn(ws[4], ws[5]), __dadd_rn(ws[6], ws[7])));
+}
+
+// One level of the pairwise sum below the root: node b = the tree of in[2048 b .. 2048 b + 2048).
+template <typename T>
+__global__ void __launch_bounds__(256)
+tree_sum_kernel(const T* __restrict__ in, int64_t count, double* __restrict__ nodes) {
+    __shared__ double ws[8];
+    const double r = tree_node(in, count, blockIdx.x, ws);
+    if (threadIdx.x == 0) nodes[blockIdx.x] = r;
 }
 
 // The General8 table in shared memory as 32 lane-interleaved replicas (entry i of replica r at
@@ -87,30 +92,44 @@ __device__ __forceinline__ uint32_t nearest_any(float xn, const float* t) {
     return idx;
 }
 
-// One warp per group of 256 outer blocks (8 per lane), persistent over the groups.
+// One warp per group of 256 outer blocks (8 per lane), persistent over the groups; every CTA
+// first forms the offset from the last level of the tree.
+template <typename T>
 __global__ void __launch_bounds__(256)
-absmax_compress_kernel(const float* __restrict__ absmax, int64_t nbo, const float* __restrict__ offset_p,
+absmax_compress_kernel(const float* __restrict__ absmax, int64_t nbo, const T* __restrict__ root_in,
+                       int64_t root_count, float* __restrict__ offset_p,
                        const float* __restrict__ code2, uint8_t* __restrict__ absmax_q,
                        float* __restrict__ absmax2) {
-    __shared__ float tr[256 * kRep];                            // 32 KB
+    __shared__ __align__(16) float tr[256 * kRep];              // 32 KB
     const float v = code2[threadIdx.x];
     const float next = threadIdx.x < 255 ? code2[threadIdx.x + 1] : v;
-#pragma unroll 8
-    for (int r = 0; r < kRep; r++) tr[threadIdx.x * kRep + ((r + threadIdx.x) & (kRep - 1))] = v;
+    // entry i's 32 replicas are 128 contiguous bytes: 8 rotated 16-byte stores per thread (the 8
+    // threads of a store phase write 8 different 16-byte columns, so no bank is hit twice)
+    static_assert(kRep == 32, "one entry is 8 float4 columns");
+    const float4 v4 = make_float4(v, v, v, v);
+#pragma unroll
+    for (int k = 0; k < 8; k++)
+        reinterpret_cast<float4*>(tr)[threadIdx.x * 8 + ((k + threadIdx.x) & 7)] = v4;
     // the barrier also makes the replicas visible
     const bool ascending = __syncthreads_and(v <= next);        // false if any entry is NaN
     const float* t = tr + (threadIdx.x & (kRep - 1));
-    const float off = *offset_p;
+    // the offset: the root of the pairwise tree over the last level (<= 2048 values), the
+    // same in every CTA; CTA 0 stores it
+    __shared__ double ws[8];
+    const float off = __double2float_rn(__ddiv_rn(tree_node(root_in, root_count, 0, ws), (double)nbo));
+    if (blockIdx.x == 0 && threadIdx.x == 0) *offset_p = off;
     const int lane = threadIdx.x & 31;
     const int64_t ngroups = (nbo + kGroup - 1) / kGroup;
     const int64_t wstride = (int64_t)gridDim.x * (blockDim.x >> 5);
-    for (int64_t g = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); g < ngroups; g += wstride) {
+    // one group: FULL groups (all 256 blocks inside nbo) need no bounds checks
+    auto group = [&](int64_t g, auto full) {
+        constexpr bool FULL = decltype(full)::value;
         float cv[8];
         float m = __int_as_float(0x7fc00000);                   // NaN: ignored by fmaxf
 #pragma unroll
         for (int j = 0; j < 8; j++) {
             const int64_t b = g * kGroup + lane + 32 * j;
-            cv[j] = b < nbo ? __fsub_rn(__ldg(absmax + b), off) : __int_as_float(0x7fc00000);
+            cv[j] = (FULL || b < nbo) ? __fsub_rn(__ldg(absmax + b), off) : __int_as_float(0x7fc00000);
             m = fmaxf(m, fabsf(cv[j]));
         }
 #pragma unroll
@@ -120,11 +139,16 @@ absmax_compress_kernel(const float* __restrict__ absmax, int64_t nbo, const floa
 #pragma unroll
         for (int j = 0; j < 8; j++) {
             const int64_t b = g * kGroup + lane + 32 * j;
-            if (b < nbo) {
+            if (FULL || b < nbo) {
                 const float xn = __fdiv_rn(cv[j], d);
                 absmax_q[b] = (uint8_t)(ascending ? nearest_ascending(xn, t) : nearest_any(xn, t));
             }
         }
+    };
+    const int64_t nfull = nbo / kGroup;
+    for (int64_t g = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); g < ngroups; g += wstride) {
+        if (g < nfull) group(g, std::true_type{});
+        else group(g, std::false_type{});
     }
 }
 
@@ -150,21 +174,29 @@ cudaError_t launch_quantize_4bit_nested(const void* A, int dtype, int64_t n, int
     double* buf_b = buf_a + tree_nodes(nbo);
     cudaError_t e = launch_quantize_4bit(A, dtype, n, log2_bs, code4, absmax, codes, vec, s);
     if (e != cudaSuccess) return e;
-    // the pairwise sum, one level per launch; the single-CTA level writes the offset
+    // the pairwise sum: one launch per level while more than 2048 values remain; the root (at
+    // most 2048 values) is formed by every CTA of the compression kernel
+    const int64_t ngroups = (nbo + kGroup - 1) / kGroup;
+    if (nbo <= kTree) {
+        const int grid = persistent_grid(absmax_compress_kernel<float>, 256, 0, ngroups, 32);
+        absmax_compress_kernel<float><<<grid, 256, 0, s>>>(absmax, nbo, absmax, nbo, offset, code2, absmax_q,
+                                                           absmax2);
+        return cudaGetLastError();
+    }
     int64_t count = tree_nodes(nbo);
-    tree_sum_kernel<float><<<(unsigned)count, 256, 0, s>>>(absmax, nbo, buf_a, nbo, offset);
+    tree_sum_kernel<float><<<(unsigned)count, 256, 0, s>>>(absmax, nbo, buf_a);
     const double* in = buf_a;
     double* out = buf_b;
-    while (count > 1) {
+    while (count > kTree) {
         const int64_t next = tree_nodes(count);
-        tree_sum_kernel<double><<<(unsigned)next, 256, 0, s>>>(in, count, out, nbo, offset);
+        tree_sum_kernel<double><<<(unsigned)next, 256, 0, s>>>(in, count, out);
         in = out;
         out = out == buf_b ? buf_a : buf_b;        // a level never outgrows the one before it
         count = next;
     }
-    const int64_t ngroups = (nbo + kGroup - 1) / kGroup;
-    const int grid = persistent_grid(absmax_compress_kernel, 256, 0, ngroups, 8);
-    absmax_compress_kernel<<<grid, 256, 0, s>>>(absmax, nbo, offset, code2, absmax_q, absmax2);
+    // 32 groups per CTA (4 per warp) amortise the 32 KB table set-up; persistent above that
+    const int grid = persistent_grid(absmax_compress_kernel<double>, 256, 0, ngroups, 32);
+    absmax_compress_kernel<double><<<grid, 256, 0, s>>>(absmax, nbo, in, count, offset, code2, absmax_q, absmax2);
     return cudaGetLastError();
 }
 

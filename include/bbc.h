@@ -221,7 +221,9 @@ int quantize_4bit(const void* A, int dtype, int64_t n, int blocksize, const floa
  *   offset     one fp32 out, a DEVICE pointer (read it back before dequantizing).
  *   workspace  DEVICE scratch of quantize_4bit_nested_workspace_bytes(n, blocksize)
  *              bytes, 256-byte aligned, caller-owned, not overlapping any argument.
- * Four launches on `stream`. Errors as quantize_4bit; a workspace that is too small
+ * Two launches on `stream` (codes, then the absmax compression, which also forms the
+ * offset) plus one per level of the offset tree above 2048 outer blocks (three at 4M
+ * outer blocks). Errors as quantize_4bit; a workspace that is too small
  * is BBC_ERR_INVALID, blocksize2 != 256 BBC_ERR_UNSUPPORTED.
  */
 size_t quantize_4bit_nested_workspace_bytes(int64_t n, int blocksize);
