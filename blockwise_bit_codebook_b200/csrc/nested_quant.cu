@@ -67,18 +67,20 @@ constexpr int kRep = 32;
 
 // First index minimising fl(|xn - t_i|) over an ascending 256-entry table (see the header).
 __device__ __forceinline__ uint32_t nearest_ascending(float xn, const float* t) {
-    if (xn != xn) return 0;                                     // NaN: no distance is below +inf
-    int p = t[255 * kRep] <= xn ? 255 : -1;                     // last index with entry p <= xn
-    if (p < 0) {
+    int p = -1;                                                 // last index with entry p <= xn
 #pragma unroll
-        for (int step = 128; step >= 1; step >>= 1)              // p + step <= 254 throughout
-            if (t[(p + step) * kRep] <= xn) p += step;
-    }
-    if (p < 0) return 0;
-    const float dp = fabsf(__fsub_rn(xn, t[p * kRep]));
-    if (p < 255 && fabsf(__fsub_rn(xn, t[(p + 1) * kRep])) < dp) return (uint32_t)p + 1;
-    int i = p;
-    while (i > 0 && fabsf(__fsub_rn(xn, t[(i - 1) * kRep])) == dp) i--;
+    for (int step = 128; step >= 1; step >>= 1)                  // p + step <= 254 throughout
+        p += t[(p + step) * kRep] <= xn ? step : 0;
+    p = t[255 * kRep] <= xn ? 255 : p;
+    // The first nearest entry is t[p] or t[p + 1]. With p clamped to 0 the same selects give 0
+    // when no entry is <= xn (t[1] is never strictly closer than t[0] below t[0]) and for a NaN
+    // xn (no comparison holds); at p = 255 the clamped neighbour is t[255] itself.
+    const int q = max(p, 0), r = min(q + 1, 255);
+    const float dq = fabsf(__fsub_rn(xn, t[q * kRep]));
+    const float dr = fabsf(__fsub_rn(xn, t[r * kRep]));
+    if (dr < dq) return (uint32_t)r;
+    int i = q;                                                  // walk down a plateau of equal distances
+    while (i > 0 && fabsf(__fsub_rn(xn, t[(i - 1) * kRep])) == dq) i--;
     return (uint32_t)i;
 }
 
@@ -121,9 +123,11 @@ absmax_compress_kernel(const float* __restrict__ absmax, int64_t nbo, const T* _
     const int lane = threadIdx.x & 31;
     const int64_t ngroups = (nbo + kGroup - 1) / kGroup;
     const int64_t wstride = (int64_t)gridDim.x * (blockDim.x >> 5);
-    // one group: FULL groups (all 256 blocks inside nbo) need no bounds checks
-    auto group = [&](int64_t g, auto full) {
+    // one group: FULL groups (all 256 blocks inside nbo) need no bounds checks; ASC selects the
+    // search (uniform over the kernel)
+    auto group = [&](int64_t g, auto full, auto asc) {
         constexpr bool FULL = decltype(full)::value;
+        constexpr bool ASC = decltype(asc)::value;
         float cv[8];
         float m = __int_as_float(0x7fc00000);                   // NaN: ignored by fmaxf
 #pragma unroll
@@ -141,14 +145,19 @@ absmax_compress_kernel(const float* __restrict__ absmax, int64_t nbo, const T* _
             const int64_t b = g * kGroup + lane + 32 * j;
             if (FULL || b < nbo) {
                 const float xn = __fdiv_rn(cv[j], d);
-                absmax_q[b] = (uint8_t)(ascending ? nearest_ascending(xn, t) : nearest_any(xn, t));
+                absmax_q[b] = (uint8_t)(ASC ? nearest_ascending(xn, t) : nearest_any(xn, t));
             }
         }
     };
     const int64_t nfull = nbo / kGroup;
-    for (int64_t g = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); g < ngroups; g += wstride) {
-        if (g < nfull) group(g, std::true_type{});
-        else group(g, std::false_type{});
+    const int64_t g0 = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    if (ascending) {
+        for (int64_t g = g0; g < ngroups; g += wstride) {
+            if (g < nfull) group(g, std::true_type{}, std::true_type{});
+            else group(g, std::false_type{}, std::true_type{});
+        }
+    } else {
+        for (int64_t g = g0; g < ngroups; g += wstride) group(g, std::false_type{}, std::false_type{});
     }
 }
 
