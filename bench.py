@@ -318,45 +318,57 @@ def run_bbc(args):
     cbs = {K: bbc.bbc_nf_codebook(K) for K in (3, 4, 5)}
     cb_dev = {K: torch.from_numpy(cbs[K]).to(dev) for K in cbs}
     ks = sorted({K for _, _, K in ops if K})
-    packed = {K: torch.empty(nb * K, dtype=torch.int32, device=dev) for K in ks}
-    absmax = {K: torch.empty(nb, dtype=torch.float32, device=dev) for K in ks}
-    absmax8 = {K: torch.empty(nb, dtype=torch.uint8, device=dev) for K in ks}
-    outs = {K: torch.empty(n, dtype=torch.bfloat16, device=dev) for K in ks}
     nested = synthetic.nested_state(n, NESTED_BS, seed=3, device=dev)
     codes, q, a2, off = nested
     code2 = synthetic.general8_table()
     code4 = cbs[4]
     code2_dev, code4_dev = torch.from_numpy(code2).to(dev), cb_dev[4]
-    nout = torch.empty(n, dtype=torch.bfloat16, device=dev)
     kinds = {kind for _, kind, _ in ops}
-    if kinds & {"quantize_4bit", "quantize_nested"}:
-        nbo4 = (n + NESTED_BS - 1) // NESTED_BS
-        q4_codes = torch.empty((n + 1) // 2, dtype=torch.uint8, device=dev)
-        q4_absmax = torch.empty(nbo4, dtype=torch.float32, device=dev)
-        nq_out = (torch.empty((n + 1) // 2, dtype=torch.uint8, device=dev),
-                  torch.empty(nbo4, dtype=torch.uint8, device=dev),
-                  torch.empty((nbo4 + 255) // 256, dtype=torch.float32, device=dev),
-                  torch.empty(1, dtype=torch.float32, device=dev))
-        nq_ws = torch.empty(bbc.quantize_4bit_nested_workspace_bytes(n, NESTED_BS), dtype=torch.uint8, device=dev)
+
+    def make_outputs():
+        """Every output (and workspace) buffer one step writes."""
+        o = {"packed": {K: torch.empty(nb * K, dtype=torch.int32, device=dev) for K in ks},
+             "absmax": {K: torch.empty(nb, dtype=torch.float32, device=dev) for K in ks},
+             "absmax8": {K: torch.empty(nb, dtype=torch.uint8, device=dev) for K in ks},
+             "outs": {K: torch.empty(n, dtype=torch.bfloat16, device=dev) for K in ks},
+             "nout": torch.empty(n, dtype=torch.bfloat16, device=dev)}
+        if kinds & {"quantize_4bit", "quantize_nested"}:
+            nbo4 = (n + NESTED_BS - 1) // NESTED_BS
+            o["q4_codes"] = torch.empty((n + 1) // 2, dtype=torch.uint8, device=dev)
+            o["q4_absmax"] = torch.empty(nbo4, dtype=torch.float32, device=dev)
+            o["nq_out"] = (torch.empty((n + 1) // 2, dtype=torch.uint8, device=dev),
+                           torch.empty(nbo4, dtype=torch.uint8, device=dev),
+                           torch.empty((nbo4 + 255) // 256, dtype=torch.float32, device=dev),
+                           torch.empty(1, dtype=torch.float32, device=dev))
+            o["nq_ws"] = torch.empty(bbc.quantize_4bit_nested_workspace_bytes(n, NESTED_BS), dtype=torch.uint8,
+                                     device=dev)
+        return o
+
+    outA = make_outputs()
+    inA = {"x": x, "codes": codes, "q": q, "a2": a2, "cb": cb_dev, "code4": code4_dev, "code2": code2_dev}
     stream = torch.cuda.current_stream(dev)
 
-    def launch(kind, K, xin=x, cin=codes, qin=q, a2in=a2, pk=packed, am=absmax, ou=outs, no=nout):
+    def launch(kind, K, inp=inA, o=outA, st=stream):
+        cb = inp["cb"]
         if kind == "quantize":
-            bbc.kbit_quantize(xin, K, cb_dev[K], absmax=am[K], packed=pk[K], stream=stream)
+            bbc.kbit_quantize(inp["x"], K, cb[K], absmax=o["absmax"][K], packed=o["packed"][K], stream=st)
         elif kind == "dequantize":
-            bbc.kbit_dequantize(pk[K], am[K], cb_dev[K], K, n, torch.bfloat16, out=ou[K], stream=stream)
+            bbc.kbit_dequantize(o["packed"][K], o["absmax"][K], cb[K], K, n, torch.bfloat16, out=o["outs"][K],
+                                stream=st)
         elif kind == "quantize_e4m4":
-            bbc.kbit_quantize_e4m4(xin, K, cb_dev[K], absmax=absmax8[K], packed=pk[K], stream=stream)
+            bbc.kbit_quantize_e4m4(inp["x"], K, cb[K], absmax=o["absmax8"][K], packed=o["packed"][K], stream=st)
         elif kind == "dequantize_e4m4":
-            bbc.kbit_dequantize_e4m4(pk[K], absmax8[K], cb_dev[K], K, n, torch.bfloat16, out=ou[K], stream=stream)
+            bbc.kbit_dequantize_e4m4(o["packed"][K], o["absmax8"][K], cb[K], K, n, torch.bfloat16,
+                                     out=o["outs"][K], stream=st)
         elif kind == "quantize_4bit":
-            bbc.quantize_4bit(xin, NESTED_BS, code4_dev, absmax=q4_absmax, codes=q4_codes, stream=stream)
+            bbc.quantize_4bit(inp["x"], NESTED_BS, inp["code4"], absmax=o["q4_absmax"], codes=o["q4_codes"],
+                              stream=st)
         elif kind == "quantize_nested":
-            bbc.quantize_4bit_nested(xin, NESTED_BS, code4_dev, code2_dev, workspace=nq_ws, out=nq_out,
-                                     stream=stream)
+            bbc.quantize_4bit_nested(inp["x"], NESTED_BS, inp["code4"], inp["code2"], workspace=o["nq_ws"],
+                                     out=o["nq_out"], stream=st)
         else:
-            bbc.dequantize_4bit_nested(cin, qin, code2_dev, a2in, float(off), code4_dev, n, NESTED_BS,
-                                       torch.bfloat16, out=no, stream=stream)
+            bbc.dequantize_4bit_nested(inp["codes"], inp["q"], inp["code2"], inp["a2"], float(off), inp["code4"], n,
+                                       NESTED_BS, torch.bfloat16, out=o["nout"], stream=st)
 
     for _ in range(args.warmup):
         for _, kind, K in ops:
@@ -431,61 +443,79 @@ def run_bbc(args):
 
     # ---- end to end through the public API with host buffers
     if not args.no_e2e:
+        # End to end through the public API from pinned host memory: every step copies its inputs
+        # in and its results out inside the timed region. Two buffer sets and three streams (copies
+        # in, compute, copies out, ordered by events) let step k + 1's input copies and kernels
+        # overlap step k's output copies: PCIe carries the two directions at once.
         pin = lambda t: t.cpu().pin_memory()  # noqa: E731
-        hx, hcodes, hq, ha2 = pin(x), pin(codes), pin(q), pin(a2)
-        hcb = {K: torch.from_numpy(cbs[K]).pin_memory() for K in (3, 4, 5)}
+        h_in = {"x": pin(x), "codes": pin(codes), "q": pin(q), "a2": pin(a2),
+                "cb": {K: torch.from_numpy(cbs[K]).pin_memory() for K in (3, 4, 5)}}
         k32 = sorted({K for _, kind, K in ops if kind in ("quantize", "dequantize")})
         k8 = sorted({K for _, kind, K in ops if kind.endswith("_e4m4")})
-        h_out = {"packed": {K: torch.empty_like(packed[K], device="cpu").pin_memory() for K in ks},
-                 "absmax": {K: torch.empty_like(absmax[K], device="cpu").pin_memory() for K in k32},
-                 "absmax8": {K: torch.empty_like(absmax8[K], device="cpu").pin_memory() for K in k8},
-                 "out": {K: torch.empty_like(outs[K], device="cpu").pin_memory() for K in ks},
-                 "nested": torch.empty_like(nout, device="cpu").pin_memory()}
-        dx, dcodes, dq, da2 = torch.empty_like(x), torch.empty_like(codes), torch.empty_like(q), torch.empty_like(a2)
-        h2d = sum(t.numel() * t.element_size() for t in (hx, hcodes, hq, ha2)) + \
-            sum(t.numel() * 4 for t in hcb.values())
-        q4_dev = ([q4_codes, q4_absmax] if "quantize_4bit" in kinds else []) + \
-            (list(nq_out) if "quantize_nested" in kinds else [])
-        q4_host = [(t, torch.empty_like(t, device="cpu").pin_memory()) for t in q4_dev]
-        d2h = sum(t.numel() * t.element_size() for K in ks for t in (packed[K], outs[K])) + \
-            sum(absmax[K].numel() * 4 for K in k32) + sum(absmax8[K].numel() for K in k8) + nout.numel() * 2 + \
-            sum(t.numel() * t.element_size() for t in q4_dev)
 
-        def e2e_step():
-            dx.copy_(hx, non_blocking=True)
-            dcodes.copy_(hcodes, non_blocking=True)
-            dq.copy_(hq, non_blocking=True)
-            da2.copy_(ha2, non_blocking=True)
-            for K in (3, 4, 5):
-                cb_dev[K].copy_(hcb[K], non_blocking=True)
+        def results(o):
+            """The device tensors a step reads back (in a fixed order)."""
+            r = [o["packed"][K] for K in ks] + [o["outs"][K] for K in ks] + [o["absmax"][K] for K in k32] + \
+                [o["absmax8"][K] for K in k8] + [o["nout"]]
+            if "quantize_4bit" in kinds:
+                r += [o["q4_codes"], o["q4_absmax"]]
+            if "quantize_nested" in kinds:
+                r += list(o["nq_out"])
+            return r
+
+        sets = []
+        for i in range(2):
+            d_in = {"x": torch.empty_like(x), "codes": torch.empty_like(codes), "q": torch.empty_like(q),
+                    "a2": torch.empty_like(a2), "cb": {K: torch.empty_like(cb_dev[K]) for K in (3, 4, 5)}}
+            d_in["code4"], d_in["code2"] = d_in["cb"][4], code2_dev
+            sets.append((d_in, outA if i == 0 else make_outputs()))
+        h_out = [torch.empty_like(t, device="cpu").pin_memory() for t in results(outA)]
+        h2d = sum(h_in[k].numel() * h_in[k].element_size() for k in ("x", "codes", "q", "a2")) + \
+            sum(t.numel() * 4 for t in h_in["cb"].values())
+        d2h = sum(t.numel() * t.element_size() for t in h_out)
+        s_in, s_comp, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+        ev_in = [torch.cuda.Event() for _ in range(2)]
+        ev_comp = [torch.cuda.Event() for _ in range(2)]
+        ev_out = [torch.cuda.Event() for _ in range(2)]
+
+        def e2e_step(k):
+            i = k % 2
+            d_in, o = sets[i]
+            s_in.wait_event(ev_comp[i])          # the set's inputs are no longer read
+            with torch.cuda.stream(s_in):
+                for key in ("x", "codes", "q", "a2"):
+                    d_in[key].copy_(h_in[key], non_blocking=True)
+                for K in (3, 4, 5):
+                    d_in["cb"][K].copy_(h_in["cb"][K], non_blocking=True)
+                ev_in[i].record(s_in)
+            s_comp.wait_event(ev_in[i])
+            s_comp.wait_event(ev_out[i])         # the set's previous results have been read back
             for _, kind, K in ops:
-                launch(kind, K, xin=dx, cin=dcodes, qin=dq, a2in=da2)
-            for K in ks:
-                h_out["packed"][K].copy_(packed[K], non_blocking=True)
-                h_out["out"][K].copy_(outs[K], non_blocking=True)
-            for K in k32:
-                h_out["absmax"][K].copy_(absmax[K], non_blocking=True)
-            for K in k8:
-                h_out["absmax8"][K].copy_(absmax8[K], non_blocking=True)
-            h_out["nested"].copy_(nout, non_blocking=True)
-            for t, h in q4_host:
-                h.copy_(t, non_blocking=True)
+                launch(kind, K, d_in, o, s_comp)
+            ev_comp[i].record(s_comp)
+            s_out.wait_event(ev_comp[i])
+            with torch.cuda.stream(s_out):
+                for h, t in zip(h_out, results(o)):
+                    h.copy_(t, non_blocking=True)
+                ev_out[i].record(s_out)
 
-        e2e_step()
+        for k in range(2):
+            e2e_step(k)
         torch.cuda.synchronize()
         if dist:
             dist.barrier()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        for _ in range(args.e2e_steps):
-            e2e_step()
-        e1.record(stream)
+        e0.record(s_in)
+        for k in range(args.e2e_steps):
+            e2e_step(k)
+        e1.record(s_out)
         torch.cuda.synchronize()
         e_ms = max_over_ranks(e0.elapsed_time(e1) / args.e2e_steps, device=dev)
         result["e2e"] = {"value": round(world * bytes_step / (e_ms * 1e-3) / 1e9, 2), "unit": "GB/s",
                          "ms_per_step": round(e_ms, 3), "h2d_bytes_per_step": h2d,
                          "d2h_bytes_per_step": d2h, "steps": args.e2e_steps,
-                         "api": "blockwise_bit_codebook_b200 (C ABI via ctypes), pinned host buffers"}
+                         "api": "blockwise_bit_codebook_b200 (C ABI via ctypes), pinned host buffers; copies in, "
+                                "kernels and copies out on three streams, two buffer sets"}
 
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         result["cpu_baseline"] = cpu_baseline(x, nested, code2, code4, cbs, args.cpu_seconds, n)
