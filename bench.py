@@ -47,7 +47,7 @@ def parse_args():
                     help="override the element count (profiling of a smaller case)")
     ap.add_argument("--ops", default=None,
                     help="comma-separated subset of quantize_k3,dequantize_k3,quantize_k5,"
-                         "dequantize_k5,nested_nf4_bs64, or the E4M4-absmax ops "
+                         "dequantize_k5,nested_nf4_bs64, {quantize,dequantize}_k{2,4}, or the E4M4-absmax ops "
                          "{quantize,dequantize}_k{3,4,5}_e4m4, or quantize_4bit_nf4_bs64, "
                          "quantize_nested_nf4_bs64 (profiling)")
     ap.add_argument("--e2e-steps", type=int, default=5)
@@ -110,7 +110,8 @@ def nested_quant_launches(n, bs=NESTED_BS):
     return 2 + levels
 
 # Selectable with --ops (not part of the default step): the E4M4-absmax codec.
-EXTRA_OPS = [(f"{k}_k{K}_e4m4", f"{k}_e4m4", K) for K in (3, 4, 5) for k in ("quantize", "dequantize")] + \
+EXTRA_OPS = [(f"{k}_k{K}", k, K) for K in (2, 4) for k in ("quantize", "dequantize")] + \
+    [(f"{k}_k{K}_e4m4", f"{k}_e4m4", K) for K in (3, 4, 5) for k in ("quantize", "dequantize")] + \
     [("quantize_4bit_nf4_bs64", "quantize_4bit", None), ("quantize_nested_nf4_bs64", "quantize_nested", None)]
 
 
@@ -315,7 +316,7 @@ def run_bbc(args):
     n = args.n or N_C5
     nb = (n + 31) // 32
     x = synthetic.weights(n, std=0.02, seed=7, dtype=torch.bfloat16, device=dev)
-    cbs = {K: bbc.bbc_nf_codebook(K) for K in (3, 4, 5)}
+    cbs = {K: bbc.bbc_nf_codebook(K) for K in (2, 3, 4, 5)}
     cb_dev = {K: torch.from_numpy(cbs[K]).to(dev) for K in cbs}
     ks = sorted({K for _, _, K in ops if K})
     nested = synthetic.nested_state(n, NESTED_BS, seed=3, device=dev)
@@ -449,7 +450,7 @@ def run_bbc(args):
         # overlap step k's output copies: PCIe carries the two directions at once.
         pin = lambda t: t.cpu().pin_memory()  # noqa: E731
         h_in = {"x": pin(x), "codes": pin(codes), "q": pin(q), "a2": pin(a2),
-                "cb": {K: torch.from_numpy(cbs[K]).pin_memory() for K in (3, 4, 5)}}
+                "cb": {K: torch.from_numpy(cbs[K]).pin_memory() for K in (2, 3, 4, 5)}}
         k32 = sorted({K for _, kind, K in ops if kind in ("quantize", "dequantize")})
         k8 = sorted({K for _, kind, K in ops if kind.endswith("_e4m4")})
 
@@ -466,7 +467,7 @@ def run_bbc(args):
         sets = []
         for i in range(2):
             d_in = {"x": torch.empty_like(x), "codes": torch.empty_like(codes), "q": torch.empty_like(q),
-                    "a2": torch.empty_like(a2), "cb": {K: torch.empty_like(cb_dev[K]) for K in (3, 4, 5)}}
+                    "a2": torch.empty_like(a2), "cb": {K: torch.empty_like(cb_dev[K]) for K in (2, 3, 4, 5)}}
             d_in["code4"], d_in["code2"] = d_in["cb"][4], code2_dev
             sets.append((d_in, outA if i == 0 else make_outputs()))
         h_out = [torch.empty_like(t, device="cpu").pin_memory() for t in results(outA)]
@@ -485,7 +486,7 @@ def run_bbc(args):
             with torch.cuda.stream(s_in):
                 for key in ("x", "codes", "q", "a2"):
                     d_in[key].copy_(h_in[key], non_blocking=True)
-                for K in (3, 4, 5):
+                for K in (2, 3, 4, 5):
                     d_in["cb"][K].copy_(h_in["cb"][K], non_blocking=True)
                 ev_in[i].record(s_in)
             s_comp.wait_event(ev_in[i])

@@ -119,3 +119,18 @@ def test_packed_matches_fp32_absmax_path(bbc):
     torch.cuda.synchronize()
     assert torch.equal(p1, p2)
     assert_bits_equal(to_host(a2), oracle.e4m4_encode(to_host(a1)), "encode of the fp32 absmax")
+
+
+def test_dequant_long_stream_half_block_path(bbc):
+    """A 16-bit output stream of at least 2^26 elements takes the half-block dequant form for K=4."""
+    K, n = 4, (1 << 26) + 37
+    nb = (n + 31) // 32
+    rng = np.random.default_rng(23)
+    packed = rng.integers(0, 2 ** 32, nb * K, dtype=np.uint64).astype(np.uint32)
+    am = rng.integers(0, 256, nb, dtype=np.uint64).astype(np.uint8)
+    cb_np = oracle.normal_float_codebook(K)
+    ref = oracle.kbit_dequantize_e4m4(packed, am, cb_np, K, n, "bf16")
+    y = bbc.kbit_dequantize_e4m4(torch.from_numpy(packed.view(np.int32)).cuda(), torch.from_numpy(am).cuda(),
+                                 torch.from_numpy(cb_np).cuda(), K, n, torch.bfloat16)
+    torch.cuda.synchronize()
+    assert_bits_equal(to_host(y)[:n], ref, "long stream e4m4 K=4 bf16")

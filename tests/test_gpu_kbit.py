@@ -308,6 +308,19 @@ def test_dequant_random_state(bbc, K, dt):
     check_dequantize(bbc, packed, absmax, cb, K, n, dt, f"random K{K}")
 
 
+@pytest.mark.parametrize("K", [2, 3, 4])
+def test_dequant_long_stream_half_block_path(bbc, K):
+    """16-bit outputs of at least 2^26 elements take the half-block path (K <= 4); an odd length
+    ends in a ragged half block."""
+    rng = np.random.default_rng(7 + K)
+    n = (1 << 26) + 37
+    nb = (n + 31) // 32
+    packed = rng.integers(0, 2**32, nb * K, dtype=np.uint64).astype(np.uint32)
+    absmax = rng.uniform(0.01, 0.1, nb).astype(np.float32)
+    cb = oracle.normal_float_codebook(K)
+    check_dequantize(bbc, packed, absmax, cb, K, n, "bf16", f"long K{K}")
+
+
 # ---------------------------------------------------------------- contract
 
 def test_no_writes_beyond_outputs_and_inputs_unchanged(bbc):
