@@ -13,11 +13,14 @@
 //      tree; each level of 2048 nodes is one launch.
 //   3. per group of 256 outer blocks, c_b = fl(absmax_b - offset): absmax2 = max |c_b| and
 //      absmax_q_b = the first nearest General8 entry to fl(c_b / fmaxf(absmax2, 1e-8f))
-//      (absmax_compress_kernel). For an ascending table the nearest entry is found exactly by
-//      binary search: fl(|xn - t_i|) does not increase up to the last t_i <= xn and does not
-//      decrease after it, so the minimum is at one of those two neighbours and the first index
-//      holding it is found by walking down a plateau of equal distances. Any other table takes
-//      the rule verbatim over all 256 entries.
+//      (absmax_compress_kernel). For an ascending table the nearest entry is found exactly from
+//      p = the last index with t_p <= xn: fl(|xn - t_i|) does not increase up to t_p and does
+//      not decrease after it, so the minimum is at t_p or t_{p+1} and the first index holding
+//      it is found by walking down a plateau of equal distances. p itself comes from a table of
+//      its values at the lower ends of 64 buckets per binade of |xn| (from 2^-24 up to 1) and a
+//      forward scan inside the bucket; comparisons t_p <= xn are exact, so this is the same p a
+//      search over all entries gives. Any other table takes the rule verbatim over all 256
+//      entries.
 #include <cfloat>
 #include <type_traits>
 
@@ -65,23 +68,61 @@ tree_sum_kernel(const T* __restrict__ in, int64_t count, double* __restrict__ no
 // never conflict. `t` below is a lane's replica base; entry i is t[i * kRep].
 constexpr int kRep = 32;
 
+// Buckets of the scaled value xn (|xn| <= 1 or NaN): 64 per binade of |xn| from 2^-24
+// (M(k) = the float with bits (k + kLutE0) << 17 is the lower edge of magnitude bucket k; all
+// smaller magnitudes fall in bucket 0), negative values first in ascending order of value:
+// bucket 1536 - k holds the negatives of magnitude in [M(k), M(k + 1)) and its lower point is
+// -M(k + 1); bucket 1537 + k holds the positives in [M(k), M(k + 1)) and its lower point is
+// M(k) (0 for k = 0). lut[j] = base | cnt << 9: base = #{i : t_i <= lower point of bucket j}
+// (0..256) and cnt = min(#{i : t_i above it and at or below the next bucket's}, 127), which
+// bounds the forward scan from base - 1 for any xn in the bucket.
+constexpr int kLutShift = 17;
+constexpr int kLutE0 = (127 - 24) << (23 - kLutShift);
+constexpr int kLutHalf = 24 << (23 - kLutShift);                // magnitude buckets 0..1536
+constexpr int kLutN = 2 * kLutHalf + 2;                         // 3074 buckets
+
+// Bucket of a value with |xn| <= 1 (NaN lands anywhere; the caller overrides it).
+__device__ __forceinline__ int lut_bucket(float xn) {
+    const uint32_t b = __float_as_uint(xn);
+    const int k = min(max((int)((b & 0x7fffffffu) >> kLutShift) - kLutE0, 0), kLutHalf);
+    return (b >> 31) ? kLutHalf - k : kLutHalf + 1 + k;
+}
+
+// First bucket whose lower point is >= x (kLutN if none), for any float x.
+__device__ __forceinline__ int lut_first_at_or_above(float x) {
+    const uint32_t b = __float_as_uint(x);
+    const int k = (int)((b & 0x7fffffffu) >> kLutShift) - kLutE0;   // M(k) <= |x| < M(k + 1) if k >= 0
+    if (x != x) return kLutN;
+    if (b >> 31) return max(kLutHalf + 1 - max(k, 0), 0);     // -M(mb + 1) >= x  <=>  mb + 1 <= k
+    if (b == 0) return kLutHalf + 1;
+    const bool edge = (b & ((1u << kLutShift) - 1)) == 0 && k >= 1;    // x == M(k)
+    return min(kLutHalf + 1 + max(edge ? k : k + 1, 1), kLutN);         // least M(mb) >= x
+}
+
 // First index minimising fl(|xn - t_i|) over an ascending 256-entry table (see the header).
-__device__ __forceinline__ uint32_t nearest_ascending(float xn, const float* t) {
-    int p = -1;                                                 // last index with entry p <= xn
-#pragma unroll
-    for (int step = 128; step >= 1; step >>= 1)                  // p + step <= 254 throughout
-        p += t[(p + step) * kRep] <= xn ? step : 0;
-    p = t[255 * kRep] <= xn ? 255 : p;
+// The common path has no branch, so the eight values a lane handles overlap their table reads.
+__device__ __forceinline__ uint32_t nearest_ascending(float xn, const float* t, const uint16_t* lut) {
+    const uint32_t e = lut[lut_bucket(xn)];
+    // p = the last index with t_p <= xn: the bucket's base less one, then a forward scan over
+    // the at most e >> 9 entries inside the bucket (one step unconditionally, more rarely)
+    int p = xn != xn ? -1 : (int)(e & 511u) - 1;
+    p += (p < 255 && t[min(p + 1, 255) * kRep] <= xn) ? 1 : 0;
+    if ((e >> 9) > 1)
+        while (p < 255 && t[(p + 1) * kRep] <= xn) p++;
     // The first nearest entry is t[p] or t[p + 1]. With p clamped to 0 the same selects give 0
     // when no entry is <= xn (t[1] is never strictly closer than t[0] below t[0]) and for a NaN
     // xn (no comparison holds); at p = 255 the clamped neighbour is t[255] itself.
     const int q = max(p, 0), r = min(q + 1, 255);
     const float dq = fabsf(__fsub_rn(xn, t[q * kRep]));
     const float dr = fabsf(__fsub_rn(xn, t[r * kRep]));
-    if (dr < dq) return (uint32_t)r;
-    int i = q;                                                  // walk down a plateau of equal distances
-    while (i > 0 && fabsf(__fsub_rn(xn, t[(i - 1) * kRep])) == dq) i--;
-    return (uint32_t)i;
+    // walk down a plateau of equal distances below q (equal entries, or distances that round
+    // alike: rare)
+    int i = q;
+    if (q > 0 && fabsf(__fsub_rn(xn, t[max(q - 1, 0) * kRep])) == dq) {
+        i--;
+        while (i > 0 && fabsf(__fsub_rn(xn, t[(i - 1) * kRep])) == dq) i--;
+    }
+    return (uint32_t)(dr < dq ? r : i);
 }
 
 __device__ __forceinline__ uint32_t nearest_any(float xn, const float* t) {
@@ -112,7 +153,46 @@ absmax_compress_kernel(const float* __restrict__ absmax, int64_t nbo, const T* _
 #pragma unroll
     for (int k = 0; k < 8; k++)
         reinterpret_cast<float4*>(tr)[threadIdx.x * 8 + ((k + threadIdx.x) & 7)] = v4;
-    // the barrier also makes the replicas visible
+    // bucket table from a histogram: h[J] = #{i : first bucket at or above t_i is J} (J = kLutN:
+    // above every bucket); with S its inclusive prefix sum, bucket j's base is S(j) (the entries
+    // at or below its lower point) and h[j + 1] = S(j + 1) - S(j) the entries inside it. Thread k
+    // owns slots [13k, 13k + 13) of the prefix sum. Meaningful only for an ascending table.
+    constexpr int kSlots = 13;
+    static_assert(kSlots * 256 >= kLutN + 1, "every slot has an owner");
+    __shared__ uint32_t hist[kLutN + 1];                        // then the table, as 16-bit entries
+    __shared__ uint32_t warp_sum[8];
+    uint16_t* const lut = reinterpret_cast<uint16_t*>(hist);
+    {
+        const int s0 = threadIdx.x * kSlots;
+#pragma unroll
+        for (int k = 0; k < kSlots; k++)
+            if (s0 + k <= kLutN) hist[s0 + k] = 0;
+        __syncthreads();
+        atomicAdd(&hist[lut_first_at_or_above(v)], 1u);
+        __syncthreads();
+        uint32_t h[kSlots + 1];
+#pragma unroll
+        for (int k = 0; k <= kSlots; k++) h[k] = s0 + k <= kLutN ? hist[s0 + k] : 0u;
+        uint32_t run = 0;                                        // total over own slots
+#pragma unroll
+        for (int k = 0; k < kSlots; k++) run += h[k];
+        uint32_t x = run;                                        // inclusive scan of thread totals
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
+            if ((threadIdx.x & 31) >= o) x += y;
+        }
+        if ((threadIdx.x & 31) == 31) warp_sum[threadIdx.x >> 5] = x;
+        __syncthreads();                                         // also: every read of hist is done
+        uint32_t sum = x - run;
+        for (int w = 0; w < (int)(threadIdx.x >> 5); w++) sum += warp_sum[w];
+#pragma unroll
+        for (int k = 0; k < kSlots; k++) {
+            sum += h[k];
+            if (s0 + k < kLutN) lut[s0 + k] = (uint16_t)(sum | min(h[k + 1], 127u) << 9);
+        }
+    }
+    // the barrier also makes the replicas and the bucket table visible
     const bool ascending = __syncthreads_and(v <= next);        // false if any entry is NaN
     const float* t = tr + (threadIdx.x & (kRep - 1));
     // the offset: the root of the pairwise tree over the last level (<= 2048 values), the
@@ -145,7 +225,7 @@ absmax_compress_kernel(const float* __restrict__ absmax, int64_t nbo, const T* _
             const int64_t b = g * kGroup + lane + 32 * j;
             if (FULL || b < nbo) {
                 const float xn = __fdiv_rn(cv[j], d);
-                absmax_q[b] = (uint8_t)(ASC ? nearest_ascending(xn, t) : nearest_any(xn, t));
+                absmax_q[b] = (uint8_t)(ASC ? nearest_ascending(xn, t, lut) : nearest_any(xn, t));
             }
         }
     };

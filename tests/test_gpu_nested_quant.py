@@ -146,3 +146,43 @@ def test_every_16bit_quotient_4bit(bbc, table, dt):
             blocks.append(blk)
     x = np.concatenate(blocks)
     check_q4(bbc, torch.from_numpy(x.view(np.int16)).view(DTYPES[dt]), 32, code4, what=f"every {dt} quotient")
+
+
+def _quotients(x_host, bs):
+    """The scaled values the General8 search sees for this input (used only to place table
+    entries on and beside them; the expected state still comes from the oracle)."""
+    _, absmax = oracle.quantize_4bit(to_host(x_host), NAMES[x_host.dtype], bs, NF4)
+    c = absmax - oracle.absmax_offset(absmax)
+    pad = (-c.size) % 256
+    d = np.abs(np.concatenate([c, np.zeros(pad, np.float32)])).reshape(-1, 256).max(axis=1)
+    d = np.maximum(d, np.float32(1e-8)).astype(np.float32)
+    return (c / np.repeat(d, 256)[:c.size]).astype(np.float32)
+
+
+@pytest.mark.parametrize("kind", ["hits", "cluster", "duplicates", "infinite_ends", "all_equal"])
+def test_nested_compression_crafted_tables(bbc, kind):
+    """Ascending tables placed around the quotients the input produces: entries equal to
+    quotients and one ulp beside them (exact and near ties), a dense cluster of 160 entries
+    around the median quotient (many entries per bucket of the search), runs of equal entries
+    (plateaus of equal distance), infinite end entries, and a table of one repeated value."""
+    bs = 64
+    x = synthetic.weights(bs * 256 * 5 + bs * 9 + 5, std=0.02, seed=31, dtype=torch.float32)
+    xn = _quotients(x, bs)
+    rng = np.random.default_rng(41)
+    picks = rng.choice(xn, 48, replace=False)
+    med = np.float32(np.median(xn))
+    if kind == "hits":
+        parts = [picks, np.nextafter(picks, np.float32(2)), np.nextafter(picks, np.float32(-2))]
+    elif kind == "cluster":
+        parts = [np.linspace(med - 2e-4, med + 2e-4, 160, dtype=np.float32), picks]
+    elif kind == "duplicates":
+        parts = [np.repeat(picks[:20], 4), np.repeat(np.float32(med), 30), picks[20:]]
+    elif kind == "infinite_ends":
+        parts = [np.array([-np.inf, np.inf], np.float32), picks]
+    else:
+        parts = [np.full(256, med, np.float32)]
+    have = np.concatenate(parts).astype(np.float32)[:256]
+    fill = rng.uniform(-1, 1, 256 - have.size).astype(np.float32)
+    table = np.sort(np.concatenate([have, fill])).astype(np.float32)
+    assert table.size == 256 and np.all(table[:-1] <= table[1:])
+    check_nested(bbc, x, bs, code2=table, what=f"crafted {kind}")
