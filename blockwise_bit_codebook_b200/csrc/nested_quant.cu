@@ -34,17 +34,44 @@ namespace {
 constexpr int kTree = 2048;            // tree leaves per CTA (256 threads x 8)
 constexpr int kGroup = 256;            // outer blocks per inner absmax
 
+// Leaves [base, base + 8) of a node (zeros past count) summed as a tree, with vector loads when
+// all eight lie inside (base is a multiple of 8 and the values 16-byte aligned).
+__device__ __forceinline__ double leaf8(const float* __restrict__ in, int64_t count, int64_t base) {
+    double v[8];
+    if (base + 8 <= count) {
+        const float4 a = __ldg(reinterpret_cast<const float4*>(in + base));
+        const float4 b = __ldg(reinterpret_cast<const float4*>(in + base + 4));
+        v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w; v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+    } else {
+#pragma unroll
+        for (int j = 0; j < 8; j++) v[j] = base + j < count ? (double)in[base + j] : 0.0;
+    }
+    return __dadd_rn(__dadd_rn(__dadd_rn(v[0], v[1]), __dadd_rn(v[2], v[3])),
+                     __dadd_rn(__dadd_rn(v[4], v[5]), __dadd_rn(v[6], v[7])));
+}
+
+__device__ __forceinline__ double leaf8(const double* __restrict__ in, int64_t count, int64_t base) {
+    double v[8];
+    if (base + 8 <= count) {
+#pragma unroll
+        for (int j = 0; j < 8; j += 2) {
+            const double2 a = __ldg(reinterpret_cast<const double2*>(in + base + j));
+            v[j] = a.x; v[j + 1] = a.y;
+        }
+    } else {
+#pragma unroll
+        for (int j = 0; j < 8; j++) v[j] = base + j < count ? in[base + j] : 0.0;
+    }
+    return __dadd_rn(__dadd_rn(__dadd_rn(v[0], v[1]), __dadd_rn(v[2], v[3])),
+                     __dadd_rn(__dadd_rn(v[4], v[5]), __dadd_rn(v[6], v[7])));
+}
+
 // Node `blk` of one level of the pairwise sum: in[2048 blk .. 2048 blk + 2048) (zeros past
 // count) summed as a binary tree by the whole CTA (8 leaves per thread as a tree, lanes by
 // xor-shuffles, warps in shared memory); the result is returned to every thread.
 template <typename T>
 __device__ __forceinline__ double tree_node(const T* __restrict__ in, int64_t count, int64_t blk, double* ws) {
-    const int64_t base = blk * kTree + threadIdx.x * 8;
-    double v[8];
-#pragma unroll
-    for (int j = 0; j < 8; j++) v[j] = base + j < count ? (double)in[base + j] : 0.0;
-    double s = __dadd_rn(__dadd_rn(__dadd_rn(v[0], v[1]), __dadd_rn(v[2], v[3])),
-                         __dadd_rn(__dadd_rn(v[4], v[5]), __dadd_rn(v[6], v[7])));
+    double s = leaf8(in, count, blk * kTree + threadIdx.x * 8);
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) s = __dadd_rn(s, __shfl_xor_sync(0xffffffffu, s, o));
     __syncthreads();                                            // ws may hold a previous use
@@ -54,13 +81,31 @@ __device__ __forceinline__ double tree_node(const T* __restrict__ in, int64_t co
                      __dadd_rn(__dadd_rn(ws[4], ws[5]), __dadd_rn(ws[6], ws[7])));
 }
 
-// One level of the pairwise sum below the root: node b = the tree of in[2048 b .. 2048 b + 2048).
+// One level of the pairwise sum below the root: node b = the tree of in[2048 b .. 2048 b + 2048),
+// kNodesPerCta consecutive nodes per CTA (their loads all in flight together), each summed
+// exactly as tree_node does.
+constexpr int kNodesPerCta = 4;
+
 template <typename T>
 __global__ void __launch_bounds__(256)
-tree_sum_kernel(const T* __restrict__ in, int64_t count, double* __restrict__ nodes) {
-    __shared__ double ws[8];
-    const double r = tree_node(in, count, blockIdx.x, ws);
-    if (threadIdx.x == 0) nodes[blockIdx.x] = r;
+tree_sum_kernel(const T* __restrict__ in, int64_t count, int64_t nnodes, double* __restrict__ nodes) {
+    __shared__ double ws[kNodesPerCta][8];
+    double s[kNodesPerCta];
+#pragma unroll
+    for (int k = 0; k < kNodesPerCta; k++)
+        s[k] = leaf8(in, count, ((int64_t)blockIdx.x * kNodesPerCta + k) * kTree + threadIdx.x * 8);
+#pragma unroll
+    for (int k = 0; k < kNodesPerCta; k++) {
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) s[k] = __dadd_rn(s[k], __shfl_xor_sync(0xffffffffu, s[k], o));
+        if ((threadIdx.x & 31) == 0) ws[k][threadIdx.x >> 5] = s[k];
+    }
+    __syncthreads();
+    const int k = threadIdx.x;
+    const int64_t blk = (int64_t)blockIdx.x * kNodesPerCta + k;
+    if (k < kNodesPerCta && blk < nnodes)
+        nodes[blk] = __dadd_rn(__dadd_rn(__dadd_rn(ws[k][0], ws[k][1]), __dadd_rn(ws[k][2], ws[k][3])),
+                               __dadd_rn(__dadd_rn(ws[k][4], ws[k][5]), __dadd_rn(ws[k][6], ws[k][7])));
 }
 
 // The General8 table in shared memory as 32 lane-interleaved replicas (entry i of replica r at
@@ -246,12 +291,13 @@ absmax_compress_kernel(const float* __restrict__ absmax, int64_t nbo, const T* _
 namespace {
 int64_t tree_nodes(int64_t count) { return (count + kTree - 1) / kTree; }
 int64_t absmax_bytes(int64_t nbo) { return ((nbo * 4 + 255) / 256) * 256; }
+int64_t even(int64_t x) { return x + (x & 1); }                // keeps the second node buffer 16-byte aligned
 }  // namespace
 
 size_t nested_quant_workspace_bytes(int64_t n, int log2_bs) {
     const int64_t nbo = (n + (1ll << log2_bs) - 1) >> log2_bs;
     const int64_t s1 = tree_nodes(nbo), s2 = tree_nodes(s1);
-    return (size_t)(absmax_bytes(nbo) + (s1 + s2) * 8);
+    return (size_t)(absmax_bytes(nbo) + (even(s1) + s2) * 8);
 }
 
 cudaError_t launch_quantize_4bit_nested(const void* A, int dtype, int64_t n, int log2_bs, const float* code4,
@@ -260,7 +306,7 @@ cudaError_t launch_quantize_4bit_nested(const void* A, int dtype, int64_t n, int
     const int64_t nbo = (n + (1ll << log2_bs) - 1) >> log2_bs;
     float* absmax = static_cast<float*>(workspace);
     double* buf_a = reinterpret_cast<double*>(static_cast<char*>(workspace) + absmax_bytes(nbo));
-    double* buf_b = buf_a + tree_nodes(nbo);
+    double* buf_b = buf_a + even(tree_nodes(nbo));
     cudaError_t e = launch_quantize_4bit(A, dtype, n, log2_bs, code4, absmax, codes, vec, s);
     if (e != cudaSuccess) return e;
     // the pairwise sum: one launch per level while more than 2048 values remain; the root (at
@@ -273,12 +319,14 @@ cudaError_t launch_quantize_4bit_nested(const void* A, int dtype, int64_t n, int
         return cudaGetLastError();
     }
     int64_t count = tree_nodes(nbo);
-    tree_sum_kernel<float><<<(unsigned)count, 256, 0, s>>>(absmax, nbo, buf_a);
+    tree_sum_kernel<float><<<(unsigned)((count + kNodesPerCta - 1) / kNodesPerCta), 256, 0, s>>>(absmax, nbo, count,
+                                                                                               buf_a);
     const double* in = buf_a;
     double* out = buf_b;
     while (count > kTree) {
         const int64_t next = tree_nodes(count);
-        tree_sum_kernel<double><<<(unsigned)next, 256, 0, s>>>(in, count, out);
+        tree_sum_kernel<double><<<(unsigned)((next + kNodesPerCta - 1) / kNodesPerCta), 256, 0, s>>>(in, count, next,
+                                                                                                    out);
         in = out;
         out = out == buf_b ? buf_a : buf_b;        // a level never outgrows the one before it
         count = next;

@@ -117,9 +117,11 @@ def test_quantize_4bit_validation(lib):
     assert q(A=P(0x1001), dt=0) == 1 and q(am=P(0x1002)) == 1
     ws = lib.quantize_4bit_nested_workspace_bytes
     assert ws(0, 64) == 0 and ws(100, 48) == 0
-    nbo = (10 ** 6 + 63) // 64
-    s1 = (nbo + 2047) // 2048
-    assert ws(10 ** 6, 64) == ((nbo * 4 + 255) // 256) * 256 + (s1 + (s1 + 2047) // 2048) * 8
+    for n in (10 ** 6, 64 * 2048 * 3):                   # 8 and 3 first-level tree nodes
+        nbo = (n + 63) // 64
+        s1 = (nbo + 2047) // 2048
+        # absmax (256-byte padded), then the two node buffers, the first padded to an even count
+        assert ws(n, 64) == ((nbo * 4 + 255) // 256) * 256 + (s1 + (s1 & 1) + (s1 + 2047) // 2048) * 8
     nq = lambda ws_ptr=P(0x100000), wsb=1 << 20, bs2=256, n=4096, off=FAKE: lib.quantize_4bit_nested(  # noqa: E731
         FAKE, 1, n, 64, FAKE, FAKE, bs2, FAKE, FAKE, FAKE, off, ws_ptr, wsb, None)
     assert nq(ws_ptr=None) == 1 and nq(off=None) == 1 and nq(n=-1) == 1

@@ -148,6 +148,15 @@ def test_every_16bit_quotient_4bit(bbc, table, dt):
     check_q4(bbc, torch.from_numpy(x.view(np.int16)).view(DTYPES[dt]), 32, code4, what=f"every {dt} quotient")
 
 
+def test_nested_state_two_tree_levels(bbc):
+    """4,198,405 outer blocks (blocksize 32): the offset tree takes two level launches (2,051
+    first-level nodes, an odd count, then 2) before the root, which reads the second node
+    buffer."""
+    nbo = 2048 * 2048 + 2048 * 2 + 5
+    x = synthetic.weights(32 * nbo - 7, std=0.02, seed=77, dtype=torch.bfloat16)
+    check_nested(bbc, x, 32, what="two tree levels")
+
+
 def _quotients(x_host, bs):
     """The scaled values the General8 search sees for this input (used only to place table
     entries on and beside them; the expected state still comes from the oracle)."""
