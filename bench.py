@@ -48,8 +48,8 @@ def parse_args():
     ap.add_argument("--ops", default=None,
                     help="comma-separated subset of quantize_k3,dequantize_k3,quantize_k5,"
                          "dequantize_k5,nested_nf4_bs64, {quantize,dequantize}_k{2,4}, or the E4M4-absmax ops "
-                         "{quantize,dequantize}_k{3,4,5}_e4m4, or quantize_4bit_nf4_bs64, "
-                         "quantize_nested_nf4_bs64 (profiling)")
+                         "{quantize,dequantize}_k{3,4,5}_e4m4, or quantize_4bit_nf4_bs{64,32}, "
+                         "quantize_nested_nf4_bs{64,32} (profiling)")
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -85,6 +85,8 @@ def op_bytes(kind, n, K=None, out_size=2, bs=NESTED_BS):
         return n * 2 + nb * K * 4 + nb
     if kind == "dequantize_e4m4":
         return nb * K * 4 + nb + n * out_size
+    if kind in ("quantize_4bit", "quantize_nested"):
+        bs = K or bs                              # these ops carry their outer blocksize as K
     nbo = (n + bs - 1) // bs
     nbi = (nbo + 255) // 256
     if kind == "quantize_4bit":                   # bf16 in; nibble codes and fp32 absmax out
@@ -112,7 +114,8 @@ def nested_quant_launches(n, bs=NESTED_BS):
 # Selectable with --ops (not part of the default step): the E4M4-absmax codec.
 EXTRA_OPS = [(f"{k}_k{K}", k, K) for K in (2, 4) for k in ("quantize", "dequantize")] + \
     [(f"{k}_k{K}_e4m4", f"{k}_e4m4", K) for K in (3, 4, 5) for k in ("quantize", "dequantize")] + \
-    [("quantize_4bit_nf4_bs64", "quantize_4bit", None), ("quantize_nested_nf4_bs64", "quantize_nested", None)]
+    [(f"quantize_4bit_nf4_bs{bs}", "quantize_4bit", bs) for bs in (64, 32)] + \
+    [(f"quantize_nested_nf4_bs{bs}", "quantize_nested", bs) for bs in (64, 32)]
 
 
 def workload_ops(only=None):
@@ -318,7 +321,7 @@ def run_bbc(args):
     x = synthetic.weights(n, std=0.02, seed=7, dtype=torch.bfloat16, device=dev)
     cbs = {K: bbc.bbc_nf_codebook(K) for K in (2, 3, 4, 5)}
     cb_dev = {K: torch.from_numpy(cbs[K]).to(dev) for K in cbs}
-    ks = sorted({K for _, _, K in ops if K})
+    ks = sorted({K for _, kind, K in ops if kind in ("quantize", "dequantize", "quantize_e4m4", "dequantize_e4m4")})
     nested = synthetic.nested_state(n, NESTED_BS, seed=3, device=dev)
     codes, q, a2, off = nested
     code2 = synthetic.general8_table()
@@ -334,14 +337,15 @@ def run_bbc(args):
              "outs": {K: torch.empty(n, dtype=torch.bfloat16, device=dev) for K in ks},
              "nout": torch.empty(n, dtype=torch.bfloat16, device=dev)}
         if kinds & {"quantize_4bit", "quantize_nested"}:
-            nbo4 = (n + NESTED_BS - 1) // NESTED_BS
+            bs4 = min(K for _, kind, K in ops if kind in ("quantize_4bit", "quantize_nested"))
+            nbo4 = (n + bs4 - 1) // bs4
             o["q4_codes"] = torch.empty((n + 1) // 2, dtype=torch.uint8, device=dev)
             o["q4_absmax"] = torch.empty(nbo4, dtype=torch.float32, device=dev)
             o["nq_out"] = (torch.empty((n + 1) // 2, dtype=torch.uint8, device=dev),
                            torch.empty(nbo4, dtype=torch.uint8, device=dev),
                            torch.empty((nbo4 + 255) // 256, dtype=torch.float32, device=dev),
                            torch.empty(1, dtype=torch.float32, device=dev))
-            o["nq_ws"] = torch.empty(bbc.quantize_4bit_nested_workspace_bytes(n, NESTED_BS), dtype=torch.uint8,
+            o["nq_ws"] = torch.empty(bbc.quantize_4bit_nested_workspace_bytes(n, bs4), dtype=torch.uint8,
                                      device=dev)
         return o
 
@@ -362,10 +366,10 @@ def run_bbc(args):
             bbc.kbit_dequantize_e4m4(o["packed"][K], o["absmax8"][K], cb[K], K, n, torch.bfloat16,
                                      out=o["outs"][K], stream=st)
         elif kind == "quantize_4bit":
-            bbc.quantize_4bit(inp["x"], NESTED_BS, inp["code4"], absmax=o["q4_absmax"], codes=o["q4_codes"],
+            bbc.quantize_4bit(inp["x"], K, inp["code4"], absmax=o["q4_absmax"], codes=o["q4_codes"],
                               stream=st)
         elif kind == "quantize_nested":
-            bbc.quantize_4bit_nested(inp["x"], NESTED_BS, inp["code4"], inp["code2"], workspace=o["nq_ws"],
+            bbc.quantize_4bit_nested(inp["x"], K, inp["code4"], inp["code2"], workspace=o["nq_ws"],
                                      out=o["nq_out"], stream=st)
         else:
             bbc.dequantize_4bit_nested(inp["codes"], inp["q"], inp["code2"], inp["a2"], float(off), inp["code4"], n,
@@ -439,7 +443,7 @@ def run_bbc(args):
               "data": "synthetic", "config": {**workload_desc(n, ops),
                                               "parallelism": f"replicas{world}" if world > 1 else "single"},
               "per_kernel": per_kernel, "roofline": roofline,
-              "gpu_launches": sum(nested_quant_launches(n) if kind == "quantize_nested" else 1
+              "gpu_launches": sum(nested_quant_launches(n, K) if kind == "quantize_nested" else 1
                                   for _, kind, _ in ops) * args.steps, "clocks": clocks}
 
     # ---- end to end through the public API with host buffers
