@@ -19,7 +19,7 @@
  *  [P2] pull request "Fuse nested 4-bit scale reconstruction on SM103",
  *       sections Summary and Implementation.
  *
- * Readings taken where the pages leave a step open (each is listed in the design doc):
+ * Readings taken where the pages leave a step open:
  *  - Nearest entry: the first index i that minimises fabsf(xn - c[i]); the scan
  *    starts from +infinity (the reference's argmin), so ties go to the lowest i.
  *  - Padding of the last k-bit block: padded lanes hold 0.0f and are quantized
@@ -353,11 +353,11 @@ int orc_dequantize_4bit(const uint8_t* codes, const float* absmax, const float* 
 
 /* ------------------------------------------------------------------ */
 /* 4-bit quantize and nested absmax compression: the inverse of the     */
-/* nested dequant. [P2] describes only the decode ("does not change ... */
-/* quantization formats"); every step below is a reading, listed in     */
-/* the k-bit rule of [P1] applied per outer block, the       */
-/* offset as a mean of the outer absmax, General8 codes of the centred  */
-/* absmax per group of blocksize2 outer blocks.                         */
+/* nested dequant. [P2] gives only the decode and leaves the stored     */
+/* formats as they were, so every step below is a reading: the k-bit    */
+/* rule of [P1] applied per outer block, the offset as a mean of the    */
+/* outer absmax, General8 codes of the centred absmax per group of      */
+/* blocksize2 outer blocks.                                             */
 /* ------------------------------------------------------------------ */
 
 /*
