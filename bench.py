@@ -23,6 +23,7 @@ import argparse
 import hashlib
 import json
 import os
+import re
 import statistics
 import subprocess
 import sys
@@ -147,6 +148,14 @@ def load_peaks():
     return FALLBACK_HBM_GBS, "fallback"
 
 
+def _code_only(text):
+    """Source text without comments and with whitespace collapsed: editing a comment leaves the
+    hash of a kernel's source alone."""
+    text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+    text = re.sub(r"//[^\n]*", " ", text)
+    return " ".join(text.split())
+
+
 def kernel_source_hash(kind):
     files = {"quantize": ["kbit_quant.cu"], "dequantize": ["kbit_dequant.cu"],
              "quantize_e4m4": ["kbit_quant.cu"], "dequantize_e4m4": ["kbit_dequant.cu"],
@@ -154,7 +163,7 @@ def kernel_source_hash(kind):
              "nested": ["nested_dequant.cu"]}[kind] + ["common.cuh"]
     h = hashlib.sha256()
     for f in files:
-        h.update(open(os.path.join(ROOT, "blockwise_bit_codebook_b200", "csrc", f), "rb").read())
+        h.update(_code_only(open(os.path.join(ROOT, "blockwise_bit_codebook_b200", "csrc", f)).read()).encode())
     return h.hexdigest()[:16]
 
 

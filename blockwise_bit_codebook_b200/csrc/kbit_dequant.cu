@@ -4,15 +4,16 @@
 // kDequantizeBlockwise_kbit): out[m] = T(codebook[idx_m] * absmax[m / 32]),
 // where idx_m is gathered from the K bit-plane words of block m / 32.
 //
-// B200 layout. For 32-byte-aligned output a thread owns a whole block: it reads
-// the block's absmax and its K words once (one vector load when the packed array
-// allows), byte-transposes them with eight permutes into four plane groups (byte
-// j of group q = plane j of elements 8q..8q+7), decodes each 4-bit index with one
+// B200 layout, two forms chosen per launch on the host. Whole blocks (K = 5, the E4M4
+// K = 3 case, and 16-bit outputs below 2^26 elements; all 32-byte aligned): a thread owns a
+// block, reads its absmax and K words once (one vector load when the packed array
+// allows), byte-transposes them with eight permutes into four plane groups (byte j
+// of group q = plane j of elements 8q..8q+7), decodes each 4-bit index with one
 // multiply-high bit gather, and writes 16 outputs per 32-byte store, so every lane
-// writes whole sectors. The next block's words are loaded before the current one
-// is decoded. The ragged last block and unaligned outputs go by half blocks (16
-// elements per thread; the two lanes of a block read the same words and keep
-// bytes 2h, 2h+1). The codebook lives in shared memory: 32 consecutive floats
+// writes whole sectors; the next block's words are loaded before the current one is
+// decoded. Half blocks (otherwise: long 16-bit streams and fp32 outputs at K = 2..4;
+// always for the ragged last block and unaligned outputs): 16 elements per thread, the
+// two lanes of a block read the same words and keep bytes 2h, 2h+1. The codebook lives in shared memory: 32 consecutive floats
 // occupy the 32 banks once, so the per-element lookup never conflicts.
 // Persistent grid-stride loops.
 #include "common.cuh"
