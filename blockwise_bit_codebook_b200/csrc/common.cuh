@@ -84,16 +84,6 @@ __device__ __forceinline__ float f16_bits_to_f32(uint32_t h16) {
     return f;
 }
 
-// Load element m of a typed array as fp32 (exact widening).
-template <int DT>
-__device__ __forceinline__ float load_as_f32(const void* A, int64_t m) {
-    if constexpr (DT == F32) return reinterpret_cast<const float*>(A)[m];
-    else {
-        uint32_t h = reinterpret_cast<const uint16_t*>(A)[m];
-        return DT == BF16 ? bf16_bits_to_f32(h) : f16_bits_to_f32(h);
-    }
-}
-
 // Store an fp32 value as element m of a typed array (one rounding to the type).
 template <int DT>
 __device__ __forceinline__ void store_from_f32(void* out, int64_t m, float v) {
@@ -115,13 +105,6 @@ __device__ __forceinline__ void pack8(const float* y, uint32_t* w) {
     }
 }
 
-// Store 8 packed elements of type DT (16 B for 16-bit types, 32 B for fp32), 16-byte aligned.
-template <int DT>
-__device__ __forceinline__ void store8_vec(void* p, const uint32_t* w) {
-    if constexpr (DT == F32) stg_v8(p, w);
-    else stg_v4(p, w[0], w[1], w[2], w[3]);
-}
-
 // Three-input NaN-propagating max of absolute values (sm_100 three-input form).
 __device__ __forceinline__ float max3_abs_nan(float a, float b, float c) {
     float r;
@@ -138,13 +121,6 @@ __device__ __forceinline__ float max_nan(float a, float b) {
 __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
     uint32_t r;
     asm("prmt.b32 %0, %1, %2, %3;" : "=r"(r) : "r"(a), "r"(b), "r"(sel));
-    return r;
-}
-
-// 0xFFFFFFFF if a >= b else 0 (false for NaN).
-__device__ __forceinline__ uint32_t set_ge(float a, float b) {
-    uint32_t r;
-    asm("set.ge.u32.f32 %0, %1, %2;" : "=r"(r) : "f"(a), "f"(b));
     return r;
 }
 
