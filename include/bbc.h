@@ -30,8 +30,8 @@
  *     kept (no flush to zero) in every step.
  *   - Device pointers need only the natural alignment of their element type.
  *     Well-aligned buffers take the vectorised path (32 bytes for the input of
- *     kbit_quantize, 16 bytes for the outputs of the dequantizers, 8 bytes for
- *     the nested codes), others a scalar path with identical results.
+ *     the quantizers and for the outputs of the dequantizers, 16 bytes for the
+ *     4-bit codes), others a scalar path with identical results.
  */
 #ifndef BBC_H
 #define BBC_H
@@ -195,7 +195,7 @@ int dequantize_4bit(const uint8_t* codes, const float* absmax, const float* code
  *   code4    [16] fp32 (NF4, FP4 or any table; ascending well-spaced tables take the
  *            fast exact path, others the rule verbatim).
  *   absmax   [ceil(n/blocksize)] fp32 out.   codes [ceil(n/2)] uint8 out.
- * Fast paths need A 32-byte and codes 8-byte aligned; other alignments give the
+ * Fast paths need A 32-byte and codes 16-byte aligned; other alignments give the
  * same results more slowly.
  */
 int quantize_4bit(const void* A, int dtype, int64_t n, int blocksize, const float* code4, float* absmax,
