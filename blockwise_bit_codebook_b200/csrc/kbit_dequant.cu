@@ -116,8 +116,13 @@ __global__ void __launch_bounds__(kThreads)
 kbit_dequant_kernel(const uint32_t* __restrict__ packed, const AT* __restrict__ absmax,
                     const float* __restrict__ codebook, int64_t n, void* __restrict__ out) {
     __shared__ float cb[32];
-    if (threadIdx.x < 32) cb[threadIdx.x] = threadIdx.x < (1u << K) ? codebook[threadIdx.x] : 0.0f;
-    __syncthreads();
+    pdl_wait();               // writes of the previous kernel in the stream are visible from here
+    // the codebook is published to shared memory after the first block's loads are issued
+    const float cbv = threadIdx.x < (1u << K) ? codebook[threadIdx.x] : 0.0f;
+    auto publish_codebook = [&]() {
+        if (threadIdx.x < 32) cb[threadIdx.x] = cbv;
+        __syncthreads();
+    };
     const char* cbb = reinterpret_cast<const char*>(cb);
 
     const int64_t nh = ((n + 31) >> 5) * 2;                       // half blocks
@@ -132,8 +137,10 @@ kbit_dequant_kernel(const uint32_t* __restrict__ packed, const AT* __restrict__ 
         const int64_t nbf = n >> 5;                                 // blocks entirely inside n
         const bool vec_words = (reinterpret_cast<uintptr_t>(packed) & (K == 4 ? 15u : 7u)) == 0;
         int64_t b = (int64_t)blockIdx.x * kThreads + threadIdx.x;
+        BlockIn<K> cb0;
+        if (b < nbf) cb0 = load_whole<K, AT>(packed, absmax, b, vec_words);
+        publish_codebook();
         if (b < nbf) {
-            BlockIn<K> cb0 = load_whole<K, AT>(packed, absmax, b, vec_words);
             while (true) {
                 const int64_t bn = b + stride;
                 BlockIn<K> cb1;
@@ -148,6 +155,7 @@ kbit_dequant_kernel(const uint32_t* __restrict__ packed, const AT* __restrict__ 
     }
     int64_t H = H0 + (int64_t)blockIdx.x * kThreads + threadIdx.x;
     BlockIn<K> cur = load_block<K, AT>(packed, absmax, H >> 1, H < nh);
+    if constexpr (!(VEC && WHOLE)) publish_codebook();
     for (; H < nh; H += stride) {
         const int64_t Hn = H + stride;
         const BlockIn<K> nxt = load_block<K, AT>(packed, absmax, Hn >> 1, Hn < nh);
@@ -213,8 +221,7 @@ cudaError_t launch_t(const uint32_t* packed, const AT* absmax, const float* code
     auto k = !vec ? kbit_dequant_kernel<K, DT, false, false, AT>
                   : whole ? kbit_dequant_kernel<K, DT, true, true, AT> : kbit_dequant_kernel<K, DT, true, false, AT>;
     const int grid = persistent_grid(k, kThreads, 0, nh, kThreads);
-    k<<<grid, kThreads, 0, s>>>(packed, absmax, codebook, n, out);
-    return cudaGetLastError();
+    return launch_pdl(k, grid, kThreads, 0, s, packed, absmax, codebook, n, out);
 }
 
 template <int K, typename AT>

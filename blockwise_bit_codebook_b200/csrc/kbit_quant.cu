@@ -79,26 +79,92 @@ constexpr int kReplicas8 = 16;           // the 8-byte table: 16 lanes per share
 // the fp32 path spilled and ran 2-10 % slower); the unaligned path keeps three.
 template <int DT, bool VEC> constexpr int kMinCtas = VEC ? 2 : 3;
 
-__device__ __forceinline__ int64_t f32_key(float f) {
-    const int32_t b = __float_as_int(f);
-    return b >= 0 ? (int64_t)b : -(int64_t)(b & 0x7fffffff) - 1;
+// Ordered 32-bit key of an fp32 value: unsigned comparison of keys is the numeric order of
+// the non-NaN values (-0 just below +0), and consecutive keys are adjacent fp32 values.
+__device__ __forceinline__ uint32_t okey(float f) {
+    const uint32_t b = __float_as_uint(f);
+    return b ^ ((uint32_t)((int32_t)b >> 31) | 0x80000000u);
 }
-__device__ __forceinline__ float key_f32(int64_t k) {
-    const uint32_t b = k >= 0 ? (uint32_t)k : ((uint32_t)(-(k + 1)) | 0x80000000u);
-    return __uint_as_float(b);
+__device__ __forceinline__ float okey_f32(uint32_t k) {
+    return __uint_as_float(k ^ ((uint32_t)((int32_t)~k >> 31) | 0x80000000u));
 }
+// The largest fp32 value below v (v finite and above -FLT_MAX).
+__device__ __forceinline__ float prev_f32(float v) { return okey_f32(okey(v) - 1u); }
 
-// Smallest fp32 v in [lo, hi] where entry `hi` beats entry `lo` under the exact
-// rule; the predicate is false at lo, true at hi and monotone in between.
-__device__ float bisect_threshold(float lo_c, float hi_c) {
-    int64_t lo = f32_key(lo_c), hi = f32_key(hi_c);
-    for (int it = 0; it < 40 && hi - lo > 1; it++) {
-        const int64_t mid = lo + ((hi - lo) >> 1);
-        const float v = key_f32(mid);
-        if (__fsub_rn(hi_c, v) < __fsub_rn(v, lo_c)) hi = mid;
-        else lo = mid;
+// The exact rule at v for two entries a < b: entry b is strictly nearer than entry a.
+__device__ __forceinline__ bool beats(float a, float b, float v) { return __fsub_rn(b, v) < __fsub_rn(v, a); }
+
+// Smallest fp32 v in (a, b] where entry b beats entry a under the exact rule, found by the 8
+// lanes of a lane group (r = lane & 7; lanes 8g .. 8g+7 of the warp; every lane of the warp
+// calls this together). The rule is false at a, true at b and monotone in between (fl(b - v)
+// does not increase and fl(v - a) does not decrease with v).
+//
+// 1. Where it can be. For v below the midpoint m = (a + b) / 2, fl(b - v) >= fl(v - a); above
+//    m + ulp(b - a) / 2 the two distances differ by more than their rounding can hide. So the
+//    threshold lies in (m, m + ulp(b - a) / 2].
+// 2. Candidates. There the rule can change only where b - v or v - a crosses a rounding boundary
+//    of fp32 near (b - a) / 2 (the midpoint beta of two neighbouring fp32 values): at v = b - beta
+//    or v = a + beta. Each lane takes one boundary (8 neighbouring ones cover the interval) and
+//    tests the smallest fp32 at or above each of its two breakpoints and the next value; the
+//    group keeps the smallest candidate where the rule holds.
+// 3. Check. It is the threshold if the rule holds there and fails one fp32 value below (the rule
+//    being monotone), however the candidates were formed. Every lane checks it (no vote needed).
+// 4. Otherwise (never seen for codebooks the fast path accepts) a search over the ordered keys
+//    from the bracket of step 1 (checked at both ends first): 8 keys per step split it into 9
+//    parts (at most 11 steps for 2^32 keys).
+// `ok` is false when even the search did not converge.
+__device__ __forceinline__ float group_threshold(float a, float b, bool live, bool& ok) {
+    const int lane = threadIdx.x & 31, r = lane & 7, gs = lane & 24;
+    uint32_t lo = okey(a), hi = okey(b);
+    const float w = __fsub_ru(b, a);
+    const double uh = (double)__uint_as_float(__float_as_uint(w) & 0x7f800000u) * 0x1p-24;   // ulp(w) / 2
+    // 2. candidates from this lane's rounding boundary of the distances
+    const double h = 0.5 * ((double)b - (double)a);
+    const uint32_t k0 = okey(__double2float_rd(h - uh)) - 1u + (uint32_t)r;
+    const double beta = 0.5 * ((double)okey_f32(k0) + (double)okey_f32(k0 + 1u));
+    const uint32_t c1 = okey(__double2float_ru((double)b - beta));
+    const uint32_t c2 = okey(__double2float_ru((double)a + beta));
+    uint32_t best = hi;
+#pragma unroll
+    for (int i = 0; i < 4; i++) {
+        const uint32_t c = (i & 2 ? c2 : c1) + (uint32_t)(i & 1);
+        if (c > lo && c < best && beats(a, b, okey_f32(c))) best = c;
     }
-    return key_f32(hi);
+    best = min(best, __shfl_xor_sync(0xffffffffu, best, 1));
+    best = min(best, __shfl_xor_sync(0xffffffffu, best, 2));
+    best = min(best, __shfl_xor_sync(0xffffffffu, best, 4));
+    // 3. the check, in every lane of the group
+    const bool done = best > lo && !beats(a, b, okey_f32(best - 1u)) && beats(a, b, okey_f32(best));
+    if (done) {
+        lo = best - 1u;
+        hi = best;
+    }
+    // 4. fallback search
+    if (__any_sync(0xffffffffu, live && !done)) {
+        const double m = 0.5 * (double)a + 0.5 * (double)b;
+        uint32_t lo1 = okey(__double2float_rd(m)) - 1u, hi1 = okey(__double2float_ru(m + uh)) + 1u;
+        lo1 = max(lo1, lo);
+        hi1 = min(hi1, hi);
+        // lane 0 checks that the rule is false at lo1, lane 1 that it is true at hi1
+        const bool p = beats(a, b, okey_f32(r == 0 ? lo1 : hi1));
+        const uint32_t g = (__ballot_sync(0xffffffffu, p) >> gs) & 0xffu;
+        if (!done && (g & 3u) == 2u && lo1 < hi1) { lo = lo1; hi = hi1; }
+        constexpr uint32_t kNinth = 477218588u;                  // floor(2^32 / 9)
+        for (int it = 0; it < 12; it++) {
+            const uint32_t range = hi - lo;
+            if (!__any_sync(0xffffffffu, live && range > 1u)) break;
+            // key lo + floor(range (r + 1) / 9) (rounded down; non-decreasing in r, below hi)
+            const uint32_t pt = lo + __umulhi(range, (uint32_t)(r + 1) * kNinth);
+            const bool q = beats(a, b, okey_f32(pt));
+            const uint32_t gq = (__ballot_sync(0xffffffffu, q) >> gs) & 0xffu;
+            const uint32_t below = 8u - (uint32_t)__popc(gq);    // points where the rule is still false
+            const uint32_t nlo = lo + __umulhi(range, below * kNinth);
+            const uint32_t nhi = below == 8u ? hi : lo + __umulhi(range, (below + 1u) * kNinth);
+            if (range > 1u) { lo = nlo; hi = nhi; }
+        }
+    }
+    ok = hi - lo <= 1u;
+    return okey_f32(hi);
 }
 
 // Bits 0..3 of v at bits 0, 8, 16, 24; for K = 5 also bit 4 of v at bit 4.
@@ -122,20 +188,51 @@ __device__ __forceinline__ uint32_t nearest_entry(float xn, const float* cb) {
     return idx;
 }
 
+// Number of thresholds thr[1 .. NE-1] below x (LESS) or at most x (!LESS): a branch-free binary
+// search over the ascending thresholds (thr[NE .. 32] hold +inf).
+template <int NE, bool LESS>
+__device__ __forceinline__ int count_thresholds(const float* thr, float x) {
+    int k = 0;
+#pragma unroll
+    for (int step = NE / 2; step >= 1; step >>= 1) {
+        const float T = thr[k + step];
+        if (LESS ? (T < x) : (T <= x)) k += step;
+    }
+    return k;
+}
+
 // Per-CTA set-up of the exact threshold method for a 2^K-entry codebook (every thread of the
 // CTA calls it; the result is CTA-uniform): loads the codebook into cb[], decides whether the
 // fast path applies (finite, strictly ascending, spaced >= 2^-19 (1 + max|c|), at most one
-// threshold per table cell), finds the thresholds by bisection and fills the 256-cell table
-// (8 replicas) whose entries are {-T, h_T, pattern(L), pattern(L + 1)}: the bit-plane spread of
-// the index for the k-bit codec, the index itself for nibble codes. With `lut8` it fills the
-// 8-byte table {-A, pattern(L)} (16 replicas) instead (see step 3 of the header).
+// threshold per table cell), finds the thresholds (one 8-lane group each, all warps at once)
+// and fills the 256-cell table (8 replicas) whose entries are {-T, h_T, pattern(L),
+// pattern(L + 1)}: the bit-plane spread of the index for the k-bit codec, the index itself for
+// nibble codes. With `lut8` it fills the 8-byte table {-A, pattern(L)} (16 replicas) instead
+// (see step 3 of the header).
+// The codebook entry a thread of warp 0 loads for the set-up (lanes >= 2^K hold 0). The load
+// goes to L2 (the coherence point), never to L1: the set-up may read the codebook before
+// griddepcontrol.wait, and the check after it (codebook_changed) must not see a stale L1 copy.
+__device__ __forceinline__ float ldg_f32_l2(const float* p) {
+    float v;
+    asm volatile("ld.global.cg.f32 %0, [%1];" : "=f"(v) : "l"(p));
+    return v;
+}
+
+template <int K>
+__device__ __forceinline__ float load_codebook_entry(const float* __restrict__ codebook) {
+    return threadIdx.x < (1u << K) ? ldg_f32_l2(codebook + threadIdx.x) : 0.0f;
+}
+
 template <int K, bool NIBBLE>
-__device__ __forceinline__ bool setup_exact_table(const float* __restrict__ codebook, float* cb, float* thr,
+__device__ __forceinline__ bool setup_exact_table(float c, float* cb, float* thr,
                                                   int* fast_ok, uint4* lut, uint2* lut8 = nullptr) {
     constexpr int NE = 1 << K;
+    static_assert((NE - 1) * 8 <= kThreads, "one 8-lane group per threshold");
     const int tid = threadIdx.x;
+    // thresholds: group j - 1 (threads 8(j-1) .. 8j-1) finds the one between entries j-1 and j
+    const int j = (tid >> 3) + 1;
+    const bool live = j < NE;
     if (tid < 32) {
-        const float c = tid < NE ? codebook[tid] : 0.0f;
         cb[tid] = c;
         float mag = tid < NE ? fabsf(c) : 0.0f;
 #pragma unroll
@@ -150,11 +247,17 @@ __device__ __forceinline__ bool setup_exact_table(const float* __restrict__ code
         ok = ok && (D <= FLT_MAX);
         const bool fast = __all_sync(0xffffffffu, ok);
         if (tid == 0) *fast_ok = fast ? 1 : 0;
-        if (fast && tid >= 1 && tid < NE) thr[tid] = bisect_threshold(prev, c);
+        if (tid >= NE) thr[tid] = __int_as_float(0x7f800000);        // +inf past the last threshold
+        if (tid == 0) thr[32] = __int_as_float(0x7f800000);
     }
     __syncthreads();
+    const float ca = live ? cb[j - 1] : 0.0f, cbv = live ? cb[j] : 1.0f;
+    bool conv = true;
+    const float T = group_threshold(ca, cbv, live, conv);
+    if (live && (tid & 7) == 0) thr[j] = T;
+    const int unconverged = __syncthreads_or(live && !conv);
     int multi = 0;
-    if (*fast_ok) {
+    if (*fast_ok && !unconverged) {
         for (int cell = tid; cell < kCells; cell += kThreads) {
             // cell cs = round(64 xn) at slot cs + 128: it holds every xn within half a cell
             const int cs = cell - 128;
@@ -162,41 +265,65 @@ __device__ __forceinline__ bool setup_exact_table(const float* __restrict__ code
             const float hi_edge = ((float)cs + 0.5f) * 0.015625f;
             const float wlo = __fsub_rn(lo_edge, 0x1p-13f + 0x1p-12f);
             const float whi = __fadd_rn(hi_edge, 0x1p-13f + 0x1p-12f);
-            int below = 0, rel = 0, relj = 0;
-            for (int j = 1; j < NE; j++) {
-                const float T = thr[j];
-                if (T < wlo) below++;
-                else if (T <= whi) { rel++; relj = j; }
-            }
+            const int below = count_thresholds<NE, true>(thr, wlo);
+            const int rel = count_thresholds<NE, false>(thr, whi) - below;
             float negT = __int_as_float(0xff800000), half = 0.0f;     // -inf, 0: never crossed
+            const float Tr = thr[below + 1];                          // the one relevant threshold
             if (rel == 1) {
-                const float T = thr[relj];
-                negT = -T;
-                half = __fmul_rn(__fsub_rn(T, key_f32(f32_key(T) - 1)), 0.5f);
+                negT = -Tr;
+                half = __fmul_rn(__fsub_rn(Tr, prev_f32(Tr)), 0.5f);
             }
             multi |= rel > 1;
             const uint32_t p0 = NIBBLE ? (uint32_t)below : spread<K>((uint32_t)below);
             const uint32_t p1 = NIBBLE ? (uint32_t)below + 1 : spread<K>((uint32_t)below + 1);
-            const uint4 ent = make_uint4(__float_as_uint(negT), __float_as_uint(half), p0, p1);
             if (!lut8) {
+                const uint4 ent = make_uint4(__float_as_uint(negT), __float_as_uint(half), p0, p1);
                 // the 8 lanes of a store phase write 8 different replicas: distinct banks
 #pragma unroll
                 for (int r = 0; r < kReplicas; r++) lut[cell * kReplicas + ((r + tid) & (kReplicas - 1))] = ent;
             } else {
                 float nA = __int_as_float(0xff800000);               // -inf: never crossed
                 if (rel == 1) {
-                    const float T = thr[relj];
-                    const float Av = T > 0.0f ? key_f32(f32_key(T) - 1) : T;
+                    const float Av = Tr > 0.0f ? prev_f32(Tr) : Tr;
                     nA = -Av;
                     multi |= !(fabsf(Av) >= 0x1p-100f);              // keep the rebuilt half-ulp normal
                 }
-                const uint2 e8 = make_uint2(__float_as_uint(nA), p0);
+                const uint32_t e = __float_as_uint(nA);
+                // replicas 2q, 2q + 1 in one 16-byte store; the 8 lanes of a store phase write 8
+                // different replica pairs: distinct banks
+                uint4* row = reinterpret_cast<uint4*>(lut8 + cell * kReplicas8);
 #pragma unroll
-                for (int r = 0; r < kReplicas8; r++) lut8[cell * kReplicas8 + ((r + tid) & (kReplicas8 - 1))] = e8;
+                for (int q = 0; q < kReplicas8 / 2; q++) row[(q + tid) & (kReplicas8 / 2 - 1)] = make_uint4(e, p0, e, p0);
             }
         }
     }
-    return (*fast_ok != 0) && !__syncthreads_or(multi);
+    return (*fast_ok != 0) && !unconverged && !__syncthreads_or(multi);
+}
+
+// After griddepcontrol.wait: true (CTA-uniform) if the codebook differs, bit for bit, from the
+// values the set-up used (read before the wait, while the previous kernel of the stream may still
+// have been writing them). The table is a function of those values alone, so when they are equal
+// it is the table that stream order defines; otherwise the caller runs the set-up again.
+template <int K>
+__device__ __forceinline__ bool codebook_changed(const float* __restrict__ codebook, const float* cb) {
+    bool diff = false;
+    if (threadIdx.x < (1u << K))
+        diff = __float_as_uint(ldg_f32_l2(codebook + threadIdx.x)) != __float_as_uint(cb[threadIdx.x]);
+    return __syncthreads_or(diff) != 0;
+}
+
+// Programmatic dependent launch, early form: lets the next kernel of the stream be scheduled once
+// every CTA of this grid has executed it. Used only by a grid that fills the GPU (every SM at this
+// kernel's occupancy), so that the next launch's CTAs take SMs only as this grid's CTAs retire
+// and run their set-up during this grid's tail.
+__device__ __forceinline__ void pdl_launch_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+// Prefetch of `bytes` (a multiple of 16, 16-byte aligned) into L2. Safe before griddepcontrol.wait:
+// nothing reaches the SM, and L2 is coherent, so the loads after the wait see current data.
+__device__ __forceinline__ void prefetch_l2(const void* p, uint32_t bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" :: "l"(p), "r"(bytes) : "memory");
 }
 
 // Raw input words of one half block (16 elements): 8 words for 16-bit types, 16 for fp32.
@@ -522,6 +649,7 @@ __device__ __forceinline__ void quantize_block(const Raw32<DT>& raw, int64_t b, 
                 // -H * d = (sign and exponent bits of -A) * (d * 2^-24), both factors exact
                 const float h0 = __uint_as_float(t0.x & 0xff800000u);
                 const float h1 = __uint_as_float(t1.x & 0xff800000u);
+                // (scalar FMAs: pairing them as f32x2 operations measured 2-7 points slower)
                 const float v0 = __fmaf_rn(h0, d24, __fmaf_rn(__uint_as_float(t0.x), d, x0));
                 const float v1 = __fmaf_rn(h1, d24, __fmaf_rn(__uint_as_float(t1.x), d, x1));
                 sv = __funnelshift_l(__float_as_uint(v0), sv, 1);                         // sign bits
@@ -593,7 +721,7 @@ __device__ __forceinline__ void quantize_block(const Raw32<DT>& raw, int64_t b, 
 template <int K, int DT, bool VEC, typename AT>
 __global__ void __launch_bounds__(kThreads, (kMinCtas<DT, VEC>))
 kbit_quant_kernel(const void* __restrict__ A, int64_t n, const float* __restrict__ codebook,
-                  AT* __restrict__ absmax, uint32_t* __restrict__ packed) {
+                  AT* __restrict__ absmax, uint32_t* __restrict__ packed, int early_trigger) {
     constexpr bool WHOLE = VEC && DT != F32;                   // whole blocks per thread: 8-byte table
     __shared__ __align__(16) uint4 lut[WHOLE ? 1 : kCells * kReplicas];     // 32 KB
     __shared__ __align__(16) uint2 lut8[WHOLE ? kCells * kReplicas8 : 1];   // 32 KB
@@ -604,9 +732,41 @@ kbit_quant_kernel(const void* __restrict__ A, int64_t n, const float* __restrict
 
     const int tid = threadIdx.x;
     const int lane = tid & 31;
+    if (early_trigger) pdl_launch_dependents();
 
-    // ---- per-CTA set-up: codebook check, thresholds, lookup table ----
-    const bool fast_cb = setup_exact_table<K, false>(codebook, cb, thr, &fast_ok, lut, WHOLE ? lut8 : nullptr);
+    // Persistent grid-stride loop over whole blocks (16-bit input, 32-byte aligned) or half blocks
+    // of whole blocks (no bounds checks), unrolled by two with ping-pong prefetch; then the
+    // ragged last block, if any.
+    const int64_t nh_full = VEC ? (n >> 5) * 2 : 0;
+    const int64_t nh = ((n + 31) >> 5) * 2;
+    const int64_t stride = (int64_t)gridDim.x * kThreads;
+    int64_t wbase = (int64_t)blockIdx.x * kThreads + (tid & ~31);
+    const int64_t bend = (n >> 5) & ~(int64_t)31;     // whole-block path: blocks of whole warp iterations
+
+    // ---- per-CTA set-up, before griddepcontrol.wait so that it overlaps the previous kernel of
+    // the stream: codebook check, thresholds, lookup table; meanwhile this warp's first two
+    // iterations of input stream into L2 ----
+    const float cbe = load_codebook_entry<K>(codebook);
+    if (VEC && lane == 0) {
+        constexpr int64_t unit = 64;                    // bytes of a block (16-bit) or half block (fp32)
+        const int64_t end = WHOLE ? bend : nh_full;
+        for (int i = 0; i < 2; i++) {
+            const int64_t u0 = wbase + i * stride;
+            if (u0 < end) prefetch_l2(static_cast<const char*>(A) + u0 * unit, (uint32_t)(min(end - u0, (int64_t)32) * unit));
+        }
+    }
+    bool fast_cb = setup_exact_table<K, false>(cbe, cb, thr, &fast_ok, lut, WHOLE ? lut8 : nullptr);
+    pdl_wait();               // writes of the previous kernel in the stream are visible from here
+    Raw32<DT> first_b;
+    Raw<DT> first_h;
+    if constexpr (WHOLE) {
+        if (wbase < bend) first_b = load_block<DT>(A, wbase + lane);
+    } else {
+        if (wbase < nh_full) first_h = load_full<DT>(A, wbase + lane, wbase + lane < nh_full);
+    }
+    if (codebook_changed<K>(codebook, cb))                  // rare: the codebook was being written
+        fast_cb = setup_exact_table<K, false>(load_codebook_entry<K>(codebook), cb, thr, &fast_ok, lut,
+                                              WHOLE ? lut8 : nullptr);
     LoopCtx c;
     c.stage = stage + (WHOLE && K == 5 ? (tid & ~31) * K : 0);
     c.lane = lane;
@@ -625,21 +785,14 @@ kbit_quant_kernel(const void* __restrict__ A, int64_t n, const float* __restrict
     c.sel_wb = c.h ? 0x3276u : 0x7632u;
     c.pair_mask = 3u << (lane & ~1);
 
-    // Persistent grid-stride loop over the half blocks of whole blocks (no bounds checks),
-    // unrolled by two with ping-pong prefetch; then the ragged last block, if any.
-    const int64_t nh_full = VEC ? (n >> 5) * 2 : 0;
-    const int64_t nh = ((n + 31) >> 5) * 2;
-    const int64_t stride = (int64_t)gridDim.x * kThreads;
-    int64_t wbase = (int64_t)blockIdx.x * kThreads + (tid & ~31);
-    if constexpr (VEC && DT != F32) {
+    if constexpr (WHOLE) {
         // whole warp iterations of 32 blocks, one block per thread, the next one prefetched;
         // what is left (at most the last partial iteration and a ragged block) goes by halves
-        const int64_t bend = (n >> 5) & ~(int64_t)31;
         int64_t wb = wbase;                                 // in blocks
         if (K == 5 && wb < bend) {
             // K = 5: one copy of the block code in the loop and a register copy of the prefetched
             // block (two unrolled copies of its larger body stalled on instruction fetch)
-            Raw32<DT> ra = load_block<DT>(A, wb + lane);
+            Raw32<DT> ra = first_b;
             while (true) {
                 const int64_t wn = wb + stride;
                 const bool more = wn < bend;
@@ -651,7 +804,7 @@ kbit_quant_kernel(const void* __restrict__ A, int64_t n, const float* __restrict
                 ra = rb;
             }
         } else if (wb < bend) {
-            Raw32<DT> ra = load_block<DT>(A, wb + lane);
+            Raw32<DT> ra = first_b;
             Raw32<DT> rb;
             while (true) {
                 int64_t wn = wb + stride;
@@ -676,7 +829,7 @@ kbit_quant_kernel(const void* __restrict__ A, int64_t n, const float* __restrict
         return;
     }
     if (wbase < nh_full) {
-        Raw<DT> ra = load_full<DT>(A, wbase + lane, wbase + lane < nh_full);
+        Raw<DT> ra = first_h;
         Raw<DT> rb;
         while (true) {
             rb = load_full<DT>(A, wbase + stride + lane, wbase + stride + lane < nh_full);
@@ -783,7 +936,7 @@ __host__ __device__ constexpr int nib_shift(int e) { return 8 * ((e & 7) >> 1) +
 template <int DT, bool VEC>
 __global__ void __launch_bounds__(kThreads, 2)
 quant4_kernel(const void* __restrict__ A, int64_t n, int log2_bs, const float* __restrict__ code4,
-              float* __restrict__ absmax, uint8_t* __restrict__ codes) {
+              float* __restrict__ absmax, uint8_t* __restrict__ codes, int early_trigger) {
     constexpr int E = kEpt<DT>;
     constexpr int NW = E / 8;                                   // code words per thread
     __shared__ __align__(16) uint2 lut8[kCells * kReplicas8];  // 32 KB: {-A, L}
@@ -801,12 +954,7 @@ quant4_kernel(const void* __restrict__ A, int64_t n, int log2_bs, const float* _
         for (int i = 0; i < 8; i++) v |= ((uint32_t)(tid >> i) & 1u) << nib_shift(i);
         nib_spread[tid] = v;                                     // kThreads == 256
     }
-    LoopCtx c;
-    c.fast_cb = setup_exact_table<4, true>(code4, cb, thr, &fast_ok, nullptr, lut8);
-    c.lut8_s = (uint32_t)__cvta_generic_to_shared(lut8);
-    c.lane8 = (uint32_t)(lane & (kReplicas8 - 1)) << 3;
-    c.lut8_c = c.lut8_s + c.lane8 + 128u * 128u - 0x4B400000u * 128u;     // mod 2^32
-
+    if (early_trigger) pdl_launch_dependents();
     const int tpb_log2 = log2_bs - (DT == F32 ? 4 : 5);        // threads per outer block
     const int tpb = 1 << tpb_log2;
     const int64_t nu = (n + E - 1) / E;                         // 64-byte slices
@@ -814,7 +962,26 @@ quant4_kernel(const void* __restrict__ A, int64_t n, int log2_bs, const float* _
     const int64_t stride = (int64_t)gridDim.x * kThreads;
     int buf = 0;
     int64_t base = (int64_t)blockIdx.x * kThreads;
+    // set-up before griddepcontrol.wait (checked after it), as in the k-bit kernel; this warp's
+    // first two slices of input stream into L2 meanwhile
+    const float cbe = load_codebook_entry<4>(code4);
+    if (VEC && lane == 0) {
+        const int64_t nfull = n / E;                            // slices entirely inside the input
+        for (int i = 0; i < 2; i++) {
+            const int64_t u0 = base + (tid & ~31) + i * stride;
+            if (u0 < nfull) prefetch_l2(static_cast<const char*>(A) + u0 * 64, (uint32_t)(min(nfull - u0, (int64_t)32) * 64));
+        }
+    }
+    LoopCtx c;
+    c.fast_cb = setup_exact_table<4, true>(cbe, cb, thr, &fast_ok, nullptr, lut8);
+    pdl_wait();               // writes of the previous kernel in the stream are visible from here
     Raw16w cur = load_slice<DT, VEC>(A, n, base + tid, base + tid < nu);
+    if (codebook_changed<4>(code4, cb))                     // rare: the table was being written
+        c.fast_cb = setup_exact_table<4, true>(load_codebook_entry<4>(code4), cb, thr, &fast_ok, nullptr, lut8);
+    c.lut8_s = (uint32_t)__cvta_generic_to_shared(lut8);
+    c.lane8 = (uint32_t)(lane & (kReplicas8 - 1)) << 3;
+    c.lut8_c = c.lut8_s + c.lane8 + 128u * 128u - 0x4B400000u * 128u;     // mod 2^32
+
     for (; base < nu; base += stride) {                         // CTA-uniform
         const int64_t U = base + tid;
         const bool active = U < nu;
@@ -859,6 +1026,7 @@ quant4_kernel(const void* __restrict__ A, int64_t n, int log2_bs, const float* _
                 // -H * d = (sign and exponent bits of -A) * (d * 2^-24), both factors exact
                 const float h0 = __uint_as_float(t0.x & 0xff800000u);
                 const float h1 = __uint_as_float(t1.x & 0xff800000u);
+                // (scalar FMAs: the paired f32x2 form spills here and was slower in the k-bit kernel)
                 const float v0 = __fmaf_rn(h0, d24, __fmaf_rn(__uint_as_float(t0.x), d, x0));
                 const float v1 = __fmaf_rn(h1, d24, __fmaf_rn(__uint_as_float(t1.x), d, x1));
                 sv = __funnelshift_l(__float_as_uint(v0), sv, 1);
@@ -900,15 +1068,13 @@ cudaError_t launch_t(const void* A, int64_t n, const float* codebook, AT* absmax
                      uint32_t* packed, bool vec, cudaStream_t s) {
     const int64_t nh = ((n + 31) >> 5) * 2;
     auto k = vec ? kbit_quant_kernel<K, DT, true, AT> : kbit_quant_kernel<K, DT, false, AT>;
-    static bool attr_set[2] = {false, false};
-    if (!attr_set[vec]) {
-        cudaFuncSetAttribute(k, cudaFuncAttributePreferredSharedMemoryCarveout,
-                             cudaSharedmemCarveoutMaxShared);
-        attr_set[vec] = true;
-    }
+    static std::atomic<uint64_t> carveout_set[2];
+    const cudaError_t e = set_attr_once(k, carveout_set[vec], cudaFuncAttributePreferredSharedMemoryCarveout,
+                                        cudaSharedmemCarveoutMaxShared);
+    if (e != cudaSuccess) return e;
+    const int cap = resident_ctas(reinterpret_cast<const void*>(k), kThreads, 0);
     const int grid = persistent_grid(k, kThreads, 0, nh, kThreads);
-    k<<<grid, kThreads, 0, s>>>(A, n, codebook, absmax, packed);
-    return cudaGetLastError();
+    return launch_pdl(k, grid, kThreads, 0, s, A, n, codebook, absmax, packed, grid >= cap ? 1 : 0);
 }
 
 template <int K, typename AT>
@@ -942,16 +1108,16 @@ cudaError_t launch_kbit_quantize(const void* A, int dtype, int64_t n, int K, con
 cudaError_t launch_quantize_4bit(const void* A, int dtype, int64_t n, int log2_bs, const float* code4,
                                  float* absmax, uint8_t* codes, bool vec, cudaStream_t s) {
     auto pick = [&](auto kv, auto kn) { return vec ? kv : kn; };
-    void (*k)(const void*, int64_t, int, const float*, float*, uint8_t*);
+    void (*k)(const void*, int64_t, int, const float*, float*, uint8_t*, int);
     switch (dtype) {
         case F16: k = pick(quant4_kernel<F16, true>, quant4_kernel<F16, false>); break;
         case BF16: k = pick(quant4_kernel<BF16, true>, quant4_kernel<BF16, false>); break;
         default: k = pick(quant4_kernel<F32, true>, quant4_kernel<F32, false>); break;
     }
     const int64_t nu = (n + 15) >> 4;                           // upper bound on 64-byte slices
+    const int cap = resident_ctas(reinterpret_cast<const void*>(k), kThreads, 0);
     const int grid = persistent_grid(k, kThreads, 0, nu, kThreads);
-    k<<<grid, kThreads, 0, s>>>(A, n, log2_bs, code4, absmax, codes);
-    return cudaGetLastError();
+    return launch_pdl(k, grid, kThreads, 0, s, A, n, log2_bs, code4, absmax, codes, grid >= cap ? 1 : 0);
 }
 
 cudaError_t launch_kbit_quantize_e4m4(const void* A, int dtype, int64_t n, int K, const float* codebook,

@@ -1,9 +1,46 @@
 // Host-side launchers of the library's kernels (called by abi.cpp after validation).
 #pragma once
+#include <atomic>
 #include <cstdint>
 #include <cuda_runtime.h>
 
 namespace bbc {
+
+// Launch with programmatic stream serialisation allowed: the kernel's CTAs may be scheduled as the
+// previous kernel of the stream finishes (once all of that kernel's CTAs have exited, before its
+// completion is signalled), so the launch latency overlaps its tail; the kernel's
+// griddepcontrol.wait (pdl_wait in common.cuh), executed before any global access, holds it until
+// that kernel has completed and its writes are visible, so stream order is kept.
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kernel)(KArgs...), unsigned grid, unsigned block, size_t dyn_smem,
+                              cudaStream_t s, Args... args) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(grid);
+    cfg.blockDim = dim3(block);
+    cfg.dynamicSmemBytes = dyn_smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
+}
+
+// Sets a function attribute of `kernel` on the current device once per device (function
+// attributes are per device): `done` holds one bit per device index below 64 (others set it on
+// every call). Concurrent first calls may both set it; the value is the same.
+template <typename Kernel>
+inline cudaError_t set_attr_once(Kernel kernel, std::atomic<uint64_t>& done, cudaFuncAttribute attr, int value) {
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    const uint64_t bit = dev < 64 ? 1ull << dev : 0ull;
+    if (bit && (done.load() & bit)) return cudaSuccess;
+    e = cudaFuncSetAttribute(kernel, attr, value);
+    if (e == cudaSuccess && bit) done.fetch_or(bit);
+    return e;
+}
 
 // Persistent grid: enough CTAs to fill every SM at the kernel's occupancy, never more than
 // the work needs. The occupancy query runs once per (kernel, device, block, smem) and is

@@ -96,15 +96,19 @@ nested_dequant_kernel(const uint8_t* __restrict__ codes, const uint8_t* __restri
                       void* __restrict__ out) {
     __shared__ float c2[256];
     __shared__ float c4[16];
-    if (NESTED) c2[threadIdx.x] = code2[threadIdx.x];
-    if (threadIdx.x < 16) c4[threadIdx.x] = code4[threadIdx.x];
-    __syncthreads();
+    pdl_wait();               // writes of the previous kernel in the stream are visible from here
+    const float c2v = NESTED ? code2[threadIdx.x] : 0.0f;
+    const float c4v = threadIdx.x < 16 ? code4[threadIdx.x] : 0.0f;
     const char* c4b = reinterpret_cast<const char*>(c4);
 
     const int64_t nu = (n + kPerThread - 1) / kPerThread;
     const int64_t stride = (int64_t)gridDim.x * kThreads;
     int64_t u = (int64_t)blockIdx.x * kThreads + threadIdx.x;
     GroupIn cur = load_group<VEC, NESTED>(codes, absmax_q, absmax2, n, u, log2_bs, u < nu);
+    // the tables are published after the first group's loads are issued
+    if (NESTED) c2[threadIdx.x] = c2v;
+    if (threadIdx.x < 16) c4[threadIdx.x] = c4v;
+    __syncthreads();
     for (; u < nu; u += stride) {
         const int64_t un = u + stride;
         const GroupIn nxt = load_group<VEC, NESTED>(codes, absmax_q, absmax2, n, un, log2_bs, un < nu);
@@ -150,8 +154,7 @@ cudaError_t launch_t(const uint8_t* codes, const uint8_t* absmax_q, const float*
     const int64_t nu = (n + kPerThread - 1) / kPerThread;
     auto k = vec ? nested_dequant_kernel<DT, true, NESTED> : nested_dequant_kernel<DT, false, NESTED>;
     const int grid = persistent_grid(k, kThreads, 0, nu, kThreads);
-    k<<<grid, kThreads, 0, s>>>(codes, absmax_q, code2, absmax2, offset, code4, n, log2_bs, out);
-    return cudaGetLastError();
+    return launch_pdl(k, grid, kThreads, 0, s, codes, absmax_q, code2, absmax2, offset, code4, n, log2_bs, out);
 }
 
 template <bool NESTED>
