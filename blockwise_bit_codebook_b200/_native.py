@@ -90,8 +90,20 @@ def _torch_dtype(dt: int):
     return {BBC_F16: torch.float16, BBC_BF16: torch.bfloat16, BBC_F32: torch.float32}[dt]
 
 
-def _ptr(t):
-    return ct.c_void_p(t.data_ptr()) if t is not None else None
+def _ptr(t, device=None, name="tensor"):
+    """Address of a tensor argument. Every tensor a call passes must be a contiguous CUDA tensor
+    on the call's device (the device of its first tensor): anything else raises ValueError here,
+    before the library is called, so that no kernel is given a host address or reads a strided
+    view as if it were contiguous."""
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor (it is on {t.device})")
+    if device is not None and t.device != device:
+        raise ValueError(f"{name} is on {t.device}, the call's other tensors on {device}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return ct.c_void_p(t.data_ptr())
 
 
 def _stream(stream, device):
@@ -105,14 +117,16 @@ def kbit_quantize(A, K: int, codebook, absmax=None, packed=None, blocksize: int 
     """k-bit quantize a CUDA tensor (any shape, contiguous). Returns (packed, absmax)."""
     import torch
     L = load_library()
+    d = A.device
     n = A.numel()
     nb = (n + blocksize - 1) // blocksize if blocksize > 0 else 0
     if absmax is None:
         absmax = torch.empty(max(nb, 1), dtype=torch.float32, device=A.device)
     if packed is None:
         packed = torch.empty(max(nb * K, 1), dtype=torch.int32, device=A.device)
-    st = L.kbit_quantize(_ptr(A), _dt(A.dtype), n, K, blocksize, _ptr(codebook), _ptr(absmax),
-                         _ptr(packed), _stream(stream, A.device))
+    st = L.kbit_quantize(_ptr(A, d, "A"), _dt(A.dtype), n, K, blocksize, _ptr(codebook, d, "codebook"),
+                         _ptr(absmax, d, "absmax"),
+                         _ptr(packed, d, "packed"), _stream(stream, A.device))
     _check("kbit_quantize", st)
     return packed, absmax
 
@@ -122,10 +136,12 @@ def kbit_dequantize(packed, absmax, codebook, K: int, n: int, dtype, out=None, b
     """Inverse of kbit_quantize; returns a 1-D CUDA tensor of n elements of `dtype`."""
     import torch
     L = load_library()
+    d = packed.device
     dt = _dt(dtype)
     if out is None:
         out = torch.empty(max(n, 1), dtype=_torch_dtype(dt), device=packed.device)
-    st = L.kbit_dequantize(_ptr(packed), _ptr(absmax), _ptr(codebook), K, blocksize, n, dt, _ptr(out),
+    st = L.kbit_dequantize(_ptr(packed, d, "packed"), _ptr(absmax, d, "absmax"), _ptr(codebook, d, "codebook"),
+                           K, blocksize, n, dt, _ptr(out, d, "out"),
                            _stream(stream, packed.device))
     _check("kbit_dequantize", st)
     return out
@@ -135,14 +151,16 @@ def kbit_quantize_e4m4(A, K: int, codebook, absmax=None, packed=None, blocksize:
     """kbit_quantize with the per-block absmax stored as one E4M4 byte. Returns (packed, absmax_u8)."""
     import torch
     L = load_library()
+    d = A.device
     n = A.numel()
     nb = (n + blocksize - 1) // blocksize if blocksize > 0 else 0
     if absmax is None:
         absmax = torch.empty(max(nb, 1), dtype=torch.uint8, device=A.device)
     if packed is None:
         packed = torch.empty(max(nb * K, 1), dtype=torch.int32, device=A.device)
-    st = L.kbit_quantize_e4m4(_ptr(A), _dt(A.dtype), n, K, blocksize, _ptr(codebook), _ptr(absmax),
-                              _ptr(packed), _stream(stream, A.device))
+    st = L.kbit_quantize_e4m4(_ptr(A, d, "A"), _dt(A.dtype), n, K, blocksize, _ptr(codebook, d, "codebook"),
+                              _ptr(absmax, d, "absmax"),
+                              _ptr(packed, d, "packed"), _stream(stream, A.device))
     _check("kbit_quantize_e4m4", st)
     return packed, absmax
 
@@ -152,10 +170,12 @@ def kbit_dequantize_e4m4(packed, absmax, codebook, K: int, n: int, dtype, out=No
     """kbit_dequantize with a uint8 E4M4 absmax; returns a 1-D CUDA tensor of n elements of `dtype`."""
     import torch
     L = load_library()
+    d = packed.device
     dt = _dt(dtype)
     if out is None:
         out = torch.empty(max(n, 1), dtype=_torch_dtype(dt), device=packed.device)
-    st = L.kbit_dequantize_e4m4(_ptr(packed), _ptr(absmax), _ptr(codebook), K, blocksize, n, dt, _ptr(out),
+    st = L.kbit_dequantize_e4m4(_ptr(packed, d, "packed"), _ptr(absmax, d, "absmax"),
+                                _ptr(codebook, d, "codebook"), K, blocksize, n, dt, _ptr(out, d, "out"),
                                 _stream(stream, packed.device))
     _check("kbit_dequantize_e4m4", st)
     return out
@@ -165,13 +185,15 @@ def quantize_4bit(A, blocksize: int, code4, absmax=None, codes=None, stream=None
     """4-bit codes (uint8[ceil(n/2)], element 2j high nibble) and fp32 absmax per outer block."""
     import torch
     L = load_library()
+    d = A.device
     n = A.numel()
     nbo = (n + blocksize - 1) // blocksize if blocksize > 0 else 1
     if absmax is None:
         absmax = torch.empty(max(nbo, 1), dtype=torch.float32, device=A.device)
     if codes is None:
         codes = torch.empty(max((n + 1) // 2, 1), dtype=torch.uint8, device=A.device)
-    st = L.quantize_4bit(_ptr(A), _dt(A.dtype), n, blocksize, _ptr(code4), _ptr(absmax), _ptr(codes),
+    st = L.quantize_4bit(_ptr(A, d, "A"), _dt(A.dtype), n, blocksize, _ptr(code4, d, "code4"),
+                         _ptr(absmax, d, "absmax"), _ptr(codes, d, "codes"),
                          _stream(stream, A.device))
     _check("quantize_4bit", st)
     return codes, absmax
@@ -187,6 +209,7 @@ def quantize_4bit_nested(A, blocksize: int, code4, code2, blocksize2: int = 256,
     CUDA tensor. `out` may hold preallocated (codes, absmax_q, absmax2, offset)."""
     import torch
     L = load_library()
+    d = A.device
     n = A.numel()
     nbo = (n + blocksize - 1) // blocksize if blocksize > 0 else 1
     nbi = (nbo + blocksize2 - 1) // blocksize2 if blocksize2 > 0 else 1
@@ -199,8 +222,10 @@ def quantize_4bit_nested(A, blocksize: int, code4, code2, blocksize2: int = 256,
     wsb = quantize_4bit_nested_workspace_bytes(n, blocksize) if n > 0 else 0
     if workspace is None:
         workspace = torch.empty(max(wsb, 1), dtype=torch.uint8, device=A.device)
-    st = L.quantize_4bit_nested(_ptr(A), _dt(A.dtype), n, blocksize, _ptr(code4), _ptr(code2), blocksize2,
-                                _ptr(codes), _ptr(absmax_q), _ptr(absmax2), _ptr(offset), _ptr(workspace),
+    st = L.quantize_4bit_nested(_ptr(A, d, "A"), _dt(A.dtype), n, blocksize, _ptr(code4, d, "code4"),
+                                _ptr(code2, d, "code2"), blocksize2, _ptr(codes, d, "codes"),
+                                _ptr(absmax_q, d, "absmax_q"), _ptr(absmax2, d, "absmax2"),
+                                _ptr(offset, d, "offset"), _ptr(workspace, d, "workspace"),
                                 workspace.numel() * workspace.element_size(), _stream(stream, A.device))
     _check("quantize_4bit_nested", st)
     return codes, absmax_q, absmax2, offset
@@ -212,12 +237,14 @@ def linear_4bit_nested(X, codes, absmax_q, code2, absmax2, offset: float, code4,
     in registers (never materialised). Returns Y [M, N] in X's dtype."""
     import torch
     L = load_library()
+    d = X.device
     M, K = X.shape
     if out is None:
         out = torch.empty((M, N), dtype=X.dtype, device=X.device)
-    st = L.linear_4bit_nested(_ptr(X), _dt(X.dtype), M, N, K, _ptr(codes), _ptr(absmax_q), _ptr(code2),
-                              _ptr(absmax2), ct.c_float(offset), _ptr(code4), blocksize, blocksize2, _ptr(out),
-                              _stream(stream, X.device))
+    st = L.linear_4bit_nested(_ptr(X, d, "X"), _dt(X.dtype), M, N, K, _ptr(codes, d, "codes"),
+                              _ptr(absmax_q, d, "absmax_q"), _ptr(code2, d, "code2"), _ptr(absmax2, d, "absmax2"),
+                              ct.c_float(offset), _ptr(code4, d, "code4"), blocksize, blocksize2,
+                              _ptr(out, d, "out"), _stream(stream, X.device))
     _check("linear_4bit_nested", st)
     return out
 
@@ -227,11 +254,13 @@ def linear_kbit(X, packed, absmax, codebook, K: int, N: int, blocksize: int = 32
     kbit_quantize (K bits, blocksize 32), decoded in registers. Returns Y [M, N] in X's dtype."""
     import torch
     L = load_library()
+    d = X.device
     M, Kin = X.shape
     if out is None:
         out = torch.empty((M, N), dtype=X.dtype, device=X.device)
-    st = L.linear_kbit(_ptr(X), _dt(X.dtype), M, N, Kin, _ptr(packed), _ptr(absmax), _ptr(codebook), K, blocksize,
-                       _ptr(out), _stream(stream, X.device))
+    st = L.linear_kbit(_ptr(X, d, "X"), _dt(X.dtype), M, N, Kin, _ptr(packed, d, "packed"),
+                       _ptr(absmax, d, "absmax"), _ptr(codebook, d, "codebook"), K, blocksize,
+                       _ptr(out, d, "out"), _stream(stream, X.device))
     _check("linear_kbit", st)
     return out
 
@@ -241,12 +270,14 @@ def dequantize_4bit_nested(codes, absmax_q, code2, absmax2, offset: float, code4
     """Nested NF4/FP4 dequant; returns a 1-D CUDA tensor of n elements of `dtype`."""
     import torch
     L = load_library()
+    d = codes.device
     dt = _dt(dtype)
     if out is None:
         out = torch.empty(max(n, 1), dtype=_torch_dtype(dt), device=codes.device)
-    st = L.dequantize_4bit_nested(_ptr(codes), _ptr(absmax_q), _ptr(code2), _ptr(absmax2),
-                                  ct.c_float(offset), _ptr(code4), n, blocksize, blocksize2, dt,
-                                  _ptr(out), _stream(stream, codes.device))
+    st = L.dequantize_4bit_nested(_ptr(codes, d, "codes"), _ptr(absmax_q, d, "absmax_q"),
+                                  _ptr(code2, d, "code2"), _ptr(absmax2, d, "absmax2"),
+                                  ct.c_float(offset), _ptr(code4, d, "code4"), n, blocksize, blocksize2, dt,
+                                  _ptr(out, d, "out"), _stream(stream, codes.device))
     _check("dequantize_4bit_nested", st)
     return out
 
@@ -255,10 +286,12 @@ def dequantize_4bit(codes, absmax, code4, n: int, blocksize: int, dtype, out=Non
     """Plain NF4/FP4 decode with an fp32 absmax per block; returns n elements of `dtype`."""
     import torch
     L = load_library()
+    d = codes.device
     dt = _dt(dtype)
     if out is None:
         out = torch.empty(max(n, 1), dtype=_torch_dtype(dt), device=codes.device)
-    st = L.dequantize_4bit(_ptr(codes), _ptr(absmax), _ptr(code4), n, blocksize, dt, _ptr(out),
+    st = L.dequantize_4bit(_ptr(codes, d, "codes"), _ptr(absmax, d, "absmax"), _ptr(code4, d, "code4"), n,
+                           blocksize, dt, _ptr(out, d, "out"),
                            _stream(stream, codes.device))
     _check("dequantize_4bit", st)
     return out
@@ -270,15 +303,18 @@ def dequantize_4bit_nested_chain(codes, absmax_q, code2, absmax2, offset: float,
     """The unfused three-launch form of dequantize_4bit_nested (same result)."""
     import torch
     L = load_library()
+    d = codes.device
     dt = _dt(dtype)
     if out is None:
         out = torch.empty(max(n, 1), dtype=_torch_dtype(dt), device=codes.device)
     if scale_workspace is None:
         scale_workspace = torch.empty(max((n + blocksize - 1) // blocksize, 1), dtype=torch.float32,
                                       device=codes.device)
-    st = L.dequantize_4bit_nested_chain(_ptr(codes), _ptr(absmax_q), _ptr(code2), _ptr(absmax2),
-                                        ct.c_float(offset), _ptr(code4), n, blocksize, blocksize2, dt,
-                                        _ptr(out), _ptr(scale_workspace), _stream(stream, codes.device))
+    st = L.dequantize_4bit_nested_chain(_ptr(codes, d, "codes"), _ptr(absmax_q, d, "absmax_q"),
+                                        _ptr(code2, d, "code2"), _ptr(absmax2, d, "absmax2"),
+                                        ct.c_float(offset), _ptr(code4, d, "code4"), n, blocksize, blocksize2, dt,
+                                        _ptr(out, d, "out"), _ptr(scale_workspace, d, "scale_workspace"),
+                                        _stream(stream, codes.device))
     _check("dequantize_4bit_nested_chain", st)
     return out
 
@@ -294,12 +330,14 @@ def dequantize_4bit_nested_chain_noalloc(codes, absmax_q, code2, absmax2, offset
     """
     import torch
     L = load_library()
+    d = codes.device
     dt = _dt(dtype)
     if out is None:
         out = torch.empty(max(n, 1), dtype=_torch_dtype(dt), device=codes.device)
-    st = L.dequantize_4bit_nested_chain_noalloc(_ptr(codes), _ptr(absmax_q), _ptr(code2), _ptr(absmax2),
-                                                ct.c_float(offset), _ptr(code4), n, blocksize, blocksize2,
-                                                dt, _ptr(out), _stream(stream, codes.device))
+    st = L.dequantize_4bit_nested_chain_noalloc(_ptr(codes, d, "codes"), _ptr(absmax_q, d, "absmax_q"),
+                                                _ptr(code2, d, "code2"), _ptr(absmax2, d, "absmax2"),
+                                                ct.c_float(offset), _ptr(code4, d, "code4"), n, blocksize, blocksize2,
+                                                dt, _ptr(out, d, "out"), _stream(stream, codes.device))
     _check("dequantize_4bit_nested_chain_noalloc", st)
     return out
 

@@ -5,6 +5,7 @@
 
 #include <cstdarg>
 #include <cstdio>
+#include <initializer_list>
 #include <string>
 
 #include "launch.h"
@@ -39,6 +40,60 @@ bool valid_dtype(int dt) { return dt == BBC_F16 || dt == BBC_BF16 || dt == BBC_F
 
 int elem_size(int dt) { return dt == BBC_F32 ? 4 : 2; }
 
+// A buffer of a call: its address, its extent in bytes and its name for messages.
+struct Buf {
+    const void* p;
+    size_t bytes;
+    const char* name;
+};
+
+bool overlap(const Buf& x, const Buf& y) {
+    const uintptr_t a = reinterpret_cast<uintptr_t>(x.p), b = reinterpret_cast<uintptr_t>(y.p);
+    return x.bytes && y.bytes && a < b + y.bytes && b < a + x.bytes;
+}
+
+// The checks of a call's buffers, after its scalar arguments passed and before anything is
+// launched: no output overlaps an input or another output (host arithmetic only), then every
+// buffer is memory of the current device (a device allocation on it, or a managed allocation),
+// as cudaPointerGetAttributes reports: host memory, pinned or not, memory of another device or an
+// address the CUDA runtime does not know is refused with BBC_ERR_INVALID rather than handed to a
+// kernel. (The extent of an allocation is not known to the runtime; only its start is checked.)
+int check_buffers(const char* fn, std::initializer_list<Buf> in, std::initializer_list<Buf> out) {
+    for (auto o = out.begin(); o != out.end(); ++o) {
+        for (const Buf& i : in)
+            if (overlap(*o, i)) return fail(BBC_ERR_INVALID, "%s: output %s overlaps input %s", fn, o->name, i.name);
+        for (auto o2 = o + 1; o2 != out.end(); ++o2)
+            if (overlap(*o, *o2))
+                return fail(BBC_ERR_INVALID, "%s: outputs %s and %s overlap", fn, o->name, o2->name);
+    }
+    int dev = -1;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) {
+        cudaGetLastError();
+        return fail(BBC_ERR_INVALID, "%s: the buffers cannot be checked as device memory: %s", fn,
+                    cudaGetErrorString(e));
+    }
+    for (const auto* list : {&in, &out})
+        for (const Buf& b : *list) {
+            cudaPointerAttributes a{};
+            e = cudaPointerGetAttributes(&a, b.p);
+            if (e != cudaSuccess) {
+                cudaGetLastError();
+                return fail(BBC_ERR_INVALID, "%s: %s is not memory the CUDA runtime knows: %s", fn, b.name,
+                            cudaGetErrorString(e));
+            }
+            if (a.type == cudaMemoryTypeManaged) continue;
+            if (a.type != cudaMemoryTypeDevice)
+                return fail(BBC_ERR_INVALID, "%s: %s is host memory; device memory is required", fn, b.name);
+            if (a.device != dev)
+                return fail(BBC_ERR_INVALID, "%s: %s is memory of device %d, the current device is %d", fn, b.name,
+                            a.device, dev);
+        }
+    return BBC_OK;
+}
+
+size_t cdiv(int64_t a, int64_t b) { return (size_t)((a + b - 1) / b); }
+
 // log2 of a 4-bit outer blocksize (a power of two in [32, 4096]), or -1.
 int log2_blocksize(int blocksize) {
     for (int l = 5; l <= 12; l++)
@@ -71,6 +126,10 @@ int kbit_quantize(const void* A, int dtype, int64_t n, int K, int blocksize,
                   const float* codebook, float* absmax, uint32_t* packed, void* stream) {
     const int st = check_kbit("kbit_quantize", A, absmax, 4, codebook, packed, n, K, dtype, blocksize, A, dtype);
     if (st != BBC_OK) return st;
+    const size_t nb = cdiv(n, 32);
+    const int sb = check_buffers("kbit_quantize", {{A, (size_t)n * elem_size(dtype), "A"}, {codebook, 4u << K, "codebook"}},
+                                 {{absmax, nb * 4, "absmax"}, {packed, nb * K * 4, "packed"}});
+    if (sb != BBC_OK) return sb;
     const bool vec = aligned(A, 32);     // 256-bit loads of 16-element groups
     return cuda_status(bbc::launch_kbit_quantize(A, dtype, n, K, codebook, absmax, packed, vec,
                                                  static_cast<cudaStream_t>(stream)),
@@ -82,6 +141,11 @@ int kbit_dequantize(const uint32_t* packed, const float* absmax, const float* co
     const int st = check_kbit("kbit_dequantize", out, absmax, 4, codebook, packed, n, K, out_dtype, blocksize,
                               out, out_dtype);
     if (st != BBC_OK) return st;
+    const size_t nb = cdiv(n, 32);
+    const int sb = check_buffers("kbit_dequantize", {{packed, nb * K * 4, "packed"}, {absmax, nb * 4, "absmax"},
+                                                     {codebook, 4u << K, "codebook"}},
+                                 {{out, (size_t)n * elem_size(out_dtype), "out"}});
+    if (sb != BBC_OK) return sb;
     const bool vec = aligned(out, 32);     // 32-byte stores of 16-element groups
     return cuda_status(bbc::launch_kbit_dequantize(packed, absmax, codebook, K, n, out_dtype, out, vec,
                                                    static_cast<cudaStream_t>(stream)),
@@ -93,6 +157,10 @@ int kbit_quantize_e4m4(const void* A, int dtype, int64_t n, int K, int blocksize
     const int st = check_kbit("kbit_quantize_e4m4", A, absmax_e4m4, 1, codebook, packed, n, K, dtype, blocksize,
                               A, dtype);
     if (st != BBC_OK) return st;
+    const size_t nb = cdiv(n, 32);
+    const int sb = check_buffers("kbit_quantize_e4m4", {{A, (size_t)n * elem_size(dtype), "A"}, {codebook, 4u << K, "codebook"}},
+                                 {{absmax_e4m4, nb, "absmax_e4m4"}, {packed, nb * K * 4, "packed"}});
+    if (sb != BBC_OK) return sb;
     const bool vec = aligned(A, 32);
     return cuda_status(bbc::launch_kbit_quantize_e4m4(A, dtype, n, K, codebook, absmax_e4m4, packed, vec,
                                                       static_cast<cudaStream_t>(stream)),
@@ -104,6 +172,11 @@ int kbit_dequantize_e4m4(const uint32_t* packed, const uint8_t* absmax_e4m4, con
     const int st = check_kbit("kbit_dequantize_e4m4", out, absmax_e4m4, 1, codebook, packed, n, K, out_dtype,
                               blocksize, out, out_dtype);
     if (st != BBC_OK) return st;
+    const size_t nb = cdiv(n, 32);
+    const int sb = check_buffers("kbit_dequantize_e4m4", {{packed, nb * K * 4, "packed"}, {absmax_e4m4, nb, "absmax_e4m4"},
+                                                          {codebook, 4u << K, "codebook"}},
+                                 {{out, (size_t)n * elem_size(out_dtype), "out"}});
+    if (sb != BBC_OK) return sb;
     const bool vec = aligned(out, 32);
     return cuda_status(bbc::launch_kbit_dequantize_e4m4(packed, absmax_e4m4, codebook, K, n, out_dtype, out, vec,
                                                         static_cast<cudaStream_t>(stream)),
@@ -130,6 +203,12 @@ int dequantize_4bit_nested(const uint8_t* codes, const uint8_t* absmax_q, const 
                     blocksize2);
     if (!aligned(out, elem_size(out_dtype)) || !aligned(code2, 4) || !aligned(absmax2, 4) || !aligned(code4, 4))
         return fail(BBC_ERR_INVALID, "dequantize_4bit_nested: pointer not aligned to its element size");
+    const size_t nbo = cdiv(n, blocksize);
+    const int sb = check_buffers("dequantize_4bit_nested",
+                                 {{codes, cdiv(n, 2), "codes"}, {absmax_q, nbo, "absmax_q"}, {code2, 1024, "code2"},
+                                  {absmax2, cdiv((int64_t)nbo, 256) * 4, "absmax2"}, {code4, 64, "code4"}},
+                                 {{out, (size_t)n * elem_size(out_dtype), "out"}});
+    if (sb != BBC_OK) return sb;
     const bool vec = aligned(out, 32) && aligned(codes, 16);   // 8/16-byte loads, 32-byte stores
     return cuda_status(bbc::launch_nested_dequantize(codes, absmax_q, code2, absmax2, offset, code4, n,
                                                      log2_bs, out_dtype, out, vec,
@@ -149,6 +228,10 @@ int dequantize_4bit(const uint8_t* codes, const float* absmax, const float* code
                     blocksize);
     if (!aligned(out, elem_size(out_dtype)) || !aligned(absmax, 4) || !aligned(code4, 4))
         return fail(BBC_ERR_INVALID, "dequantize_4bit: pointer not aligned to its element size");
+    const int sb = check_buffers("dequantize_4bit",
+                                 {{codes, cdiv(n, 2), "codes"}, {absmax, cdiv(n, blocksize) * 4, "absmax"}, {code4, 64, "code4"}},
+                                 {{out, (size_t)n * elem_size(out_dtype), "out"}});
+    if (sb != BBC_OK) return sb;
     const bool vec = aligned(out, 32) && aligned(codes, 16);
     return cuda_status(bbc::launch_dequantize_4bit(codes, absmax, code4, n, log2_bs, out_dtype, out, vec,
                                                    static_cast<cudaStream_t>(stream)),
@@ -166,6 +249,9 @@ int quantize_4bit(const void* A, int dtype, int64_t n, int blocksize, const floa
         return fail(BBC_ERR_INVALID, "%s: blocksize must be a power of two in [32, 4096] (got %d)", fn, blocksize);
     if (!aligned(A, elem_size(dtype)) || !aligned(absmax, 4) || !aligned(code4, 4))
         return fail(BBC_ERR_INVALID, "%s: pointer not aligned to its element size", fn);
+    const int sb = check_buffers(fn, {{A, (size_t)n * elem_size(dtype), "A"}, {code4, 64, "code4"}},
+                                 {{absmax, cdiv(n, blocksize) * 4, "absmax"}, {codes, cdiv(n, 2), "codes"}});
+    if (sb != BBC_OK) return sb;
     const bool vec = aligned(A, 32) && aligned(codes, 16);     // 256-bit loads, 8/16-byte code stores
     return cuda_status(bbc::launch_quantize_4bit(A, dtype, n, log2_bs, code4, absmax, codes, vec,
                                                  static_cast<cudaStream_t>(stream)),
@@ -197,6 +283,12 @@ int quantize_4bit_nested(const void* A, int dtype, int64_t n, int blocksize, con
     if (!aligned(A, elem_size(dtype)) || !aligned(code4, 4) || !aligned(code2, 4) || !aligned(absmax2, 4) ||
         !aligned(offset, 4) || !aligned(workspace, 256))
         return fail(BBC_ERR_INVALID, "%s: pointer not aligned (elements; workspace to 256 bytes)", fn);
+    const size_t nbo = cdiv(n, blocksize);
+    const int sb = check_buffers(fn, {{A, (size_t)n * elem_size(dtype), "A"}, {code4, 64, "code4"}, {code2, 1024, "code2"}},
+                                 {{codes, cdiv(n, 2), "codes"}, {absmax_q, nbo, "absmax_q"},
+                                  {absmax2, cdiv((int64_t)nbo, 256) * 4, "absmax2"}, {offset, 4, "offset"},
+                                  {workspace, need, "workspace"}});
+    if (sb != BBC_OK) return sb;
     const bool vec = aligned(A, 32) && aligned(codes, 16);
     return cuda_status(bbc::launch_quantize_4bit_nested(A, dtype, n, log2_bs, code4, code2, codes, absmax_q,
                                                         absmax2, offset, workspace, vec,
@@ -226,6 +318,12 @@ int linear_4bit_nested(const void* X, int dtype, int64_t M, int64_t N, int64_t K
     if (!aligned(X, 16) || !aligned(codes, 16) || !aligned(Y, 2) || !aligned(code2, 4) || !aligned(absmax2, 4) ||
         !aligned(code4, 4))
         return fail(BBC_ERR_INVALID, "%s: X and codes must be 16-byte aligned (others: element size)", fn);
+    const int sb = check_buffers(fn, {{X, (size_t)(M * K) * 2, "X"}, {codes, (size_t)(N * K / 2), "codes"},
+                                      {absmax_q, cdiv(N * K, blocksize), "absmax_q"}, {code2, 1024, "code2"},
+                                      {absmax2, cdiv((int64_t)cdiv(N * K, blocksize), 256) * 4, "absmax2"},
+                                      {code4, 64, "code4"}},
+                                 {{Y, (size_t)(M * N) * 2, "Y"}});
+    if (sb != BBC_OK) return sb;
     return cuda_status(bbc::launch_linear_4bit_nested(X, dtype, (int)M, N, K, codes, absmax_q, code2, absmax2,
                                                       offset, code4, log2_bs, Y, static_cast<cudaStream_t>(stream)),
                        "linear_4bit_nested launch");
@@ -247,6 +345,10 @@ int linear_kbit(const void* X, int dtype, int64_t M, int64_t N, int64_t K, const
                     fn, (long long)M, (long long)N, (long long)K);
     if (!aligned(X, 16) || !aligned(packed, 16) || !aligned(Y, 2) || !aligned(absmax, 4) || !aligned(codebook, 4))
         return fail(BBC_ERR_INVALID, "%s: X and packed must be 16-byte aligned (others: element size)", fn);
+    const int sb = check_buffers(fn, {{X, (size_t)(M * K) * 2, "X"}, {packed, (size_t)(N * K / 32) * bits * 4, "packed"},
+                                      {absmax, (size_t)(N * K / 32) * 4, "absmax"}, {codebook, 4u << bits, "codebook"}},
+                                 {{Y, (size_t)(M * N) * 2, "Y"}});
+    if (sb != BBC_OK) return sb;
     return cuda_status(bbc::launch_linear_kbit(X, dtype, (int)M, N, K, packed, absmax, codebook, bits, Y,
                                                static_cast<cudaStream_t>(stream)),
                        "linear_kbit launch");
@@ -273,6 +375,12 @@ int dequantize_4bit_nested_chain(const uint8_t* codes, const uint8_t* absmax_q, 
     if (!aligned(out, elem_size(out_dtype)) || !aligned(code2, 4) || !aligned(absmax2, 4) ||
         !aligned(code4, 4) || !aligned(scale_workspace, 4))
         return fail(BBC_ERR_INVALID, "dequantize_4bit_nested_chain: pointer not aligned to its element size");
+    const size_t nbo = cdiv(n, blocksize);
+    const int sb = check_buffers("dequantize_4bit_nested_chain",
+                                 {{codes, cdiv(n, 2), "codes"}, {absmax_q, nbo, "absmax_q"}, {code2, 1024, "code2"},
+                                  {absmax2, cdiv((int64_t)nbo, 256) * 4, "absmax2"}, {code4, 64, "code4"}},
+                                 {{out, (size_t)n * elem_size(out_dtype), "out"}, {scale_workspace, nbo * 4, "scale_workspace"}});
+    if (sb != BBC_OK) return sb;
     const bool vec = aligned(out, 32) && aligned(codes, 16);
     return cuda_status(bbc::launch_nested_dequantize_chain(codes, absmax_q, code2, absmax2, offset, code4, n,
                                                            log2_bs, out_dtype, out, scale_workspace, vec,
@@ -303,6 +411,10 @@ int dequantize_4bit_nested_chain_noalloc(const uint8_t* codes, const uint8_t* ab
                     fn, (long long)nbo, (long long)n, blocksize, BBC_NOALLOC_SCRATCH_FLOATS);
     if (!aligned(out, elem_size(out_dtype)) || !aligned(code2, 4) || !aligned(absmax2, 4) || !aligned(code4, 4))
         return fail(BBC_ERR_INVALID, "%s: pointer not aligned to its element size", fn);
+    const int sb = check_buffers(fn, {{codes, cdiv(n, 2), "codes"}, {absmax_q, (size_t)nbo, "absmax_q"}, {code2, 1024, "code2"},
+                                      {absmax2, cdiv(nbo, 256) * 4, "absmax2"}, {code4, 64, "code4"}},
+                                 {{out, (size_t)n * elem_size(out_dtype), "out"}});
+    if (sb != BBC_OK) return sb;
     const bool vec = aligned(out, 32) && aligned(codes, 16);
     return cuda_status(bbc::launch_nested_dequantize_chain_noalloc(codes, absmax_q, code2, absmax2, offset,
                                                                    code4, n, log2_bs, out_dtype, out, vec,
