@@ -26,6 +26,7 @@ from ._native import (  # noqa: F401
     BBCError,
     bbc_last_error,
     bbc_nf_codebook,
+    bbc_wait_timeouts,
     dequantize_4bit,
     dequantize_4bit_nested,
     dequantize_4bit_nested_chain,

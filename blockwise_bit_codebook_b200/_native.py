@@ -60,6 +60,8 @@ def load_library():
     L.dequantize_4bit_nested_chain_noalloc.restype = I
     L.bbc_nf_codebook.argtypes = [I, P]
     L.bbc_nf_codebook.restype = I
+    L.bbc_wait_timeouts.argtypes = [ct.POINTER(ct.c_uint)]
+    L.bbc_wait_timeouts.restype = I
     L.bbc_last_error.argtypes = []
     L.bbc_last_error.restype = ct.c_char_p
     _lib = L
@@ -233,8 +235,9 @@ def quantize_4bit_nested(A, blocksize: int, code4, code2, blocksize2: int = 256,
 
 def linear_4bit_nested(X, codes, absmax_q, code2, absmax2, offset: float, code4, N: int, blocksize: int,
                        blocksize2: int = 256, out=None, stream=None):
-    """Y = X @ W^T for X [M, K] (fp16/bf16, M <= 32) and W [N, K] the nested 4-bit weight, decoded
-    in registers (never materialised). Returns Y [M, N] in X's dtype."""
+    """Y = X @ W^T for X [M, K] (fp16/bf16) and W [N, K] the nested 4-bit weight, decoded on the
+    fly (never materialised; M > 32 on the tensor cores, N % 128 == 0). Returns Y [M, N] in X's
+    dtype."""
     import torch
     L = load_library()
     d = X.device
@@ -250,8 +253,9 @@ def linear_4bit_nested(X, codes, absmax_q, code2, absmax2, offset: float, code4,
 
 
 def linear_kbit(X, packed, absmax, codebook, K: int, N: int, blocksize: int = 32, out=None, stream=None):
-    """Y = X @ W^T for X [M, Kin] (fp16/bf16, M <= 32) and W [N, Kin] the k-bit weight of
-    kbit_quantize (K bits, blocksize 32), decoded in registers. Returns Y [M, N] in X's dtype."""
+    """Y = X @ W^T for X [M, Kin] (fp16/bf16) and W [N, Kin] the k-bit weight of kbit_quantize
+    (K bits, blocksize 32), decoded on the fly (M > 32 on the tensor cores, N % 128 == 0).
+    Returns Y [M, N] in X's dtype."""
     import torch
     L = load_library()
     d = X.device
@@ -340,6 +344,15 @@ def dequantize_4bit_nested_chain_noalloc(codes, absmax_q, code2, absmax2, offset
                                                 dt, _ptr(out, d, "out"), _stream(stream, codes.device))
     _check("dequantize_4bit_nested_chain_noalloc", st)
     return out
+
+
+def bbc_wait_timeouts() -> int:
+    """Bounded in-kernel waits that gave up on the current device since the last call (the
+    count is reset); 0 when every wait completed."""
+    L = load_library()
+    c = ct.c_uint(0)
+    _check("bbc_wait_timeouts", L.bbc_wait_timeouts(ct.byref(c)))
+    return int(c.value)
 
 
 def bbc_nf_codebook(K: int) -> np.ndarray:

@@ -4,6 +4,7 @@
 #include <cuda_runtime.h>
 
 #include <cstdarg>
+#include <cstdint>
 #include <cstdio>
 #include <initializer_list>
 #include <string>
@@ -307,8 +308,9 @@ int linear_4bit_nested(const void* X, int dtype, int64_t M, int64_t N, int64_t K
                     (long long)N, (long long)K);
     if (dtype != BBC_F16 && dtype != BBC_BF16)
         return fail(BBC_ERR_UNSUPPORTED, "%s: activations must be fp16 or bf16 (got dtype %d)", fn, dtype);
-    if (M > 32 || N % 16 != 0 || K % 64 != 0)
-        return fail(BBC_ERR_UNSUPPORTED, "%s: needs M <= 32, N %% 16 == 0, K %% 64 == 0 (got %lld, %lld, %lld)",
+    if (N % 16 != 0 || K % 64 != 0 || (M > 32 && N % 128 != 0) || M > INT32_MAX || K > INT32_MAX)
+        return fail(BBC_ERR_UNSUPPORTED,
+                    "%s: needs K %% 64 == 0 and N %% 16 == 0 (N %% 128 == 0 when M > 32) (got M=%lld, N=%lld, K=%lld)",
                     fn, (long long)M, (long long)N, (long long)K);
     const int log2_bs = log2_blocksize(blocksize);
     if (log2_bs < 0)
@@ -340,8 +342,9 @@ int linear_kbit(const void* X, int dtype, int64_t M, int64_t N, int64_t K, const
     if (blocksize != 32) return fail(BBC_ERR_UNSUPPORTED, "%s: blocksize must be 32 (got %d)", fn, blocksize);
     if (dtype != BBC_F16 && dtype != BBC_BF16)
         return fail(BBC_ERR_UNSUPPORTED, "%s: activations must be fp16 or bf16 (got dtype %d)", fn, dtype);
-    if (M > 32 || N % 16 != 0 || K % 64 != 0)
-        return fail(BBC_ERR_UNSUPPORTED, "%s: needs M <= 32, N %% 16 == 0, K %% 64 == 0 (got %lld, %lld, %lld)",
+    if (N % 16 != 0 || K % 64 != 0 || (M > 32 && N % 128 != 0) || M > INT32_MAX || K > INT32_MAX)
+        return fail(BBC_ERR_UNSUPPORTED,
+                    "%s: needs K %% 64 == 0 and N %% 16 == 0 (N %% 128 == 0 when M > 32) (got M=%lld, N=%lld, K=%lld)",
                     fn, (long long)M, (long long)N, (long long)K);
     if (!aligned(X, 16) || !aligned(packed, 16) || !aligned(Y, 2) || !aligned(absmax, 4) || !aligned(codebook, 4))
         return fail(BBC_ERR_INVALID, "%s: X and packed must be 16-byte aligned (others: element size)", fn);
@@ -420,6 +423,11 @@ int dequantize_4bit_nested_chain_noalloc(const uint8_t* codes, const uint8_t* ab
                                                                    code4, n, log2_bs, out_dtype, out, vec,
                                                                    static_cast<cudaStream_t>(stream)),
                        fn);
+}
+
+int bbc_wait_timeouts(unsigned int* count) {
+    if (!count) return fail(BBC_ERR_INVALID, "bbc_wait_timeouts: null pointer argument");
+    return cuda_status(bbc::wait_timeouts(count), "bbc_wait_timeouts");
 }
 
 const char* bbc_last_error(void) { return g_last_error.c_str(); }

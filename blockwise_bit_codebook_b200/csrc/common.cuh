@@ -183,4 +183,38 @@ __device__ __forceinline__ uint32_t plane_offset4(uint32_t B, uint32_t B3) {
     return __umulhi(src & mask, mult) & 0x3Cu;
 }
 
+
+// ---- k-bit weights of a 32-element block: plane groups and per-element decode ----
+
+// Element 8q + E of a block as fp32 (codebook entry times absmax, one rounding), from plane group
+// Bq (byte j = plane j of elements 8q .. 8q+7, Bqs = Bq << 3) and, for K = 5, p4q (bit i = plane
+// 4 of element 8q + i); cbb is the codebook in shared memory (byte address).
+template <int KB, int DT, int E>
+__device__ __forceinline__ float kbit_elem(uint32_t Bq, uint32_t Bqs, uint32_t p4q, float am, const char* cbb) {
+    uint32_t off = plane_offset4<E>(Bq, Bqs);
+    if constexpr (KB == 5) off |= (E <= 6 ? (p4q << (6 - E)) : (p4q >> (E - 6))) & 0x40u;
+    return __fmul_rn(*reinterpret_cast<const float*>(cbb + off), am);
+}
+// The plane groups of a lane's run: all four for a 32-element run; for a 16-element run, the
+// two groups of half h of the block.
+template <int KB, int R>
+__device__ __forceinline__ void kbit_groups(const uint32_t (&w)[KB], int h, uint32_t (&G)[R / 8], uint32_t& p4) {
+    const uint32_t w0 = w[0], w1 = w[1 % KB], w2 = KB > 2 ? w[2 % KB] : 0u, w3 = KB > 3 ? w[3 % KB] : 0u;
+    p4 = KB == 5 ? w[4 % KB] : 0u;
+    if constexpr (R == 32) {
+        const uint32_t t0 = prmt(w0, w1, 0x5140u), t1 = prmt(w0, w1, 0x7362u);
+        const uint32_t t2 = prmt(w2, w3, 0x5140u), t3 = prmt(w2, w3, 0x7362u);
+        G[0] = prmt(t0, t2, 0x5410u);
+        G[1] = prmt(t0, t2, 0x7632u);
+        G[2] = prmt(t1, t3, 0x5410u);
+        G[3] = prmt(t1, t3, 0x7632u);
+    } else {
+        const uint32_t sel = h ? 0x7362u : 0x5140u;            // bytes 2h, 2h + 1 of two words
+        const uint32_t tl = prmt(w0, w1, sel), th = prmt(w2, w3, sel);
+        G[0] = prmt(tl, th, 0x5410u);
+        G[1] = prmt(tl, th, 0x7632u);
+        p4 >>= 16 * h;
+    }
+}
+
 }  // namespace bbc

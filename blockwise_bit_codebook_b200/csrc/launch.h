@@ -44,13 +44,14 @@ inline cudaError_t set_attr_once(Kernel kernel, std::atomic<uint64_t>& done, cud
 
 // Persistent grid: enough CTAs to fill every SM at the kernel's occupancy, never more than
 // the work needs. The occupancy query runs once per (kernel, device, block, smem) and is
-// cached (grid.cpp).
+// cached (grid.cpp); if it fails both return 0 (an empty grid, whose launch then fails).
 int resident_ctas(const void* kernel, int block, size_t dyn_smem);
 
 template <typename Kernel>
 inline int persistent_grid(Kernel kernel, int block, size_t dyn_smem, int64_t work_items,
                            int items_per_cta) {
     const int64_t cap = resident_ctas(reinterpret_cast<const void*>(kernel), block, dyn_smem);
+    if (cap < 1) return 0;
     int64_t need = (work_items + items_per_cta - 1) / items_per_cta;
     if (need < 1) need = 1;
     return (int)(need < cap ? need : cap);
@@ -85,6 +86,18 @@ cudaError_t launch_linear_4bit_nested(const void* X, int dtype, int M, int64_t N
 
 cudaError_t launch_linear_kbit(const void* X, int dtype, int M, int64_t N, int64_t K, const uint32_t* packed,
                                const float* absmax, const float* codebook, int KB, void* Y, cudaStream_t s);
+
+// The same two layers for M > 32 on the tensor cores (tcgen05; N % 128 == 0, K % 64 == 0, X 16-byte
+// aligned): linear_tc.cu.
+cudaError_t launch_linear_4bit_nested_tc(const void* X, int dtype, int M, int64_t N, int64_t K, const uint8_t* codes,
+                                         const uint8_t* absmax_q, const float* code2, const float* absmax2,
+                                         float offset, const float* code4, int log2_bs, void* Y, cudaStream_t s);
+cudaError_t launch_linear_kbit_tc(const void* X, int dtype, int M, int64_t N, int64_t K, const uint32_t* packed,
+                                  const float* absmax, const float* codebook, int KB, void* Y, cudaStream_t s);
+
+// Bounded waits (mbarrier waits of the tensor-core kernels) that gave up on the current device
+// since the last call; reads and resets the device's count (synchronous).
+cudaError_t wait_timeouts(unsigned int* count);
 
 // The same two operations with the per-block absmax stored as one E4M4 byte.
 cudaError_t launch_kbit_quantize_e4m4(const void* A, int dtype, int64_t n, int K, const float* codebook,

@@ -331,14 +331,6 @@ __device__ __forceinline__ void load_kwin(KWin<KB>& r, const uint32_t* packed, c
     r.amb = __ldg(absmax + bb);
 }
 
-// Eight weights (elements 8q .. 8q+7 of a block) as four packed pairs of T, from plane group Bq
-// (byte j = plane j of those elements) and, for K = 5, p4q (bit i = plane 4 of element 8q + i).
-template <int KB, int DT, int E>
-__device__ __forceinline__ float kbit_elem(uint32_t Bq, uint32_t Bqs, uint32_t p4q, float am, const char* cbb) {
-    uint32_t off = plane_offset4<E>(Bq, Bqs);
-    if constexpr (KB == 5) off |= (E <= 6 ? (p4q << (6 - E)) : (p4q >> (E - 6))) & 0x40u;
-    return __fmul_rn(*reinterpret_cast<const float*>(cbb + off), am);
-}
 template <int KB, int DT>
 __device__ __forceinline__ void kbit_group(uint32_t Bq, uint32_t p4q, float am, const char* cbb, uint32_t (&pr)[4]) {
     const uint32_t Bqs = Bq << 3;
@@ -369,28 +361,6 @@ __device__ __forceinline__ void kbit_group_pairs(uint32_t Bq, float am, uint32_t
         const float2 v = *reinterpret_cast<const float2*>(table + (sel | lane_off));
         const float2 p = __fmul2_rn(v, sc);
         pr[i] = DT == BF16 ? pack_bf16x2(p.x, p.y) : pack_f16x2(p.x, p.y);
-    }
-}
-
-// The plane groups of a lane's run: all four for a 32-element run; for a 16-element run, the
-// two groups of half h of the block.
-template <int KB, int R>
-__device__ __forceinline__ void kbit_groups(const uint32_t (&w)[KB], int h, uint32_t (&G)[R / 8], uint32_t& p4) {
-    const uint32_t w0 = w[0], w1 = w[1 % KB], w2 = KB > 2 ? w[2 % KB] : 0u, w3 = KB > 3 ? w[3 % KB] : 0u;
-    p4 = KB == 5 ? w[4 % KB] : 0u;
-    if constexpr (R == 32) {
-        const uint32_t t0 = prmt(w0, w1, 0x5140u), t1 = prmt(w0, w1, 0x7362u);
-        const uint32_t t2 = prmt(w2, w3, 0x5140u), t3 = prmt(w2, w3, 0x7362u);
-        G[0] = prmt(t0, t2, 0x5410u);
-        G[1] = prmt(t0, t2, 0x7632u);
-        G[2] = prmt(t1, t3, 0x5410u);
-        G[3] = prmt(t1, t3, 0x7632u);
-    } else {
-        const uint32_t sel = h ? 0x7362u : 0x5140u;            // bytes 2h, 2h + 1 of two words
-        const uint32_t tl = prmt(w0, w1, sel), th = prmt(w2, w3, sel);
-        G[0] = prmt(tl, th, 0x5410u);
-        G[1] = prmt(tl, th, 0x7632u);
-        p4 >>= 16 * h;
     }
 }
 
@@ -596,6 +566,9 @@ cudaError_t launch_linear_4bit_nested(const void* X, int dtype, int M, int64_t N
                                       const uint8_t* codes, const uint8_t* absmax_q, const float* code2,
                                       const float* absmax2, float offset, const float* code4, int log2_bs,
                                       void* Y, cudaStream_t s) {
+    if (M > 32)
+        return launch_linear_4bit_nested_tc(X, dtype, M, N, K, codes, absmax_q, code2, absmax2, offset, code4, log2_bs,
+                                            Y, s);
     const uint16_t* x = static_cast<const uint16_t*>(X);
     uint16_t* y = static_cast<uint16_t*>(Y);
     if (dtype == BF16) return launch_dt<BF16>(x, M, N, K, codes, absmax_q, code2, absmax2, offset, code4, log2_bs, y, s);
@@ -604,6 +577,7 @@ cudaError_t launch_linear_4bit_nested(const void* X, int dtype, int M, int64_t N
 
 cudaError_t launch_linear_kbit(const void* X, int dtype, int M, int64_t N, int64_t K, const uint32_t* packed,
                                const float* absmax, const float* codebook, int KB, void* Y, cudaStream_t s) {
+    if (M > 32) return launch_linear_kbit_tc(X, dtype, M, N, K, packed, absmax, codebook, KB, Y, s);
     const uint16_t* x = static_cast<const uint16_t*>(X);
     uint16_t* y = static_cast<uint16_t*>(Y);
     if (dtype == BF16) return launch_kbit_dt<BF16>(x, M, N, K, packed, absmax, codebook, KB, y, s);

@@ -195,9 +195,12 @@ static __device__ __align__(256) float g_chain_scale_scratch[BBC_NOALLOC_SCRATCH
 
 }  // namespace
 
-// Device address of this device's copy of the scratch array, looked up once per device with
-// that device current; nullptr if the lookup failed (the error is returned in *err).
-static float* scratch_address(cudaError_t* err) {
+// Device address of this device's copy of the scratch array, looked up with that device current;
+// nullptr if the lookup failed (the error is returned in *err). A call made while `s` is not being
+// captured looks the address up again (cheap once the module is loaded), so that after the
+// device's context has been torn down and the module reloaded (cudaDeviceReset) the new address
+// is used; a call during capture takes the one the last such call found.
+static float* scratch_address(cudaStream_t s, cudaError_t* err) {
     static std::mutex mu;
     static float* addr[64] = {};
     int dev = 0;
@@ -207,8 +210,11 @@ static float* scratch_address(cudaError_t* err) {
         *err = cudaErrorInvalidDevice;
         return nullptr;
     }
+    cudaStreamCaptureStatus cap = cudaStreamCaptureStatusNone;
+    *err = cudaStreamIsCapturing(s, &cap);
+    if (*err != cudaSuccess) return nullptr;
     std::lock_guard<std::mutex> lock(mu);
-    if (!addr[dev]) {
+    if (!addr[dev] || cap == cudaStreamCaptureStatusNone) {
         void* p = nullptr;
         *err = cudaGetSymbolAddress(&p, g_chain_scale_scratch);
         if (*err != cudaSuccess) return nullptr;
@@ -222,7 +228,7 @@ cudaError_t launch_nested_dequantize_chain_noalloc(const uint8_t* codes, const u
                                                    const float* code4, int64_t n, int log2_bs,
                                                    int out_dtype, void* out, bool vec, cudaStream_t s) {
     cudaError_t err = cudaSuccess;
-    float* scale = scratch_address(&err);
+    float* scale = scratch_address(s, &err);
     if (!scale) return err;
     return launch_nested_dequantize_chain(codes, absmax_q, code2, absmax2, offset, code4, n, log2_bs,
                                           out_dtype, out, scale, vec, s);

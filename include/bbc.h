@@ -274,9 +274,11 @@ int dequantize_4bit_nested_chain(const uint8_t* codes, const uint8_t* absmax_q, 
  * without scale_workspace. In addition:
  *   - ceil(n / blocksize) must not exceed BBC_NOALLOC_SCRATCH_FLOATS; larger
  *     requests return BBC_ERR_UNSUPPORTED and launch nothing.
- *   - The first call on each device looks up that device's copy of the array
- *     (once, with the device current); make that first call before capturing
- *     any stream. It allocates nothing.
+ *   - Each call made while `stream` is not being captured looks up the
+ *     current device's copy of the array (so that it stays right after
+ *     cudaDeviceReset reloads the library's module); a call during stream
+ *     capture uses the address the last such call found, so make the first call
+ *     on each device before capturing any stream. Neither allocates anything.
  *   - All calls share the one array per device and it keeps whatever the last
  *     call left there. Each call writes every scale it later reads, so nothing
  *     needs clearing, but calls whose work can overlap on the GPU (different
@@ -303,10 +305,17 @@ int dequantize_4bit_nested_chain_noalloc(const uint8_t* codes, const uint8_t* ab
  * accumulation, a fixed order: the same inputs give the same bits); each Y
  * element is rounded once to T. Not bit-exact against a float64 sum: the error
  * is at most 2*K*2^-24*sum_k |x w| plus half an ulp of T.
+ * M <= 32 runs warp-level MMAs on weights decoded in registers; M > 32 runs the
+ * fifth-generation tensor cores (tcgen05, accumulators in tensor memory) on
+ * 128-row weight tiles decoded into shared memory, with activation tiles loaded
+ * by TMA and, when there are few output tiles, K split over a thread-block
+ * cluster whose partial sums are added in a fixed order in distributed shared
+ * memory (no workspace). Its mbarrier waits are bounded: see bbc_wait_timeouts.
  *
  *   X        [M][K] activations, row-major, dtype BBC_F16 or BBC_BF16 (T),
  *            16-byte aligned.
- *   M        1..32.   N: a multiple of 16.   K: a multiple of 64.
+ *   M        >= 1.   N: a multiple of 16 (of 128 when M > 32).
+ *   K        a multiple of 64.
  *   codes    [N*K/2] uint8 (element 2j in the high nibble of byte j),
  *            16-byte aligned.
  *   absmax_q [ceil(N*K/blocksize)] uint8.   code2 [256] fp32.
@@ -315,8 +324,8 @@ int dequantize_4bit_nested_chain_noalloc(const uint8_t* codes, const uint8_t* ab
  *   blocksize  power of two in [32, 4096].   blocksize2: must be 256.
  *   Y        [M][N] out, row-major, dtype T.
  * One launch on `stream`. Errors: null pointers, M/N/K < 1, a bad blocksize or
- * misaligned X/codes -> BBC_ERR_INVALID; another dtype, M > 32, N % 16 != 0,
- * K % 64 != 0 or blocksize2 != 256 -> BBC_ERR_UNSUPPORTED.
+ * misaligned X/codes -> BBC_ERR_INVALID; another dtype, N % 16 != 0 (N % 128
+ * != 0 when M > 32), K % 64 != 0 or blocksize2 != 256 -> BBC_ERR_UNSUPPORTED.
  */
 int linear_4bit_nested(const void* X, int dtype, int64_t M, int64_t N, int64_t K, const uint8_t* codes,
                        const uint8_t* absmax_q, const float* code2, const float* absmax2, float offset,
@@ -331,21 +340,23 @@ int linear_4bit_nested(const void* X, int dtype, int64_t M, int64_t N, int64_t K
  * public paths ("Fuse nested 4-bit scale reconstruction on SM103", Summary).
  * Each weight is exactly the element kbit_dequantize would write in the
  * activation type T: w[n][k] = T(fl(codebook[idx(m)] * absmax[m / 32])) for the
- * flattened element m = n*K + k of the N x K row-major weight. Accumulation and
- * error bound as linear_4bit_nested (fp32 tensor-core sums in a fixed order,
- * at most 2*K*2^-24*sum_k |x w| plus half an ulp of T from the float64 result).
+ * flattened element m = n*K + k of the N x K row-major weight. Accumulation,
+ * error bound and the two paths (M <= 32, M > 32) as linear_4bit_nested (fp32
+ * tensor-core sums in a fixed order, at most 2*K*2^-24*sum_k |x w| plus half an
+ * ulp of T from the float64 result).
  *
  *   X        [M][K] activations, row-major, dtype BBC_F16 or BBC_BF16 (T),
  *            16-byte aligned.
- *   M        1..32.   N: a multiple of 16.   K: a multiple of 64.
+ *   M        >= 1.   N: a multiple of 16 (of 128 when M > 32).
+ *   K        a multiple of 64.
  *   packed   [N*K/32 * bits] uint32 bit-plane words (kbit_quantize layout),
  *            16-byte aligned.
  *   absmax   [N*K/32] fp32.   codebook: [2^bits] fp32.
  *   bits     2..5 (the K of kbit_quantize).   blocksize: must be 32.
  *   Y        [M][N] out, row-major, dtype T.
  * One launch on `stream`. Errors: null pointers, M/N/K < 1, bits outside 2..5
- * or misaligned X/packed -> BBC_ERR_INVALID; another dtype, M > 32,
- * N % 16 != 0, K % 64 != 0 or blocksize != 32 -> BBC_ERR_UNSUPPORTED.
+ * or misaligned X/packed -> BBC_ERR_INVALID; another dtype, N % 16 != 0 (N % 128
+ * != 0 when M > 32), K % 64 != 0 or blocksize != 32 -> BBC_ERR_UNSUPPORTED.
  */
 int linear_kbit(const void* X, int dtype, int64_t M, int64_t N, int64_t K, const uint32_t* packed,
                 const float* absmax, const float* codebook, int bits, int blocksize, void* Y, void* stream);
@@ -363,6 +374,21 @@ int linear_kbit(const void* X, int dtype, int64_t M, int64_t N, int64_t K, const
  * Host-only: no CUDA call is made.
  */
 int bbc_nf_codebook(int K, float* codebook_out);
+
+/*
+ * bbc_wait_timeouts - failure detection for the kernels that wait on one
+ * another's progress inside a CTA (the tensor-core linear layers: mbarrier
+ * waits between the TMA, decode, MMA and epilogue roles). Every such wait gives
+ * up after a bounded number of polls instead of hanging, counts itself in a
+ * per-device counter and lets the kernel wind down (its results are then not
+ * meaningful). No counterpart on the pages.
+ *
+ *   count  HOST pointer: receives the number of waits that gave up on the
+ *          current device since the previous call; the counter is reset.
+ * Synchronous (a device-to-host copy on the legacy stream). Errors: a null
+ * pointer -> BBC_ERR_INVALID; a failed copy -> BBC_ERR_CUDA.
+ */
+int bbc_wait_timeouts(unsigned int* count);
 
 /* Message for the last non-OK status returned on the calling thread ("" if none). */
 const char* bbc_last_error(void);

@@ -97,7 +97,7 @@ def test_invalid_arguments(bbc):
     x = torch.zeros(33, 64, dtype=torch.bfloat16, device="cuda")
     z8 = torch.zeros(4096, dtype=torch.uint8, device="cuda")
     f = torch.zeros(256, device="cuda")
-    with pytest.raises(BBCError, match="M <= 32"):
+    with pytest.raises(BBCError, match="N % 128"):           # M > 32: the tensor-core path
         bbc.linear_4bit_nested(x, z8, z8, f, f, 0.0, f, 16, 64)
     with pytest.raises(BBCError, match="N % 16"):
         bbc.linear_4bit_nested(x[:4], z8, z8, f, f, 0.0, f, 24, 64)
@@ -118,7 +118,7 @@ def test_kbit_invalid_arguments(bbc):
     f = torch.zeros(256, device="cuda")
     with pytest.raises(BBCError, match="bits"):
         bbc.linear_kbit(x, pk, f, f, 6, 16)
-    with pytest.raises(BBCError, match="M <= 32"):
+    with pytest.raises(BBCError, match="N % 128"):
         bbc.linear_kbit(torch.zeros(33, 64, dtype=torch.bfloat16, device="cuda"), pk, f, f, 4, 16)
     with pytest.raises(BBCError, match="aligned"):
         bbc.linear_kbit(x, pk[2:], f, f, 4, 16)
