@@ -56,11 +56,22 @@ def test_c4_matrix_reduced(bbc, fmt, bs, dt):
     run_both(bbc, n, bs, dt, fmt, seed=bs, all_codes=True)
 
 
-@pytest.mark.parametrize("fmt", ["nf4", "fp4"])
-@pytest.mark.parametrize("bs", [64, 4096])
-def test_c4_full_size_odd(bbc, fmt, bs):
-    """8192*8192 + 37 elements: partial last outer block and inner group; bf16 output."""
-    run_both(bbc, 8192 * 8192 + 37, bs, "bf16", fmt, seed=11, all_codes=True)
+@pytest.mark.parametrize("bs", [32, 64, 128, 256, 1024, 4096])
+def test_c4_full_size_odd(bbc, bs):
+    """The whole C4 matrix at its own size, 8192*8192 + 37 elements (a partial last outer block
+    and inner group): both value tables and all three output types, every General8 code present."""
+    n = 8192 * 8192 + 37
+    codes, q, a2, off = synthetic.nested_state(n, bs, seed=11, device="cuda", all_codes=True)
+    hc, hq, ha2 = to_host(codes), to_host(q), to_host(a2)
+    out = {dt: torch.empty(n, dtype=DTYPES[dt], device="cuda") for dt in ("f16", "bf16", "f32")}
+    for fmt in ("nf4", "fp4"):
+        code2, code4 = tables(fmt)
+        c2d, c4d = torch.from_numpy(code2).cuda(), torch.from_numpy(code4).cuda()
+        for dt in ("f16", "bf16", "f32"):
+            ref = oracle.nested_dequantize(hc, hq, code2, ha2, float(off), code4, n, bs, 256, dt)
+            y = bbc.dequantize_4bit_nested(codes, q, c2d, a2, float(off), c4d, n, bs, DTYPES[dt], out=out[dt])
+            torch.cuda.synchronize()
+            assert_bits_equal(to_host(y), ref, f"nested full-size odd n bs={bs} {fmt} {dt}")
 
 
 @pytest.mark.parametrize("dt", ["f16", "bf16", "f32"])
