@@ -54,6 +54,11 @@ def parse_args():
     ap.add_argument("--e2e-steps", type=int, default=5)
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-per-config", action="store_true",
+                    help="skip the c1-c4 cells that the default 1-GPU line carries in per_config")
+    ap.add_argument("--linear-case", default=None, metavar="FMT:M[:N:K]",
+                    help="profiling case: build one fused-linear weight (FMT nested or kbit4, bf16 "
+                         "activations, N = K = 4096 unless given) and call the entry point 4 times")
     ap.add_argument("--linear", action="store_true",
                     help="fused nested 4-bit dequant + linear vs dequant then cuBLAS, on the pull "
                          "request's public-path control shapes (one JSON line per case)")
@@ -128,9 +133,10 @@ def workload_ops(only=None):
     return ops
 
 
-def workload_desc(n, ops):
+def workload_desc(n, ops, world=1):
     full = n == N_C5 and len(ops) == len(ALL_OPS)
     return {
+        "parallelism": f"replicas{world}" if world > 1 else "single",
         "workload": ("c5: 16384x16384 bf16 weight ~ N(0,0.02) seed 7; k-bit quantize+dequantize at "
                      "K=3 and K=5 (blocksize 32, normal-float codebooks) and nested NF4 dequant "
                      "(outer blocksize 64, inner 256) of the same size, bf16 outputs")
@@ -449,8 +455,7 @@ def run_bbc(args):
     result = {"metric": METRIC, "value": round(value, 1), "unit": "GB/s", "n_gpus": world,
               "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 5),
               "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32",
-              "data": "synthetic", "config": {**workload_desc(n, ops),
-                                              "parallelism": f"replicas{world}" if world > 1 else "single"},
+              "data": "synthetic", "config": workload_desc(n, ops, world),
               "per_kernel": per_kernel, "roofline": roofline,
               "gpu_launches": sum(nested_quant_launches(n, K) if kind == "quantize_nested" else 1
                                   for _, kind, _ in ops) * args.steps, "clocks": clocks}
@@ -535,6 +540,11 @@ def run_bbc(args):
         result["cpu_baseline"] = cpu_baseline(x, nested, code2, code4, cbs, args.cpu_seconds, n)
     elif rank == 0:
         result["cpu_baseline"] = None
+
+    if rank == 0 and world == 1 and not args.no_per_config and args.ops is None and n == N_C5:
+        # the other configurations, each timed on its own after the c5 step (one GPU)
+        torch.cuda.empty_cache()
+        result["per_config"] = per_config_summary(config_cells(dev, peak))
 
     if dist:
         dist.barrier()
@@ -649,6 +659,42 @@ def run_linear(args):
                               "max_rel_diff_vs_unfused": round(rel, 6)}), flush=True)
 
 
+def run_linear_case(args):
+    """One fused-linear case for a profiler: the weight state of `--linear-case FMT:M[:N:K]` (FMT
+    nested: NF4, outer blocksize 64, General8 absmax; kbit4: K = 4, blocksize 32, fp32 absmax),
+    bf16 activations ~ N(0,1), then four calls of the public entry point."""
+    import torch
+
+    import blockwise_bit_codebook_b200 as bbc
+    from blockwise_bit_codebook_b200 import synthetic
+
+    parts = args.linear_case.split(":")
+    fmt, M = parts[0], int(parts[1])
+    N, K = (int(parts[2]), int(parts[3])) if len(parts) == 4 else (4096, 4096)
+    dev = torch.device("cuda", 0)
+    x = synthetic.weights(M * K, std=1.0, seed=4, dtype=torch.bfloat16, device=dev).reshape(M, K)
+    if fmt == "nested":
+        codes, q, a2, off = synthetic.nested_state(N * K, NESTED_BS, seed=3, device=dev)
+        c4 = torch.from_numpy(bbc.bbc_nf_codebook(4)).to(dev)
+        c2 = torch.from_numpy(synthetic.general8_table()).to(dev)
+
+        def f():
+            return bbc.linear_4bit_nested(x, codes, q, c2, a2, float(off), c4, N, NESTED_BS)
+    elif fmt == "kbit4":
+        pk, am = synthetic.kbit_state(N * K, 4, seed=3, device=dev)
+        cb = torch.from_numpy(bbc.bbc_nf_codebook(4)).to(dev)
+
+        def f():
+            return bbc.linear_kbit(x, pk, am, cb, 4, N)
+    else:
+        raise SystemExit(f"unknown format {fmt} (nested or kbit4)")
+    for _ in range(4):
+        y = f()
+    torch.cuda.synchronize()
+    print(json.dumps({"linear_case": args.linear_case, "M": M, "N": N, "K": K,
+                      "y_abs_sum": float(y.float().abs().sum())}), flush=True)
+
+
 def _graph_time(fns, rounds=7):
     """Median, p10 and p90 device time (us) of one call, from CUDA-graph replays of `fns` (one
     call per element, cycling through buffer sets), 7 rounds."""
@@ -673,38 +719,36 @@ def _graph_time(fns, rounds=7):
     return statistics.median(samples), pct_of(samples, 0.1), pct_of(samples, 0.9)
 
 
-def run_matrix(args):
-    """The timed configuration cells other than the c5 step.
+def _cell(cfg, op, dt_name, K, n, nbytes, t, nsets, peak, **extra):
+    med, p10, p90 = t
+    return {"config": cfg, "op": op, "dtype": dt_name, "K": K, "n": n, **extra,
+            "us_median": round(med, 2), "us_p10_p90": [round(p10, 2), round(p90, 2)],
+            "GB/s": round(nbytes / med / 1e3, 1), "Gelem/s": round(n / med / 1e3, 1),
+            "frac_of_measured_hbm": round(nbytes / med / 1e3 / peak, 4), "buffer_sets": nsets}
+
+
+def config_cells(dev, peak, c4_blocksizes=(64,), c4_formats=("nf4", "fp4"), c2_dtypes=None):
+    """The timed configuration cells other than the c5 step, as a list of dicts.
 
     c1: 1,048,576 fp32 ~ N(0,1) (seed 0), K=4 quantize and dequantize to fp32: 4.9 MB, so
         L2-resident: reported as latency, not against the HBM roofline.
     c2: 4096x4096 ~ N(0,0.02) (seed 1) with 0.1 % outliers x20 (seed 2), K = 2..5 x fp16 / bf16 /
         fp32, quantize then dequantize; every cell cycles through >= 4 buffer sets holding more
         than twice the 126 MB L2, so each launch streams from HBM.
-    c4: nested dequant of 8192x8192 (every General8 code present, all 16 value codes), NF4 and
-        FP4, outer blocksizes 32 .. 4096, bf16 and fp32 outputs (>= 168 MB per launch, no reuse).
-    Each cell: CUDA-graph replays (one call per buffer set, host launch cost excluded), 7 rounds,
-    median / p10 / p90; GB/s = algorithmic bytes / median time."""
+    c3: nested NF4 dequant of 4096x11008 (outer blocksize 64), fp16 / bf16 / fp32 outputs.
+    c4: nested dequant of 8192x8192 (every General8 code present, all 16 value codes) at the
+        given outer blocksizes and formats, bf16 and fp32 outputs (>= 168 MB per launch).
+    Each cell: CUDA-graph replays of back-to-back calls (one per buffer set; host launch cost
+    excluded), 7 rounds, median / p10 / p90; GB/s = algorithmic bytes / median time."""
     import torch
 
     import blockwise_bit_codebook_b200 as bbc
     from blockwise_bit_codebook_b200 import synthetic
 
-    dev = torch.device("cuda", 0)
-    torch.cuda.set_device(dev)
-    bbc.load_library()
-    peak, _ = load_peaks()
     l2 = torch.cuda.get_device_properties(dev).L2_cache_size
     sizes = {torch.float16: 2, torch.bfloat16: 2, torch.float32: 4}
     names = {torch.float16: "fp16", torch.bfloat16: "bf16", torch.float32: "fp32"}
-
-    def emit(cfg, op, dt, K, n, nbytes, t, nsets, **extra):
-        med, p10, p90 = t
-        print(json.dumps({"config": cfg, "op": op, "dtype": names[dt], "K": K, "n": n, **extra,
-                          "us_median": round(med, 2), "us_p10_p90": [round(p10, 2), round(p90, 2)],
-                          "GB/s": round(nbytes / med / 1e3, 1), "Gelem/s": round(n / med / 1e3, 1),
-                          "frac_of_measured_hbm": round(nbytes / med / 1e3 / peak, 4),
-                          "buffer_sets": nsets}), flush=True)
+    cells = []
 
     def kbit_cells(cfg, n, dt, Ks, x0, l2_resident, reps_per_set):
         s_in = sizes[dt]
@@ -719,12 +763,32 @@ def run_matrix(args):
             outs = [torch.empty(n, dtype=dt, device=dev) for _ in range(nsets)]
             qf = [(lambda i=i: bbc.kbit_quantize(xs[i], K, cb, absmax=absmax[i], packed=packed[i]))
                   for i in range(nsets)] * reps_per_set
-            emit(cfg, "quantize", dt, K, n, qb, _graph_time(qf), nsets)
+            cells.append(_cell(cfg, "quantize", names[dt], K, n, qb, _graph_time(qf), nsets, peak))
             df = [(lambda i=i: bbc.kbit_dequantize(packed[i], absmax[i], cb, K, n, dt, out=outs[i]))
                   for i in range(nsets)] * reps_per_set
-            emit(cfg, "dequantize", dt, K, n, qb, _graph_time(df), nsets)
+            cells.append(_cell(cfg, "dequantize", names[dt], K, n, qb, _graph_time(df), nsets, peak))
             del xs, packed, absmax, outs
             torch.cuda.empty_cache()
+
+    def nested_cells(cfg, n, bs, fmts, dts, seed, all_codes, reps):
+        codes, q, a2, off = synthetic.nested_state(n, bs, seed=seed, device=dev, all_codes=all_codes)
+        code2 = torch.from_numpy(synthetic.general8_table()).to(dev)
+        tabs = {"nf4": bbc.bbc_nf_codebook(4), "fp4": synthetic.fp4_table()}
+        for fmt in fmts:
+            code4 = torch.from_numpy(tabs[fmt]).to(dev)
+            for dt in dts:
+                # inputs and outputs both rotate through sets holding more than twice the L2
+                nbytes = op_bytes("nested", n, out_size=sizes[dt], bs=bs)
+                nsets = max(2, -(-2 * l2 // nbytes))
+                sets = [(codes.clone(), q.clone(), a2.clone(), torch.empty(n, dtype=dt, device=dev))
+                        for _ in range(nsets)]
+                fns = [(lambda s=s: bbc.dequantize_4bit_nested(s[0], s[1], code2, s[2], float(off), code4, n, bs, dt,
+                                                               out=s[3])) for s in sets] * reps
+                cells.append(_cell(cfg, "nested_dequant", names[dt], None, n, nbytes, _graph_time(fns), nsets, peak,
+                                   format=fmt, blocksize=bs))
+                del sets
+        del codes, q, a2
+        torch.cuda.empty_cache()
 
     # c1: L2-resident, one buffer set
     n1 = 1 << 20
@@ -732,25 +796,49 @@ def run_matrix(args):
     kbit_cells("c1", n1, torch.float32, [4], x1, True, 200)
     # c2: the k-bit sweep
     n2 = 4096 * 4096
-    for dt in (torch.float16, torch.bfloat16, torch.float32):
+    for dt in (c2_dtypes or (torch.float16, torch.bfloat16, torch.float32)):
         x2 = synthetic.weights(n2, std=0.02, seed=1, dtype=dt, device=dev, outlier_frac=0.001)
         kbit_cells("c2", n2, dt, [2, 3, 4, 5], x2, False, 8)
         del x2
-    # c4: nested dequant, blocksize sweep
-    n4 = 8192 * 8192
-    code2 = torch.from_numpy(synthetic.general8_table()).to(dev)
-    tabs = {"nf4": bbc.bbc_nf_codebook(4), "fp4": synthetic.fp4_table()}
-    for bs in (32, 64, 128, 256, 1024, 4096):
-        codes, q, a2, off = synthetic.nested_state(n4, bs, seed=3, device=dev, all_codes=True)
-        for fmt, tab in tabs.items():
-            code4 = torch.from_numpy(tab).to(dev)
-            for dt in (torch.bfloat16, torch.float32):
-                out = torch.empty(n4, dtype=dt, device=dev)
-                nbytes = op_bytes("nested", n4, out_size=sizes[dt], bs=bs)
-                fns = [lambda: bbc.dequantize_4bit_nested(codes, q, code2, a2, float(off), code4, n4, bs, dt,
-                                                          out=out)] * 20
-                emit("c4", "nested_dequant", dt, None, n4, nbytes, _graph_time(fns), 1, format=fmt, blocksize=bs)
-                del out
+    # c3: the headline nested cell (the output buffers rotate so writes do not stay in L2)
+    nested_cells("c3", 4096 * 11008, 64, ("nf4",), (torch.float16, torch.bfloat16, torch.float32), 3, False, 10)
+    # c4: 8192x8192 at the given outer blocksizes
+    for bs in c4_blocksizes:
+        nested_cells("c4", 8192 * 8192, bs, c4_formats, (torch.bfloat16, torch.float32), 3, True, 10)
+    return cells
+
+
+def run_matrix(args):
+    """Every timed configuration cell besides the c5 step (config_cells), the c4 sweep over all
+    six outer blocksizes, one JSON line per cell."""
+    import torch
+
+    import blockwise_bit_codebook_b200 as bbc
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    bbc.load_library()
+    peak, _ = load_peaks()
+    for c in config_cells(dev, peak, c4_blocksizes=(32, 64, 128, 256, 1024, 4096)):
+        print(json.dumps(c), flush=True)
+
+
+def per_config_summary(cells):
+    """The default line's per_config block: every cell by name, and the lowest fraction of the
+    measured HBM copy bandwidth per (config, op) over the HBM-bound configurations."""
+    out, lows = {}, {}
+    for c in cells:
+        name = ":".join(str(x) for x in (c["config"], c["op"], c["dtype"], f"K{c['K']}" if c["K"] else None,
+                                         c.get("format"), f"bs{c['blocksize']}" if c.get("blocksize") else None)
+                        if x)
+        out[name] = {"us": c["us_median"], "GB/s": c["GB/s"], "Gelem/s": c["Gelem/s"],
+                     "frac_of_measured_hbm": c["frac_of_measured_hbm"], "buffer_sets": c["buffer_sets"]}
+        if c["config"] != "c1":
+            key = f"{c['config']}:{c['op']}"
+            lows[key] = min(lows.get(key, 1e9), c["frac_of_measured_hbm"])
+    return {"cells": out, "min_frac_of_measured_hbm": lows,
+            "method": "CUDA-graph replays of back-to-back calls over rotating buffer sets (> 2x L2 for c2, "
+                      "c3, c4), 7 rounds, medians; c1 is L2-resident (latency, not an HBM fraction)"}
 
 
 def run_nested_matrix(args):
@@ -873,16 +961,36 @@ def run_reference(args):
         "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s",
         "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(tot_t / args.steps * 1e3, 3), "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "f32", "data": "synthetic", "config": workload_desc(N_C5, ALL_OPS),
+        "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": workload_desc(N_C5, ALL_OPS, int(os.environ.get("WORLD_SIZE", "1"))),
         "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": C, "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }), flush=True)
 
 
+def relaunch_under_torchrun(args):
+    """`bench.py --gpus N` (N > 1) started without torchrun starts N ranks itself, one per GPU, as
+    the driver does (torchrun on 127.0.0.1); rank 0 prints the line."""
+    import subprocess
+    import sys
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={args.gpus}",
+           "--master-addr", "127.0.0.1", "--master-port", os.environ.get("BBC_BENCH_PORT", "29513"),
+           os.path.abspath(__file__), *sys.argv[1:]]
+    sys.exit(subprocess.call(cmd))
+
+
 if __name__ == "__main__":
     a = parse_args()
-    if a.linear:
+    if a.gpus > 1 and "WORLD_SIZE" not in os.environ and a.impl == "bbc" and not (
+            a.linear or a.linear_case or a.matrix or a.nested_matrix):
+        relaunch_under_torchrun(a)
+    world_env = int(os.environ.get("WORLD_SIZE", "1"))
+    if a.impl == "bbc" and "WORLD_SIZE" in os.environ and world_env != a.gpus:
+        raise SystemExit(f"--gpus {a.gpus} but WORLD_SIZE={world_env}: start one rank per GPU")
+    if a.linear_case:
+        run_linear_case(a)
+    elif a.linear:
         run_linear(a)
     elif a.matrix:
         run_matrix(a)

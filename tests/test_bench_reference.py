@@ -50,3 +50,20 @@ def test_algorithmic_bytes_and_launch_counts():
     assert b.nested_quant_launches(2048 * 64, 64) == 2          # the root alone, inside the compression
     names = [o[0] for o in b.workload_ops("quantize_nested_nf4_bs32,quantize_4bit_nf4_bs64,dequantize_k4")]
     assert names == ["dequantize_k4", "quantize_4bit_nf4_bs64", "quantize_nested_nf4_bs32"]
+
+
+def test_both_arms_name_the_same_config():
+    bench = _bench_module()
+    ops = bench.ALL_OPS
+    assert bench.workload_desc(bench.N_C5, ops, 1) == bench.workload_desc(bench.N_C5, list(ops), 1)
+    assert bench.workload_desc(bench.N_C5, ops, 1)["parallelism"] == "single"
+    assert bench.workload_desc(bench.N_C5, ops, 4)["parallelism"] == "replicas4"
+
+
+def test_gpus_must_match_the_ranks_started():
+    import subprocess
+    import sys
+    env = dict(os.environ, WORLD_SIZE="1", RANK="0", LOCAL_RANK="0")
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--gpus", "2", "--steps", "1"],
+                       capture_output=True, text=True, env=env, timeout=300)
+    assert r.returncode != 0 and "WORLD_SIZE=1" in r.stderr

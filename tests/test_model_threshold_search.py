@@ -3,12 +3,14 @@
 The fast quantize path needs, for each pair of neighbouring codebook entries a < b, the
 smallest fp32 value T at which entry b is strictly nearer than entry a under the exact rule of
 the k-bit patch series (kQuantizeBlockwise_kbit: fp32 distance fabsf(xn - c), first index on
-ties), i.e. fl(b - T) < fl(T - a). The kernel finds T with 8 lanes per threshold: a narrow
-bracket around the midpoint (checked before use), then 9-way splits of the ordered-key range.
-This file restates that arithmetic on the host (uint32 keys, fp32 subtractions, fp64 midpoint,
-directed conversions) and checks that it returns exactly the brute-force T (bisection over all
-fp32 keys with the rule itself) within its step bound, for the codebooks the library uses and
-for adversarial pairs. No GPU is involved.
+ties), i.e. fl(b - T) < fl(T - a). The kernel finds T with 8 lanes per threshold: candidates
+at the rounding boundaries of the two distances near (b - a) / 2, the smallest one where the
+rule holds kept if the rule fails one fp32 value below it; otherwise a checked bracket around
+the midpoint and 9-way splits of its ordered keys. This file restates that arithmetic on the
+host (uint32 keys, fp32 subtractions, fp64 breakpoints, directed conversions) and checks that it
+returns exactly the brute-force T (bisection over all fp32 keys with the rule itself) within
+its step bound, for the codebooks the library uses and for adversarial pairs. No GPU is
+involved.
 """
 from fractions import Fraction
 
