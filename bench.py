@@ -59,6 +59,8 @@ def parse_args():
     ap.add_argument("--linear-case", default=None, metavar="FMT:M[:N:K]",
                     help="profiling case: build one fused-linear weight (FMT nested or kbit4, bf16 "
                          "activations, N = K = 4096 unless given) and call the entry point 4 times")
+    ap.add_argument("--linear-shapes", default=None, metavar="M,M,...",
+                    help="with --linear: only the control shapes with these activation counts")
     ap.add_argument("--linear", action="store_true",
                     help="fused nested 4-bit dequant + linear vs dequant then cuBLAS, on the pull "
                          "request's public-path control shapes (one JSON line per case)")
@@ -579,9 +581,13 @@ def run_linear(args):
     bs = NESTED_BS
     KB = 4
     cbk = torch.from_numpy(bbc.bbc_nf_codebook(KB)).to(dev)
-    for (M, N, K, label) in [(1, 4096, 4096, "recurrent grad_A M=1"), (8, 4096, 4096, "recurrent grad_A M=8"),
-                             (32, 4096, 4096, "fallback forward M=32"),
-                             (32, 11008, 4096, "fallback forward M=32 N=11008")]:
+    shapes = [(1, 4096, 4096, "recurrent grad_A M=1"), (8, 4096, 4096, "recurrent grad_A M=8"),
+              (32, 4096, 4096, "fallback forward M=32"), (32, 11008, 4096, "fallback forward M=32 N=11008"),
+              (64, 4096, 4096, "batch M=64"), (128, 4096, 4096, "batch M=128"), (256, 4096, 4096, "batch M=256"),
+              (256, 11008, 4096, "batch M=256 N=11008")]
+    if args.linear_shapes:
+        shapes = [s for s in shapes if s[0] in {int(m) for m in args.linear_shapes.split(",")}]
+    for (M, N, K, label) in shapes:
         x = synthetic.weights(M * K, std=1.0, seed=4, dtype=torch.bfloat16, device=dev).reshape(M, K)
         w = torch.empty(N * K, dtype=torch.bfloat16, device=dev)
         y_f = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
@@ -645,7 +651,10 @@ def run_linear(args):
             med = {k: statistics.median(v) for k, v in samples.items()}
             nbytes = wbytes + M * K * 2 + M * N * 2
             rel = float((y_f.float() - y_u.float()).abs().max() / y_u.float().abs().max())
+            flops = 2.0 * M * N * K
             print(json.dumps({"case": label, "format": fmt, "M": M, "N": N, "K": K, "dtype": "bf16",
+                              "fused_TFLOPs": round(flops / med["fused"] / 1e6, 1),
+                              "unfused_TFLOPs": round(flops / med["unfused"] / 1e6, 1),
                               "fused_us_median": round(med["fused"], 2), "unfused_us_median": round(med["unfused"], 2),
                               "unfused_over_fused": round(med["unfused"] / med["fused"], 3),
                               "fused_GBs": round(nbytes / med["fused"] / 1e3, 1),

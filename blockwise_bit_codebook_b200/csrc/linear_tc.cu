@@ -6,15 +6,19 @@
 // exactly the values the unfused dequantize-then-linear path materialises; here W never exists
 // in global memory.
 //
-// Tiling (weight rows on the MMA's M side): a CTA owns 128 rows of W and NT (64, 128 or 256)
-// activation rows; its accumulator D[128 x NT] (fp32) lives in tensor memory. K advances in
-// 64-wide stages through a 4-deep shared-memory ring:
-//   * warp 0, one thread: TMA load of the X tile (NT rows x 64 k, 128-byte swizzle);
-//   * warps 2..9 (256 threads): decode the W tile (thread = one weight row and one half of the
-//     64 k: 16 code bytes or one k-bit block) straight into the same swizzled K-major layout;
-//   * warp 1, one thread: four tcgen05.mma (kind::f16, K = 16 each) per stage, then a commit that
-//     frees the stage when the MMAs have read it.
-// Full and empty stages are tracked with mbarriers; every wait is bounded (on expiry it counts a
+// Tiling (weight rows on the MMA's M side): a CTA owns 128 rows of W and NT (16, 32, 64, 128 or
+// 256) activation rows; its accumulator D[128 x NT] (fp32) lives in tensor memory. K advances in
+// 64-wide stages:
+//   * warp 0, one thread: TMA loads of the X tiles (NT rows x 64 k, 128-byte swizzle) into a ring
+//     of 6-8 shared-memory stages;
+//   * warps 2..17 (512 threads): decode the W tile (thread = one weight row and a quarter of the
+//     64 k: 8 code bytes or half a k-bit block, loaded 4 stages ahead into registers) and write it
+//     straight into tensor memory (tcgen05.st: the row is the thread's lane), a ring of 8 A tiles;
+//     no shared memory and no proxy fence sits between a decoder's loads and the MMA;
+//   * warp 1, one thread: four tcgen05.mma (kind::f16, K = 16 each, A from tensor memory, B from
+//     the swizzled X tile) per stage, then commits that free the X and W slots when the MMAs have
+//     read them.
+// Full and empty slots are tracked with mbarriers; every wait is bounded (on expiry it counts a
 // timeout, see bbc_wait_timeouts, and the kernel winds down instead of hanging).
 //
 // Split K over a thread-block cluster: with few output tiles the S CTAs of a cluster (S <= 8)
@@ -27,6 +31,7 @@
 
 #include <atomic>
 #include <mutex>
+#include <type_traits>
 
 #include "common.cuh"
 #include "launch.h"
@@ -40,11 +45,11 @@ namespace {
 
 constexpr int kTcRows = 128;              // weight rows per CTA (the MMA's M)
 constexpr int kTcBK = 64;                 // k per stage: one 128-byte swizzle row of 16-bit values
-constexpr int kTcStages = 4;
-constexpr int kTcDecoders = 256;          // warps 2..9
+constexpr int kTcDecoders = 512;          // warps 2..17
 constexpr int kTcThreads = 64 + kTcDecoders;
-constexpr int kTcWTile = kTcRows * kTcBK * 2;      // 16 KB
-constexpr uint32_t kWaitLimit = 1u << 20;          // try_wait rounds before a wait gives up
+constexpr uint32_t kWaitRoundNs = 100000;          // suspend-time hint of one try_wait round (100 us)
+constexpr uint32_t kWaitLimit = 1u << 13;          // rounds before a wait gives up
+constexpr int kPrefetch = 4;                       // stages of decoder inputs loaded ahead
 
 // ---- mbarriers ----
 
@@ -57,14 +62,16 @@ __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
 __device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
     asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" :: "r"(bar), "r"(bytes) : "memory");
 }
+// One round of waiting: the thread is suspended until the phase completes or kWaitRoundNs pass
+// (it does not spin, so waiting roles take no issue slots from the decoders).
 __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
     uint32_t ok;
-    asm volatile("{ .reg .pred p; mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2; selp.u32 %0, 1, 0, p; }"
-                 : "=r"(ok) : "r"(bar), "r"(parity) : "memory");
+    asm volatile("{ .reg .pred p; mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3; selp.u32 %0, 1, 0, p; }"
+                 : "=r"(ok) : "r"(bar), "r"(parity), "r"(kWaitRoundNs) : "memory");
     return ok != 0;
 }
 // Waits for the phase of `bar` with the given parity; false (and one timeout counted) if it did
-// not complete within kWaitLimit rounds.
+// not complete within kWaitLimit rounds (about a second).
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
     for (uint32_t i = 0; i < kWaitLimit; i++)
         if (mbar_try_wait(bar, parity)) return true;
@@ -99,14 +106,27 @@ __device__ __forceinline__ void mma_f16(uint32_t tmem_d, uint64_t a, uint64_t b,
                  "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p; }"
                  :: "r"(tmem_d), "l"(a), "l"(b), "r"(idesc), "r"(acc) : "memory");
 }
+// The same with A in tensor memory (lane = row of A, 32-bit column c = elements 2c, 2c + 1 of the
+// row's K slice, element 2c in the low half).
+__device__ __forceinline__ void mma_f16_ta(uint32_t tmem_d, uint32_t tmem_a, uint64_t b, uint32_t idesc, uint32_t acc) {
+    asm volatile("{ .reg .pred p; setp.ne.b32 p, %4, 0;\n"
+                 "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p; }"
+                 :: "r"(tmem_d), "r"(tmem_a), "l"(b), "r"(idesc), "r"(acc) : "memory");
+}
+// Eight consecutive 32-bit columns of this thread's tensor-memory lane, from registers
+// (asynchronous: tmem_wait_st waits for this thread's stores to complete).
+__device__ __forceinline__ void tmem_st8(uint32_t addr, const uint32_t (&v)[8]) {
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};"
+                 :: "r"(addr), "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7])
+                 : "memory");
+}
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 // Arrives on `bar` once every tcgen05.mma this thread issued before has completed.
 __device__ __forceinline__ void mma_commit(uint32_t bar) {
     asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" :: "r"(bar) : "memory");
 }
 __device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
 __device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
-// Generic-proxy writes to shared memory made visible to the tensor cores (async proxy).
-__device__ __forceinline__ void fence_async_smem() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
 
 // 16 consecutive fp32 accumulator columns of this thread's tensor-memory lane.
 __device__ __forceinline__ void tmem_ld16(uint32_t addr, float (&v)[16]) {
@@ -155,68 +175,86 @@ struct KbitW {
     const float* codebook;
 };
 
-// Byte address, in a K-major 128-byte-swizzled tile (rows of 128 bytes, 8-row atoms of 1024
-// bytes), of 16-byte chunk c (k 8c .. 8c + 7) of row r: chunk c of row r sits at position
-// c ^ (r mod 8) of its row. The 8 rows of a 16-byte store phase (consecutive r, same c) hit 8
-// different chunk positions: no bank conflicts.
-__device__ __forceinline__ uint32_t sw128_chunk(uint32_t tile, int r, int c) {
-    return tile + (uint32_t)((r >> 3) * 1024 + (r & 7) * 128 + ((c ^ (r & 7)) << 4));
-}
-
-__device__ __forceinline__ void sts128(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
-    asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" :: "r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
-}
-
 template <int DT>
 __device__ __forceinline__ uint32_t pack2(float lo, float hi) {
     return DT == BF16 ? pack_bf16x2(lo, hi) : pack_f16x2(lo, hi);
 }
 
-// The 32 weights m0 .. m0 + 31 of a nested 4-bit row (m0 a multiple of 32, so they share one
-// outer block) as 16 packed pairs of T: one 16-byte code load, one scale
-// fl(fl(code2[q] * absmax2) + offset), then per code byte the pair (code4[hi], code4[lo]) times the
-// scale (one paired multiply) and one paired conversion. c4s holds code4 in shared memory (16
-// entries in 16 banks: lanes never conflict).
-template <int DT>
-__device__ __forceinline__ void decode_nested32(const NestedW& w, int64_t m0, const float* c2s, const float* c4s,
-                                                uint32_t (&out)[16]) {
-    const uint4 c = __ldg(reinterpret_cast<const uint4*>(w.codes + (m0 >> 1)));
+// The inputs of the 16 weights m0 .. m0 + 15 of a nested 4-bit row (m0 a multiple of 16, so they
+// share one outer block b): 8 code bytes, the General8 code of b and the inner absmax of b.
+// Loaded several stages ahead of their use (the decoder's prefetch ring).
+struct NestedIn {
+    uint2 c;
+    uint32_t q;
+    float a2;
+};
+__device__ __forceinline__ NestedIn load_nested16(const NestedW& w, int64_t m0) {
+    NestedIn r;
+    r.c = __ldg(reinterpret_cast<const uint2*>(w.codes + (m0 >> 1)));
     const int64_t b = m0 >> w.log2_bs;
-    const float s = __fadd_rn(__fmul_rn(c2s[__ldg(w.absmax_q + b)], __ldg(w.absmax2 + (b >> 8))), w.offset);
+    r.q = __ldg(w.absmax_q + b);
+    r.a2 = __ldg(w.absmax2 + (b >> 8));
+    return r;
+}
+
+// The decode table: entry (byte, r) = (code4[byte >> 4], code4[byte & 15]) at byte offset
+// byte * 128 + r * 8, 16 interleaved replicas: the 16 lanes of an 8-byte shared-load phase read
+// replica lane & 15, so they never conflict.
+constexpr int kPairBytes = 256 * 16 * 8;           // 32 KB
+
+// Those 16 weights as 8 packed pairs of T: the scale fl(fl(code2[q] * absmax2) + offset), then per
+// code byte one table read of (code4[hi], code4[lo]) (its address: the byte moved to bits 7..14 or-ed
+// with the lane's replica), times the scale (one paired multiply), one paired conversion.
+template <int DT>
+__device__ __forceinline__ void decode_nested16(const NestedIn& in, float offset, const float* c2s,
+                                                const unsigned char* pairs, uint32_t lane_off, uint32_t (&out)[8]) {
+    const float s = __fadd_rn(__fmul_rn(c2s[in.q], in.a2), offset);
     const float2 s2 = make_float2(s, s);
-    const uint32_t words[4] = {c.x, c.y, c.z, c.w};
+    const uint32_t words[2] = {in.c.x, in.c.y};
 #pragma unroll
-    for (int i = 0; i < 4; i++)
+    for (int i = 0; i < 2; i++)
 #pragma unroll
         for (int j = 0; j < 4; j++) {
-            const uint32_t hi = (words[i] >> (8 * j + 4)) & 15u, lo = (words[i] >> (8 * j)) & 15u;
-            const float2 p = __fmul2_rn(make_float2(c4s[hi], c4s[lo]), s2);
+            const uint32_t sel = (j == 0 ? (words[i] << 7) : (words[i] >> (8 * j - 7))) & 0x7f80u;
+            const float2 p = __fmul2_rn(*reinterpret_cast<const float2*>(pairs + (sel | lane_off)), s2);
             out[4 * i + j] = pack2<DT>(p.x, p.y);
         }
 }
 
-// The 32 weights of k-bit block b as 16 packed pairs of T (elements 2i, 2i + 1 in word i): the
-// block's K plane words transposed into four plane groups, each index gathered by one
-// multiply-high (plane_offset4), the codebook entry (cbb, shared) times the absmax.
-template <int DT, int KB>
-__device__ __forceinline__ void decode_kbit32(const KbitW& w, int64_t b, const char* cbb, uint32_t (&out)[16]) {
-    uint32_t wd[KB];
+// The inputs of the 32 weights of k-bit block b: its K plane words and its absmax.
+template <int KB>
+struct KbitIn {
+    uint32_t w[KB];
+    float am;
+};
+template <int KB>
+__device__ __forceinline__ KbitIn<KB> load_kbit32(const KbitW& w, int64_t b) {
+    KbitIn<KB> r;
     const uint32_t* p = w.packed + b * KB;
     if constexpr (KB == 4) {
         const uint4 v = __ldg(reinterpret_cast<const uint4*>(p));
-        wd[0] = v.x; wd[1 % KB] = v.y; wd[2 % KB] = v.z; wd[3 % KB] = v.w;
+        r.w[0] = v.x; r.w[1 % KB] = v.y; r.w[2 % KB] = v.z; r.w[3 % KB] = v.w;
     } else if constexpr (KB == 2) {
         const uint2 v = __ldg(reinterpret_cast<const uint2*>(p));
-        wd[0] = v.x; wd[1 % KB] = v.y;
+        r.w[0] = v.x; r.w[1 % KB] = v.y;
     } else {
 #pragma unroll
-        for (int j = 0; j < KB; j++) wd[j] = __ldg(p + j);
+        for (int j = 0; j < KB; j++) r.w[j] = __ldg(p + j);
     }
-    const float am = __ldg(w.absmax + b);
-    uint32_t G[4], p4;
-    kbit_groups<KB, 32>(wd, 0, G, p4);
+    r.am = __ldg(w.absmax + b);
+    return r;
+}
+
+// Half hb of those 32 weights (elements 16 hb .. 16 hb + 15) as 8 packed pairs of T (elements 2i,
+// 2i + 1 in word i): the K plane words transposed into the half's two plane groups, each index
+// gathered by one multiply-high (plane_offset4), the codebook entry (cbb, shared) times the absmax.
+template <int DT, int KB>
+__device__ __forceinline__ void decode_kbit16(const KbitIn<KB>& in, int hb, const char* cbb, uint32_t (&out)[8]) {
+    uint32_t G[2], p4;
+    kbit_groups<KB, 16>(in.w, hb, G, p4);
+    const float am = in.am;
 #pragma unroll
-    for (int q = 0; q < 4; q++) {
+    for (int q = 0; q < 2; q++) {
         const uint32_t B = G[q], Bs = B << 3, P = p4 >> (8 * q);
         out[4 * q + 0] = pack2<DT>(kbit_elem<KB, DT, 0>(B, Bs, P, am, cbb), kbit_elem<KB, DT, 1>(B, Bs, P, am, cbb));
         out[4 * q + 1] = pack2<DT>(kbit_elem<KB, DT, 2>(B, Bs, P, am, cbb), kbit_elem<KB, DT, 3>(B, Bs, P, am, cbb));
@@ -234,24 +272,42 @@ __device__ __forceinline__ bool warp_wait(uint32_t bar, uint32_t parity) {
     return false;
 }
 
+__device__ __forceinline__ void st_cluster_v4(uint32_t addr, float a, float b, float c, float d) {
+    asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" :: "r"(addr), "f"(a), "f"(b), "f"(c), "f"(d)
+                 : "memory");
+}
 __device__ __forceinline__ void st_cluster_f32(uint32_t addr, float v) {
     asm volatile("st.shared::cluster.f32 [%0], %1;" :: "r"(addr), "f"(v) : "memory");
 }
 
-// Shared memory of a CTA (dynamic, rounded up to a 1024-byte boundary for the swizzle atoms):
-// kTcStages stages of {W tile 16 KB, X tile NT x 128 bytes}, then the mbarriers, the tensor-memory
-// address and the tables. After the main loop the stage area holds the split-K receive buffer.
+// Tensor memory of a CTA (512 columns): the accumulator D[128 x NT] in columns 0 .. NT-1, and a ring
+// of kTcWStages = 8 decoded weight tiles (A operands: 128 rows x 64 k of 16-bit values = 32 columns
+// each) in columns 256 .. 511.
+constexpr int kTmemCols = 512;
+constexpr int kTmemA = 256;
+constexpr int kTcWStages = 8;
+
+// Shared memory of a CTA (dynamic, rounded up to a 1024-byte boundary for the swizzle atoms): a
+// ring of kXStages X tiles (NT rows x 128 bytes), the nested decode table, then the mbarriers, the
+// tensor-memory address and the other tables. After the main loop the X area holds the split-K receive buffer.
 template <int NT>
 struct TcSmem {
-    static constexpr int kXTile = NT * 128;
-    static constexpr int kStage = kTcWTile + kXTile;              // a multiple of 1024
-    static constexpr int kBars = kTcStages * kStage;             // x_full[4], w_full[4], empty[4], acc_full
-    static constexpr int kTmemSlot = kBars + 13 * 8;
-    static constexpr int kTables = kBars + 128;                  // code2 (256 floats), code4 / codebook (32)
+    static constexpr int kXTile = NT * 128;                       // a multiple of 1024 for NT >= 8
+    static constexpr int kXStages = NT >= 256 ? 6 : 8;
+    static constexpr int kPairs = kXStages * kXTile;             // the 32 KB decode table (nested weights)
+    static constexpr int kBars = kPairs + kPairBytes;            // x_full, x_empty, w_full, w_empty, acc_full
+    static constexpr int kNumBars = 2 * kXStages + 2 * kTcWStages + 1;   // at most 33
+    static constexpr int kTmemSlot = kBars + 272;
+    static constexpr int kTables = kBars + 288;                  // code2 (256 floats), code4 / codebook (32)
+    static_assert(kNumBars * 8 <= 272, "barriers before the tensor-memory slot");
     static constexpr int kBytes = kTables + (256 + 32) * 4;
     static constexpr int kAlloc = kBytes + 1024;                  // with the alignment slack
-    static_assert(kStage % 1024 == 0, "stages start on swizzle-atom boundaries");
-    static_assert(NT * kTcRows * 4 <= kTcStages * kStage, "the receive buffer fits in the stage area");
+    static_assert(kXTile % 1024 == 0, "X tiles start on swizzle-atom boundaries");
+    // the split-K receive buffer, S x 128 rows x (NT / S + 4) floats at most (S <= 8)
+    static constexpr int kRecvMax = kTcRows * 4 * (NT + 4 * 8);
+    // (below NT = 64 the bound is loose: W < 16 needs no padding, so S x 128 x W x 4 = 512 NT bytes)
+    static_assert(kRecvMax <= kXStages * kXTile || NT * kTcRows * 4 <= kXStages * kXTile, "receive buffer fits");
+    static_assert(kTables % 16 == 0, "tables aligned");
 };
 
 template <int DT, int NT, bool NESTED, int KB>
@@ -259,14 +315,16 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 linear_tc_kernel(const __grid_constant__ CUtensorMap tmx, int M, int64_t N, int64_t K, NestedW nw, KbitW kw,
                  uint16_t* __restrict__ Y) {
     using L = TcSmem<NT>;
+    constexpr int XS = L::kXStages, WS = kTcWStages;
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = (uint32_t)__cvta_generic_to_shared(smem_raw);
     const uint32_t base = (raw + 1023u) & ~1023u;
     uint8_t* const base_p = smem_raw + (base - raw);
     auto x_full = [&](int s) { return base + L::kBars + 8u * s; };
-    auto w_full = [&](int s) { return base + L::kBars + 32u + 8u * s; };
-    auto empty = [&](int s) { return base + L::kBars + 64u + 8u * s; };
-    const uint32_t acc_full = base + L::kBars + 96u;
+    auto x_empty = [&](int s) { return base + L::kBars + 8u * (XS + s); };
+    auto w_full = [&](int s) { return base + L::kBars + 8u * (2 * XS + s); };
+    auto w_empty = [&](int s) { return base + L::kBars + 8u * (2 * XS + WS + s); };
+    const uint32_t acc_full = base + L::kBars + 8u * (2 * XS + 2 * WS);
     float* const c2s = reinterpret_cast<float*>(base_p + L::kTables);
     float* const c4s = c2s + 256;
 
@@ -280,23 +338,36 @@ linear_tc_kernel(const __grid_constant__ CUtensorMap tmx, int M, int64_t N, int6
     const int nchunks = (int)(C * (rank + 1) / S - c_lo);
 
     // ---- set-up: tables, barriers, tensor memory ----
-    if (NESTED)
+    unsigned char* const pairs = base_p + L::kPairs;
+    if (NESTED) {
         for (int i = threadIdx.x; i < 256; i += kTcThreads) c2s[i] = nw.code2[i];
+        if (threadIdx.x < 256) {
+            // thread i writes the 16 replicas of entry i as 8 rotated 16-byte stores
+            const int byte = threadIdx.x;
+            const float hi = nw.code4[byte >> 4], lo = nw.code4[byte & 15];
+            const float4 v = make_float4(hi, lo, hi, lo);
+#pragma unroll
+            for (int r = 0; r < 8; r++) *reinterpret_cast<float4*>(pairs + byte * 128 + ((r + byte) & 7) * 16) = v;
+        }
+    }
     if (threadIdx.x < 32)
         c4s[threadIdx.x] = NESTED ? (threadIdx.x < 16 ? nw.code4[threadIdx.x] : 0.0f)
                                   : (threadIdx.x < (1 << KB) ? kw.codebook[threadIdx.x] : 0.0f);
     if (threadIdx.x == 0) {
-        for (int s = 0; s < kTcStages; s++) {
+        for (int s = 0; s < XS; s++) {
             mbar_init(x_full(s), 1);                        // the TMA thread's arrive (+ the bytes)
+            mbar_init(x_empty(s), 1);                       // the MMA thread's commit
+        }
+        for (int s = 0; s < WS; s++) {
             mbar_init(w_full(s), kTcDecoders / 32);         // one arrive per decoder warp
-            mbar_init(empty(s), 1);                         // the MMA thread's commit
+            mbar_init(w_empty(s), 1);                       // the MMA thread's commit
         }
         mbar_init(acc_full, 1);
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     if (warp == 1) {
         asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
-                     :: "r"(base + (uint32_t)L::kTmemSlot), "r"((uint32_t)NT) : "memory");
+                     :: "r"(base + (uint32_t)L::kTmemSlot), "r"((uint32_t)kTmemCols) : "memory");
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
     }
     __syncthreads();
@@ -309,59 +380,93 @@ linear_tc_kernel(const __grid_constant__ CUtensorMap tmx, int M, int64_t N, int6
             asm volatile("prefetch.tensormap [%0];" :: "l"(reinterpret_cast<uint64_t>(&tmx)) : "memory");
             int issued = 0;
             for (int i = 0; i < nchunks; i++) {
-                const int s = i % kTcStages, r = i / kTcStages;
-                if (r > 0 && !mbar_wait(empty(s), (r & 1) ^ 1)) break;
+                const int s = i % XS, r = i / XS;
+                if (r > 0 && !mbar_wait(x_empty(s), (r & 1) ^ 1)) break;
                 mbar_arrive_expect_tx(x_full(s), L::kXTile);
-                tma_load_2d(base + s * L::kStage + kTcWTile, &tmx, (int)((c_lo + i) * kTcBK), m_tile0, x_full(s));
+                tma_load_2d(base + s * L::kXTile, &tmx, (int)((c_lo + i) * kTcBK), m_tile0, x_full(s));
                 issued = i + 1;
             }
             // the last loads in flight have landed before the CTA moves on (bounded)
-            for (int i = issued > kTcStages ? issued - kTcStages : 0; i < issued; i++)
-                mbar_wait(x_full(i % kTcStages), (i / kTcStages) & 1);
+            for (int i = issued > XS ? issued - XS : 0; i < issued; i++) mbar_wait(x_full(i % XS), (i / XS) & 1);
         }
     } else if (warp == 1) {
-        // ---- the MMAs: D[128 x NT] += W[128 x 64] X[NT x 64]^T per stage ----
+        // ---- the MMAs: D[128 x NT] += W[128 x 64] X[NT x 64]^T per stage, W from tensor memory ----
         if (lane == 0) {
             constexpr uint32_t idesc = mma_idesc(DT == BF16 ? 1 : 0, NT);
             for (int i = 0; i < nchunks; i++) {
-                const int s = i % kTcStages, r = i / kTcStages;
-                if (!mbar_wait(x_full(s), r & 1) || !mbar_wait(w_full(s), r & 1)) break;
+                const int sx = i % XS, rx = i / XS, sw = i % WS, rw = i / WS;
+                if (!mbar_wait(x_full(sx), rx & 1) || !mbar_wait(w_full(sw), rw & 1)) break;
                 tc_fence_after();
-                const uint32_t wa = base + s * L::kStage, xa = wa + kTcWTile;
+                const uint32_t xa = base + sx * L::kXTile, wa = tmem + kTmemA + 32u * sw;
 #pragma unroll
                 for (int kk = 0; kk < kTcBK / 16; kk++)
-                    mma_f16(tmem, smem_desc_sw128(wa + 32 * kk), smem_desc_sw128(xa + 32 * kk), idesc,
-                            (i > 0 || kk > 0) ? 1u : 0u);
-                mma_commit(empty(s));
+                    mma_f16_ta(tmem, wa + 8u * kk, smem_desc_sw128(xa + 32 * kk), idesc, (i > 0 || kk > 0) ? 1u : 0u);
+                mma_commit(x_empty(sx));
+                mma_commit(w_empty(sw));
             }
             mma_commit(acc_full);          // once every MMA issued above has completed
         }
     } else {
-        // ---- W tiles decoded into shared memory ----
-        const int row = 32 * (warp & 3) + lane;                   // also this warp's tensor-memory lane
-        const int h = (warp - 2) >> 2;                            // which 32 of a stage's 64 k
+        // ---- W tiles decoded into tensor memory ----
+        // Thread: one weight row (its tensor-memory lane) and one quarter (16 k) of a stage's 64 k,
+        // i.e. 8 of the stage's 32 A columns. Its inputs are loaded kPrefetch stages ahead of their
+        // decode (a register ring); no shared memory and no proxy fence is involved.
+        const int row = 32 * (warp & 3) + lane;
+        const int qk = (warp - 2) >> 2;                           // which 16 of a stage's 64 k
         const int64_t n = n0 + row;
-        for (int i = 0; i < nchunks; i++) {
-            const int s = i % kTcStages, r = i / kTcStages;
-            if (r > 0 && !warp_wait(empty(s), (r & 1) ^ 1)) break;
-            const int64_t m0 = n * K + (c_lo + i) * kTcBK + 32 * h;
-            uint32_t v[16];
-            if constexpr (NESTED) decode_nested32<DT>(nw, m0, c2s, c4s, v);
-            else decode_kbit32<DT, KB>(kw, m0 >> 5, reinterpret_cast<const char*>(c4s), v);
-            const uint32_t tile = base + s * L::kStage;
+        const int64_t mrow = n * K + c_lo * kTcBK + 16 * qk;      // first weight of this thread's stage 0
+        const uint32_t lane_a = tmem + ((uint32_t)(32 * (warp & 3)) << 16) + kTmemA + 8u * qk;
+        using In = std::conditional_t<NESTED, NestedIn, KbitIn<KB>>;
+        auto load_in = [&](int i) -> In {
+            const int64_t m0 = mrow + (int64_t)i * kTcBK;
+            if constexpr (NESTED) return load_nested16(nw, m0);
+            else return load_kbit32<KB>(kw, m0 >> 5);
+        };
+        In pre[kPrefetch];
 #pragma unroll
-            for (int c = 0; c < 4; c++)
-                sts128(sw128_chunk(tile, row, 4 * h + c), v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
-            fence_async_smem();
+        for (int j = 0; j < kPrefetch; j++)
+            if (j < nchunks) pre[j] = load_in(j);
+        const uint32_t lane_off = (uint32_t)(lane & 15) * 8u;
+        bool live = true;
+        int done_to = 0;                                          // stages whose stores were issued
+        for (int i0 = 0; i0 < nchunks && live; i0 += kPrefetch) {
+#pragma unroll
+            for (int j = 0; j < kPrefetch; j++) {
+                const int i = i0 + j;
+                if (i >= nchunks) break;
+                const int s = i % WS, r = i / WS;
+                if (r > 0 && !warp_wait(w_empty(s), (r & 1) ^ 1)) {
+                    live = false;
+                    break;
+                }
+                uint32_t v[8];
+                if constexpr (NESTED) decode_nested16<DT>(pre[j], nw.offset, c2s, pairs, lane_off, v);
+                else decode_kbit16<DT, KB>(pre[j], qk & 1, reinterpret_cast<const char*>(c4s), v);
+                if (i + kPrefetch < nchunks) pre[j] = load_in(i + kPrefetch);
+                // the previous stage's tensor-memory stores completed while this one was decoded:
+                // signal it now, then start this stage's stores
+                if (i > 0) {
+                    tmem_wait_st();
+                    tc_fence_before();
+                    __syncwarp();
+                    if (lane == 0) mbar_arrive(w_full((i - 1) % WS));
+                }
+                tmem_st8(lane_a + 32u * s, v);
+                done_to = i + 1;
+            }
+        }
+        if (done_to > 0) {
+            tmem_wait_st();
+            tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(w_full(s));
+            if (lane == 0) mbar_arrive(w_full((done_to - 1) % WS));
         }
     }
 
     // ---- epilogue (decoder warps): accumulator -> Y, summed over the cluster for split K ----
     const bool epi = warp >= 2;
     const int row = 32 * (warp & 3) + lane;
-    const int g = (warp - 2) >> 2;                                // which half of the columns
+    const int g = (warp - 2) >> 2;                                // which of four column groups
     const int64_t n = n0 + row;
     const uint32_t lane_tmem = tmem + ((uint32_t)(32 * (warp & 3)) << 16);
     auto store = [&](int col, float v) {
@@ -374,40 +479,53 @@ linear_tc_kernel(const __grid_constant__ CUtensorMap tmx, int M, int64_t N, int6
     }
     if (S == 1) {
         if (epi)
-            for (int c = g * (NT / 2); c < (g + 1) * (NT / 2); c += 16) {
+            for (int c = 16 * g; c < NT; c += 64) {                // 16-column chunks, rotating groups
                 float v[16];
                 tmem_ld16(lane_tmem + c, v);
 #pragma unroll
                 for (int i = 0; i < 16; i++) store(c + i, v[i]);
             }
     } else {
-        // receive buffer of this CTA: [S][W][128] floats, partial of rank s for owned column c at
-        // [s][c - rank * W][row]
-        const int W = NT / (int)S;
+        // CTA `rank` owns columns [rank W, rank W + W) (W = NT / S >= 2); its receive buffer holds the
+        // partial of rank s for owned column c at [s][row][c - rank W], rows WP floats apart (WP = W + 4
+        // when W >= 16: 16-byte accesses of 8 consecutive rows then hit different banks)
+        const int W = NT / (int)S, own0 = (int)rank * W, WP = W >= 16 ? W + 4 : W;
         cluster_sync();                                           // every CTA is past its main loop
         if (epi)
-            for (int c = g * (NT / 2); c < (g + 1) * (NT / 2); c += 16) {
-                const uint32_t owner = (uint32_t)(c / W);
-                if (owner == rank) continue;
+            for (int c = 16 * g; c < NT; c += 64) {
+                if (c >= own0 && c + 16 <= own0 + W) continue;    // all of this chunk stays here
                 float v[16];
                 tmem_ld16(lane_tmem + c, v);
-                const uint32_t dst = map_to_rank(base, owner);
+                if (W >= 16) {                                    // the chunk has one owner: 16-byte stores
+                    const int owner = c / W;
+                    const uint32_t dst = map_to_rank(base, (uint32_t)owner) +
+                                         (uint32_t)((((int)rank * kTcRows + row) * WP + (c - owner * W)) * 4);
 #pragma unroll
-                for (int i = 0; i < 16; i++)
-                    st_cluster_f32(dst + (uint32_t)(((rank * W + (c - (int)owner * W) + i) * kTcRows + row) * 4), v[i]);
+                    for (int i = 0; i < 16; i += 4) st_cluster_v4(dst + 4u * i, v[i], v[i + 1], v[i + 2], v[i + 3]);
+                } else {
+#pragma unroll
+                    for (int i = 0; i < 16; i++) {
+                        const int owner = (c + i) / W;
+                        if (owner == (int)rank) continue;
+                        const uint32_t dst = map_to_rank(base, (uint32_t)owner);
+                        st_cluster_f32(dst + (uint32_t)((((int)rank * kTcRows + row) * WP + (c + i - owner * W)) * 4),
+                                       v[i]);
+                    }
+                }
             }
         cluster_sync();                                           // every partial has arrived
         if (epi) {
             const float* recv = reinterpret_cast<const float*>(base_p);
-            for (int c = (int)rank * W + g * (W / 2); c < (int)rank * W + (g + 1) * (W / 2); c += 16) {
+            for (int c = (own0 & ~15) + 16 * g; c < own0 + W; c += 64) {
                 float v[16];
                 tmem_ld16(lane_tmem + c, v);
 #pragma unroll
                 for (int i = 0; i < 16; i++) {
-                    const int cl = c - (int)rank * W + i;
-                    float acc = rank == 0 ? v[i] : recv[(0 * W + cl) * kTcRows + row];
+                    const int cl = c + i - own0;
+                    if (cl < 0 || cl >= W) continue;
+                    float acc = rank == 0 ? v[i] : recv[row * WP + cl];
                     for (uint32_t s = 1; s < S; s++)
-                        acc = __fadd_rn(acc, s == rank ? v[i] : recv[((int)s * W + cl) * kTcRows + row]);
+                        acc = __fadd_rn(acc, s == rank ? v[i] : recv[((int)s * kTcRows + row) * WP + cl]);
                     store(c + i, acc);
                 }
             }
@@ -416,7 +534,8 @@ linear_tc_kernel(const __grid_constant__ CUtensorMap tmx, int M, int64_t N, int6
     tc_fence_before();
     __syncthreads();
     if (warp == 1)
-        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" :: "r"(tmem), "r"((uint32_t)NT) : "memory");
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" :: "r"(tmem), "r"((uint32_t)kTmemCols)
+                     : "memory");
 }
 
 // ---- host side ----
@@ -443,12 +562,12 @@ EncodeTiled tensor_map_encoder(cudaError_t* err) {
 
 // Split factor S (a cluster of S CTAs shares an output tile along K): the S in {1, 2, 4, 8} that
 // fills the machine best (output tiles x S CTAs over waves of `cap` resident CTAs), with at least
-// 32 accumulator columns and two K stages per CTA; a larger S only when it is 5 % better.
-int pick_split(int64_t tiles, int cap, int nt, int64_t stages_k) {
+// two K stages per CTA; a larger S only when it is 5 % better.
+int pick_split(int64_t tiles, int cap, int64_t stages_k) {
     int best = 1;
     double best_eff = 0.0;
     for (int S = 1; S <= 8; S *= 2) {
-        if (S > nt / 32 || stages_k < 2 * S) break;
+        if (stages_k < 2 * S) break;
         const int64_t ctas = tiles * S;
         const int64_t waves = (ctas + cap - 1) / cap;
         const double eff = (double)ctas / (double)(waves * cap);
@@ -485,7 +604,7 @@ cudaError_t launch_tc(const uint16_t* X, int M, int64_t N, int64_t K, const Nest
     const int64_t mtiles = (M + NT - 1) / NT, ntiles = N / kTcRows;
     const int cap = resident_ctas(reinterpret_cast<const void*>(k), kTcThreads, L::kAlloc);
     if (cap < 1) return cudaErrorInvalidConfiguration;
-    const int S = pick_split(ntiles * mtiles, cap, NT, K / kTcBK);
+    const int S = pick_split(ntiles * mtiles, cap, K / kTcBK);
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)S, (unsigned)ntiles, (unsigned)mtiles);
     cfg.blockDim = dim3(kTcThreads);
@@ -504,6 +623,8 @@ cudaError_t launch_tc(const uint16_t* X, int M, int64_t N, int64_t K, const Nest
 template <int DT, bool NESTED, int KB>
 cudaError_t launch_tc_nt(const uint16_t* X, int M, int64_t N, int64_t K, const NestedW& nw, const KbitW& kw,
                          uint16_t* Y, cudaStream_t s) {
+    if (M <= 16) return launch_tc<DT, 16, NESTED, KB>(X, M, N, K, nw, kw, Y, s);
+    if (M <= 32) return launch_tc<DT, 32, NESTED, KB>(X, M, N, K, nw, kw, Y, s);
     if (M <= 64) return launch_tc<DT, 64, NESTED, KB>(X, M, N, K, nw, kw, Y, s);
     if (M <= 128) return launch_tc<DT, 128, NESTED, KB>(X, M, N, K, nw, kw, Y, s);
     return launch_tc<DT, 256, NESTED, KB>(X, M, N, K, nw, kw, Y, s);
