@@ -12,7 +12,8 @@
 //      lanes by xor-shuffles and warps in shared memory computes exactly the nodes of that
 //      tree; each level of 2048 nodes is one launch.
 //   3. per group of 256 outer blocks, c_b = fl(absmax_b - offset): absmax2 = max |c_b| and
-//      absmax_q_b = the first nearest General8 entry to fl(c_b / fmaxf(absmax2, 1e-8f))
+//      absmax_q_b = the first nearest General8 entry to fl(c_b / fmaxf(absmax2, 1e-8f)) (the
+//      quotient correctly rounded from one reciprocal per group and Markstein's correction)
 //      (absmax_compress_kernel). For an ascending table the nearest entry is found exactly from
 //      p = the last index with t_p <= xn: fl(|xn - t_i|) does not increase up to t_p and does
 //      not decrease after it, so the minimum is at t_p or t_{p+1} and the first index holding
@@ -90,6 +91,7 @@ template <typename T>
 __global__ void __launch_bounds__(256)
 tree_sum_kernel(const T* __restrict__ in, int64_t count, int64_t nnodes, double* __restrict__ nodes) {
     __shared__ double ws[kNodesPerCta][8];
+    pdl_wait();               // the values come from the launch just before this one
     double s[kNodesPerCta];
 #pragma unroll
     for (int k = 0; k < kNodesPerCta; k++)
@@ -239,6 +241,10 @@ absmax_compress_kernel(const float* __restrict__ absmax, int64_t nbo, const T* _
     }
     // the barrier also makes the replicas and the bucket table visible
     const bool ascending = __syncthreads_and(v <= next);        // false if any entry is NaN
+    // Everything above reads only the General8 table, an input written before the quantize's
+    // first launch; the outer absmax and the tree nodes below come from the launches just before
+    // this one (programmatic dependent launch: this set-up overlaps their end).
+    pdl_wait();
     const float* t = tr + (threadIdx.x & (kRep - 1));
     // the offset: the root of the pairwise tree over the last level (<= 2048 values), the
     // same in every CTA; CTA 0 stores it
@@ -265,11 +271,18 @@ absmax_compress_kernel(const float* __restrict__ absmax, int64_t nbo, const T* _
         for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
         if (lane == 0) absmax2[g] = m;
         const float d = fmaxf(m, 1e-8f);
+        // xn = RN(c / d) from the correctly rounded reciprocal y: q0 = RN(c y), r = c - d q0 (exact
+        // by the fma), xn = RN(q0 + r y) is the correctly rounded quotient by Markstein's theorem
+        // (y within half an ulp of 1/d, q0 within one ulp of c / d, no underflow); zero, tiny and
+        // NaN quotients take the IEEE division instead
+        const float y = __frcp_rn(d);
 #pragma unroll
         for (int j = 0; j < 8; j++) {
             const int64_t b = g * kGroup + lane + 32 * j;
             if (FULL || b < nbo) {
-                const float xn = __fdiv_rn(cv[j], d);
+                const float q0 = __fmul_rn(cv[j], y);
+                float xn = __fmaf_rn(__fmaf_rn(-d, q0, cv[j]), y, q0);
+                if (!(fabsf(q0) >= 0x1p-100f)) xn = __fdiv_rn(cv[j], d);
                 absmax_q[b] = (uint8_t)(ASC ? nearest_ascending(xn, t, lut) : nearest_any(xn, t));
             }
         }
@@ -314,27 +327,28 @@ cudaError_t launch_quantize_4bit_nested(const void* A, int dtype, int64_t n, int
     const int64_t ngroups = (nbo + kGroup - 1) / kGroup;
     if (nbo <= kTree) {
         const int grid = persistent_grid(absmax_compress_kernel<float>, 256, 0, ngroups, 32);
-        absmax_compress_kernel<float><<<grid, 256, 0, s>>>(absmax, nbo, absmax, nbo, offset, code2, absmax_q,
-                                                           absmax2);
-        return cudaGetLastError();
+        return launch_pdl(absmax_compress_kernel<float>, grid, 256, 0, s, absmax, nbo, absmax, nbo, offset, code2,
+                          absmax_q, absmax2);
     }
     int64_t count = tree_nodes(nbo);
-    tree_sum_kernel<float><<<(unsigned)((count + kNodesPerCta - 1) / kNodesPerCta), 256, 0, s>>>(absmax, nbo, count,
-                                                                                               buf_a);
+    e = launch_pdl(tree_sum_kernel<float>, (unsigned)((count + kNodesPerCta - 1) / kNodesPerCta), 256, 0, s, absmax,
+                   nbo, count, buf_a);
+    if (e != cudaSuccess) return e;
     const double* in = buf_a;
     double* out = buf_b;
     while (count > kTree) {
         const int64_t next = tree_nodes(count);
-        tree_sum_kernel<double><<<(unsigned)((next + kNodesPerCta - 1) / kNodesPerCta), 256, 0, s>>>(in, count, next,
-                                                                                                    out);
+        e = launch_pdl(tree_sum_kernel<double>, (unsigned)((next + kNodesPerCta - 1) / kNodesPerCta), 256, 0, s, in,
+                       count, next, out);
+        if (e != cudaSuccess) return e;
         in = out;
         out = out == buf_b ? buf_a : buf_b;        // a level never outgrows the one before it
         count = next;
     }
     // 32 groups per CTA (4 per warp) amortise the 32 KB table set-up; persistent above that
     const int grid = persistent_grid(absmax_compress_kernel<double>, 256, 0, ngroups, 32);
-    absmax_compress_kernel<double><<<grid, 256, 0, s>>>(absmax, nbo, in, count, offset, code2, absmax_q, absmax2);
-    return cudaGetLastError();
+    return launch_pdl(absmax_compress_kernel<double>, grid, 256, 0, s, absmax, nbo, in, count, offset, code2, absmax_q,
+                      absmax2);
 }
 
 }  // namespace bbc
