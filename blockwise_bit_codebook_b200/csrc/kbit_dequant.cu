@@ -4,17 +4,18 @@
 // kDequantizeBlockwise_kbit): out[m] = T(codebook[idx_m] * absmax[m / 32]),
 // where idx_m is gathered from the K bit-plane words of block m / 32.
 //
-// B200 layout, two forms chosen per launch on the host. Whole blocks (K = 5, the E4M4
-// K = 3 case, and 16-bit outputs below 2^26 elements; all 32-byte aligned): a thread owns a
+// B200 layout, two forms chosen per launch on the host. Whole blocks (16-bit outputs, 32-byte
+// aligned, at K = 5, for the E4M4 K = 3 case and below 2^26 elements): a thread owns a
 // block, reads its absmax and K words once (one vector load when the packed array
 // allows), byte-transposes them with eight permutes into four plane groups (byte j
 // of group q = plane j of elements 8q..8q+7), decodes each 4-bit index with one
 // multiply-high bit gather, and writes 16 outputs per 32-byte store, so every lane
 // writes whole sectors; the next block's words are loaded before the current one is
-// decoded. Half blocks (otherwise: long 16-bit streams and fp32 outputs at K = 2..4;
+// decoded. Half blocks (otherwise: long 16-bit streams and all fp32 outputs;
 // always for the ragged last block and unaligned outputs): 16 elements per thread, the
-// two lanes of a block read the same words and keep bytes 2h, 2h+1. The codebook lives in shared memory: 32 consecutive floats
-// occupy the 32 banks once, so the per-element lookup never conflicts.
+// two lanes of a block read the same words and keep bytes 2h, 2h+1. The codebook lives in
+// shared memory: 32 consecutive floats occupy the 32 banks once, so the per-element lookup
+// never conflicts.
 // Persistent grid-stride loops.
 #include "common.cuh"
 #include "launch.h"
@@ -214,10 +215,11 @@ cudaError_t launch_t(const uint32_t* packed, const AT* absmax, const float* code
     const int64_t nh = ((n + 31) >> 5) * 2;
     // Whole blocks per thread or half blocks (measured, c5 = 268 M bf16 outputs / c2 = 16.8 M):
     // half blocks write 32 contiguous bytes per lane and were faster on long streams (c5, K = 2..4:
-    // +1 to +7 points) and for fp32 outputs (c2: 20 % faster), whole blocks on short 16-bit
-    // streams (c2: 6-20 % faster) and at K = 5 (five words re-read by both lanes of a block) and
-    // for the E4M4 absmax at K = 3.
-    const bool whole = K == 5 || (sizeof(AT) == 1 && K == 3) || (DT != F32 && n < (int64_t(1) << 26));
+    // +1 to +7 points) and for every fp32 output (c2: 20 % faster at K = 2..4, 22 % at K = 5, where
+    // a whole block's 128 output bytes per lane spread one store instruction over 4 KB), whole
+    // blocks for 16-bit outputs on short streams (c2: 6-20 % faster), at K = 5 (five words
+    // re-read by both lanes of a block) and for the E4M4 absmax at K = 3.
+    const bool whole = DT != F32 && (K == 5 || (sizeof(AT) == 1 && K == 3) || n < (int64_t(1) << 26));
     auto k = !vec ? kbit_dequant_kernel<K, DT, false, false, AT>
                   : whole ? kbit_dequant_kernel<K, DT, true, true, AT> : kbit_dequant_kernel<K, DT, true, false, AT>;
     const int grid = persistent_grid(k, kThreads, 0, nh, kThreads);
