@@ -130,6 +130,16 @@ __device__ __forceinline__ float max_nan(float a, float b) {
     return r;
 }
 
+// Ordered 32-bit key of an fp32 value: unsigned comparison of keys is the numeric order of
+// the non-NaN values (-0 just below +0), and consecutive keys are adjacent fp32 values.
+__device__ __forceinline__ uint32_t okey(float f) {
+    const uint32_t b = __float_as_uint(f);
+    return b ^ ((uint32_t)((int32_t)b >> 31) | 0x80000000u);
+}
+__device__ __forceinline__ float okey_f32(uint32_t k) {
+    return __uint_as_float(k ^ ((uint32_t)((int32_t)~k >> 31) | 0x80000000u));
+}
+
 // Byte permute.
 __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
     uint32_t r;

@@ -1,4 +1,4 @@
-// Occupancy cache for persistent grids.
+// Occupancy and SM-count caches for persistent grids.
 #include <cuda_runtime.h>
 
 #include <map>
@@ -31,6 +31,24 @@ int resident_ctas(const void* kernel, int block, size_t dyn_smem) {
     std::lock_guard<std::mutex> lock(mu);
     cache[key] = ctas;
     return ctas;
+}
+
+// Streaming multiprocessors of the current device (0 when the query fails; not cached then).
+int sm_count() {
+    static std::mutex mu;
+    static std::map<int, int> cache;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+    {
+        std::lock_guard<std::mutex> lock(mu);
+        auto it = cache.find(dev);
+        if (it != cache.end()) return it->second;
+    }
+    int sms = 0;
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms < 1) return 0;
+    std::lock_guard<std::mutex> lock(mu);
+    cache[dev] = sms;
+    return sms;
 }
 
 }  // namespace bbc

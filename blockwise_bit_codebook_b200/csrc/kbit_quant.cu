@@ -79,15 +79,6 @@ constexpr int kReplicas8 = 16;           // the 8-byte table: 16 lanes per share
 // the fp32 path spilled and ran 2-10 % slower); the unaligned path keeps three.
 template <int DT, bool VEC> constexpr int kMinCtas = VEC ? 2 : 3;
 
-// Ordered 32-bit key of an fp32 value: unsigned comparison of keys is the numeric order of
-// the non-NaN values (-0 just below +0), and consecutive keys are adjacent fp32 values.
-__device__ __forceinline__ uint32_t okey(float f) {
-    const uint32_t b = __float_as_uint(f);
-    return b ^ ((uint32_t)((int32_t)b >> 31) | 0x80000000u);
-}
-__device__ __forceinline__ float okey_f32(uint32_t k) {
-    return __uint_as_float(k ^ ((uint32_t)((int32_t)~k >> 31) | 0x80000000u));
-}
 // The largest fp32 value below v (v finite and above -FLT_MAX).
 __device__ __forceinline__ float prev_f32(float v) { return okey_f32(okey(v) - 1u); }
 

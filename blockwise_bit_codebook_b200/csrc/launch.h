@@ -46,6 +46,7 @@ inline cudaError_t set_attr_once(Kernel kernel, std::atomic<uint64_t>& done, cud
 // the work needs. The occupancy query runs once per (kernel, device, block, smem) and is
 // cached (grid.cpp); if it fails both return 0 (an empty grid, whose launch then fails).
 int resident_ctas(const void* kernel, int block, size_t dyn_smem);
+int sm_count();
 
 template <typename Kernel>
 inline int persistent_grid(Kernel kernel, int block, size_t dyn_smem, int64_t work_items,

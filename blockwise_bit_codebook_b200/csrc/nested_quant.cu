@@ -14,14 +14,19 @@
 //   3. per group of 256 outer blocks, c_b = fl(absmax_b - offset): absmax2 = max |c_b| and
 //      absmax_q_b = the first nearest General8 entry to fl(c_b / fmaxf(absmax2, 1e-8f)) (the
 //      quotient correctly rounded from one reciprocal per group and Markstein's correction)
-//      (absmax_compress_kernel). For an ascending table the nearest entry is found exactly from
+//      (absmax_compress_kernel). For a strictly ascending table whose neighbouring gaps are
+//      within a factor 2^20 of each other (the fast form; the General8 stand-in and tables built
+//      by decades are) the first nearest entry is the number of switch points D_i <= xn, D_i the
+//      smallest fp32 at which t_i beats t_{i-1} in fp32 distances, found per CTA by bisection
+//      over ordered keys; a bucket table (64 buckets per binade of |xn| from 2^-24 up to 1)
+//      holds per bucket the switch points below it and the first one inside it, so a value
+//      costs one table read and one comparison. Other ascending tables take an exact search:
 //      p = the last index with t_p <= xn: fl(|xn - t_i|) does not increase up to t_p and does
 //      not decrease after it, so the minimum is at t_p or t_{p+1} and the first index holding
-//      it is found by walking down a plateau of equal distances. p itself comes from a table of
-//      its values at the lower ends of 64 buckets per binade of |xn| (from 2^-24 up to 1) and a
-//      forward scan inside the bucket; comparisons t_p <= xn are exact, so this is the same p a
-//      search over all entries gives. Any other table takes the rule verbatim over all 256
-//      entries.
+//      it is found by walking down a plateau of equal distances; p comes from the same buckets
+//      holding the entries and a forward scan (comparisons t_p <= xn are exact). Any other table
+//      takes the rule verbatim over all 256 entries.
+#include <algorithm>
 #include <cfloat>
 #include <type_traits>
 
@@ -91,6 +96,8 @@ template <typename T>
 __global__ void __launch_bounds__(256)
 tree_sum_kernel(const T* __restrict__ in, int64_t count, int64_t nnodes, double* __restrict__ nodes) {
     __shared__ double ws[kNodesPerCta][8];
+    // (no early trigger: letting the compression's CTAs in beside these ones to run their table
+    // set-up measured 2-4 us slower at 4.2 M outer blocks)
     pdl_wait();               // the values come from the launch just before this one
     double s[kNodesPerCta];
 #pragma unroll
@@ -131,8 +138,9 @@ constexpr int kLutN = 2 * kLutHalf + 2;                         // 3074 buckets
 // Bucket of a value with |xn| <= 1 (NaN lands anywhere; the caller overrides it).
 __device__ __forceinline__ int lut_bucket(float xn) {
     const uint32_t b = __float_as_uint(xn);
-    const int k = min(max((int)((b & 0x7fffffffu) >> kLutShift) - kLutE0, 0), kLutHalf);
-    return (b >> 31) ? kLutHalf - k : kLutHalf + 1 + k;
+    const int k = min(max((int)((b << 1) >> (kLutShift + 1)) - kLutE0, 0), kLutHalf);
+    // kLutHalf - k for a set sign bit (k ^ -1 = -k - 1), kLutHalf + 1 + k otherwise
+    return kLutHalf + 1 + (k ^ ((int)b >> 31));
 }
 
 // First bucket whose lower point is >= x (kLutN if none), for any float x.
@@ -182,40 +190,115 @@ __device__ __forceinline__ uint32_t nearest_any(float xn, const float* t) {
     return idx;
 }
 
-// One warp per group of 256 outer blocks (8 per lane), persistent over the groups; every CTA
-// first forms the offset from the last level of the tree.
+// Switch point of the exact rule between neighbouring entries a < b of a strictly ascending
+// table: the smallest fp32 xn in (a, b] at which b is strictly nearer, fl(b - xn) < fl(xn - a).
+// Both rounded distances are monotone in xn, so the comparison is false at a, true at b and
+// changes once in between; a bisection over the ordered keys finds the change (at most 32 steps,
+// from a checked bracket 4).
+__device__ __forceinline__ float switch_point(float a, float b) {
+    uint32_t lo = okey(a), hi = okey(b);
+    // The change usually lies within a few ulps of the midpoint: a bracket of 16 keys around it,
+    // taken only if the comparison is false at its low end and true at its high end, leaves four
+    // steps (near zero, or across binades, the whole interval is searched).
+    const uint32_t c = okey(__double2float_rn(0.5 * ((double)a + (double)b)));   // finite: no wrap below
+    const uint32_t l2 = max(lo, c - 8u), h2 = min(hi, c + 8u);
+    const float vl = okey_f32(l2), vh = okey_f32(h2);
+    if (l2 < h2 && !(__fsub_rn(b, vl) < __fsub_rn(vl, a)) && __fsub_rn(b, vh) < __fsub_rn(vh, a)) {
+        lo = l2;
+        hi = h2;
+    }
+    while (hi - lo > 1u) {
+        const uint32_t mid = lo + ((hi - lo) >> 1);
+        const float v = okey_f32(mid);
+        if (__fsub_rn(b, v) < __fsub_rn(v, a)) hi = mid; else lo = mid;
+    }
+    return okey_f32(hi);
+}
+
+// First nearest entry from the switch-point table (the fast form): the index is the number of
+// switch points at or below xn; ent[bucket] = {the first switch point above the bucket's lower
+// point (+inf if none), base | min(cnt, 127) << 9} with base the switch points at or below that
+// point and cnt those up to the next bucket's; dsw[1..255] the switch points. A NaN xn takes 0
+// (no comparison of the verbatim rule holds, so its first entry stays).
+__device__ __forceinline__ uint32_t nearest_fast(float xn, const uint2* ent, const float* dsw) {
+    const uint2 e = ent[lut_bucket(xn)];
+    uint32_t idx = (e.y & 511u) + (xn >= __uint_as_float(e.x) ? 1u : 0u);
+    if (e.y >= (2u << 9))                                       // two or more in the bucket: rare
+        while (idx < 255u && xn >= dsw[idx + 1]) idx++;
+    return xn == xn ? idx : 0u;
+}
+
+// One warp per group of 256 outer blocks (8 consecutive ones per lane), persistent over the
+// groups; every CTA first forms the offset from the last level of the tree.
+//
+// Table forms (CTA-uniform, decided from the General8 table alone):
+//  * fast: finite, strictly ascending, every two neighbouring gaps within a factor 2^20 of each
+//    other, and, when the last entry is below 1, a last gap of at least 2^-20 (1 + |t_254|).
+//    For xn in [t_{i-1}, t_i] the rounded distance to any other entry then exceeds the smaller
+//    of the two neighbours' (a gap g beyond a distance below g' >= 2^-20 g exceeds an ulp of
+//    their sum), so the verbatim rule picks i - 1 or i, by the switch point D_i; below t_0 it
+//    picks 0 (ties go to the first index) and above t_255 (up to xn = 1) entry 255. Hence
+//    index = #{i : D_i <= xn}.
+//  * ascending otherwise: nearest_ascending over 32 replicas of the table and the 16-bit bucket
+//    table of the entries.
+//  * anything else: the verbatim rule over all 256 entries.
 template <typename T>
 __global__ void __launch_bounds__(256)
 absmax_compress_kernel(const float* __restrict__ absmax, int64_t nbo, const T* __restrict__ root_in,
                        int64_t root_count, float* __restrict__ offset_p,
                        const float* __restrict__ code2, uint8_t* __restrict__ absmax_q,
                        float* __restrict__ absmax2) {
-    __shared__ __align__(16) float tr[256 * kRep];              // 32 KB
-    const float v = code2[threadIdx.x];
-    const float next = threadIdx.x < 255 ? code2[threadIdx.x + 1] : v;
-    // entry i's 32 replicas are 128 contiguous bytes: 8 rotated 16-byte stores per thread (the 8
-    // threads of a store phase write 8 different 16-byte columns, so no bank is hit twice)
-    static_assert(kRep == 32, "one entry is 8 float4 columns");
-    const float4 v4 = make_float4(v, v, v, v);
+    // 32 KB: the 32 replicas of the table, or (fast form) the bucket entries and switch points
+    __shared__ __align__(16) float tr[256 * kRep];
+    static_assert(2 * kLutN + 257 <= 256 * kRep, "bucket entries and switch points fit");
+    __shared__ uint32_t hist[kLutN + 1];                        // then the 16-bit bucket table
+    __shared__ uint32_t warp_sum[8];
+    uint2* const ent = reinterpret_cast<uint2*>(tr);            // 8-byte aligned: tr is 16-byte aligned
+    float* const dsw = tr + 2 * kLutN;                          // D_i at dsw[i], i = 1 .. 255
+    uint16_t* const lut = reinterpret_cast<uint16_t*>(hist);
+    const int tid = threadIdx.x;
+    const float v = code2[tid];
+    const float prev = tid > 0 ? code2[tid - 1] : v;
+    const float next = tid < 255 ? code2[tid + 1] : v;
+    const bool ascending = __syncthreads_and(v <= next);        // false if any entry is NaN
+    bool ok = fabsf(v) <= FLT_MAX && (tid == 255 || v < next);
+    if (tid > 0 && tid < 255) {
+        // fp64 gaps: exact to 2^-53 relative, far inside the factor-4 margin of the bound used
+        const double g0 = (double)v - (double)prev, g1 = (double)next - (double)v;
+        ok = ok && g0 >= 0x1p-20 * g1 && g1 >= 0x1p-20 * g0;
+    }
+    if (tid == 255 && v < 1.0f) ok = ok && (double)v - (double)prev >= 0x1p-20 * (1.0 + fabs((double)prev));
+    const bool fast = __syncthreads_and(ok) != 0;
+    // the value this thread enters into the bucket histogram: its switch point, or its entry
+    float key = v;
+    if (fast) {
+        if (tid > 0) {
+            key = switch_point(prev, v);
+            dsw[tid] = key;
+        }
+    } else {
+        // entry i's 32 replicas are 128 contiguous bytes: 8 rotated 16-byte stores per thread (the
+        // 8 threads of a store phase write 8 different 16-byte columns, so no bank is hit twice)
+        static_assert(kRep == 32, "one entry is 8 float4 columns");
+        const float4 v4 = make_float4(v, v, v, v);
 #pragma unroll
-    for (int k = 0; k < 8; k++)
-        reinterpret_cast<float4*>(tr)[threadIdx.x * 8 + ((k + threadIdx.x) & 7)] = v4;
-    // bucket table from a histogram: h[J] = #{i : first bucket at or above t_i is J} (J = kLutN:
-    // above every bucket); with S its inclusive prefix sum, bucket j's base is S(j) (the entries
-    // at or below its lower point) and h[j + 1] = S(j + 1) - S(j) the entries inside it. Thread k
-    // owns slots [13k, 13k + 13) of the prefix sum. Meaningful only for an ascending table.
+        for (int k = 0; k < 8; k++)
+            reinterpret_cast<float4*>(tr)[tid * 8 + ((k + tid) & 7)] = v4;
+    }
+    // Bucket table from a histogram: h[J] = #{keys whose first bucket at or above them is J}
+    // (J = kLutN: above every bucket); with S its inclusive prefix sum, bucket j's base is S(j)
+    // (the keys at or below its lower point) and h[j + 1] = S(j + 1) - S(j) the keys inside it.
+    // Thread k owns slots [13k, 13k + 13) of the prefix sum. Meaningful only for an ascending
+    // table (the keys then ascend too).
     constexpr int kSlots = 13;
     static_assert(kSlots * 256 >= kLutN + 1, "every slot has an owner");
-    __shared__ uint32_t hist[kLutN + 1];                        // then the table, as 16-bit entries
-    __shared__ uint32_t warp_sum[8];
-    uint16_t* const lut = reinterpret_cast<uint16_t*>(hist);
     {
-        const int s0 = threadIdx.x * kSlots;
+        const int s0 = tid * kSlots;
 #pragma unroll
         for (int k = 0; k < kSlots; k++)
             if (s0 + k <= kLutN) hist[s0 + k] = 0;
-        __syncthreads();
-        atomicAdd(&hist[lut_first_at_or_above(v)], 1u);
+        __syncthreads();                                        // also: the switch points are visible
+        if (!fast || tid > 0) atomicAdd(&hist[lut_first_at_or_above(key)], 1u);
         __syncthreads();
         uint32_t h[kSlots + 1];
 #pragma unroll
@@ -227,46 +310,71 @@ absmax_compress_kernel(const float* __restrict__ absmax, int64_t nbo, const T* _
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
             const uint32_t y = __shfl_up_sync(0xffffffffu, x, o);
-            if ((threadIdx.x & 31) >= o) x += y;
+            if ((tid & 31) >= o) x += y;
         }
-        if ((threadIdx.x & 31) == 31) warp_sum[threadIdx.x >> 5] = x;
+        if ((tid & 31) == 31) warp_sum[tid >> 5] = x;
         __syncthreads();                                         // also: every read of hist is done
         uint32_t sum = x - run;
-        for (int w = 0; w < (int)(threadIdx.x >> 5); w++) sum += warp_sum[w];
+        for (int w = 0; w < (tid >> 5); w++) sum += warp_sum[w];
 #pragma unroll
         for (int k = 0; k < kSlots; k++) {
             sum += h[k];
-            if (s0 + k < kLutN) lut[s0 + k] = (uint16_t)(sum | min(h[k + 1], 127u) << 9);
+            if (s0 + k < kLutN) {
+                const uint32_t e = sum | min(h[k + 1], 127u) << 9;
+                if (fast)        // a bucket with keys inside holds the first of them (sum + 1 <= 255)
+                    ent[s0 + k] = make_uint2(h[k + 1] ? __float_as_uint(dsw[sum + 1]) : 0x7f800000u, e);
+                else
+                    lut[s0 + k] = (uint16_t)e;
+            }
         }
     }
-    // the barrier also makes the replicas and the bucket table visible
-    const bool ascending = __syncthreads_and(v <= next);        // false if any entry is NaN
+    __syncthreads();                                            // the tables are complete
     // Everything above reads only the General8 table, an input written before the quantize's
     // first launch; the outer absmax and the tree nodes below come from the launches just before
     // this one (programmatic dependent launch: this set-up overlaps their end).
     pdl_wait();
-    const float* t = tr + (threadIdx.x & (kRep - 1));
+    const float* t = tr + (tid & (kRep - 1));
+    const int lane = tid & 31;
+    const int64_t ngroups = (nbo + kGroup - 1) / kGroup;
+    const int64_t nfull = nbo / kGroup;
+    const int64_t wstride = (int64_t)gridDim.x * (blockDim.x >> 5);
+    const int64_t g0 = (int64_t)blockIdx.x * (blockDim.x >> 5) + (tid >> 5);
+    const bool q_vec = (reinterpret_cast<uintptr_t>(absmax_q) & 7u) == 0;
+    // A full group's 8 absmax values of this lane: two 16-byte loads (absmax is 256-byte aligned).
+    auto load_full = [&](int64_t g, float4& x0, float4& x1) {
+        const float* p = absmax + g * kGroup + lane * 8;
+        x0 = __ldg(reinterpret_cast<const float4*>(p));
+        x1 = __ldg(reinterpret_cast<const float4*>(p + 4));
+    };
+    // the first full group's values go out before the root is formed, so the loads overlap
+    const float4 z = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+    float4 n0 = z, n1 = z;
+    if (g0 < nfull) load_full(g0, n0, n1);
     // the offset: the root of the pairwise tree over the last level (<= 2048 values), the
     // same in every CTA; CTA 0 stores it
     __shared__ double ws[8];
     const float off = __double2float_rn(__ddiv_rn(tree_node(root_in, root_count, 0, ws), (double)nbo));
-    if (blockIdx.x == 0 && threadIdx.x == 0) *offset_p = off;
-    const int lane = threadIdx.x & 31;
-    const int64_t ngroups = (nbo + kGroup - 1) / kGroup;
-    const int64_t wstride = (int64_t)gridDim.x * (blockDim.x >> 5);
-    // one group: FULL groups (all 256 blocks inside nbo) need no bounds checks; ASC selects the
-    // search (uniform over the kernel)
-    auto group = [&](int64_t g, auto full, auto asc) {
+    if (blockIdx.x == 0 && tid == 0) *offset_p = off;
+    // one group: FULL groups (all 256 blocks inside nbo) need no bounds checks and take their
+    // values from x0, x1; FORM is the table form (0 fast, 1 ascending, 2 any), uniform over the
+    // kernel
+    auto group = [&](int64_t g, auto full, auto form, float4 x0, float4 x1) {
         constexpr bool FULL = decltype(full)::value;
-        constexpr bool ASC = decltype(asc)::value;
+        constexpr int FORM = decltype(form)::value;
+        const int64_t b0 = g * kGroup + lane * 8;
         float cv[8];
+        if constexpr (FULL) {
+            const float xs[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+#pragma unroll
+            for (int j = 0; j < 8; j++) cv[j] = __fsub_rn(xs[j], off);
+        } else {
+#pragma unroll
+            for (int j = 0; j < 8; j++)
+                cv[j] = b0 + j < nbo ? __fsub_rn(__ldg(absmax + b0 + j), off) : __int_as_float(0x7fc00000);
+        }
         float m = __int_as_float(0x7fc00000);                   // NaN: ignored by fmaxf
 #pragma unroll
-        for (int j = 0; j < 8; j++) {
-            const int64_t b = g * kGroup + lane + 32 * j;
-            cv[j] = (FULL || b < nbo) ? __fsub_rn(__ldg(absmax + b), off) : __int_as_float(0x7fc00000);
-            m = fmaxf(m, fabsf(cv[j]));
-        }
+        for (int j = 0; j < 8; j++) m = fmaxf(m, fabsf(cv[j]));
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
         if (lane == 0) absmax2[g] = m;
@@ -275,28 +383,66 @@ absmax_compress_kernel(const float* __restrict__ absmax, int64_t nbo, const T* _
         // by the fma), xn = RN(q0 + r y) is the correctly rounded quotient by Markstein's theorem
         // (y within half an ulp of 1/d, q0 within one ulp of c / d, no underflow); zero, tiny and
         // NaN quotients take the IEEE division instead
+        // (the rare cases are collected per warp and handled behind one vote, off the common path)
         const float y = __frcp_rn(d);
+        float xn[8];
+        bool rare = false;
 #pragma unroll
         for (int j = 0; j < 8; j++) {
-            const int64_t b = g * kGroup + lane + 32 * j;
-            if (FULL || b < nbo) {
-                const float q0 = __fmul_rn(cv[j], y);
-                float xn = __fmaf_rn(__fmaf_rn(-d, q0, cv[j]), y, q0);
-                if (!(fabsf(q0) >= 0x1p-100f)) xn = __fdiv_rn(cv[j], d);
-                absmax_q[b] = (uint8_t)(ASC ? nearest_ascending(xn, t, lut) : nearest_any(xn, t));
+            const float q0 = __fmul_rn(cv[j], y);
+            xn[j] = __fmaf_rn(__fmaf_rn(-d, q0, cv[j]), y, q0);
+            rare |= !(fabsf(q0) >= 0x1p-100f);
+        }
+        if (__any_sync(0xffffffffu, rare)) {
+#pragma unroll
+            for (int j = 0; j < 8; j++)
+                if (!(fabsf(__fmul_rn(cv[j], y)) >= 0x1p-100f)) xn[j] = __fdiv_rn(cv[j], d);
+        }
+        uint32_t q[8];
+        if constexpr (FORM == 0) {
+            // one table read and one comparison per value; buckets holding two or more switch
+            // points and NaN quotients redo the value through nearest_fast
+            bool redo = false;
+#pragma unroll
+            for (int j = 0; j < 8; j++) {
+                const uint2 e = ent[lut_bucket(xn[j])];
+                q[j] = (e.y & 511u) + (xn[j] >= __uint_as_float(e.x) ? 1u : 0u);
+                redo |= e.y >= (2u << 9) || xn[j] != xn[j];
             }
+            if (__any_sync(0xffffffffu, redo)) {
+#pragma unroll
+                for (int j = 0; j < 8; j++) q[j] = nearest_fast(xn[j], ent, dsw);
+            }
+        } else {
+#pragma unroll
+            for (int j = 0; j < 8; j++) q[j] = FORM == 1 ? nearest_ascending(xn[j], t, lut) : nearest_any(xn[j], t);
+        }
+        if (FULL && q_vec) {
+            const uint32_t w0 = q[0] | q[1] << 8 | q[2] << 16 | q[3] << 24;
+            const uint32_t w1 = q[4] | q[5] << 8 | q[6] << 16 | q[7] << 24;
+            asm volatile("st.global.v2.u32 [%0], {%1,%2};" :: "l"(absmax_q + b0), "r"(w0), "r"(w1) : "memory");
+        } else {
+#pragma unroll
+            for (int j = 0; j < 8; j++)
+                if (FULL || b0 + j < nbo) absmax_q[b0 + j] = (uint8_t)q[j];
         }
     };
-    const int64_t nfull = nbo / kGroup;
-    const int64_t g0 = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-    if (ascending) {
-        for (int64_t g = g0; g < ngroups; g += wstride) {
-            if (g < nfull) group(g, std::true_type{}, std::true_type{});
-            else group(g, std::false_type{}, std::true_type{});
+    using Fast = std::integral_constant<int, 0>;
+    using Asc = std::integral_constant<int, 1>;
+    using Any = std::integral_constant<int, 2>;
+    int64_t g = g0;
+    // full groups with the next group's values in flight, then the partial last group
+    auto run = [&](auto form) {
+        for (; g < nfull; g += wstride) {
+            const float4 c0 = n0, c1 = n1;
+            if (g + wstride < nfull) load_full(g + wstride, n0, n1);
+            group(g, std::true_type{}, form, c0, c1);
         }
-    } else {
-        for (int64_t g = g0; g < ngroups; g += wstride) group(g, std::false_type{}, std::false_type{});
-    }
+        for (; g < ngroups; g += wstride) group(g, std::false_type{}, form, z, z);
+    };
+    if (fast) run(Fast{});
+    else if (ascending) run(Asc{});
+    else for (; g < ngroups; g += wstride) group(g, std::false_type{}, Any{}, z, z);
 }
 
 }  // namespace
@@ -326,7 +472,7 @@ cudaError_t launch_quantize_4bit_nested(const void* A, int dtype, int64_t n, int
     // most 2048 values) is formed by every CTA of the compression kernel
     const int64_t ngroups = (nbo + kGroup - 1) / kGroup;
     if (nbo <= kTree) {
-        const int grid = persistent_grid(absmax_compress_kernel<float>, 256, 0, ngroups, 32);
+        const int grid = std::min(persistent_grid(absmax_compress_kernel<float>, 256, 0, ngroups, 32), 2 * sm_count());
         return launch_pdl(absmax_compress_kernel<float>, grid, 256, 0, s, absmax, nbo, absmax, nbo, offset, code2,
                           absmax_q, absmax2);
     }
@@ -345,8 +491,9 @@ cudaError_t launch_quantize_4bit_nested(const void* A, int dtype, int64_t n, int
         out = out == buf_b ? buf_a : buf_b;        // a level never outgrows the one before it
         count = next;
     }
-    // 32 groups per CTA (4 per warp) amortise the 32 KB table set-up; persistent above that
-    const int grid = persistent_grid(absmax_compress_kernel<double>, 256, 0, ngroups, 32);
+    // at least 32 groups per CTA (4 per warp) amortise the per-CTA table set-up; persistent
+    // above that, two CTAs per SM (every SM the same share; more CTAs only repeat the set-up)
+    const int grid = std::min(persistent_grid(absmax_compress_kernel<double>, 256, 0, ngroups, 32), 2 * sm_count());
     return launch_pdl(absmax_compress_kernel<double>, grid, 256, 0, s, absmax, nbo, in, count, offset, code2, absmax_q,
                       absmax2);
 }

@@ -168,6 +168,36 @@ def _quotients(x_host, bs):
     return (c / np.repeat(d, 256)[:c.size]).astype(np.float32)
 
 
+@pytest.mark.parametrize("kind", ["straddle", "decade", "scaled"])
+def test_nested_compression_switch_point_tables(bbc, kind):
+    """Tables in the compression's fast form (finite, strictly ascending, neighbouring gaps within
+    a factor 2^20): entry pairs straddling 48 of the quotients the input produces, so that switch
+    points fall on and one ulp beside them; a table built by decades from 1e-7 to 1; and the
+    stand-in table scaled by 0.9, so that the quotients +-1 of every group's largest block lie
+    beyond both end entries."""
+    from tests.test_model_compression_switch_points import decade_table, fast_form_ok
+    bs = 64
+    x = synthetic.weights(bs * 256 * 5 + bs * 9 + 5, std=0.02, seed=33, dtype=torch.float32)
+    if kind == "straddle":
+        xn = _quotients(x, bs)
+        rng = np.random.default_rng(43)
+        picks = np.unique(rng.choice(xn[np.abs(xn) < 0.95], 48, replace=False))
+        delta = (np.abs(picks) * 1e-3 + 1e-7).astype(np.float32)
+        lo, hi = (picks - delta).astype(np.float32), (picks + delta).astype(np.float32)
+        # symmetric pairs put the switch point one ulp above the pick (the tie stays with the
+        # lower entry); lowering every other lower entry by two ulps puts it on the pick
+        lo[1::2] = np.nextafter(np.nextafter(lo[1::2], np.float32(-2)), np.float32(-2))
+        pairs = np.concatenate([lo, hi]).astype(np.float32)
+        fill = np.linspace(-1, 1, 256 - pairs.size).astype(np.float32)
+        table = np.sort(np.concatenate([pairs, fill])).astype(np.float32)
+    elif kind == "decade":
+        table = decade_table()
+    else:
+        table = (G8 * np.float32(0.9)).astype(np.float32)
+    assert table.size == 256 and fast_form_ok(table)
+    check_nested(bbc, x, bs, code2=table, what=f"fast form {kind}")
+
+
 @pytest.mark.parametrize("kind", ["hits", "cluster", "duplicates", "infinite_ends", "all_equal"])
 def test_nested_compression_crafted_tables(bbc, kind):
     """Ascending tables placed around the quotients the input produces: entries equal to
