@@ -27,6 +27,8 @@ from ._native import (  # noqa: F401
     bbc_last_error,
     bbc_nf_codebook,
     bbc_wait_timeouts,
+    bbc_debug_status,
+    bbc_is_debug_build,
     dequantize_4bit,
     dequantize_4bit_nested,
     dequantize_4bit_nested_chain,

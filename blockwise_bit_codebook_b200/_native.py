@@ -62,6 +62,10 @@ def load_library():
     L.bbc_nf_codebook.restype = I
     L.bbc_wait_timeouts.argtypes = [ct.POINTER(ct.c_uint)]
     L.bbc_wait_timeouts.restype = I
+    L.bbc_debug_status.argtypes = [ct.POINTER(ct.c_uint), ct.c_int]
+    L.bbc_debug_status.restype = I
+    L.bbc_is_debug_build.argtypes = []
+    L.bbc_is_debug_build.restype = I
     L.bbc_last_error.argtypes = []
     L.bbc_last_error.restype = ct.c_char_p
     _lib = L
@@ -353,6 +357,20 @@ def bbc_wait_timeouts() -> int:
     c = ct.c_uint(0)
     _check("bbc_wait_timeouts", L.bbc_wait_timeouts(ct.byref(c)))
     return int(c.value)
+
+
+def bbc_debug_status(reset: bool = False) -> int:
+    """Bits of the debug build's bounds guards that failed on the current device (0 in a release
+    build); `reset` clears them after reading."""
+    L = load_library()
+    c = ct.c_uint(0)
+    _check("bbc_debug_status", L.bbc_debug_status(ct.byref(c), 1 if reset else 0))
+    return int(c.value)
+
+
+def bbc_is_debug_build() -> bool:
+    """True when the loaded library was compiled with the bounds guards."""
+    return bool(load_library().bbc_is_debug_build())
 
 
 def bbc_nf_codebook(K: int) -> np.ndarray:

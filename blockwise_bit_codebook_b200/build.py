@@ -2,7 +2,10 @@
 
 Each source is compiled by nvcc (no relocatable device code: every kernel and
 its launcher share a translation unit), then linked into one shared library
-next to this file. `python -m blockwise_bit_codebook_b200.build [--force]`.
+next to this file. `python -m blockwise_bit_codebook_b200.build [--force] [--debug]`.
+--debug builds libbbc_debug.so instead: the same sources with -DBBC_DEBUG, whose
+kernels check every computed global address against its buffer's extent and
+report failures through bbc_debug_status (load it with BBC_LIBRARY=...).
 """
 import concurrent.futures as cf
 import glob
@@ -17,6 +20,7 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.environ.get("BBC_BUILD_OUTPUT") or os.path.join(HERE, "libbbc.so")
+LIB_DEBUG = os.path.join(HERE, "libbbc_debug.so")
 
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
@@ -28,18 +32,21 @@ def sources():
     return sorted(glob.glob(os.path.join(CSRC, "*.cu")) + glob.glob(os.path.join(CSRC, "*.cpp")))
 
 
-def _stale() -> bool:
-    if not os.path.exists(LIB):
+def _stale(lib: str) -> bool:
+    if not os.path.exists(lib):
         return True
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     deps = sources() + glob.glob(os.path.join(CSRC, "*.h")) + glob.glob(os.path.join(CSRC, "*.cuh")) \
         + [os.path.join(INCLUDE, "bbc.h"), __file__]
     return any(os.path.getmtime(d) > t for d in deps)
 
 
-def build(force: bool = False, verbose: bool = False, extra=()) -> str:
-    if not force and not _stale():
-        return LIB
+def build(force: bool = False, verbose: bool = False, extra=(), debug: bool = False) -> str:
+    lib = LIB_DEBUG if debug else LIB
+    if debug:
+        extra = (*extra, "-DBBC_DEBUG")
+    if not force and not _stale(lib):
+        return lib
     tmp = tempfile.mkdtemp(prefix="bbc_build_")
     try:
         def compile_one(src):
@@ -57,12 +64,13 @@ def build(force: bool = False, verbose: bool = False, extra=()) -> str:
         out = os.path.join(tmp, "libbbc.so")
         cmd = [NVCC, *ARCH, "-shared", "-o", out, *objs]
         subprocess.run(cmd, check=True)
-        shutil.move(out, LIB)
+        shutil.move(out, lib)
     finally:
         shutil.rmtree(tmp, ignore_errors=True)
-    return LIB
+    return lib
 
 
 if __name__ == "__main__":
     extra = ["-Xptxas", "-v"] if "--ptxas" in sys.argv else []
-    print(build(force="--force" in sys.argv or bool(extra), verbose="-v" in sys.argv or bool(extra), extra=extra))
+    print(build(force="--force" in sys.argv or bool(extra), verbose="-v" in sys.argv or bool(extra), extra=extra,
+                debug="--debug" in sys.argv))

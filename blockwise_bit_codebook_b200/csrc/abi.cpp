@@ -430,6 +430,30 @@ int bbc_wait_timeouts(unsigned int* count) {
     return cuda_status(bbc::wait_timeouts(count), "bbc_wait_timeouts");
 }
 
+int bbc_debug_status(unsigned int* status, int reset) {
+    if (!status) return fail(BBC_ERR_INVALID, "bbc_debug_status: null pointer argument");
+    cudaError_t (*const words[])(unsigned int*, bool) = {
+        bbc::guard_status_kbit_quant, bbc::guard_status_kbit_dequant, bbc::guard_status_nested_dequant,
+        bbc::guard_status_nested_quant, bbc::guard_status_linear, bbc::guard_status_linear_tc};
+    unsigned int all = 0;
+    for (auto word : words) {
+        unsigned int v = 0;
+        const cudaError_t e = word(&v, reset != 0);
+        if (e != cudaSuccess) return cuda_status(e, "bbc_debug_status");
+        all |= v;
+    }
+    *status = all;
+    return BBC_OK;
+}
+
+int bbc_is_debug_build(void) {
+#ifdef BBC_DEBUG
+    return 1;
+#else
+    return 0;
+#endif
+}
+
 const char* bbc_last_error(void) { return g_last_error.c_str(); }
 
 }  // extern "C"

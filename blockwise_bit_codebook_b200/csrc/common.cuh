@@ -227,4 +227,40 @@ __device__ __forceinline__ void kbit_groups(const uint32_t (&w)[KB], int h, uint
     }
 }
 
+// ---- debug builds (-DBBC_DEBUG): bounds guards -------------------------------
+//
+// In a debug build every global access whose address a kernel computes is checked against the
+// extent the launch's arguments give that buffer; a failed check sets its bit in this
+// translation unit's status word and skips the access (no trap: the context stays usable), and
+// bbc_debug_status reads the words. In a release build a guard is the constant true.
+enum GuardBit : unsigned {
+    kGuardQuantIn = 1u << 0,      // quantize input loads (k-bit and 4-bit), L2 prefetches
+    kGuardQuantOut = 1u << 1,     // quantize stores: plane words, codes, absmax
+    kGuardDequantIn = 1u << 2,    // k-bit dequant loads: plane words, absmax
+    kGuardDequantOut = 1u << 3,   // k-bit dequant output stores
+    kGuardNestedIn = 1u << 4,     // nested dequant loads (fused and three-launch)
+    kGuardNestedOut = 1u << 5,    // nested dequant stores (output, scale workspace)
+    kGuardTree = 1u << 6,         // offset tree loads and node stores
+    kGuardCompress = 1u << 7,     // General8 compression loads and stores
+    kGuardLinear = 1u << 8,       // fused linear weight loads (both linear kernels)
+};
+#ifdef BBC_DEBUG
+static __device__ unsigned int g_bbc_guard;      // one status word per translation unit
+#define BBC_GUARD(cond, bit) ((cond) || (atomicOr(&::bbc::g_bbc_guard, (unsigned)(bit)), false))
+#define BBC_GUARD_ACCESSOR(name)                                                              \
+    cudaError_t name(unsigned int* v, bool reset) {                                           \
+        cudaError_t e = cudaMemcpyFromSymbol(v, g_bbc_guard, sizeof(unsigned int));           \
+        if (e != cudaSuccess || !reset) return e;                                             \
+        const unsigned int zero = 0;                                                          \
+        return cudaMemcpyToSymbol(g_bbc_guard, &zero, sizeof(unsigned int));                  \
+    }
+#else
+#define BBC_GUARD(cond, bit) (true)
+#define BBC_GUARD_ACCESSOR(name)                                                              \
+    cudaError_t name(unsigned int* v, bool) {                                                 \
+        *v = 0;                                                                               \
+        return cudaSuccess;                                                                   \
+    }
+#endif
+
 }  // namespace bbc

@@ -34,9 +34,9 @@ struct BlockIn {
 
 template <int K, typename AT>
 __device__ __forceinline__ BlockIn<K> load_block(const uint32_t* packed, const AT* absmax,
-                                                 int64_t b, bool active) {
+                                                 int64_t b, bool active, int64_t nb) {
     BlockIn<K> r;
-    if (active) {
+    if (active && BBC_GUARD(b >= 0 && b < nb, kGuardDequantIn)) {
         r.am = load_absmax(absmax, b);          // fp32 as stored, or the exact E4M4 value
         const uint32_t* wp = packed + b * K;
 #pragma unroll
@@ -53,8 +53,14 @@ __device__ __forceinline__ BlockIn<K> load_block(const uint32_t* packed, const A
 // words when `packed` allows it (K = 2: 8-byte, K = 4: 16-byte alignment of the array).
 template <int K, typename AT>
 __device__ __forceinline__ BlockIn<K> load_whole(const uint32_t* packed, const AT* absmax, int64_t b,
-                                                 bool vec_words) {
+                                                 bool vec_words, int64_t n) {
     BlockIn<K> r;
+    if (!BBC_GUARD(b >= 0 && (b + 1) * 32 <= n, kGuardDequantIn)) {
+        r.am = 0.0f;
+#pragma unroll
+        for (int j = 0; j < K; j++) r.w[j] = 0u;
+        return r;
+    }
     r.am = load_absmax(absmax, b);
     const uint32_t* wp = packed + b * K;
     if (K == 4 && vec_words) {
@@ -139,14 +145,15 @@ kbit_dequant_kernel(const uint32_t* __restrict__ packed, const AT* __restrict__ 
         const bool vec_words = (reinterpret_cast<uintptr_t>(packed) & (K == 4 ? 15u : 7u)) == 0;
         int64_t b = (int64_t)blockIdx.x * kThreads + threadIdx.x;
         BlockIn<K> cb0;
-        if (b < nbf) cb0 = load_whole<K, AT>(packed, absmax, b, vec_words);
+        if (b < nbf) cb0 = load_whole<K, AT>(packed, absmax, b, vec_words, n);
         publish_codebook();
         if (b < nbf) {
             while (true) {
                 const int64_t bn = b + stride;
                 BlockIn<K> cb1;
-                if (bn < nbf) cb1 = load_whole<K, AT>(packed, absmax, bn, vec_words);
-                decode_whole<K, DT>(cb0, cbb, reinterpret_cast<char*>(out) + b * 32 * dtype_size(DT));
+                if (bn < nbf) cb1 = load_whole<K, AT>(packed, absmax, bn, vec_words, n);
+                if (BBC_GUARD((b + 1) * 32 <= n, kGuardDequantOut))
+                    decode_whole<K, DT>(cb0, cbb, reinterpret_cast<char*>(out) + b * 32 * dtype_size(DT));
                 b = bn;
                 if (b >= nbf) break;
                 cb0 = cb1;
@@ -155,11 +162,12 @@ kbit_dequant_kernel(const uint32_t* __restrict__ packed, const AT* __restrict__ 
         H0 = 2 * nbf;
     }
     int64_t H = H0 + (int64_t)blockIdx.x * kThreads + threadIdx.x;
-    BlockIn<K> cur = load_block<K, AT>(packed, absmax, H >> 1, H < nh);
+    const int64_t nb = nh >> 1;
+    BlockIn<K> cur = load_block<K, AT>(packed, absmax, H >> 1, H < nh, nb);
     if constexpr (!(VEC && WHOLE)) publish_codebook();
     for (; H < nh; H += stride) {
         const int64_t Hn = H + stride;
-        const BlockIn<K> nxt = load_block<K, AT>(packed, absmax, Hn >> 1, Hn < nh);
+        const BlockIn<K> nxt = load_block<K, AT>(packed, absmax, Hn >> 1, Hn < nh, nb);
 
         uint32_t B0, B1;
         if constexpr (K == 2) {
@@ -248,6 +256,8 @@ cudaError_t launch_any(const uint32_t* packed, const AT* absmax, const float* co
 }
 
 }  // namespace
+
+BBC_GUARD_ACCESSOR(guard_status_kbit_dequant)
 
 cudaError_t launch_kbit_dequantize(const uint32_t* packed, const float* absmax,
                                    const float* codebook, int K, int64_t n, int out_dtype,

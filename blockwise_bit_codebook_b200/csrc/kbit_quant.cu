@@ -357,9 +357,9 @@ __device__ __forceinline__ Raw<DT> load_raw(const void* A, int64_t n, int64_t H,
 // Exact fp32 values of the two 16-bit elements packed in w (element 2i in the low half).
 // Raw words of a half block that lies entirely inside the input (vector loads only).
 template <int DT>
-__device__ __forceinline__ Raw<DT> load_full(const void* A, int64_t H, bool active) {
+__device__ __forceinline__ Raw<DT> load_full(const void* A, int64_t H, bool active, int64_t n) {
     Raw<DT> r;
-    if (active) {
+    if (active && BBC_GUARD(H >= 0 && (H + 1) * 16 <= n, kGuardQuantIn)) {
         const char* p = reinterpret_cast<const char*>(A) + H * 16 * dtype_size(DT);
         const u32x8 a = ldg_stream_v8(p);
 #pragma unroll
@@ -437,6 +437,7 @@ struct LoopCtx {
     bool packed_v4;
     uint32_t* stage;        // this warp's 32 * 5 words (whole-block path, K = 5)
     int lane;
+    int64_t nb;             // blocks of the input (bounds guards of debug builds)
 };
 
 // The table entry of the cell whose index sits in bits 7..14 of `fbits`.
@@ -562,14 +563,15 @@ __device__ __forceinline__ void quantize_half(const Raw<DT>& raw, int64_t H, boo
 
     const int64_t b = H >> 1;
     uint32_t* out = packed + b * K;
+    const bool st = active && BBC_GUARD(b >= 0 && b < c.nb, kGuardQuantOut);
     if (K == 4 && c.packed_v2) {
-        if (active) asm volatile("st.global.v2.u32 [%0], {%1,%2};" :: "l"(out + 2 * c.h), "r"(wa), "r"(wb) : "memory");
+        if (st) asm volatile("st.global.v2.u32 [%0], {%1,%2};" :: "l"(out + 2 * c.h), "r"(wa), "r"(wb) : "memory");
     } else {
-        if (active && 2 * c.h < K) out[2 * c.h] = wa;
-        if (active && 2 * c.h + 1 < K) out[2 * c.h + 1] = wb;
-        if constexpr (K == 5) { if (active && c.h == 0) out[4] = w4; }
+        if (st && 2 * c.h < K) out[2 * c.h] = wa;
+        if (st && 2 * c.h + 1 < K) out[2 * c.h + 1] = wb;
+        if constexpr (K == 5) { if (st && c.h == 0) out[4] = w4; }
     }
-    if (active && c.h == 0) store_absmax(absmax, b, amax);
+    if (st && c.h == 0) store_absmax(absmax, b, amax);
 }
 
 // ---- one whole block (32 elements of a 16-bit type) per thread ----
@@ -579,8 +581,13 @@ template <int DT>
 struct Raw32 { uint32_t w[16]; };
 
 template <int DT>
-__device__ __forceinline__ Raw32<DT> load_block(const void* A, int64_t b) {
+__device__ __forceinline__ Raw32<DT> load_block(const void* A, int64_t b, int64_t n) {
     Raw32<DT> r;
+    if (!BBC_GUARD(b >= 0 && (b + 1) * 32 <= n, kGuardQuantIn)) {
+#pragma unroll
+        for (int i = 0; i < 16; i++) r.w[i] = 0u;
+        return r;
+    }
     const char* p = reinterpret_cast<const char*>(A) + b * 64;
     const u32x8 a = ldg_stream_v8(p);
     const u32x8 q = ldg_stream_v8(p + 32);
@@ -684,29 +691,42 @@ __device__ __forceinline__ void quantize_block(const Raw32<DT>& raw, int64_t b, 
         }
     }
     uint32_t* out = packed + b * K;
+    // the K = 5 transpose stores the warp's 32 consecutive blocks b - lane .. b - lane + 31
+    const bool st = BBC_GUARD(b >= 0 && b < c.nb && (K != 5 || (b - c.lane >= 0 && b - c.lane + 32 <= c.nb)),
+                              kGuardQuantOut);
     if constexpr (K == 2) {
-        if (c.packed_v2) asm volatile("st.global.v2.u32 [%0], {%1,%2};" :: "l"(out), "r"(w[0]), "r"(w[1]) : "memory");
+        if (!st) {
+        } else if (c.packed_v2) asm volatile("st.global.v2.u32 [%0], {%1,%2};" :: "l"(out), "r"(w[0]), "r"(w[1]) : "memory");
         else { out[0] = w[0]; out[1] = w[1]; }
     } else if constexpr (K == 4) {
-        if (c.packed_v4) stg_v4(out, w[0], w[1], w[2], w[3]);
+        if (!st) {
+        } else if (c.packed_v4) stg_v4(out, w[0], w[1], w[2], w[3]);
         else { out[0] = w[0]; out[1] = w[1]; out[2] = w[2]; out[3] = w[3]; }
     } else if constexpr (K == 5) {
         // the warp's 32 consecutive blocks are 160 contiguous words: transposed through shared
         // memory so that each store instruction writes 128 contiguous bytes (five 4-byte stores
         // at a 20-byte lane stride left the K = 5 kernel 2-3 points slower)
-        uint32_t* st = c.stage;
+        uint32_t* stg = c.stage;
 #pragma unroll
-        for (int j = 0; j < K; j++) st[c.lane * K + j] = w[j];
+        for (int j = 0; j < K; j++) stg[c.lane * K + j] = w[j];
         __syncwarp();
         uint32_t* outw = packed + (b - c.lane) * K;
+#ifdef BBC_DEBUG
+        const bool st_warp = __all_sync(0xffffffffu, st);
+#else
+        const bool st_warp = true;
+#endif
+        if (st_warp) {
 #pragma unroll
-        for (int j = 0; j < K; j++) outw[j * 32 + c.lane] = st[j * 32 + c.lane];
+            for (int j = 0; j < K; j++) outw[j * 32 + c.lane] = stg[j * 32 + c.lane];
+        }
         __syncwarp();
     } else {
 #pragma unroll
-        for (int j = 0; j < K; j++) out[j] = w[j];
+        for (int j = 0; j < K; j++)
+            if (st) out[j] = w[j];
     }
-    store_absmax(absmax, b, amax);
+    if (st) store_absmax(absmax, b, amax);
 }
 
 template <int K, int DT, bool VEC, typename AT>
@@ -743,7 +763,8 @@ kbit_quant_kernel(const void* __restrict__ A, int64_t n, const float* __restrict
         const int64_t end = WHOLE ? bend : nh_full;
         for (int i = 0; i < 2; i++) {
             const int64_t u0 = wbase + i * stride;
-            if (u0 < end) prefetch_l2(static_cast<const char*>(A) + u0 * unit, (uint32_t)(min(end - u0, (int64_t)32) * unit));
+            if (u0 < end && BBC_GUARD((u0 + min(end - u0, (int64_t)32)) * unit <= n * dtype_size(DT), kGuardQuantIn))
+                prefetch_l2(static_cast<const char*>(A) + u0 * unit, (uint32_t)(min(end - u0, (int64_t)32) * unit));
         }
     }
     bool fast_cb = setup_exact_table<K, false>(cbe, cb, thr, &fast_ok, lut, WHOLE ? lut8 : nullptr);
@@ -751,9 +772,9 @@ kbit_quant_kernel(const void* __restrict__ A, int64_t n, const float* __restrict
     Raw32<DT> first_b;
     Raw<DT> first_h;
     if constexpr (WHOLE) {
-        if (wbase < bend) first_b = load_block<DT>(A, wbase + lane);
+        if (wbase < bend) first_b = load_block<DT>(A, wbase + lane, n);
     } else {
-        if (wbase < nh_full) first_h = load_full<DT>(A, wbase + lane, wbase + lane < nh_full);
+        if (wbase < nh_full) first_h = load_full<DT>(A, wbase + lane, wbase + lane < nh_full, n);
     }
     if (codebook_changed<K>(codebook, cb))                  // rare: the codebook was being written
         fast_cb = setup_exact_table<K, false>(load_codebook_entry<K>(codebook), cb, thr, &fast_ok, lut,
@@ -775,6 +796,7 @@ kbit_quant_kernel(const void* __restrict__ A, int64_t n, const float* __restrict
     c.sel_wa = c.h ? 0x1054u : 0x5410u;
     c.sel_wb = c.h ? 0x3276u : 0x7632u;
     c.pair_mask = 3u << (lane & ~1);
+    c.nb = (n + 31) >> 5;
 
     if constexpr (WHOLE) {
         // whole warp iterations of 32 blocks, one block per thread, the next one prefetched;
@@ -788,7 +810,7 @@ kbit_quant_kernel(const void* __restrict__ A, int64_t n, const float* __restrict
                 const int64_t wn = wb + stride;
                 const bool more = wn < bend;
                 Raw32<DT> rb;
-                if (more) rb = load_block<DT>(A, wn + lane);
+                if (more) rb = load_block<DT>(A, wn + lane, n);
                 quantize_block<K, DT, AT>(ra, wb + lane, c, cb, absmax, packed);
                 wb = wn;
                 if (!more) break;
@@ -800,13 +822,13 @@ kbit_quant_kernel(const void* __restrict__ A, int64_t n, const float* __restrict
             while (true) {
                 int64_t wn = wb + stride;
                 bool more = wn < bend;
-                if (more) rb = load_block<DT>(A, wn + lane);
+                if (more) rb = load_block<DT>(A, wn + lane, n);
                 quantize_block<K, DT, AT>(ra, wb + lane, c, cb, absmax, packed);
                 wb = wn;
                 if (!more) break;
                 wn = wb + stride;
                 more = wn < bend;
-                if (more) ra = load_block<DT>(A, wn + lane);
+                if (more) ra = load_block<DT>(A, wn + lane, n);
                 quantize_block<K, DT, AT>(rb, wb + lane, c, cb, absmax, packed);
                 wb = wn;
                 if (!more) break;
@@ -823,11 +845,11 @@ kbit_quant_kernel(const void* __restrict__ A, int64_t n, const float* __restrict
         Raw<DT> ra = first_h;
         Raw<DT> rb;
         while (true) {
-            rb = load_full<DT>(A, wbase + stride + lane, wbase + stride + lane < nh_full);
+            rb = load_full<DT>(A, wbase + stride + lane, wbase + stride + lane < nh_full, n);
             quantize_half<K, DT, AT>(ra, wbase + lane, wbase + lane < nh_full, c, cb, absmax, packed);
             wbase += stride;
             if (wbase >= nh_full) break;
-            ra = load_full<DT>(A, wbase + stride + lane, wbase + stride + lane < nh_full);
+            ra = load_full<DT>(A, wbase + stride + lane, wbase + stride + lane < nh_full, n);
             quantize_half<K, DT, AT>(rb, wbase + lane, wbase + lane < nh_full, c, cb, absmax, packed);
             wbase += stride;
             if (wbase >= nh_full) break;
@@ -960,7 +982,8 @@ quant4_kernel(const void* __restrict__ A, int64_t n, int log2_bs, const float* _
         const int64_t nfull = n / E;                            // slices entirely inside the input
         for (int i = 0; i < 2; i++) {
             const int64_t u0 = base + (tid & ~31) + i * stride;
-            if (u0 < nfull) prefetch_l2(static_cast<const char*>(A) + u0 * 64, (uint32_t)(min(nfull - u0, (int64_t)32) * 64));
+            if (u0 < nfull && BBC_GUARD((u0 + min(nfull - u0, (int64_t)32)) * 64 <= n * dtype_size(DT), kGuardQuantIn))
+                prefetch_l2(static_cast<const char*>(A) + u0 * 64, (uint32_t)(min(nfull - u0, (int64_t)32) * 64));
         }
     }
     LoopCtx c;
@@ -1048,7 +1071,9 @@ quant4_kernel(const void* __restrict__ A, int64_t n, int log2_bs, const float* _
                 for (int j = 0; j < E / 2; j++)
                     if (U * (E / 2) + j < nbytes) cp[j] = (uint8_t)(acc[j / 4] >> (8 * (j & 3)));
             }
-            if ((tid & (tpb - 1)) == 0) absmax[U >> tpb_log2] = amax;
+            if ((tid & (tpb - 1)) == 0 &&
+                BBC_GUARD((U >> tpb_log2) < ((n + (int64_t(1) << log2_bs) - 1) >> log2_bs), kGuardQuantOut))
+                absmax[U >> tpb_log2] = amax;
         }
         cur = nxt;
     }
@@ -1090,6 +1115,8 @@ cudaError_t launch_any(const void* A, int dtype, int64_t n, int K, const float* 
 }
 
 }  // namespace
+
+BBC_GUARD_ACCESSOR(guard_status_kbit_quant)
 
 cudaError_t launch_kbit_quantize(const void* A, int dtype, int64_t n, int K, const float* codebook,
                                  float* absmax, uint32_t* packed, bool vec, cudaStream_t s) {

@@ -128,4 +128,13 @@ cudaError_t launch_nested_dequantize_chain_noalloc(const uint8_t* codes, const u
                                                    const float* code4, int64_t n, int log2_bs,
                                                    int out_dtype, void* out, bool vec, cudaStream_t s);
 
+// Debug builds: each translation unit's guard status word (0 in a release build), read and
+// optionally cleared on the current device; abi.cpp ors them for bbc_debug_status.
+cudaError_t guard_status_kbit_quant(unsigned int* v, bool reset);
+cudaError_t guard_status_kbit_dequant(unsigned int* v, bool reset);
+cudaError_t guard_status_nested_dequant(unsigned int* v, bool reset);
+cudaError_t guard_status_nested_quant(unsigned int* v, bool reset);
+cudaError_t guard_status_linear(unsigned int* v, bool reset);
+cudaError_t guard_status_linear_tc(unsigned int* v, bool reset);
+
 }  // namespace bbc

@@ -80,8 +80,13 @@ struct Win {
 // ea, eb: flattened index of the window's first weight in rows g and g + 8.
 template <int W>
 __device__ __forceinline__ void load_win(Win<W>& r, const uint8_t* codes, const uint8_t* absmax_q,
-                                         const float* absmax2, int log2_bs, int64_t ea, int64_t eb, int t) {
+                                         const float* absmax2, int log2_bs, int64_t ea, int64_t eb, int t,
+                                         int64_t nw) {
     const int64_t la = ea + (W / 4) * t, lb = eb + (W / 4) * t;
+    if (!BBC_GUARD(la >= 0 && lb >= 0 && la + W / 4 <= nw && lb + W / 4 <= nw, kGuardLinear)) {
+        r = Win<W>{};
+        return;
+    }
     if constexpr (W == 128) {
         const uint4 a = __ldg(reinterpret_cast<const uint4*>(codes + (la >> 1)));
         const uint4 b = __ldg(reinterpret_cast<const uint4*>(codes + (lb >> 1)));
@@ -242,7 +247,7 @@ linear4_nested_kernel(const uint16_t* __restrict__ X, int M, int64_t N, int64_t 
     for (int i = 0; i < B; i++)
         if (w_lo + i < w_hi)
             load_win<WM>(wc[i], codes, absmax_q, absmax2, log2_bs, ea0 + (w_lo + i) * WM,
-                         eb0 + (w_lo + i) * WM, t);
+                         eb0 + (w_lo + i) * WM, t, N * K);
     {
         // thread i writes the 16 replicas of entry i as 8 rotated 16-byte stores (each store
         // phase of 8 threads covers all 32 banks)
@@ -277,13 +282,13 @@ linear4_nested_kernel(const uint16_t* __restrict__ X, int M, int64_t N, int64_t 
             // the slot is refilled with the window B ahead once this one is decoded
             if (win + B < w_hi)
                 load_win<WM>(wc[i], codes, absmax_q, absmax2, log2_bs, ea0 + (win + B) * WM,
-                             eb0 + (win + B) * WM, t);
+                             eb0 + (win + B) * WM, t, N * K);
         }
     }
     if (WM == 128 && (K & 64) && warp == kNWarp - 1) {
         // the last 64 k of every row
         Win<64> tw;
-        load_win<64>(tw, codes, absmax_q, absmax2, log2_bs, ea0 + K - 64, eb0 + K - 64, t);
+        load_win<64>(tw, codes, absmax_q, absmax2, log2_bs, ea0 + K - 64, eb0 + K - 64, t, N * K);
         run_win<DT, NT, 64>(acc, tw, c2s, offset, table, lane_off, xr, K - 64, t);
     }
     // the partials overlay the decode table, which no warp reads any more after the barrier
@@ -311,8 +316,12 @@ struct KWin {
 // aligned, so block b's words start on a 16-byte (K = 4) or 8-byte (K = 2) boundary.
 template <int KB, int W>
 __device__ __forceinline__ void load_kwin(KWin<KB>& r, const uint32_t* packed, const float* absmax, int64_t ea,
-                                          int64_t eb, int t) {
+                                          int64_t eb, int t, int64_t nw) {
     const int64_t ba = (ea + (W / 4) * t) >> 5, bb = (eb + (W / 4) * t) >> 5;
+    if (!BBC_GUARD(ba >= 0 && bb >= 0 && (ba + 1) * 32 <= nw && (bb + 1) * 32 <= nw, kGuardLinear)) {
+        r = KWin<KB>{};
+        return;
+    }
     const uint32_t* pa = packed + ba * KB;
     const uint32_t* pb = packed + bb * KB;
     if constexpr (KB == 4) {
@@ -427,7 +436,7 @@ linear_kbit_kernel(const uint16_t* __restrict__ X, int M, int64_t N, int64_t K,
     KWin<KB> wc[B];
 #pragma unroll
     for (int i = 0; i < B; i++)
-        if (w_lo + i < w_hi) load_kwin<KB, WM>(wc[i], packed, absmax, ea0 + (w_lo + i) * WM, eb0 + (w_lo + i) * WM, t);
+        if (w_lo + i < w_hi) load_kwin<KB, WM>(wc[i], packed, absmax, ea0 + (w_lo + i) * WM, eb0 + (w_lo + i) * WM, t, N * K);
     if (threadIdx.x < 32) cbs[threadIdx.x] = threadIdx.x < (1 << KB) ? __ldg(codebook + threadIdx.x) : 0.0f;
     if constexpr (PAIRS) {
         // thread i writes the 16 replicas of entry i (rotated 16-byte stores, as the nested table)
@@ -466,12 +475,12 @@ linear_kbit_kernel(const uint16_t* __restrict__ X, int M, int64_t N, int64_t K,
             if (win >= w_hi) break;
             run_kwin<DT, NT, KB, WM>(acc, wc[i], cbb, table, lane_off, xr, win * WM, t);
             if (win + B < w_hi)
-                load_kwin<KB, WM>(wc[i], packed, absmax, ea0 + (win + B) * WM, eb0 + (win + B) * WM, t);
+                load_kwin<KB, WM>(wc[i], packed, absmax, ea0 + (win + B) * WM, eb0 + (win + B) * WM, t, N * K);
         }
     }
     if (WM == 128 && (K & 64) && warp == kNWarp - 1) {
         KWin<KB> tw;
-        load_kwin<KB, 64>(tw, packed, absmax, ea0 + K - 64, eb0 + K - 64, t);
+        load_kwin<KB, 64>(tw, packed, absmax, ea0 + K - 64, eb0 + K - 64, t, N * K);
         run_kwin<DT, NT, KB, 64>(acc, tw, cbb, table, lane_off, xr, K - 64, t);
     }
     // with the pair table the partials overlay it (no warp reads it after the barrier)
@@ -583,5 +592,7 @@ cudaError_t launch_linear_kbit(const void* X, int dtype, int M, int64_t N, int64
     if (dtype == BF16) return launch_kbit_dt<BF16>(x, M, N, K, packed, absmax, codebook, KB, y, s);
     return launch_kbit_dt<F16>(x, M, N, K, packed, absmax, codebook, KB, y, s);
 }
+
+BBC_GUARD_ACCESSOR(guard_status_linear)
 
 }  // namespace bbc

@@ -419,6 +419,7 @@ linear_tc_kernel(const __grid_constant__ CUtensorMap tmx, int M, int64_t N, int6
         using In = std::conditional_t<NESTED, NestedIn, KbitIn<KB>>;
         auto load_in = [&](int i) -> In {
             const int64_t m0 = mrow + (int64_t)i * kTcBK;
+            if (!BBC_GUARD(m0 >= 0 && m0 + 16 <= N * K, kGuardLinear)) return In{};
             if constexpr (NESTED) return load_nested16(nw, m0);
             else return load_kbit32<KB>(kw, m0 >> 5);
         };
@@ -666,5 +667,7 @@ cudaError_t wait_timeouts(unsigned int* count) {
     const unsigned int zero = 0;
     return cudaMemcpyToSymbol(g_wait_timeouts, &zero, sizeof(unsigned int));
 }
+
+BBC_GUARD_ACCESSOR(guard_status_linear_tc)
 
 }  // namespace bbc

@@ -79,6 +79,7 @@ __device__ __forceinline__ GroupIn load_group(const uint8_t* codes, const uint8_
         g.c = make_uint4(wb[0], wb[1], wb[2], wb[3]);
     }
     const int64_t b = m0 >> log2_bs;
+    if (!BBC_GUARD(m0 < n && b < ((n + (int64_t(1) << log2_bs) - 1) >> log2_bs), kGuardNestedIn)) return g;
     if constexpr (NESTED) {
         g.q = __ldg(absmax_q + b);
         g.a2 = __ldg(absmax2 + (b >> 8));
@@ -194,6 +195,8 @@ add_offset_kernel(float* __restrict__ scale, int64_t nbo, float offset) {
 static __device__ __align__(256) float g_chain_scale_scratch[BBC_NOALLOC_SCRATCH_FLOATS];
 
 }  // namespace
+
+BBC_GUARD_ACCESSOR(guard_status_nested_dequant)
 
 // Device address of this device's copy of the scratch array, looked up with that device current;
 // nullptr if the lookup failed (the error is returned in *err). A call made while `s` is not being

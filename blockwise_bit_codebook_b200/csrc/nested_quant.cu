@@ -342,6 +342,7 @@ absmax_compress_kernel(const float* __restrict__ absmax, int64_t nbo, const T* _
     const bool q_vec = (reinterpret_cast<uintptr_t>(absmax_q) & 7u) == 0;
     // A full group's 8 absmax values of this lane: two 16-byte loads (absmax is 256-byte aligned).
     auto load_full = [&](int64_t g, float4& x0, float4& x1) {
+        if (!BBC_GUARD(g >= 0 && (g + 1) * kGroup <= nbo, kGuardCompress)) return;
         const float* p = absmax + g * kGroup + lane * 8;
         x0 = __ldg(reinterpret_cast<const float4*>(p));
         x1 = __ldg(reinterpret_cast<const float4*>(p + 4));
@@ -377,7 +378,7 @@ absmax_compress_kernel(const float* __restrict__ absmax, int64_t nbo, const T* _
         for (int j = 0; j < 8; j++) m = fmaxf(m, fabsf(cv[j]));
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-        if (lane == 0) absmax2[g] = m;
+        if (lane == 0 && BBC_GUARD(g >= 0 && g < ngroups, kGuardCompress)) absmax2[g] = m;
         const float d = fmaxf(m, 1e-8f);
         // xn = RN(c / d) from the correctly rounded reciprocal y: q0 = RN(c y), r = c - d q0 (exact
         // by the fma), xn = RN(q0 + r y) is the correctly rounded quotient by Markstein's theorem
@@ -420,11 +421,12 @@ absmax_compress_kernel(const float* __restrict__ absmax, int64_t nbo, const T* _
         if (FULL && q_vec) {
             const uint32_t w0 = q[0] | q[1] << 8 | q[2] << 16 | q[3] << 24;
             const uint32_t w1 = q[4] | q[5] << 8 | q[6] << 16 | q[7] << 24;
-            asm volatile("st.global.v2.u32 [%0], {%1,%2};" :: "l"(absmax_q + b0), "r"(w0), "r"(w1) : "memory");
+            if (BBC_GUARD(b0 + 8 <= nbo, kGuardCompress))
+                asm volatile("st.global.v2.u32 [%0], {%1,%2};" :: "l"(absmax_q + b0), "r"(w0), "r"(w1) : "memory");
         } else {
 #pragma unroll
             for (int j = 0; j < 8; j++)
-                if (FULL || b0 + j < nbo) absmax_q[b0 + j] = (uint8_t)q[j];
+                if ((FULL && BBC_GUARD(b0 + j < nbo, kGuardCompress)) || b0 + j < nbo) absmax_q[b0 + j] = (uint8_t)q[j];
         }
     };
     using Fast = std::integral_constant<int, 0>;
@@ -446,6 +448,8 @@ absmax_compress_kernel(const float* __restrict__ absmax, int64_t nbo, const T* _
 }
 
 }  // namespace
+
+BBC_GUARD_ACCESSOR(guard_status_nested_quant)
 
 namespace {
 int64_t tree_nodes(int64_t count) { return (count + kTree - 1) / kTree; }

@@ -390,6 +390,29 @@ int bbc_nf_codebook(int K, float* codebook_out);
  */
 int bbc_wait_timeouts(unsigned int* count);
 
+/*
+ * bbc_debug_status - the bounds guards of a debug build (the library compiled
+ * with -DBBC_DEBUG, libbbc_debug.so next to libbbc.so). In that build every
+ * global load and store whose address a kernel computes is checked against the
+ * extent its launch's arguments give that buffer; a failed check skips the
+ * access (no trap: the context stays usable) and sets a bit in a per-device
+ * status word: 1 quantize input loads and prefetches, 2 quantize stores, 4 k-bit
+ * dequant loads, 8 k-bit dequant stores, 16 nested dequant loads, 32 nested
+ * dequant stores, 64 offset tree, 128 General8 compression, 256 fused linear
+ * weight loads. Outputs of a launch that set a bit are not meaningful. A release
+ * build has no guards and always reports 0. No counterpart on the pages.
+ *
+ *   status HOST pointer: receives the OR of the bits set on the current device
+ *          since the last reset.
+ *   reset  nonzero: clear the bits after reading them.
+ * Synchronous (device-to-host copies on the legacy stream). Errors: a null
+ * pointer -> BBC_ERR_INVALID; a failed copy -> BBC_ERR_CUDA.
+ */
+int bbc_debug_status(unsigned int* status, int reset);
+
+/* 1 in a debug build (bounds guards compiled in, see bbc_debug_status), else 0. */
+int bbc_is_debug_build(void);
+
 /* Message for the last non-OK status returned on the calling thread ("" if none). */
 const char* bbc_last_error(void);
 

@@ -204,3 +204,22 @@ def test_nf_codebook_rejects_bad_k(lib):
     assert lib.bbc_nf_codebook(0, out.ctypes.data_as(P)) == 1
     assert lib.bbc_nf_codebook(9, out.ctypes.data_as(P)) == 1
     assert lib.bbc_nf_codebook(4, None) == 1
+
+
+def test_debug_build_exports_the_same_boundary():
+    """libbbc_debug.so (the bounds-guarded build) exports every declared function and says it is
+    the debug build; the release library says it is not (no CUDA call is made)."""
+    import subprocess
+    from blockwise_bit_codebook_b200 import build, load_library
+    dbg_path = build.build(debug=True)
+    out = subprocess.run(["nm", "-D", "--defined-only", dbg_path], capture_output=True, text=True).stdout
+    syms = {line.split()[-1] for line in out.splitlines() if line.strip()}
+    for name in declared_functions():
+        assert name in syms, name
+    dbg = ct.CDLL(dbg_path)
+    assert dbg.bbc_is_debug_build() == 1
+    assert load_library().bbc_is_debug_build() == 0
+
+
+def test_debug_status_rejects_a_null_pointer(lib):
+    assert lib.bbc_debug_status(None, 0) == 1
