@@ -3,10 +3,11 @@ the device) that bench.py times, through the same calls on whole tensors, so eve
 in the launch configuration the bench measures.
 
 Every k-bit block depends only on its own 32 inputs and every nested inner group (256 outer
-blocks of 64) only on its own state, so the oracle recomputes a seeded sample of them one by
-one (plus the first and the last). Properties that hold at any size are checked on the whole
-outputs on the device. The nested quantize's offset depends on every outer block, so its whole
-state is compared.
+blocks of 64) only on its own state, so the oracle recomputes them in ranges: a seeded sample
+(plus the first and the last) in the quick tests, and every block and group on all host cores in
+the whole-tensor tests. Properties that hold at any size are also checked on the whole outputs
+on the device. The nested quantize's offset depends on every outer block, so its whole state is
+compared.
 """
 import numpy as np
 import pytest
@@ -97,3 +98,61 @@ def test_c5_nested_quantize_whole_state(bbc, x):
     assert_bits_equal(to_host(a2)[:ref[2].size], ref[2], "c5 absmax2")
     assert_bits_equal(to_host(q)[:ref[1].size], ref[1], "c5 absmax_q")
     assert_bits_equal(to_host(codes)[:ref[0].size], ref[0], "c5 nested codes")
+
+
+def _chunks(total, parts):
+    step = -(-total // parts)
+    return [(a, min(total, a + step)) for a in range(0, total, step)]
+
+
+def _on_all_cores(fn, total):
+    """fn(lo, hi) over contiguous ranges of [0, total) on every host core (the oracle's ctypes
+    calls release the interpreter lock)."""
+    import os
+    from concurrent.futures import ThreadPoolExecutor
+    with ThreadPoolExecutor(max_workers=os.cpu_count() or 1) as ex:
+        list(ex.map(lambda r: fn(*r), _chunks(total, 4 * (os.cpu_count() or 1))))
+
+
+@pytest.mark.parametrize("K", [3, 5])
+def test_c5_kbit_whole_tensor(bbc, x, K):
+    """Every one of the 8,388,608 blocks of the c5 tensor, quantized and dequantized, against the
+    oracle bit for bit (ranges of whole blocks on all host cores)."""
+    cb = oracle.normal_float_codebook(K)
+    cb_dev = torch.from_numpy(cb).cuda()
+    packed, absmax = bbc.kbit_quantize(x, K, cb_dev)
+    y = bbc.kbit_dequantize(packed, absmax, cb_dev, K, N, torch.bfloat16)
+    torch.cuda.synchronize()
+    xh = to_host(x)
+    got_p, got_a, got_y = to_host(packed)[: NB * K], to_host(absmax)[:NB], to_host(y)[:N]
+    bad = []
+
+    def check(lo, hi):          # blocks [lo, hi)
+        rp, ra = oracle.kbit_quantize(xh[lo * 32:hi * 32], "bf16", K, cb)
+        ry = oracle.kbit_dequantize(rp, ra, cb, K, (hi - lo) * 32, "bf16")
+        if not (np.array_equal(got_p[lo * K:hi * K], rp) and np.array_equal(got_a[lo:hi].view(np.uint32),
+                                                                              ra.view(np.uint32))
+                and np.array_equal(got_y[lo * 32:hi * 32], ry)):
+            bad.append((lo, hi))
+    _on_all_cores(check, NB)
+    assert not bad, f"K={K}: block ranges differing from the oracle: {sorted(bad)[:4]}"
+
+
+def test_c5_nested_dequant_whole_tensor(bbc):
+    """Every inner group of the c5 nested state (16,384 groups of 256 outer blocks of 64) against
+    the oracle bit for bit."""
+    codes, q, a2, off = synthetic.nested_state(N, BS, seed=3, device="cuda")
+    y = bbc.dequantize_4bit_nested(codes, q, torch.from_numpy(G8).cuda(), a2, float(off),
+                                   torch.from_numpy(NF4).cuda(), N, BS, torch.bfloat16)
+    torch.cuda.synchronize()
+    ch, qh, a2h, got = to_host(codes), to_host(q), to_host(a2), to_host(y)[:N]
+    ngroups = N // GROUP
+    bad = []
+
+    def check(lo, hi):          # inner groups [lo, hi)
+        ref = oracle.nested_dequantize(ch[lo * GROUP // 2:hi * GROUP // 2], qh[lo * 256:hi * 256], G8, a2h[lo:hi],
+                                       float(off), NF4, (hi - lo) * GROUP, BS, 256, "bf16")
+        if not np.array_equal(got[lo * GROUP:hi * GROUP], ref):
+            bad.append((lo, hi))
+    _on_all_cores(check, ngroups)
+    assert not bad, f"group ranges differing from the oracle: {sorted(bad)[:4]}"
