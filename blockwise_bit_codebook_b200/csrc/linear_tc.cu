@@ -561,20 +561,25 @@ EncodeTiled tensor_map_encoder(cudaError_t* err) {
     return fn;
 }
 
-// Split factor S (a cluster of S CTAs shares an output tile along K): the S in {1, 2, 4, 8} that
-// fills the machine best (output tiles x S CTAs over waves of `cap` resident CTAs), with at least
-// two K stages per CTA; a larger S only when it is 5 % better.
-int pick_split(int64_t tiles, int cap, int64_t stages_k) {
+// Split factor S (a cluster of S CTAs shares an output tile along K): the S in {1, 2, 4, 8}, with at
+// least two K stages per CTA, of the least estimated time, in units of one 64-wide K stage (~0.6 us
+// per CTA, measured with in-kernel timestamps): per wave of `cap` resident CTAs, a CTA's set-up (~5
+// stages), its K stages, and its epilogue — a direct store (~NT/128 + 1) or, for S > 1, the
+// exchange of partial sums through distributed shared memory and the wait for the cluster's
+// slowest CTA (~NT/16: 9 us at NT = 256). A larger S must be 5 % better. (Counting only how well
+// the CTAs fill the waves picked S = 8 for 86 row tiles of N = 11008 at M = 256: five waves of
+// short CTAs dominated by set-up and epilogue, 158 us against ~45 us with S = 1.)
+int pick_split(int64_t tiles, int cap, int64_t stages_k, int nt) {
     int best = 1;
-    double best_eff = 0.0;
+    double best_t = 0.0;
     for (int S = 1; S <= 8; S *= 2) {
-        if (stages_k < 2 * S) break;
-        const int64_t ctas = tiles * S;
-        const int64_t waves = (ctas + cap - 1) / cap;
-        const double eff = (double)ctas / (double)(waves * cap);
-        if (eff > best_eff * 1.05) {
+        if (S > 1 && stages_k < 2 * S) break;
+        const int64_t waves = (tiles * S + cap - 1) / cap;
+        const double per_cta = 5.0 + (double)stages_k / S + (S == 1 ? nt / 128.0 + 1.0 : nt / 16.0);
+        const double t = (double)waves * per_cta;
+        if (S == 1 || t < best_t * 0.95) {
             best = S;
-            best_eff = eff;
+            best_t = t;
         }
     }
     return best;
@@ -605,7 +610,7 @@ cudaError_t launch_tc(const uint16_t* X, int M, int64_t N, int64_t K, const Nest
     const int64_t mtiles = (M + NT - 1) / NT, ntiles = N / kTcRows;
     const int cap = resident_ctas(reinterpret_cast<const void*>(k), kTcThreads, L::kAlloc);
     if (cap < 1) return cudaErrorInvalidConfiguration;
-    const int S = pick_split(ntiles * mtiles, cap, K / kTcBK);
+    const int S = pick_split(ntiles * mtiles, cap, K / kTcBK, NT);
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)S, (unsigned)ntiles, (unsigned)mtiles);
     cfg.blockDim = dim3(kTcThreads);

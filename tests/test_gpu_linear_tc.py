@@ -25,6 +25,8 @@ def _no_timeouts(bbc):
     (300, 1024, 2048, 4096, "f16"),     # two activation tiles, the second mostly past M
     (64, 11008, 4096, 64, "bf16"),      # the N = 11008 control shape at M = 64
     (200, 128, 8192, 64, "bf16"),       # a single output tile: eight CTAs share K
+    (300, 4096, 4096, 64, "bf16"),      # 2 x 32 output tiles: K split over a pair of CTAs
+    (256, 11008, 4096, 64, "f16"),      # 86 row tiles of 256 activations: no split
 ])
 def test_nested_tensor_core_path(bbc, M, N, K, bs, dt):
     run_case(bbc, M, N, K, bs, dt, seed=M + K)
