@@ -520,14 +520,37 @@ linear_tc_kernel(const __grid_constant__ CUtensorMap tmx, int M, int64_t N, int6
             for (int c = (own0 & ~15) + 16 * g; c < own0 + W; c += 64) {
                 float v[16];
                 tmem_ld16(lane_tmem + c, v);
+                if (W >= 16) {
+                    // the chunk lies inside the owned columns (both 16-aligned): the partials are read
+                    // four columns at a time, 16-byte loads whose 8-row phases hit different banks
+                    // (WP = W + 4); the sum keeps rank order
 #pragma unroll
-                for (int i = 0; i < 16; i++) {
-                    const int cl = c + i - own0;
-                    if (cl < 0 || cl >= W) continue;
-                    float acc = rank == 0 ? v[i] : recv[row * WP + cl];
-                    for (uint32_t s = 1; s < S; s++)
-                        acc = __fadd_rn(acc, s == rank ? v[i] : recv[((int)s * kTcRows + row) * WP + cl]);
-                    store(c + i, acc);
+                    for (int i = 0; i < 16; i += 4) {
+                        const int cl = c + i - own0;
+                        float4 acc = rank == 0 ? make_float4(v[i], v[i + 1], v[i + 2], v[i + 3])
+                                               : *reinterpret_cast<const float4*>(recv + row * WP + cl);
+                        for (uint32_t s = 1; s < S; s++) {
+                            const float4 p = s == rank ? make_float4(v[i], v[i + 1], v[i + 2], v[i + 3])
+                                                       : *reinterpret_cast<const float4*>(
+                                                             recv + ((int)s * kTcRows + row) * WP + cl);
+                            acc = make_float4(__fadd_rn(acc.x, p.x), __fadd_rn(acc.y, p.y), __fadd_rn(acc.z, p.z),
+                                              __fadd_rn(acc.w, p.w));
+                        }
+                        store(c + i, acc.x);
+                        store(c + i + 1, acc.y);
+                        store(c + i + 2, acc.z);
+                        store(c + i + 3, acc.w);
+                    }
+                } else {
+#pragma unroll
+                    for (int i = 0; i < 16; i++) {
+                        const int cl = c + i - own0;
+                        if (cl < 0 || cl >= W) continue;
+                        float acc = rank == 0 ? v[i] : recv[row * WP + cl];
+                        for (uint32_t s = 1; s < S; s++)
+                            acc = __fadd_rn(acc, s == rank ? v[i] : recv[((int)s * kTcRows + row) * WP + cl]);
+                        store(c + i, acc);
+                    }
                 }
             }
         }
