@@ -233,6 +233,7 @@ linear4_nested_kernel(const uint16_t* __restrict__ X, int M, int64_t N, int64_t 
     __shared__ float c2s[256];
     extern __shared__ __align__(16) uint16_t xs[];              // [M][K + 8] staged X (XS only)
 
+    pdl_wait();               // writes of the previous kernel in the stream are visible from here
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int g = lane >> 2, t = lane & 3;
     const int64_t r0 = (int64_t)blockIdx.x * 16;
@@ -425,6 +426,7 @@ linear_kbit_kernel(const uint16_t* __restrict__ X, int M, int64_t N, int64_t K,
     __shared__ __align__(16) float red5[PAIRS ? 1 : kNWarp * 32 * 4 * NT];     // split-K partials (K = 5)
     extern __shared__ __align__(16) uint16_t xs[];              // [M][K + 8] staged X (XS only)
 
+    pdl_wait();               // writes of the previous kernel in the stream are visible from here
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int g = lane >> 2, t = lane & 3;
     const int64_t r0 = (int64_t)blockIdx.x * 16;
@@ -513,9 +515,8 @@ cudaError_t launch_nt(const uint16_t* X, int M, int64_t N, int64_t K, const uint
     const cudaError_t e = allow_dyn_smem(k, attr, XS ? kMaxXs : 0);
     if (e != cudaSuccess) return e;
     const size_t dyn = XS ? (size_t)M * (size_t)(K + 8) * 2 : 0;
-    k<<<(unsigned)(N / 16), kLinThreads, dyn, s>>>(X, M, N, K, codes, absmax_q, code2, absmax2, offset, code4,
-                                                   log2_bs, Y);
-    return cudaGetLastError();
+    return launch_pdl(k, (unsigned)(N / 16), kLinThreads, dyn, s, X, M, N, K, codes, absmax_q, code2, absmax2, offset,
+                      code4, log2_bs, Y);
 }
 
 template <int DT>
@@ -541,8 +542,7 @@ cudaError_t launch_kbit_nt(const uint16_t* X, int M, int64_t N, int64_t K, const
     const cudaError_t e = allow_dyn_smem(k, attr, XS ? kMaxXs : 0);
     if (e != cudaSuccess) return e;
     const size_t dyn = XS ? (size_t)M * (size_t)(K + 8) * 2 : 0;
-    k<<<(unsigned)(N / 16), kLinThreads, dyn, s>>>(X, M, N, K, packed, absmax, codebook, Y);
-    return cudaGetLastError();
+    return launch_pdl(k, (unsigned)(N / 16), kLinThreads, dyn, s, X, M, N, K, packed, absmax, codebook, Y);
 }
 
 template <int DT, int KB>

@@ -314,6 +314,7 @@ template <int DT, int NT, bool NESTED, int KB>
 __global__ void __launch_bounds__(kTcThreads, 1)
 linear_tc_kernel(const __grid_constant__ CUtensorMap tmx, int M, int64_t N, int64_t K, NestedW nw, KbitW kw,
                  uint16_t* __restrict__ Y) {
+    pdl_wait();               // writes of the previous kernel in the stream are visible from here
     using L = TcSmem<NT>;
     constexpr int XS = L::kXStages, WS = kTcWStages;
     extern __shared__ uint8_t smem_raw[];
@@ -639,13 +640,17 @@ cudaError_t launch_tc(const uint16_t* X, int M, int64_t N, int64_t K, const Nest
     cfg.blockDim = dim3(kTcThreads);
     cfg.dynamicSmemBytes = L::kAlloc;
     cfg.stream = s;
-    cudaLaunchAttribute attr_c[1];
-    attr_c[0].id = cudaLaunchAttributeClusterDimension;
-    attr_c[0].val.clusterDim.x = (unsigned)S;
-    attr_c[0].val.clusterDim.y = 1;
-    attr_c[0].val.clusterDim.z = 1;
+    // programmatic stream serialisation (the kernel's first act is griddepcontrol.wait), and the
+    // cluster of the K split when there is one
+    cudaLaunchAttribute attr_c[2];
+    attr_c[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr_c[0].val.programmaticStreamSerializationAllowed = 1;
+    attr_c[1].id = cudaLaunchAttributeClusterDimension;
+    attr_c[1].val.clusterDim.x = (unsigned)S;
+    attr_c[1].val.clusterDim.y = 1;
+    attr_c[1].val.clusterDim.z = 1;
     cfg.attrs = attr_c;
-    cfg.numAttrs = S > 1 ? 1 : 0;
+    cfg.numAttrs = S > 1 ? 2 : 1;
     return cudaLaunchKernelEx(&cfg, k, map, M, N, K, nw, kw, Y);
 }
 
