@@ -338,6 +338,24 @@ linear_tc_kernel(const __grid_constant__ CUtensorMap tmx, int M, int64_t N, int6
     const int64_t c_lo = C * rank / S;
     const int nchunks = (int)(C * (rank + 1) / S - c_lo);
 
+    // Decoder thread (warps 2..): one weight row (its tensor-memory lane) and one quarter (16 k) of a
+    // stage's 64 k. Its first kPrefetch stages of inputs are loaded before the set-up below, so that
+    // their latency overlaps the tables, the barriers and the tensor-memory allocation.
+    const int64_t d_mrow = (n0 + 32 * (warp & 3) + lane) * K + c_lo * kTcBK + 16 * ((warp - 2) >> 2);
+    using In = std::conditional_t<NESTED, NestedIn, KbitIn<KB>>;
+    auto load_in = [&](int i) -> In {
+        const int64_t m0 = d_mrow + (int64_t)i * kTcBK;
+        if (!BBC_GUARD(m0 >= 0 && m0 + 16 <= N * K, kGuardLinear)) return In{};
+        if constexpr (NESTED) return load_nested16(nw, m0);
+        else return load_kbit32<KB>(kw, m0 >> 5);
+    };
+    In pre[kPrefetch];
+    if (warp >= 2) {
+#pragma unroll
+        for (int j = 0; j < kPrefetch; j++)
+            if (j < nchunks) pre[j] = load_in(j);
+    }
+
     // ---- set-up: tables, barriers, tensor memory ----
     unsigned char* const pairs = base_p + L::kPairs;
     if (NESTED) {
@@ -409,25 +427,11 @@ linear_tc_kernel(const __grid_constant__ CUtensorMap tmx, int M, int64_t N, int6
         }
     } else {
         // ---- W tiles decoded into tensor memory ----
-        // Thread: one weight row (its tensor-memory lane) and one quarter (16 k) of a stage's 64 k,
-        // i.e. 8 of the stage's 32 A columns. Its inputs are loaded kPrefetch stages ahead of their
-        // decode (a register ring); no shared memory and no proxy fence is involved.
-        const int row = 32 * (warp & 3) + lane;
+        // 8 of a stage's 32 A columns per thread (see d_mrow above). Its inputs are loaded kPrefetch
+        // stages ahead of their decode (a register ring); no shared memory and no proxy fence is
+        // involved.
         const int qk = (warp - 2) >> 2;                           // which 16 of a stage's 64 k
-        const int64_t n = n0 + row;
-        const int64_t mrow = n * K + c_lo * kTcBK + 16 * qk;      // first weight of this thread's stage 0
         const uint32_t lane_a = tmem + ((uint32_t)(32 * (warp & 3)) << 16) + kTmemA + 8u * qk;
-        using In = std::conditional_t<NESTED, NestedIn, KbitIn<KB>>;
-        auto load_in = [&](int i) -> In {
-            const int64_t m0 = mrow + (int64_t)i * kTcBK;
-            if (!BBC_GUARD(m0 >= 0 && m0 + 16 <= N * K, kGuardLinear)) return In{};
-            if constexpr (NESTED) return load_nested16(nw, m0);
-            else return load_kbit32<KB>(kw, m0 >> 5);
-        };
-        In pre[kPrefetch];
-#pragma unroll
-        for (int j = 0; j < kPrefetch; j++)
-            if (j < nchunks) pre[j] = load_in(j);
         const uint32_t lane_off = (uint32_t)(lane & 15) * 8u;
         bool live = true;
         int done_to = 0;                                          // stages whose stores were issued
