@@ -223,3 +223,13 @@ def test_debug_build_exports_the_same_boundary():
 
 def test_debug_status_rejects_a_null_pointer(lib):
     assert lib.bbc_debug_status(None, 0) == 1
+
+
+def test_debug_status_without_a_device_reports_a_cuda_error(lib):
+    """With no usable device the status read fails cleanly (BBC_ERR_CUDA), it does not crash; on
+    a device the release build reports 0."""
+    c = ct.c_uint(123)
+    st = lib.bbc_debug_status(ct.byref(c), 1)
+    assert st in (0, 3), st
+    if st == 0:
+        assert c.value == 0
